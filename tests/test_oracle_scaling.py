@@ -1,0 +1,282 @@
+"""Pins for the oracle's scaling modes (amax, scale, quantize, dequantize, history).
+
+What pins them, other than the oracle itself:
+- the relative-error table printed by the handbook page ("FP8 training")
+- the handbook's exercise 2 (0.01 under a 5000 outlier becomes 0)
+- torch CPU ops restating the handbook's per_tensor / per_block steps (reshape,
+  amax, clamp, the library's float8 cast) with this library's multiply form
+- the closed form of delayed scaling (PyTorch-FP8 page, s4.2 DelayedScaler)
+- invariants: each block whose amax is above eps holds a +-max code; an all
+  zero block gives code 0 and scale max/eps
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import golden_rows
+from fine_grained_block_b200 import inputs
+
+TORCH_FP8 = {oracle.E4M3: torch.float8_e4m3fn, oracle.E5M2: torch.float8_e5m2}
+EPS32 = np.float32(1e-12)
+
+
+def rel_err(q, x):
+    q = np.asarray(q, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    return float(np.linalg.norm(q - x) / np.linalg.norm(x))
+
+
+# -- handbook "FP8 training": per-tensor vs 1x128 relative error ----------------
+
+def test_handbook_relative_error_table():
+    printed = {float(f): (float(t), float(b)) for f, t, b in golden_rows("p3_relerr.txt")}
+    for factor, a in inputs.relerr_outlier_tensors():
+        x = a.numpy()
+        q, s, _ = oracle.quantize_per_tensor(x, oracle.E4M3)
+        y_t = oracle.dequantize(q, oracle.E4M3, np.array([s]))
+        qb, sb = oracle.quantize_blockwise(x, 1, 128, oracle.E4M3)
+        y_b = oracle.dequantize(qb, oracle.E4M3, sb, 1, 128)
+        t = rel_err(y_t[:, 128:], x[:, 128:]) * 100
+        b = rel_err(y_b[:, 128:], x[:, 128:]) * 100
+        want_t, want_b = printed[factor]
+        # the page prints one decimal
+        assert round(t, 1) == want_t, (factor, t)
+        assert round(b, 1) == want_b, (factor, b)
+    # per-tensor error grows with the outlier; the block error stays at the format's precision
+    errs = []
+    for factor, a in inputs.relerr_outlier_tensors():
+        x = a.numpy()
+        q, s, _ = oracle.quantize_per_tensor(x, oracle.E4M3)
+        errs.append(rel_err(oracle.dequantize(q, oracle.E4M3, np.array([s]))[:, 128:], x[:, 128:]))
+    assert errs[0] < errs[1] < errs[2]
+
+
+def test_handbook_exercise_small_value_flushes():
+    for amax, value, fmt, expect in golden_rows("exercise_outlier.txt"):
+        assert fmt == "e4m3fn"
+        rng = np.random.default_rng(5)
+        x = rng.uniform(-1, 1, size=4096).astype(np.float32)
+        x[17] = np.float32(amax)
+        x[100] = np.float32(value)
+        q, s, a = oracle.quantize_per_tensor(x, oracle.E4M3)
+        assert a == np.float32(amax)
+        assert s == np.float32(448.0 / float(amax))
+        got = oracle.decode(int(q[100]), oracle.E4M3)
+        assert got == float(expect) and math.copysign(1, got) == math.copysign(1, float(expect))
+        # the page's reasoning: value * s is below half the smallest subnormal
+        assert abs(float(value)) * float(s) < 2.0 ** -10
+        # and a good share of the values in [-1, 1] land in the subnormal range or at 0,
+        # keeping at most the 3 mantissa bits of a subnormal
+        dec = oracle.decode_table(oracle.E4M3)[q]
+        small = np.abs(x) < 1
+        assert np.mean(np.abs(dec[small]) < 2.0 ** -6) > 0.1
+
+
+# -- torch restatements of the handbook's per_tensor / per_block -------------------
+
+def torch_blockwise(x: torch.Tensor, br: int, bc: int, fmt: int):
+    """The handbook's per_block with reshape / amax / clamp(1e-12), scale = MAX / amax multiplied in.
+
+    Ragged edges are handled by zero padding (zeros never raise an amax)."""
+    MAX = oracle.MAX[fmt]
+    x = x.to(torch.float32)
+    R, C = x.shape
+    Rp, Cp = -(-R // br) * br, -(-C // bc) * bc
+    xp = torch.zeros(Rp, Cp, dtype=torch.float32)
+    xp[:R, :C] = x
+    b = xp.reshape(Rp // br, br, Cp // bc, bc)
+    amax = b.abs().amax(dim=(1, 3), keepdim=True).clamp(min=1e-12)
+    s = torch.tensor(MAX, dtype=torch.float32) / amax
+    q = (b * s).clamp(-MAX, MAX).to(TORCH_FP8[fmt]).view(torch.uint8)
+    return q.reshape(Rp, Cp)[:R, :C].numpy(), s.reshape(Rp // br, Cp // bc).numpy()
+
+
+def torch_per_tensor(x: torch.Tensor, fmt: int, scale=None):
+    MAX = oracle.MAX[fmt]
+    x = x.to(torch.float32)
+    amax = x.abs().max() if x.numel() else torch.tensor(0.0)
+    s = (torch.tensor(MAX, dtype=torch.float32) / amax.clamp(min=1e-12)) if scale is None \
+        else torch.tensor(scale, dtype=torch.float32)
+    q = (x * s).clamp(-MAX, MAX).to(TORCH_FP8[fmt]).view(torch.uint8)
+    return q.numpy(), s.item(), amax.item()
+
+
+def as_oracle_input(t: torch.Tensor):
+    if t.dtype == torch.bfloat16:
+        return inputs.bf16_bits(t)
+    return t.numpy()
+
+
+SHAPES = [(1, 128), (3, 256), (128, 128), (130, 384), (257, 640), (64, 100), (200, 77), (5, 1)]
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("block", [(1, 128), (128, 128)])
+def test_blockwise_vs_torch_handbook_form(fmt, dtype, block):
+    br, bc = block
+    for i, (R, C) in enumerate(SHAPES):
+        x = inputs.random_matrix(R, C, seed=100 + i, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        q, s = oracle.quantize_blockwise(as_oracle_input(x), br, bc, fmt)
+        qt, st = torch_blockwise(x, br, bc, fmt)
+        assert np.array_equal(s, st), (R, C)
+        assert np.array_equal(q, qt), (R, C)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_per_tensor_vs_torch_handbook_form(fmt, dtype):
+    for i, n in enumerate([1, 7, 128, 1000, 65537]):
+        x = inputs.random_matrix(1, n, seed=200 + i, dtype=dtype, outlier_frac=0.002, factor=1e4)
+        q, s, a = oracle.quantize_per_tensor(as_oracle_input(x), fmt)
+        qt, st, at = torch_per_tensor(x, fmt)
+        assert a == np.float32(at) and s == np.float32(st)
+        assert np.array_equal(q, qt)
+        # delayed form: a given scale, values may saturate
+        q2, s2, a2 = oracle.quantize_per_tensor(as_oracle_input(x), fmt, scale=3.0)
+        qt2, _, _ = torch_per_tensor(x, fmt, scale=3.0)
+        assert s2 == np.float32(3.0) and a2 == a
+        assert np.array_equal(q2, qt2)
+
+
+def test_empty_inputs():
+    q, s, a = oracle.quantize_per_tensor(np.zeros(0, dtype=np.float32), oracle.E4M3)
+    assert q.size == 0 and a == 0.0 and s == np.float32(448.0 / np.float64(EPS32))
+    q, s = oracle.quantize_blockwise(np.zeros((0, 256), dtype=np.float32), 1, 128, oracle.E4M3)
+    assert q.size == 0 and s.shape == (0, 2)
+    q, s = oracle.quantize_blockwise(np.zeros((4, 0), dtype=np.float32), 128, 128, oracle.E4M3)
+    assert q.size == 0 and s.shape == (1, 0)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_block_invariants(fmt):
+    top = oracle.top_code(fmt)
+    x = inputs.random_matrix(256, 512, seed=11, dtype=torch.bfloat16, outlier_frac=0.003, factor=1e3)
+    xb = inputs.bf16_bits(x).copy()
+    # zero out a whole 1x128 block and a whole 128x128 block
+    xb[5, 128:256] = 0
+    xb[128:256, 384:512] = 0x8000  # negative zeros
+    for br, bc in ((1, 128), (128, 128)):
+        q, s = oracle.quantize_blockwise(xb, br, bc, fmt)
+        for bi in range(s.shape[0]):
+            for bj in range(s.shape[1]):
+                blk = q[bi * br:(bi + 1) * br, bj * bc:(bj + 1) * bc]
+                xv = (xb[bi * br:(bi + 1) * br, bj * bc:(bj + 1) * bc].astype(np.uint32) << 16).view(np.float32)
+                if np.abs(xv).max() == 0:
+                    assert s[bi, bj] == np.float32(oracle.MAX[fmt] / np.float64(EPS32))
+                    assert np.all((blk & 0x7F) == 0)
+                else:
+                    assert np.any((blk & 0x7F) == top), (br, bi, bj)
+                    assert np.all((blk & 0x7F) <= top)
+
+
+# -- dequantize ---------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_dequantize_vs_torch(fmt):
+    rng = np.random.default_rng(21 + fmt)
+    top = oracle.top_code(fmt)
+    R, C = 256, 384
+    codes = rng.integers(0, top + 1, size=(R, C)).astype(np.uint8) | (rng.integers(0, 2, size=(R, C)) * 0x80).astype(np.uint8)
+    scales_1x128 = np.exp2(rng.uniform(-30, 40, size=(R, 3))).astype(np.float32)
+    scales_128 = np.exp2(rng.uniform(-30, 40, size=(2, 3))).astype(np.float32)
+    qv = torch.from_numpy(codes).view(TORCH_FP8[fmt]).to(torch.float32)
+    cases = [
+        (1, 128, scales_1x128, torch.from_numpy(np.repeat(scales_1x128, 128, axis=1))),
+        (128, 128, scales_128, torch.from_numpy(np.repeat(np.repeat(scales_128, 128, 0), 128, 1))),
+        (0, 0, scales_128.reshape(-1)[:1], torch.from_numpy(scales_128.reshape(-1)[:1])),
+    ]
+    for br, bc, sc, sfull in cases:
+        ref = qv / sfull  # fp32 division, the page's "/ scale"
+        y = oracle.dequantize(codes, fmt, sc, br, bc, out_dtype=oracle.F32)
+        assert np.array_equal(y.view(np.uint32), ref.numpy().view(np.uint32))
+        yb = oracle.dequantize(codes, fmt, sc, br, bc, out_dtype=oracle.BF16)
+        refb = ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(yb, refb)
+
+
+def test_round_trip_error_bound():
+    """Quantize then dequantize stays within half a code spacing of x * s, divided back by s."""
+    x = inputs.random_matrix(128, 1024, seed=31, dtype=torch.float32).numpy()
+    q, s = oracle.quantize_blockwise(x, 1, 128, oracle.E4M3)
+    y = oracle.dequantize(q, oracle.E4M3, s, 1, 128)
+    srep = np.repeat(s, 128, axis=1).astype(np.float64)
+    xs = x.astype(np.float64) * srep
+    err = np.abs(y.astype(np.float64) * srep - xs)
+    # E4M3: normal spacing is 2^(e-3); allow the fp32 rounding of the product and of the quotient
+    bound = np.maximum(np.exp2(np.floor(np.log2(np.maximum(np.abs(xs), 2.0 ** -6))) - 4), 2.0 ** -10)
+    assert np.all(err <= bound * (1 + 1e-6) + np.abs(xs) * 2.0 ** -22)
+
+
+# -- delayed scaling: closed form -----------------------------------------------
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_delayed_scaling_closed_form(fmt):
+    W, steps = 16, 32
+    base = inputs.gradient_base(rows=64, cols=256)
+    hist = oracle.AmaxHistory(W, fmt)
+    amaxes, used = [], []
+    for k in range(steps):
+        g = inputs.gradient_step(base, k)
+        s_used = hist.scale[0]
+        q, s, a = oracle.quantize_per_tensor(inputs.bf16_bits(g), fmt, scale=float(s_used))
+        qt, _, at = torch_per_tensor(g, fmt, scale=float(s_used))
+        assert np.array_equal(q, qt) and a == np.float32(at)
+        used.append(s)
+        amaxes.append(float(a))
+        hist.update(a)
+    MAX = oracle.MAX[fmt]
+    for k in range(steps):
+        if k < W:
+            assert used[k] == np.float32(1.0), k
+        else:
+            window = max(amaxes[k - W:k])
+            assert used[k] == np.float32(MAX / max(window, float(EPS32))), k
+    assert hist.state[1] == W and hist.state[0] == steps % W
+
+
+def test_delayed_scaling_underflow_then_recovers():
+    """Gradients of 1e-6 flush to zero in E5M2 at scale 1, and survive once the window scale applies."""
+    base = inputs.gradient_base(rows=64, cols=256)
+    g = inputs.gradient_step(base, 0)
+    gb = inputs.bf16_bits(g)
+    q1, _, _ = oracle.quantize_per_tensor(gb, oracle.E5M2, scale=1.0)
+    frac_zero_s1 = np.mean((q1 & 0x7F) == 0)
+    q2, s2, _ = oracle.quantize_per_tensor(gb, oracle.E5M2)
+    frac_zero_cur = np.mean((q2 & 0x7F) == 0)
+    assert frac_zero_s1 > 0.1 and frac_zero_cur == 0.0
+
+
+# -- the fp32 product rounds before the cast -------------------------------------
+
+def test_product_rounded_to_fp32_before_cast():
+    """x * s is an fp32 op in the pages' code, so it rounds to fp32 before the cast.
+
+    Find products whose exact value lies just off an E4M3 midpoint but whose
+    fp32 rounding lands on it.  The oracle must follow the fp32 value (and agree
+    with torch's x * s then cast); rounding the exact product instead would pick
+    the neighbour on the exact value's side, which differs for some of them."""
+    rng = np.random.default_rng(3)
+    found = differs = 0
+    for _ in range(400_000):
+        x = np.float32(rng.uniform(1, 2))
+        j = int(rng.integers(0, 7))
+        target = np.float32(1.0625 + 0.125 * j)  # midpoint between E4M3 codes 0x38+j and 0x39+j
+        s = np.float32(target / x)
+        p32 = np.float32(np.float64(x) * np.float64(s))
+        exact = np.float64(x) * np.float64(s)
+        if p32 != target or exact == np.float64(target):
+            continue
+        found += 1
+        code = int(oracle.quantize_per_tensor(np.array([x]), oracle.E4M3, scale=float(s))[0][0])
+        ref = (torch.tensor([x]) * torch.tensor(s)).to(torch.float8_e4m3fn).view(torch.uint8).item()
+        assert code == ref
+        assert code in (0x38 + j, 0x39 + j) and code % 2 == 0  # the tie went to the even code
+        exact_side = 0x39 + j if exact > np.float64(target) else 0x38 + j
+        differs += int(exact_side != code)
+        if found >= 60:
+            break
+    assert found >= 20 and differs >= 5
