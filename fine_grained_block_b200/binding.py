@@ -1,0 +1,189 @@
+"""ctypes binding of ``libfp8q.so`` -- argument marshalling only.
+
+Two layers with the C names:
+
+* ``lib()`` returns the loaded ``ctypes.CDLL`` whose functions take the exact
+  C arguments (device pointers as ints, sizes, enums, a stream handle).
+* ``fp8_quantize_per_tensor``, ``fp8_quantize_blockwise``, ``fp8_dequantize``
+  and ``fp8_amax_history_update`` below take torch CUDA tensors, allocate any
+  output the caller did not pass (``torch.empty`` on the input's device), pass
+  pointers and the current stream to the C function, and raise ``FP8Error`` on
+  a nonzero status.  All computation happens in the library's kernels; there
+  is no CPU fallback, and a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+E4M3, E5M2 = 0, 1
+F32, BF16 = 0, 1
+FP8_MAX = {E4M3: 448.0, E5M2: 57344.0}
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp8q.so")
+_lib = None
+
+# Declared in include/fp8q.h: name -> (restype, argtypes)
+_c_int, _i64, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+SIGNATURES = {
+    "fp8_quantize_per_tensor": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _vp, _vp]),
+    "fp8_quantize_blockwise": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "fp8_dequantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _c_int, _vp]),
+    "fp8_amax_history_update": (_c_int, [_vp, _vp, _c_int, _vp, _c_int, _vp, _vp]),
+    "fp8_status_string": (ctypes.c_char_p, [_c_int]),
+}
+
+
+class FP8Error(RuntimeError):
+    """A libfp8q call returned an error status."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({fp8_status_string(status)})")
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libfp8q.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(
+            f"{p} is missing: build it with `python -m fine_grained_block_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = L
+    return L
+
+
+lib = load_library
+
+
+def fp8_status_string(status: int) -> str:
+    return load_library().fp8_status_string(int(status)).decode()
+
+
+# -- marshalling helpers ----------------------------------------------------------
+
+_DTYPE_CODE = {torch.float32: F32, torch.bfloat16: BF16}
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libfp8q works on CUDA tensors only")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("libfp8q needs contiguous tensors")
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise FP8Error(fn, status)
+
+
+# -- entry points -------------------------------------------------------------------
+
+def fp8_quantize_per_tensor(x: torch.Tensor, fmt: int = E4M3, scale_in: torch.Tensor | None = None,
+                            q: torch.Tensor | None = None, scale_out: torch.Tensor | None = None,
+                            amax_out: torch.Tensor | None = None, want_amax: bool = True, stream=None):
+    """Per-tensor quantize.  scale_in None = current scaling, else delayed (a 1-element fp32 CUDA tensor).
+
+    Returns (q uint8 like x, scale_out [1] fp32, amax_out [1] fp32 or None)."""
+    _need_cuda(x, scale_in, q, scale_out, amax_out)
+    dev = x.device
+    q = torch.empty(x.shape, dtype=torch.uint8, device=dev) if q is None else q
+    scale_out = torch.empty(1, dtype=torch.float32, device=dev) if scale_out is None else scale_out
+    if amax_out is None and (want_amax or scale_in is None):
+        amax_out = torch.empty(1, dtype=torch.float32, device=dev)
+    st = load_library().fp8_quantize_per_tensor(_ptr(x), _DTYPE_CODE[x.dtype], x.numel(), fmt, _ptr(scale_in),
+                                                _ptr(q), _ptr(scale_out), _ptr(amax_out), _stream(stream))
+    _check("fp8_quantize_per_tensor", st)
+    return q, scale_out, amax_out
+
+
+def fp8_quantize_blockwise(x: torch.Tensor, block=(1, 128), fmt: int = E4M3, q: torch.Tensor | None = None,
+                           scales: torch.Tensor | None = None, stream=None):
+    """Blockwise quantize of a 2-D tensor with (1, 128) or (128, 128) blocks.  Returns (q, scales)."""
+    _need_cuda(x, q, scales)
+    if x.dim() != 2:
+        raise ValueError("blockwise quantize takes a 2-D tensor")
+    R, C = x.shape
+    br, bc = block
+    q = torch.empty((R, C), dtype=torch.uint8, device=x.device) if q is None else q
+    if scales is None:
+        scales = torch.empty((math.ceil(R / br), math.ceil(C / bc)), dtype=torch.float32, device=x.device)
+    st = load_library().fp8_quantize_blockwise(_ptr(x), _DTYPE_CODE[x.dtype], R, C, br, bc, fmt, _ptr(q),
+                                               _ptr(scales), _stream(stream))
+    _check("fp8_quantize_blockwise", st)
+    return q, scales
+
+
+def fp8_dequantize(q: torch.Tensor, scales: torch.Tensor, block=(0, 0), fmt: int = E4M3,
+                   out_dtype=torch.bfloat16, y: torch.Tensor | None = None, stream=None):
+    """Dequantize codes; block (0, 0) = per-tensor (scales[0]).  Returns y."""
+    _need_cuda(q, scales, y)
+    if q.dim() == 1:
+        R, C = 1, q.shape[0]
+    elif q.dim() == 2:
+        R, C = q.shape
+    else:
+        raise ValueError("dequantize takes a 1-D or 2-D tensor")
+    y = torch.empty(q.shape, dtype=out_dtype, device=q.device) if y is None else y
+    st = load_library().fp8_dequantize(_ptr(q), fmt, R, C, block[0], block[1], _ptr(scales), _ptr(y),
+                                       _DTYPE_CODE[y.dtype], _stream(stream))
+    _check("fp8_dequantize", st)
+    return y
+
+
+def fp8_amax_history_update(history: torch.Tensor, state: torch.Tensor, amax: torch.Tensor, scale: torch.Tensor,
+                            fmt: int = E4M3, stream=None):
+    """Push amax into the history ring and refresh scale in place (all 4 are CUDA tensors)."""
+    _need_cuda(history, state, amax, scale)
+    st = load_library().fp8_amax_history_update(_ptr(history), _ptr(state), history.numel(), _ptr(amax), fmt,
+                                                _ptr(scale), _stream(stream))
+    _check("fp8_amax_history_update", st)
+    return scale
+
+
+class DelayedScaler:
+    """Device-resident delayed-scaling state (history ring, {pos, count}, scale), after the
+    PyTorch-FP8 page's DelayedScaler (s4.2).  step(x) quantizes x with the current scale, then
+    pushes amax(x) into the history -- all on the device, no host round trip."""
+
+    def __init__(self, window: int = 16, fmt: int = E5M2, device="cuda"):
+        self.fmt = fmt
+        self.history = torch.zeros(window, dtype=torch.float32, device=device)
+        self.state = torch.zeros(2, dtype=torch.int32, device=device)
+        self.scale = torch.ones(1, dtype=torch.float32, device=device)
+        self.amax = torch.zeros(1, dtype=torch.float32, device=device)
+        self.scale_used = torch.ones(1, dtype=torch.float32, device=device)
+
+    def step(self, x: torch.Tensor, q: torch.Tensor | None = None, stream=None):
+        q, s, _ = fp8_quantize_per_tensor(x, self.fmt, scale_in=self.scale, q=q, scale_out=self.scale_used,
+                                          amax_out=self.amax, stream=stream)
+        fp8_amax_history_update(self.history, self.state, self.amax, self.scale, self.fmt, stream=stream)
+        return q, self.scale_used

@@ -1,0 +1,141 @@
+// fp8q_abi.cu -- the C ABI of libfp8q (declared in include/fp8q.h).
+//
+// Each entry point checks every argument on the host, then enqueues its
+// kernels on the caller's stream and returns.  Nothing here allocates,
+// synchronizes or keeps state between calls, apart from a per-device cache of
+// the SM count.
+
+#include <atomic>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "fp8q.h"
+#include "fp8q_launch.h"
+
+namespace fp8q {
+
+int device_sm_count() {
+    static std::atomic<int> cache[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+}  // namespace fp8q
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool fmt_ok(int fmt) { return fmt == FP8_E4M3 || fmt == FP8_E5M2; }
+bool dtype_ok(int dt) { return dt == FP8_F32 || dt == FP8_BF16; }
+
+// rows * cols without overflow (both >= 0); -1 if it would overflow.
+int64_t checked_count(int64_t rows, int64_t cols) {
+    if (rows == 0 || cols == 0) return 0;
+    if (rows > INT64_MAX / cols) return -1;
+    return rows * cols;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int fp8_quantize_per_tensor(const void* x, int dtype, int64_t n, int fmt, const float* scale_in, uint8_t* q,
+                            float* scale_out, float* amax_out, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (scale_out == nullptr) return FP8_ERR_NULL;
+    if (scale_in == nullptr && amax_out == nullptr) return FP8_ERR_NULL;
+    if (n > 0 && (x == nullptr || q == nullptr)) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale_out, 4) || !aligned(scale_in, 4) ||
+        !aligned(amax_out, 4))
+        return FP8_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (amax_out != nullptr) {
+        cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), st);
+        if (e != cudaSuccess) return FP8_ERR_CUDA;
+    }
+    if (scale_in == nullptr && n > 0) {
+        cudaError_t e = fp8q::launch_tensor_amax(x, dtype, n, amax_out, st);
+        if (e != cudaSuccess) return FP8_ERR_CUDA;
+    }
+    return status_of(fp8q::launch_tensor_cast(x, dtype, n, fmt, scale_in, amax_out, q, scale_out,
+                                              scale_in ? amax_out : nullptr, st));
+}
+
+int fp8_quantize_blockwise(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows, int block_cols,
+                           int fmt, uint8_t* q, float* scales, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    if (!((block_rows == 1 || block_rows == 128) && block_cols == 128)) return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (n == 0) return FP8_OK;  // no element, no block, no scale
+    if (x == nullptr || q == nullptr || scales == nullptr) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scales, 4)) return FP8_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (cols % 128 != 0) {
+        e = fp8q::launch_quant_block_general(x, dtype, rows, cols, block_rows, block_cols, fmt, q, scales, st);
+    } else if (block_rows == 1) {
+        e = fp8q::launch_quant_1x128(x, dtype, n / 128, fmt, q, scales, st);
+    } else {
+        e = fp8q::launch_quant_128x128(x, dtype, rows, cols, fmt, q, scales, st);
+    }
+    return status_of(e);
+}
+
+int fp8_dequantize(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int block_rows, int block_cols,
+                   const float* scales, void* y, int out_dtype, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(out_dtype)) return FP8_ERR_DTYPE;
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    int mode;
+    if (block_rows == 0 && block_cols == 0) mode = 0;
+    else if (block_rows == 1 && block_cols == 128) mode = 1;
+    else if (block_rows == 128 && block_cols == 128) mode = 2;
+    else return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (n == 0) return FP8_OK;
+    if (q == nullptr || scales == nullptr || y == nullptr) return FP8_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(y, 16) || !aligned(scales, 4)) return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_dequant(q, fmt, rows, cols, mode, scales, y, out_dtype,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_amax_history_update(float* history, int32_t* state, int window, const float* amax, int fmt, float* scale,
+                            void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (window <= 0 || window > 65536) return FP8_ERR_ARG;
+    if (history == nullptr || state == nullptr || amax == nullptr || scale == nullptr) return FP8_ERR_NULL;
+    if (!aligned(history, 4) || !aligned(state, 4) || !aligned(amax, 4) || !aligned(scale, 4)) return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_amax_history_update(history, state, window, amax, fmt, scale,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
+const char* fp8_status_string(int status) {
+    switch (status) {
+        case FP8_OK: return "ok";
+        case FP8_ERR_NULL: return "a required pointer is NULL";
+        case FP8_ERR_SHAPE: return "invalid size or unsupported block shape";
+        case FP8_ERR_ALIGN: return "pointer not aligned (tensors: 16 bytes, scalars: 4 bytes)";
+        case FP8_ERR_FORMAT: return "fmt is not FP8_E4M3 or FP8_E5M2";
+        case FP8_ERR_DTYPE: return "dtype is not FP8_F32 or FP8_BF16";
+        case FP8_ERR_CUDA: return "a CUDA call or kernel launch failed";
+        case FP8_ERR_ARG: return "invalid argument";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// fp8q_launch.h -- internal host-side launchers of libfp8q (not part of the ABI).
+//
+// The C ABI (fp8q_abi.cu) validates arguments and calls these; each one picks
+// a launch shape for the current device and enqueues kernels on `stream`.
+// They return the first CUDA error seen (cudaSuccess when all launches went
+// in).  None of them allocates or synchronizes.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8q {
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+// 1x128 blocks over a [rows, cols] tensor with cols % 128 == 0: the blocks
+// are the n / 128 consecutive 128-element runs, scales are one per run.
+cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fmt,
+                               uint8_t* q, float* scales, cudaStream_t stream);
+
+// 128x128 blocks over [rows, cols], cols % 128 == 0, any rows.
+cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
+                                 uint8_t* q, float* scales, cudaStream_t stream);
+
+// Any block shape, any cols (ragged right edge), element-wise accesses.
+cudaError_t launch_quant_block_general(const void* x, int dtype, int64_t rows, int64_t cols,
+                                       int block_rows, int block_cols, int fmt,
+                                       uint8_t* q, float* scales, cudaStream_t stream);
+
+// Per-tensor: amax of x into *amax_out (which the caller has zeroed).
+cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_out,
+                               cudaStream_t stream);
+
+// Per-tensor cast.  scale_in == nullptr: s from *amax_in (current scaling);
+// else s = *scale_in (delayed), and amax_out (if non-null, zeroed by the
+// caller) receives amax(x) from the same pass.  *scale_out = s.
+cudaError_t launch_tensor_cast(const void* x, int dtype, int64_t n, int fmt,
+                               const float* scale_in, const float* amax_in,
+                               uint8_t* q, float* scale_out, float* amax_out,
+                               cudaStream_t stream);
+
+// Dequantize.  mode 0: per-tensor; 1: 1x128; 2: 128x128.
+cudaError_t launch_dequant(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int mode,
+                           const float* scales, void* y, int out_dtype, cudaStream_t stream);
+
+// Delayed-scaling history update (one warp).
+cudaError_t launch_amax_history_update(float* history, int32_t* state, int window,
+                                       const float* amax, int fmt, float* scale,
+                                       cudaStream_t stream);
+
+}  // namespace fp8q

@@ -1,0 +1,166 @@
+/*
+ * fp8q.h -- C ABI of libfp8q, FP8 scaled quantization on NVIDIA B200 (sm_100a).
+ *
+ * The library computes the data-parallel path of FP8 mixed-precision
+ * training described on two pages:
+ *   [FP8-native]  PyTorch native FP8 dtypes (m.nxbn.cn/news/137885):
+ *                 s1.2 format table, s1.3 finite-only saturation,
+ *                 s4.1 scale = max_val / amax, s4.2 delayed scaling.
+ *   [MP-handbook] Mixed precision and FP8 training (anrans.github.io,
+ *                 ai-infra-handbooks/train/practice/mixed-precision),
+ *                 section "FP8 training": per-tensor vs 1x128 / 128x128
+ *                 block scaling (quant, per_tensor, per_block).
+ *
+ * Arithmetic, identical in every entry point:
+ *   amax  = max |x| over the scaled group (a block, or the whole tensor)
+ *   s     = fp32( MAX / max(amax, 1e-12f) ),  MAX = 448 (E4M3), 57344 (E5M2)
+ *   q     = fp8_rne_satfinite( fp32(x * s) )   x widened to fp32 exactly
+ *   y     = fp32( decode(q) / s ),  bf16 output = bf16_rne(y)
+ * The stored scale is the multiplier s (not its reciprocal).  Casts round to
+ * nearest-even and saturate: no Inf is ever produced, and E4M3 has no Inf.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or keeps them.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream), never synchronizes, and is
+ *     safe to call from several host threads.  Calls that touch the same
+ *     buffers must be ordered by the caller (same stream or events).
+ *   - Tensors are contiguous and row-major, [rows, cols] with cols innermost.
+ *   - x, q and y must be 16-byte aligned; scale, amax and history pointers
+ *     4-byte aligned.  Anything else returns FP8_ERR_ALIGN.
+ *   - Arguments are checked before anything is launched; on an error return
+ *     nothing has been enqueued.  A launch failure returns FP8_ERR_CUDA.
+ *     Faults inside a kernel surface at the caller's next synchronization,
+ *     as with any CUDA work.
+ *   - Element counts may be 0 (nothing is launched unless a scale or amax
+ *     output has to be written).
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* FP8 formats ([FP8-native] s1.2): E4M3 = float8_e4m3fn (bias 7, max 448,
+ * no Inf, 0x7F/0xFF are NaN); E5M2 = float8_e5m2 (bias 15, max 57344). */
+enum fp8_format { FP8_E4M3 = 0, FP8_E5M2 = 1 };
+
+/* Element types of high-precision tensors. */
+enum fp8_dtype { FP8_F32 = 0, FP8_BF16 = 1 };
+
+/* Status codes.  0 is success; every error is negative. */
+enum fp8_status {
+    FP8_OK = 0,
+    FP8_ERR_NULL = -1,          /* a required pointer is NULL */
+    FP8_ERR_SHAPE = -2,         /* negative size, or an unsupported block shape */
+    FP8_ERR_ALIGN = -3,         /* a pointer is not aligned as stated above */
+    FP8_ERR_FORMAT = -4,        /* fmt is not an fp8_format */
+    FP8_ERR_DTYPE = -5,         /* dtype is not an fp8_dtype */
+    FP8_ERR_CUDA = -6,          /* a CUDA call or launch failed */
+    FP8_ERR_ARG = -7            /* any other invalid argument (e.g. window <= 0) */
+};
+
+/*
+ * Per-tensor quantization: one scale for the whole tensor.
+ * Follows [MP-handbook] "FP8 training" per_tensor and [FP8-native] s4.1-s4.2.
+ *
+ *   x          [n] input, dtype FP8_F32 or FP8_BF16 (any n >= 0)
+ *   scale_in   NULL: current scaling -- s is computed from amax(x) in this
+ *              call (two passes over x: amax, then cast).
+ *              non-NULL: delayed scaling -- device pointer to one fp32 scale
+ *              made from earlier steps (e.g. by fp8_amax_history_update);
+ *              x is cast with it in one pass, values beyond range saturate.
+ *   q          [n] output codes (uint8 bit patterns of fmt)
+ *   scale_out  [1] output: the scale used.  May equal scale_in.
+ *   amax_out   [1] output: amax(x) (0 for n == 0).  Required with current
+ *              scaling; with delayed scaling it may be NULL, which skips the
+ *              amax reduction.
+ * Errors: FP8_ERR_NULL (x or q NULL with n > 0, scale_out NULL, amax_out
+ * NULL with scale_in NULL), FP8_ERR_SHAPE (n < 0), FP8_ERR_ALIGN,
+ * FP8_ERR_FORMAT, FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_quantize_per_tensor(const void *x, int dtype, int64_t n, int fmt,
+                            const float *scale_in, uint8_t *q,
+                            float *scale_out, float *amax_out, void *stream);
+
+/*
+ * Fine-grained (blockwise) quantization: one scale per block_rows x
+ * block_cols block, in one fused pass (amax, scale, cast, scale store).
+ * Follows [MP-handbook] "FP8 training" per_block: 1x128 blocks for
+ * activations, 128x128 blocks for weights.
+ *
+ *   x          [rows, cols] input, FP8_F32 or FP8_BF16
+ *   block_rows, block_cols   (1, 128) or (128, 128); anything else is
+ *              FP8_ERR_SHAPE
+ *   q          [rows, cols] output codes
+ *   scales     [ceil(rows / block_rows), ceil(cols / 128)] fp32, row-major;
+ *              scales[i][j] is the s of the block whose top-left element is
+ *              (i * block_rows, j * 128).
+ * Ragged edges: when rows or cols is not a multiple of the block, the last
+ * blocks hold only the elements inside the tensor (their amax is taken over
+ * those elements).  cols % 128 == 0 takes the fast kernels; other widths
+ * take a slower general kernel with the same results.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_FORMAT,
+ * FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_quantize_blockwise(const void *x, int dtype, int64_t rows, int64_t cols,
+                           int block_rows, int block_cols, int fmt,
+                           uint8_t *q, float *scales, void *stream);
+
+/*
+ * Dequantization: y = fp32(decode(q) / s), with s the scale of q's block.
+ * Follows [FP8-native] s4.1 (divide by the scale to restore) and s4.2
+ * quantize() (.to(dtype) / scale).
+ *
+ *   q          [rows, cols] codes of fmt
+ *   block_rows, block_cols   (0, 0): per-tensor, scales[0] for everything;
+ *              (1, 128) or (128, 128): the scale layout of
+ *              fp8_quantize_blockwise.
+ *   scales     fp32 scales (multipliers, as produced by the quantizers)
+ *   y          [rows, cols] output, out_dtype FP8_F32 or FP8_BF16 (bf16 is
+ *              the fp32 quotient rounded to nearest-even)
+ * Results are bit-exact IEEE quotients for every scale.  NaN codes give NaN.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_FORMAT,
+ * FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_dequantize(const uint8_t *q, int fmt, int64_t rows, int64_t cols,
+                   int block_rows, int block_cols, const float *scales,
+                   void *y, int out_dtype, void *stream);
+
+/*
+ * Delayed scaling: push one amax into the amax history and refresh the scale.
+ * Follows [FP8-native] s4.2 DelayedScaler.update: the last `window` amax
+ * values are kept; once `window` of them have been seen, the scale becomes
+ * MAX / max(max(history), 1e-12f); before that it is left unchanged.
+ *
+ *   history    [window] fp32 ring buffer (device)
+ *   state      [2] int32 (device): state[0] = next slot, state[1] = number
+ *              of valid entries (saturates at window)
+ *   amax       [1] fp32 (device): this step's amax, e.g. the amax_out of
+ *              fp8_quantize_per_tensor
+ *   scale      [1] fp32 (device), in/out
+ * Before the first step the caller zeroes history and state and sets
+ * *scale = 1.0f.  The state is plain device memory: copying history, state
+ * and scale checkpoints and restores it.  A state outside its range is
+ * clamped into range on the device (pos taken modulo window, count clamped
+ * to [0, window]) rather than faulting.
+ * One single-warp launch; runs entirely on the device, no host sync.
+ * Errors: FP8_ERR_NULL, FP8_ERR_ALIGN, FP8_ERR_FORMAT, FP8_ERR_ARG
+ * (window <= 0 or window > 65536), FP8_ERR_CUDA.
+ */
+int fp8_amax_history_update(float *history, int32_t *state, int window,
+                            const float *amax, int fmt, float *scale,
+                            void *stream);
+
+/* Static, human-readable text for a status code (never NULL). */
+const char *fp8_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -1,0 +1,138 @@
+"""The C-ABI library loads, exports every function include/fp8q.h declares, and
+rejects bad arguments on the host before touching CUDA.  No compute runs here:
+these calls return before any kernel launch, so they work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fine_grained_block_b200 import build as fbuild
+from fine_grained_block_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_FORMAT, ERR_DTYPE, ERR_CUDA, ERR_ARG = 0, -1, -2, -3, -4, -5, -6, -7
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fp8_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return binding.load_library()
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(["fp8_quantize_per_tensor", "fp8_quantize_blockwise", "fp8_dequantize",
+                                           "fp8_amax_history_update", "fp8_status_string"])
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in binding.SIGNATURES
+    assert set(binding.SIGNATURES) == set(declared_functions())
+
+
+def test_exported_symbols_are_c_linkage():
+    out = os.popen(f"nm -D --defined-only {binding.LIB_PATH}").read()
+    exported = set(re.findall(r" T (fp8_\w+)$", out, flags=re.M))
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(L):
+    for st in (OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_FORMAT, ERR_DTYPE, ERR_CUDA, ERR_ARG):
+        s = binding.fp8_status_string(st)
+        assert s and s != "unknown status"
+    assert binding.fp8_status_string(12345) == "unknown status"
+
+
+# Fake (never dereferenced) device addresses: validation rejects before any use.
+A16 = 0x7F0000000000
+A4 = A16 + 4
+A1 = A16 + 1
+
+
+def test_blockwise_validation(L):
+    f = L.fp8_quantize_blockwise
+    assert f(A16, 1, 4, 256, 1, 128, 7, A16, A16, None) == ERR_FORMAT
+    assert f(A16, 3, 4, 256, 1, 128, 0, A16, A16, None) == ERR_DTYPE
+    assert f(A16, 1, -1, 256, 1, 128, 0, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 4, 256, 2, 128, 0, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 4, 256, 1, 64, 0, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 4, 256, 128, 256, 0, A16, A16, None) == ERR_SHAPE
+    assert f(None, 1, 4, 256, 1, 128, 0, A16, A16, None) == ERR_NULL
+    assert f(A16, 1, 4, 256, 1, 128, 0, None, A16, None) == ERR_NULL
+    assert f(A16, 1, 4, 256, 1, 128, 0, A16, None, None) == ERR_NULL
+    assert f(A1, 1, 4, 256, 1, 128, 0, A16, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 4, 256, 1, 128, 0, A4, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 4, 256, 1, 128, 0, A16, A1, None) == ERR_ALIGN
+    assert f(A16, 1, 1 << 62, 1 << 62, 1, 128, 0, A16, A16, None) == ERR_SHAPE
+    # empty tensors: nothing to do, nothing launched, null pointers allowed
+    assert f(None, 1, 0, 256, 1, 128, 0, None, None, None) == OK
+    assert f(None, 1, 4, 0, 128, 128, 0, None, None, None) == OK
+
+
+def test_dequant_validation(L):
+    f = L.fp8_dequantize
+    assert f(A16, 2, 4, 256, 1, 128, A16, A16, 1, None) == ERR_FORMAT
+    assert f(A16, 0, 4, 256, 1, 128, A16, A16, 2, None) == ERR_DTYPE
+    assert f(A16, 0, 4, 256, 1, 64, A16, A16, 1, None) == ERR_SHAPE
+    assert f(A16, 0, 4, 256, 0, 128, A16, A16, 1, None) == ERR_SHAPE
+    assert f(A16, 0, -4, 256, 0, 0, A16, A16, 1, None) == ERR_SHAPE
+    assert f(None, 0, 4, 256, 0, 0, A16, A16, 1, None) == ERR_NULL
+    assert f(A16, 0, 4, 256, 0, 0, None, A16, 1, None) == ERR_NULL
+    assert f(A16, 0, 4, 256, 0, 0, A16, None, 1, None) == ERR_NULL
+    assert f(A4, 0, 4, 256, 0, 0, A16, A16, 1, None) == ERR_ALIGN
+    assert f(A16, 0, 4, 256, 0, 0, A16, A4, 1, None) == ERR_ALIGN
+    assert f(A16, 0, 4, 256, 0, 0, A1, A16, 1, None) == ERR_ALIGN
+    assert f(None, 0, 0, 0, 0, 0, None, None, 1, None) == OK
+
+
+def test_per_tensor_validation(L):
+    f = L.fp8_quantize_per_tensor
+    assert f(A16, 1, 16, 5, None, A16, A16, A16, None) == ERR_FORMAT
+    assert f(A16, 9, 16, 0, None, A16, A16, A16, None) == ERR_DTYPE
+    assert f(A16, 1, -16, 0, None, A16, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 16, 0, None, A16, None, A16, None) == ERR_NULL      # scale_out required
+    assert f(A16, 1, 16, 0, None, A16, A16, None, None) == ERR_NULL      # amax_out required for current scaling
+    assert f(None, 1, 16, 0, A16, A16, A16, None, None) == ERR_NULL
+    assert f(A16, 1, 16, 0, A16, None, A16, None, None) == ERR_NULL
+    assert f(A1, 1, 16, 0, None, A16, A16, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, None, A4, A16, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, A1, A16, A16, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, None, A16, A1, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, None, A16, A16, A1, None) == ERR_ALIGN
+
+
+def test_history_validation(L):
+    f = L.fp8_amax_history_update
+    assert f(A16, A16, 16, A16, 3, A16, None) == ERR_FORMAT
+    assert f(A16, A16, 0, A16, 1, A16, None) == ERR_ARG
+    assert f(A16, A16, 70000, A16, 1, A16, None) == ERR_ARG
+    assert f(None, A16, 16, A16, 1, A16, None) == ERR_NULL
+    assert f(A16, None, 16, A16, 1, A16, None) == ERR_NULL
+    assert f(A16, A16, 16, None, 1, A16, None) == ERR_NULL
+    assert f(A16, A16, 16, A16, 1, None, None) == ERR_NULL
+    assert f(A1, A16, 16, A16, 1, A16, None) == ERR_ALIGN
+    assert f(A16, A16 + 2, 16, A16, 1, A16, None) == ERR_ALIGN
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.fp8_quantize_blockwise(x)
+    with pytest.raises(ValueError):
+        binding.fp8_quantize_per_tensor(x)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no fallback"):
+        binding.load_library(str(tmp_path / "nope.so"))

@@ -1,0 +1,124 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the benchmark uses.
+
+Full element-by-element comparison with the (threaded) oracle up to 2^26
+elements; the 2^30 sweep point is compared on sampled rows / tile rows (each
+block's result depends only on its block, and the per-tensor scale comes from
+the oracle's amax over the whole tensor), plus invariants over every block.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fine_grained_block_b200 import binding as B
+from fine_grained_block_b200 import inputs
+from parity_util import (assert_bytes_equal, fp32_bits, host_input, oracle_amax, oracle_blockwise, oracle_dequant,
+                         oracle_per_tensor, to_cuda)
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def test_activations_16384x7168_1x128():
+    a = inputs.activation_outlier_channels()
+    xh = host_input(a)
+    x = to_cuda(a)
+    q, s = B.fp8_quantize_blockwise(x, (1, 128), B.E4M3)
+    assert tuple(s.shape) == (16384, 56)
+    oq, os_ = oracle_blockwise(xh, 1, 128, oracle.E4M3)
+    assert_bytes_equal(s, fp32_bits(os_), "scales")
+    assert_bytes_equal(q, oq, "codes")
+    y = B.fp8_dequantize(q, s, (1, 128), B.E4M3, torch.bfloat16)
+    assert_bytes_equal(y, oracle_dequant(oq, oracle.E4M3, os_, 1, 128, oracle.BF16), "dequant bf16")
+
+
+def test_gradients_8192_delayed_e5m2_32_steps():
+    W, steps = 16, 32
+    base = inputs.gradient_base()
+    sc = B.DelayedScaler(window=W, fmt=B.E5M2)
+    ref = oracle.AmaxHistory(W, oracle.E5M2)
+    q = torch.empty(8192, 8192, dtype=torch.uint8, device="cuda")
+    zero_frac = []
+    for k in range(steps):
+        g = inputs.gradient_step(base, k)
+        gh = host_input(g)
+        s_ref = ref.scale[0]
+        q, s_used = sc.step(to_cuda(g), q=q)
+        oq, os_, oa = oracle_per_tensor(gh, oracle.E5M2, scale=float(s_ref))
+        ref.update(oa)
+        torch.cuda.synchronize()
+        assert_bytes_equal(s_used, fp32_bits([os_]), f"step {k} scale used")
+        assert_bytes_equal(sc.amax, fp32_bits([oa]), f"step {k} amax")
+        assert_bytes_equal(sc.scale, fp32_bits(ref.scale), f"step {k} next scale")
+        assert_bytes_equal(q, oq, f"step {k} codes")
+        zero_frac.append(float(((q & 0x7F) == 0).float().mean()))
+    assert sc.state.cpu().tolist() == ref.state.tolist()
+    assert_bytes_equal(sc.history, fp32_bits(ref.history), "history")
+    # with s = 1 the smallest gradients flush to zero; with the window scale they do not
+    assert min(zero_frac[:W]) > 0.1 and max(zero_frac[W:]) < 1e-3
+
+
+@pytest.mark.parametrize("log2_n", [20, 24, 26])
+def test_sweep_full(log2_n):
+    t = inputs.sweep_tensor(log2_n)
+    xh = host_input(t)
+    x = to_cuda(t)
+    for block in ((1, 128), (128, 128)):
+        q, s = B.fp8_quantize_blockwise(x, block, B.E4M3)
+        oq, os_ = oracle_blockwise(xh, *block, oracle.E4M3)
+        assert_bytes_equal(s, fp32_bits(os_), f"{block} scales")
+        assert_bytes_equal(q, oq, f"{block} codes")
+        y = B.fp8_dequantize(q, s, block, B.E4M3, torch.bfloat16)
+        assert_bytes_equal(y, oracle_dequant(oq, oracle.E4M3, os_, *block, oracle.BF16), f"{block} dequant")
+    q, s, a = B.fp8_quantize_per_tensor(x, B.E5M2)
+    oq, os_, oa = oracle_per_tensor(xh, oracle.E5M2)
+    assert_bytes_equal(a, fp32_bits([oa]), "amax")
+    assert_bytes_equal(s, fp32_bits([os_]), "scale")
+    assert_bytes_equal(q, oq, "per-tensor codes")
+    y = B.fp8_dequantize(q, s, (0, 0), B.E5M2, torch.bfloat16)
+    assert_bytes_equal(y, oracle_dequant(oq, oracle.E5M2, np.array([os_], np.float32), 0, 0, oracle.BF16),
+                       "per-tensor dequant")
+
+
+def test_sweep_2pow30_sampled():
+    t = inputs.sweep_tensor(30)
+    xh = host_input(t)
+    R, C = xh.shape
+    x = to_cuda(t)
+    del t
+    rng = np.random.default_rng(30)
+    top_e4 = oracle.top_code(oracle.E4M3)
+    # 1x128: sampled rows, plus the first and last
+    q, s = B.fp8_quantize_blockwise(x, (1, 128), B.E4M3)
+    rows = np.unique(np.concatenate([[0, R - 1], rng.integers(0, R, 254)]))
+    for r in rows:
+        oq, os_ = oracle.quantize_blockwise(xh[r:r + 1], 1, 128, oracle.E4M3)
+        assert_bytes_equal(q[r:r + 1], oq, f"1x128 row {r}")
+        assert_bytes_equal(s[r:r + 1], fp32_bits(os_), f"1x128 scales row {r}")
+    assert bool(((q & 0x7F).view(R, C // 128, 128).amax(dim=2) == top_e4).all())
+    y = B.fp8_dequantize(q, s, (1, 128), B.E4M3, torch.bfloat16)
+    for r in rows[:32]:
+        oq = q[r:r + 1].cpu().numpy()
+        assert_bytes_equal(y[r:r + 1], oracle.dequantize(oq, oracle.E4M3, s[r:r + 1].cpu().numpy(), 1, 128,
+                                                         oracle.BF16), f"1x128 dequant row {r}")
+    del q, s, y
+    # 128x128: sampled tile rows, plus the first and last
+    q, s = B.fp8_quantize_blockwise(x, (128, 128), B.E4M3)
+    for tr in np.unique(np.concatenate([[0, R // 128 - 1], rng.integers(0, R // 128, 6)])):
+        sl = slice(tr * 128, tr * 128 + 128)
+        oq, os_ = oracle_blockwise(xh[sl], 128, 128, oracle.E4M3)
+        assert_bytes_equal(q[sl], oq, f"128x128 tile row {tr}")
+        assert_bytes_equal(s[tr:tr + 1], fp32_bits(os_), f"128x128 scales tile row {tr}")
+    mag = (q & 0x7F).view(R // 128, 128, C // 128, 128)
+    assert bool((mag.amax(dim=(1, 3)) == top_e4).all())
+    del q, s, mag
+    # per-tensor E5M2: amax over the whole tensor from the oracle; codes on sampled rows
+    q, s, a = B.fp8_quantize_per_tensor(x, B.E5M2)
+    oa = oracle_amax(xh)
+    os_ = oracle.scale_from_amax(oa, oracle.E5M2)
+    assert_bytes_equal(a, fp32_bits([oa]), "amax 2^30")
+    assert_bytes_equal(s, fp32_bits([os_]), "scale 2^30")
+    for r in rows[:64]:
+        oq, _, _ = oracle.quantize_per_tensor(xh[r], oracle.E5M2, scale=float(os_))
+        assert_bytes_equal(q[r], oq, f"per-tensor row {r}")

@@ -1,0 +1,314 @@
+"""GPU parity: the CUDA library (called through its C ABI) against the CPU oracle.
+
+Bar: FP8 codes bit-exact, fp32 scales and amax bit-exact, dequantized fp32 /
+bf16 bit-exact (0 ulp), on the same seeded inputs.  Output buffers carry guard
+bands that must come back untouched.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fine_grained_block_b200 import binding as B
+from fine_grained_block_b200 import inputs
+from parity_util import (Guarded, assert_bytes_equal, fp32_bits, host_input, oracle_blockwise, oracle_dequant,
+                         oracle_per_tensor, to_cuda)
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [oracle.E4M3, oracle.E5M2]
+DT = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16}
+
+
+def run_blockwise(x_cpu: torch.Tensor, block, fmt):
+    R, C = x_cpu.shape
+    br, bc = block
+    x = to_cuda(x_cpu)
+    gq = Guarded((R, C), torch.uint8)
+    gs = Guarded((math.ceil(R / br), math.ceil(C / bc)), torch.float32)
+    B.fp8_quantize_blockwise(x, block, fmt, q=gq.t, scales=gs.t)
+    torch.cuda.synchronize()
+    gq.check()
+    gs.check()
+    return gq.t, gs.t
+
+
+def run_dequant(q: torch.Tensor, scales: torch.Tensor, block, fmt, out_dtype):
+    gy = Guarded(tuple(q.shape), out_dtype)
+    B.fp8_dequantize(q, scales, block, fmt, out_dtype, y=gy.t)
+    torch.cuda.synchronize()
+    gy.check()
+    return gy.t
+
+
+def check_blockwise_roundtrip(x_cpu, block, fmt, what, dequant=True):
+    br, bc = block
+    xh = host_input(x_cpu)
+    q, s = run_blockwise(x_cpu, block, fmt)
+    oq, os_ = oracle_blockwise(xh, br, bc, fmt)
+    assert_bytes_equal(s, fp32_bits(os_), f"{what} scales")
+    assert_bytes_equal(q, oq, f"{what} codes")
+    if dequant:
+        for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
+            y = run_dequant(q, s, block, fmt, out_dtype)
+            oy = oracle_dequant(oq, fmt, os_, br, bc, oc)
+            assert_bytes_equal(y, oy, f"{what} dequant {out_dtype}")
+    return q, s
+
+
+def run_per_tensor(x_cpu: torch.Tensor, fmt, scale=None):
+    x = to_cuda(x_cpu)
+    gq = Guarded(tuple(x.shape), torch.uint8)
+    s_out = torch.empty(1, dtype=torch.float32, device="cuda")
+    a_out = torch.empty(1, dtype=torch.float32, device="cuda")
+    s_in = None if scale is None else torch.tensor([scale], dtype=torch.float32, device="cuda")
+    B.fp8_quantize_per_tensor(x, fmt, scale_in=s_in, q=gq.t, scale_out=s_out, amax_out=a_out)
+    torch.cuda.synchronize()
+    gq.check()
+    return gq.t, s_out, a_out
+
+
+def check_per_tensor(x_cpu, fmt, what, scale=None, dequant=True):
+    xh = host_input(x_cpu)
+    q, s, a = run_per_tensor(x_cpu, fmt, scale)
+    oq, os_, oa = oracle_per_tensor(xh, fmt, scale)
+    assert_bytes_equal(a, fp32_bits([oa]), f"{what} amax")
+    assert_bytes_equal(s, fp32_bits([os_]), f"{what} scale")
+    assert_bytes_equal(q, oq, f"{what} codes")
+    if dequant:
+        q2 = q.reshape(-1) if q.dim() != 2 else q
+        oq2 = oq.reshape(q2.shape)
+        for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
+            y = run_dequant(q2, s, (0, 0), fmt, out_dtype)
+            oy = oracle_dequant(oq2, fmt, np.array([os_], np.float32), 0, 0, oc)
+            assert_bytes_equal(y, oy, f"{what} dequant {out_dtype}")
+    return q, s, a
+
+
+# -- the scalar experiment (PyTorch-FP8 page s2.2) and special values ------------
+
+def special_values():
+    v = list(inputs.SCALAR_VALUES)
+    v += [-x for x in inputs.SCALAR_VALUES]
+    v += [0.0, -0.0, 1e4, 6e4, 1e6, 3.0e38, -3.0e38, 464.0, 480.0, 61440.0, 2.0 ** -10, 2.0 ** -17,
+          1e-40, -1e-40, 1.0625, 1.1875, 0.0009765625, 0.00146484375, 2.0 ** -9 * 0.5, 2.0 ** -16 * 0.5,
+          float("inf"), float("-inf")]
+    return torch.tensor(v, dtype=torch.float32)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_scalar_cast_at_scale_one(fmt):
+    x = special_values()
+    q, s, a = run_per_tensor(x, fmt, scale=1.0)
+    want = np.array([oracle.encode(float(v), fmt) for v in x.numpy()], dtype=np.uint8)
+    assert_bytes_equal(q, want, "scale-1 cast")
+    assert s.item() == 1.0
+
+
+# -- config: fp32 256x1024 with outlier columns (handbook "FP8 training") ---------
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_outlier_tensors_per_tensor_and_1x128(fmt):
+    for factor, a in inputs.relerr_outlier_tensors():
+        check_per_tensor(a, fmt, f"per-tensor x{factor}")
+        check_blockwise_roundtrip(a, (1, 128), fmt, f"1x128 x{factor}")
+        check_blockwise_roundtrip(a, (128, 128), fmt, f"128x128 x{factor}")
+
+
+def test_outlier_tensors_relative_error_from_gpu():
+    """The handbook's printed table, reproduced from the GPU's own round trip."""
+    from conftest import golden_rows
+    printed = {float(f): (float(t), float(b)) for f, t, b in golden_rows("p3_relerr.txt")}
+    for factor, a in inputs.relerr_outlier_tensors():
+        x = to_cuda(a)
+        q, s, _ = B.fp8_quantize_per_tensor(x, B.E4M3)
+        yt = B.fp8_dequantize(q, s, (0, 0), B.E4M3, torch.float32)
+        qb, sb = B.fp8_quantize_blockwise(x, (1, 128), B.E4M3)
+        yb = B.fp8_dequantize(qb, sb, (1, 128), B.E4M3, torch.float32)
+        n = x[:, 128:].double()
+        t = ((yt[:, 128:].double() - n).norm() / n.norm()).item() * 100
+        b = ((yb[:, 128:].double() - n).norm() / n.norm()).item() * 100
+        assert (round(t, 1), round(b, 1)) == printed[factor]
+
+
+# -- config: bf16 weight 4096x4096, N(0, 0.02^2), 128x128 ------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_weight_4096_128x128(fmt):
+    w = inputs.weight_4096()
+    check_blockwise_roundtrip(w, (128, 128), fmt, "weight 128x128")
+
+
+def test_weight_4096_1x128_and_per_tensor():
+    w = inputs.weight_4096()
+    check_blockwise_roundtrip(w, (1, 128), oracle.E4M3, "weight 1x128")
+    check_per_tensor(w, oracle.E5M2, "weight per-tensor")
+
+
+# -- ragged shapes, both dtypes, both formats --------------------------------------
+
+SHAPES = [(1, 128), (3, 256), (128, 128), (130, 384), (257, 640), (129, 1280), (64, 100), (200, 77), (5, 1),
+          (1, 8), (2, 136), (300, 4096)]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("block", [(1, 128), (128, 128)])
+def test_ragged_blockwise(fmt, dtype, block):
+    for i, (R, C) in enumerate(SHAPES):
+        x = inputs.random_matrix(R, C, seed=1000 + i, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        check_blockwise_roundtrip(x, block, fmt, f"{block} {R}x{C} {dtype}")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_ragged_per_tensor(fmt, dtype):
+    for i, n in enumerate([1, 3, 7, 8, 9, 127, 4096, 4097, 65536 + 5, 1 << 20, (1 << 20) + 3]):
+        x = inputs.random_matrix(1, n, seed=2000 + i, dtype=dtype, outlier_frac=0.001, factor=1e3).reshape(-1)
+        check_per_tensor(x, fmt, f"per-tensor n={n} {dtype}")
+        check_per_tensor(x, fmt, f"delayed n={n} {dtype}", scale=7.5)
+
+
+def test_empty_inputs():
+    x = torch.zeros(0, dtype=torch.bfloat16, device="cuda")
+    q, s, a = B.fp8_quantize_per_tensor(x, B.E4M3)
+    torch.cuda.synchronize()
+    assert a.item() == 0.0
+    assert fp32_bits([s.item()])[0] == fp32_bits([oracle.scale_from_amax(0.0, oracle.E4M3)])[0]
+    q, s, a = B.fp8_quantize_per_tensor(x, B.E5M2, scale_in=torch.tensor([3.0], device="cuda"))
+    torch.cuda.synchronize()
+    assert s.item() == 3.0 and a.item() == 0.0
+    q, s = B.fp8_quantize_blockwise(torch.zeros(0, 256, dtype=torch.bfloat16, device="cuda"))
+    assert q.numel() == 0 and s.numel() == 0
+    y = B.fp8_dequantize(torch.zeros(0, 128, dtype=torch.uint8, device="cuda"),
+                         torch.ones(1, device="cuda"), (0, 0))
+    assert y.numel() == 0
+
+
+# -- edge values -------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_edge_value_blocks(fmt):
+    R, C = 256, 512
+    x = inputs.random_matrix(R, C, seed=77, dtype=torch.float32)
+    x[0, :128] = 0.0                       # all-zero block
+    x[1, :128] = -0.0                      # all negative zero
+    x[2, :128] = 1e-42                     # fp32 subnormals only
+    x[3, :128] = torch.linspace(-1e-30, 1e-30, 128)
+    x[4, 128:256] = 3.0e38                 # near fp32 max
+    x[5, 256:384] = torch.tensor([2.0 ** k for k in range(-64, 64)])
+    x[6, :] = 1.0                           # constant row: every element hits MAX
+    x[128:256, 384:512] = 0.0              # an all-zero 128x128 tile
+    x[7, 5] = 1e-45
+    for block in ((1, 128), (128, 128)):
+        check_blockwise_roundtrip(x, block, fmt, f"edge {block}")
+        check_blockwise_roundtrip(x.to(torch.bfloat16), block, fmt, f"edge bf16 {block}")
+    check_per_tensor(x, fmt, "edge per-tensor")
+    check_per_tensor(x, fmt, "edge delayed saturating", scale=1e30)
+    check_per_tensor(x, fmt, "edge delayed tiny scale", scale=1e-30)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_dequant_every_code_with_extreme_scales(fmt):
+    """All finite codes against scales across the whole fp32 range (the bit-exact division)."""
+    top = oracle.top_code(fmt)
+    codes = np.array([c for c in range(256) if (c & 0x7F) <= top], dtype=np.uint8)
+    R = 64
+    q = np.ascontiguousarray(np.tile(codes, (R, 2))[:, :256])  # every finite code in each row
+    scales = np.exp2(np.linspace(-126, 127, R)).astype(np.float32).reshape(R, 1)
+    scales = np.repeat(scales, 2, axis=1)
+    scales[5, 0] = 1.4e-45   # subnormal scale
+    scales[6, 1] = 3.4e38
+    scales[7, 0] = 448.0 / 1e-12
+    qg = to_cuda(torch.from_numpy(q))
+    sg = to_cuda(torch.from_numpy(scales))
+    for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
+        y = run_dequant(qg, sg, (1, 128), fmt, out_dtype)
+        oy = oracle.dequantize(q, fmt, scales, 1, 128, oc)
+        assert_bytes_equal(y, oy, f"dequant extremes {out_dtype}")
+        y0 = run_dequant(qg, sg[7:8, 0].contiguous(), (0, 0), fmt, out_dtype)
+        oy0 = oracle.dequantize(q, fmt, scales[7:8, 0], 0, 0, oc)
+        assert_bytes_equal(y0, oy0, f"dequant per-tensor {out_dtype}")
+
+
+# -- invariants that hold at any size ----------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_every_block_holds_a_max_code(fmt):
+    x = to_cuda(inputs.random_matrix(1024, 2048, seed=5, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e3))
+    top = oracle.top_code(fmt)
+    for block in ((1, 128), (128, 128)):
+        q, s = B.fp8_quantize_blockwise(x, block, fmt)
+        br, bc = block
+        mag = (q & 0x7F).view(q.shape[0] // br, br, q.shape[1] // bc, bc)
+        assert bool((mag.amax(dim=(1, 3)) == top).all())
+        assert bool((mag <= top).all())
+
+
+# -- delayed scaling: history kernel --------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("window", [1, 3, 16, 33, 1024])
+def test_history_update_matches_oracle(fmt, window):
+    rng = np.random.default_rng(window + 10 * fmt)
+    steps = window * 2 + 5
+    amaxes = np.exp(rng.uniform(np.log(1e-14), np.log(1e4), size=steps)).astype(np.float32)
+    amaxes[3 % steps] = 0.0
+    h = torch.zeros(window, dtype=torch.float32, device="cuda")
+    st = torch.zeros(2, dtype=torch.int32, device="cuda")
+    sc = torch.ones(1, dtype=torch.float32, device="cuda")
+    am = torch.empty(1, dtype=torch.float32, device="cuda")
+    ref = oracle.AmaxHistory(window, fmt)
+    for k in range(steps):
+        am.fill_(float(amaxes[k]))
+        B.fp8_amax_history_update(h, st, am, sc, fmt)
+        ref.update(amaxes[k])
+        torch.cuda.synchronize()
+        assert_bytes_equal(sc, fp32_bits(ref.scale), f"scale step {k}")
+        assert st.cpu().tolist() == ref.state.tolist()
+        assert_bytes_equal(h, fp32_bits(ref.history), f"history step {k}")
+
+
+def test_history_state_out_of_range_is_clamped():
+    W = 8
+    h = torch.arange(W, dtype=torch.float32, device="cuda")
+    st = torch.tensor([-3, 999], dtype=torch.int32, device="cuda")
+    sc = torch.ones(1, device="cuda")
+    am = torch.tensor([100.0], device="cuda")
+    B.fp8_amax_history_update(h, st, am, sc, B.E4M3)
+    torch.cuda.synchronize()
+    # pos -3 mod 8 = 5, count clamped to 8 (full) -> slot 5 takes 100, scale from max = 100
+    ref = oracle.AmaxHistory(W, oracle.E4M3)
+    ref.history[:] = np.arange(W, dtype=np.float32)
+    ref.state[:] = [5, 8]
+    ref.update(100.0)
+    assert st.cpu().tolist() == ref.state.tolist()
+    assert_bytes_equal(h, fp32_bits(ref.history), "history")
+    assert_bytes_equal(sc, fp32_bits(ref.scale), "scale")
+
+
+# -- boundary behaviour on the device ---------------------------------------------------
+
+def test_misaligned_device_pointers_rejected():
+    buf = torch.zeros(4096 + 64, dtype=torch.uint8, device="cuda")
+    x = buf[1:1 + 2 * 1024].view(torch.uint8)
+    L = B.load_library()
+    stream = torch.cuda.current_stream().cuda_stream
+    q = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    s = torch.empty(8, dtype=torch.float32, device="cuda")
+    assert L.fp8_quantize_blockwise(x.data_ptr(), 1, 8, 128, 1, 128, 0, q.data_ptr(), s.data_ptr(), stream) == -3
+    assert L.fp8_dequantize(buf[3:].data_ptr(), 0, 8, 128, 1, 128, s.data_ptr(), q.data_ptr(), 1, stream) == -3
+
+
+def test_runs_on_a_side_stream():
+    x = to_cuda(inputs.random_matrix(512, 1024, seed=9, dtype=torch.bfloat16))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        q, s = B.fp8_quantize_blockwise(x, (1, 128), B.E4M3)
+    side.synchronize()
+    oq, os_ = oracle_blockwise(host_input(x.cpu()), 1, 128, oracle.E4M3)
+    assert_bytes_equal(q, oq, "side-stream codes")
+    assert_bytes_equal(s, fp32_bits(os_), "side-stream scales")
