@@ -35,7 +35,10 @@ SIGNATURES = {
     "fp8_dequantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _c_int, _vp]),
     "fp8_amax_history_update": (_c_int, [_vp, _vp, _c_int, _vp, _c_int, _vp, _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_c_int]),
+    "fp8_device_status": (_c_int, [_vp, _c_int, _vp]),
+    "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
 }
+DEVICE_STATUS_WAIT_TIMEOUT = 0x1
 
 
 class FP8Error(RuntimeError):
@@ -167,6 +170,18 @@ def fp8_amax_history_update(history: torch.Tensor, state: torch.Tensor, amax: to
                                                 _ptr(scale), _stream(stream))
     _check("fp8_amax_history_update", st)
     return scale
+
+
+def fp8_device_status(clear: bool = False, device=None, stream=None) -> int:
+    """The device status word (FP8_DEVICE_STATUS_* bits); synchronizes the stream to read it."""
+    out = torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+    _check("fp8_device_status", load_library().fp8_device_status(_ptr(out), 1 if clear else 0, _stream(stream)))
+    return int(out.item())
+
+
+def fp8_selftest_wait_timeout(timeout_us: int = 1000, stream=None):
+    """Launch a wait that can only time out (sets DEVICE_STATUS_WAIT_TIMEOUT after timeout_us)."""
+    _check("fp8_selftest_wait_timeout", load_library().fp8_selftest_wait_timeout(int(timeout_us), _stream(stream)))
 
 
 class DelayedScaler:

@@ -41,32 +41,39 @@ def _headers():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile and link the library if anything is stale; return its path."""
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, defines: dict | None = None, out: str | None = None) -> str:
+    """Compile and link the library if anything is stale; return its path.
+
+    defines / out build a variant with extra -D tuning macros into another
+    location (objects under _build/variants/<name of out's folder>)."""
+    lib_path = out or LIB
+    build_dir = BUILD if out is None else os.path.join(ROOT, "_build", "variants", os.path.basename(os.path.dirname(out)))
+    flags = list(NVCC_FLAGS) + [f"-D{k}={v}" for k, v in (defines or {}).items()]
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0.0)
     objects = []
-    relinked = force or not os.path.exists(LIB)
+    relinked = force or not os.path.exists(lib_path)
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objects.append(obj)
         stale = force or not os.path.exists(obj) or \
             os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header)
         if stale:
-            cmd = [nvcc(), *NVCC_FLAGS, "-c", src, "-o", obj]
+            cmd = [nvcc(), *flags, "-c", src, "-o", obj]
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
                 print(" ".join(cmd), file=sys.stderr)
             subprocess.run(cmd, check=True)
             relinked = True
-    if not relinked and os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objects):
+    if not relinked and os.path.getmtime(lib_path) < max(os.path.getmtime(o) for o in objects):
         relinked = True
     if relinked:
-        tmp = LIB + f".tmp{os.getpid()}"
+        os.makedirs(os.path.dirname(lib_path), exist_ok=True)
+        tmp = lib_path + f".tmp{os.getpid()}"
         subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objects], check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":

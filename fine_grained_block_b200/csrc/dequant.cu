@@ -1,9 +1,21 @@
 // dequant.cu -- FP8 dequantization kernels.
 //
 // PyTorch-FP8 page, s4.1 (divide by the scale to restore the value) and s4.2
-// quantize() (.to(dtype) / scale): y = fp32(decode(q) / s), one IEEE
-// round-to-nearest division per element, then (bf16 output) one more
-// round-to-nearest-even to bf16.
+// quantize() (.to(dtype) / scale): y = fp32(decode(q) / s), the correctly
+// rounded IEEE quotient, then (bf16 output) one more round-to-nearest-even to
+// bf16.
+//
+// The quotient is formed without a division per element.  Each thread takes
+// r = RN(1/s) once for its group of codes and then, per element,
+//     y0 = RN(q * r);  e = RN(q - s * y0) (fma);  y = RN(y0 + e * r) (fma).
+// Every FP8 value is (1 + j/8) * 2^a, so with no step leaving the normal range
+// the scheme is exact for all codes iff it is exact for the 8 mantissas of q
+// against every one of the 2^23 mantissas of s -- 8 * 2^23 cases, all checked
+// exhaustively by tests/c/recip_division_exhaustive.c.  The normal-range
+// condition holds for |s| in [2^-100, 2^101), which covers every scale the
+// quantizers produce except for amax above ~2^108; other scales, and E5M2
+// Inf codes (whose fma residual would be Inf - Inf), take the per-element IEEE
+// division instead.
 //
 // Each thread turns one group of codes into one 16-byte output vector: 8 codes
 // for bf16 output, 4 codes for fp32 output.  Consecutive lanes therefore read
@@ -14,79 +26,157 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "lane_vec.cuh"
 
 namespace fp8q {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+// Code groups loaded per trip per thread.
+#ifndef FP8Q_DEQ_UNROLL
+#define FP8Q_DEQ_UNROLL 4
+#endif
+constexpr int kUnroll = FP8Q_DEQ_UNROLL;
 
-template <int OUT>  // 0 = fp32, 1 = bf16
-struct DOut;
+// |s| in [2^-100, 2^101): r, q * r, the residual and the result all stay normal.
+__device__ __forceinline__ bool scale_fast_ok(float s) {
+    const uint32_t ex = (__float_as_uint(s) >> 23) & 0xFFu;
+    return ex >= 27u && ex <= 227u;
+}
 
+// True when any of the 4 codes in w is an E5M2 Inf/NaN code (exponent field all ones).
+__device__ __forceinline__ bool e5m2_has_special(uint32_t w) {
+    return (((w & 0x7C7C7C7Cu) + 0x04040404u) & 0x80808080u) != 0u;
+}
+
+// Two codes (low 16 bits of c2) -> two exact quotients RN(q / s), from
+// r2 = {RN(1/s)} x2 and ns2 = {-s} x2:
+//   y0 = q * r;  e = q - s * y0 (fma);  y = y0 + e * r (fma)
+// For q = +-0 the last fma would give +0 for -0, so the sign is taken from
+// y0, which carries the quotient's sign for every q.
+template <int FMT>
+__device__ __forceinline__ float2 dequant2_fast(uint32_t c2, uint64_t r2, uint64_t ns2) {
+    const float2 a = fp8x2_to_float2<FMT>(c2);
+    const uint64_t q2 = f32x2(a.x, a.y);
+    const uint64_t y0 = mul_f32x2(q2, r2);
+    const uint64_t e = fma_f32x2(y0, ns2, q2);
+    const float2 y = f32x2_split(fma_f32x2(e, r2, y0));
+    const float2 z = f32x2_split(y0);
+    return make_float2(copysignf(y.x, z.x), copysignf(y.y, z.y));
+}
+
+template <int FMT>
+__device__ __forceinline__ float2 dequant2_div(uint32_t c2, float s) {
+    const float2 a = fp8x2_to_float2<FMT>(c2);
+    return make_float2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s));
+}
+
+template <int NW>
+__device__ __forceinline__ void unpack_codes(const typename CodeWords<NW>::T& c, uint32_t* w);
 template <>
-struct DOut<0> {
-    static constexpr int kCodes = 4;  // 4 codes -> 16 B of fp32
-    using In = uint32_t;
+__device__ __forceinline__ void unpack_codes<1>(const uint32_t& c, uint32_t* w) { w[0] = c; }
+template <>
+__device__ __forceinline__ void unpack_codes<2>(const uint2& c, uint32_t* w) { w[0] = c.x; w[1] = c.y; }
+template <>
+__device__ __forceinline__ void unpack_codes<4>(const uint4& c, uint32_t* w) {
+    w[0] = c.x; w[1] = c.y; w[2] = c.z; w[3] = c.w;
+}
+
+__device__ __forceinline__ void store_words(void* p, const Words<4>& v) {
+    st_stream(static_cast<uint4*>(p), make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
+}
+__device__ __forceinline__ void store_words(void* p, const Words<8>& v) {
+    V32 o;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o.w[k] = v.w[k];
+    st32_stream(p, o);
+}
+
+// One lane's group of codes -> one OB-byte output vector (OUT 0 = fp32, 1 = bf16).
+template <int OUT, int OB>
+struct DOut {
+    static constexpr int kOutElem = OUT == 0 ? 4 : 2;
+    static constexpr int kCodes = OB / kOutElem;
+    static constexpr int kCodeWords = kCodes / 4;
+    using In = typename CodeWords<kCodeWords>::T;
+    using Out = Words<OB / 4>;
+
     template <int FMT>
-    static __device__ __forceinline__ uint4 convert(In c, float s) {
-        const float2 a = fp8x2_to_float2<FMT>(c & 0xFFFFu);
-        const float2 b = fp8x2_to_float2<FMT>(c >> 16);
-        return make_uint4(__float_as_uint(__fdiv_rn(a.x, s)), __float_as_uint(__fdiv_rn(a.y, s)),
-                          __float_as_uint(__fdiv_rn(b.x, s)), __float_as_uint(__fdiv_rn(b.y, s)));
+    static __device__ __forceinline__ void put(Out& o, int pair, float2 y) {
+        if (OUT == 1) {
+            o.w[pair] = pack_bf16x2(y.x, y.y);
+        } else {
+            o.w[2 * pair] = __float_as_uint(y.x);
+            o.w[2 * pair + 1] = __float_as_uint(y.y);
+        }
+    }
+
+    template <int FMT>
+    static __device__ __forceinline__ Out convert(const In& cin, float s) {
+        uint32_t cw[kCodeWords];
+        unpack_codes<kCodeWords>(cin, cw);
+        bool fast = scale_fast_ok(s);
+        if (FMT == kE5M2) {
+#pragma unroll
+            for (int k = 0; k < kCodeWords; ++k) fast = fast && !e5m2_has_special(cw[k]);
+        }
+        Out o;
+        if (fast) {
+            const float r = __frcp_rn(s);
+            const uint64_t r2 = f32x2(r, r);
+            const uint64_t ns2 = f32x2(-s, -s);
+#pragma unroll
+            for (int k = 0; k < kCodeWords; ++k) {
+                put<FMT>(o, 2 * k, dequant2_fast<FMT>(cw[k] & 0xFFFFu, r2, ns2));
+                put<FMT>(o, 2 * k + 1, dequant2_fast<FMT>(cw[k] >> 16, r2, ns2));
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < kCodeWords; ++k) {
+                put<FMT>(o, 2 * k, dequant2_div<FMT>(cw[k] & 0xFFFFu, s));
+                put<FMT>(o, 2 * k + 1, dequant2_div<FMT>(cw[k] >> 16, s));
+            }
+        }
+        return o;
     }
 };
 
-template <>
-struct DOut<1> {
-    static constexpr int kCodes = 8;  // 8 codes -> 16 B of bf16
-    using In = uint2;
-    template <int FMT>
-    static __device__ __forceinline__ uint32_t pair(uint32_t c2, float s) {
-        const float2 a = fp8x2_to_float2<FMT>(c2);
-        return pack_bf16x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s));
-    }
-    template <int FMT>
-    static __device__ __forceinline__ uint4 convert(In c, float s) {
-        return make_uint4(pair<FMT>(c.x & 0xFFFFu, s), pair<FMT>(c.x >> 16, s),
-                          pair<FMT>(c.y & 0xFFFFu, s), pair<FMT>(c.y >> 16, s));
-    }
-};
-
-__device__ __forceinline__ uint32_t ld_codes(const uint32_t* p) { return __ldcs(reinterpret_cast<const unsigned int*>(p)); }
+__device__ __forceinline__ uint32_t ld_codes(const uint32_t* p) {
+    return __ldcs(reinterpret_cast<const unsigned int*>(p));
+}
 __device__ __forceinline__ uint2 ld_codes(const uint2* p) { return __ldcs(p); }
+__device__ __forceinline__ uint4 ld_codes(const uint4* p) { return __ldcs(p); }
 
 // One code -> fp32 (for tails and the general kernel).
 template <int FMT>
 __device__ __forceinline__ float decode1(uint8_t c) { return fp8x2_to_float2<FMT>(c).x; }
 
 // Per-tensor (MODE 0) and 1x128 (MODE 1, cols % 128 == 0) over a flat range
-// of ngroups code groups; a per-tensor tail of < kCodes codes goes to CTA 0.
-template <int FMT, int OUT, int MODE>
+// of ngroups code groups.  Each CTA owns kThreads x kUnroll consecutive groups
+// and issues all its loads before converting; a per-tensor tail of < kCodes
+// codes goes to CTA 0.
+template <int FMT, int OUT, int OB, int MODE>
 __global__ void __launch_bounds__(kThreads)
-k_dequant_flat(const typename DOut<OUT>::In* __restrict__ q, int64_t ngroups,
+k_dequant_flat(const typename DOut<OUT, OB>::In* __restrict__ q, int64_t ngroups,
                const uint8_t* __restrict__ q_tail, int tail_n, const float* __restrict__ scales,
-               uint4* __restrict__ y, void* __restrict__ y_tail) {
-    using D = DOut<OUT>;
+               typename DOut<OUT, OB>::Out* __restrict__ y, void* __restrict__ y_tail) {
+    using D = DOut<OUT, OB>;
     constexpr int kGroupsPerBlock = 128 / D::kCodes;
-    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x;
     const float s0 = (MODE == 0) ? scales[0] : 0.0f;
-    for (int64_t i0 = tid; i0 < ngroups; i0 += nthreads * kUnroll) {
-        typename D::In c[kUnroll];
-        float s[kUnroll];
+    typename D::In c[kUnroll];
+    float s[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t g = i0 + u * nthreads;
-            const bool ok = g < ngroups;
-            c[u] = ok ? ld_codes(q + g) : typename D::In{};
-            s[u] = (MODE == 0) ? s0 : (ok ? scales[g / kGroupsPerBlock] : 1.0f);
-        }
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t g = base + u * kThreads;
+        const bool ok = g < ngroups;
+        c[u] = ok ? ld_codes(q + g) : typename D::In{};
+        s[u] = (MODE == 0) ? s0 : (ok ? scales[g / kGroupsPerBlock] : 1.0f);
+    }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t g = i0 + u * nthreads;
-            if (g < ngroups) st_stream(y + g, D::template convert<FMT>(c[u], s[u]));
-        }
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t g = base + u * kThreads;
+        if (g < ngroups) store_words(y + g, D::template convert<FMT>(c[u], s[u]));
     }
     if (MODE == 0 && blockIdx.x == 0 && threadIdx.x < tail_n) {
         const float v = __fdiv_rn(decode1<FMT>(q_tail[threadIdx.x]), s0);
@@ -97,14 +187,16 @@ k_dequant_flat(const typename DOut<OUT>::In* __restrict__ q, int64_t ngroups,
 
 // 128x128 (cols % 128 == 0): one CTA per tile, one scale per CTA.  A tile row
 // is 128 codes = kGroupsPerRow groups; the CTA sweeps the tile's 128 rows.
-template <int FMT, int OUT>
+template <int FMT, int OUT, int OB>
 __global__ void __launch_bounds__(kThreads)
-k_dequant_128x128(const typename DOut<OUT>::In* __restrict__ q, const float* __restrict__ scales,
-                  uint4* __restrict__ y, int64_t rows, int64_t cols) {
-    using D = DOut<OUT>;
-    constexpr int kGroupsPerRow = 128 / D::kCodes;             // 16 (bf16 out) or 32 (fp32 out)
-    constexpr int kRowsPerPass = kThreads / kGroupsPerRow;      // 16 or 8
-    constexpr int kPasses = 128 / kRowsPerPass;                 // 8 or 16
+k_dequant_128x128(const typename DOut<OUT, OB>::In* __restrict__ q, const float* __restrict__ scales,
+                  typename DOut<OUT, OB>::Out* __restrict__ y, int64_t rows, int64_t cols) {
+    using D = DOut<OUT, OB>;
+    constexpr int kGroupsPerRow = 128 / D::kCodes;
+    constexpr int kRowsPerPass = kThreads / kGroupsPerRow;
+    constexpr int kPasses = 128 / kRowsPerPass;
+    constexpr int kTileUnroll = 4;  // passes per batch of loads
+    static_assert(kPasses % kTileUnroll == 0, "the unrolled passes must stay inside the tile");
     const int64_t tiles_c = cols >> 7;
     const int64_t tr = blockIdx.x / tiles_c;
     const int64_t tc = blockIdx.x - tr * tiles_c;
@@ -113,17 +205,20 @@ k_dequant_128x128(const typename DOut<OUT>::In* __restrict__ q, const float* __r
     const int64_t r0 = tr * 128 + threadIdx.x / kGroupsPerRow;
     const int64_t g0 = r0 * groups_per_tensor_row + tc * kGroupsPerRow + threadIdx.x % kGroupsPerRow;
 #pragma unroll
-    for (int p0 = 0; p0 < kPasses; p0 += kUnroll) {
-        typename D::In c[kUnroll];
+    for (int p0 = 0; p0 < kPasses; p0 += kTileUnroll) {
+        typename D::In c[kTileUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kTileUnroll; ++u) {
             const int64_t r = r0 + (p0 + u) * kRowsPerPass;
-            c[u] = (r < rows) ? ld_codes(q + g0 + (p0 + u) * kRowsPerPass * groups_per_tensor_row) : typename D::In{};
+            c[u] = (r < rows) ? ld_codes(q + g0 + (p0 + u) * kRowsPerPass * groups_per_tensor_row)
+                              : typename D::In{};
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kTileUnroll; ++u) {
             const int64_t r = r0 + (p0 + u) * kRowsPerPass;
-            if (r < rows) st_stream(y + g0 + (p0 + u) * kRowsPerPass * groups_per_tensor_row, D::template convert<FMT>(c[u], s));
+            if (r < rows)
+                store_words(y + g0 + (p0 + u) * kRowsPerPass * groups_per_tensor_row,
+                            D::template convert<FMT>(c[u], s));
         }
     }
 }
@@ -146,41 +241,41 @@ k_dequant_general(const uint8_t* __restrict__ q, int64_t rows, int64_t cols, int
     }
 }
 
-template <typename Kernel>
-int64_t flat_grid(Kernel k, int64_t ngroups) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, 0) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    const int64_t full = static_cast<int64_t>(device_sm_count()) * per_sm;
-    const int64_t need = (ngroups + static_cast<int64_t>(kThreads) * kUnroll - 1) / (static_cast<int64_t>(kThreads) * kUnroll);
-    return std::max<int64_t>(1, std::min(full, need));
+template <int FMT, int OUT, int OB>
+cudaError_t dequant_fast(const uint8_t* q, int64_t rows, int64_t cols, int mode, const float* scales, void* y,
+                         cudaStream_t st) {
+    using D = DOut<OUT, OB>;
+    const int64_t n = rows * cols;
+    if (mode == 2) {
+        const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
+        if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        k_dequant_128x128<FMT, OUT, OB><<<static_cast<unsigned>(tiles), kThreads, 0, st>>>(
+            reinterpret_cast<const typename D::In*>(q), scales, static_cast<typename D::Out*>(y), rows, cols);
+        return cudaGetLastError();
+    }
+    const int64_t ngroups = n / D::kCodes;
+    const int tail_n = static_cast<int>(n - ngroups * D::kCodes);
+    const size_t osz = D::kOutElem;
+    const int64_t per_cta = static_cast<int64_t>(kThreads) * kUnroll;
+    const int64_t grid = std::max<int64_t>(1, (ngroups + per_cta - 1) / per_cta);
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    auto launch = [&](auto kern) {
+        kern<<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
+            reinterpret_cast<const typename D::In*>(q), ngroups, q + ngroups * D::kCodes, tail_n, scales,
+            static_cast<typename D::Out*>(y), static_cast<char*>(y) + ngroups * D::kCodes * osz);
+    };
+    if (mode == 0) launch(k_dequant_flat<FMT, OUT, OB, 0>);
+    else launch(k_dequant_flat<FMT, OUT, OB, 1>);
+    return cudaGetLastError();
 }
 
 template <int FMT, int OUT>
 cudaError_t dequant_typed(const uint8_t* q, int64_t rows, int64_t cols, int mode, const float* scales, void* y,
                           cudaStream_t st) {
-    using D = DOut<OUT>;
     const int64_t n = rows * cols;
-    const size_t osz = OUT == 0 ? 4 : 2;
-    if (mode == 0 || (mode == 1 && cols % 128 == 0)) {
-        const int64_t ngroups = (mode == 0) ? n / D::kCodes : n / D::kCodes;
-        const int tail_n = static_cast<int>(n - ngroups * D::kCodes);
-        auto launch = [&](auto kern) {
-            const int64_t grid = flat_grid(kern, ngroups);
-            kern<<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
-                reinterpret_cast<const typename D::In*>(q), ngroups, q + ngroups * D::kCodes, tail_n, scales,
-                static_cast<uint4*>(y), static_cast<char*>(y) + ngroups * D::kCodes * osz);
-        };
-        if (mode == 0) launch(k_dequant_flat<FMT, OUT, 0>);
-        else launch(k_dequant_flat<FMT, OUT, 1>);
-        return cudaGetLastError();
-    }
-    if (mode == 2 && cols % 128 == 0) {
-        const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
-        if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-        k_dequant_128x128<FMT, OUT><<<static_cast<unsigned>(tiles), kThreads, 0, st>>>(
-            reinterpret_cast<const typename D::In*>(q), scales, static_cast<uint4*>(y), rows, cols);
-        return cudaGetLastError();
+    if (mode == 0 || cols % 128 == 0) {
+        if ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) return dequant_fast<FMT, OUT, 32>(q, rows, cols, mode, scales, y, st);
+        return dequant_fast<FMT, OUT, 16>(q, rows, cols, mode, scales, y, st);
     }
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((n + kThreads - 1) / kThreads,
                                                                 static_cast<int64_t>(device_sm_count()) * 8));

@@ -108,9 +108,95 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Running max of |x| over packed bf16 pairs with one instruction per pair:
+// max.xorsign.abs takes the larger magnitude (its sign bit is the xor of the
+// inputs' signs and is cleared at the end by bf16x2_absmax_finish).  A NaN
+// operand yields the other operand.  Exact.
+__device__ __forceinline__ uint32_t xabsmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ float bf16x2_absmax_finish(uint32_t m) {
+    return bf16x2_hmax(m & 0x7FFF7FFFu);
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE round-to-nearest
+// results per instruction, denormals kept)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ float2 f32x2_split(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return make_float2(lo, hi);
+}
+
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// A packed bf16 pair (lo element in the low half) scaled by s2 = {s, s} in
+// fp32 and cast to two FP8 codes (low 16 bits, lo code in the low byte):
+// q = fp8(fp32(x * s)) for both elements.
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_cast_bf16x2(uint32_t w, uint64_t s2) {
+    const float2 p = f32x2_split(mul_f32x2(f32x2(bf16_lo(w), bf16_hi(w)), s2));
+    return cvt_fp8x2<FMT>(p.x, p.y);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_cast_f32x2(uint32_t a, uint32_t b, uint64_t s2) {
+    const float2 p = f32x2_split(mul_f32x2(f32x2(__uint_as_float(a), __uint_as_float(b)), s2));
+    return cvt_fp8x2<FMT>(p.x, p.y);
+}
+
 // ---------------------------------------------------------------------------
 // memory access
 // ---------------------------------------------------------------------------
+
+// 32-byte vector (one 256-bit access per lane).
+struct V32 {
+    uint32_t w[8];
+};
+
+__device__ __forceinline__ V32 ld32_stream(const void* p) {
+    V32 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+                   "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st32_stream(void* p, const V32& v) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+                    "r"(v.w[6]), "r"(v.w[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ V32 v32_zero() {
+    V32 v;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v.w[k] = 0u;
+    return v;
+}
 
 // Streaming 16-byte load: read once, do not keep in L1.
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {

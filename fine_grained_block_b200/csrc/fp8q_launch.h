@@ -23,6 +23,19 @@ cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fm
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                  uint8_t* q, float* scales, cudaStream_t stream);
 
+// 128x128 blocks with TMA-staged tiles (bf16, cols % 128 == 0, rows and cols
+// below 2^31, and a driver that provides the tensor-map encoder).
+bool tma_128x128_supported(int dtype, int64_t rows, int64_t cols);
+cudaError_t launch_quant_128x128_tma(const void* x, int64_t rows, int64_t cols, int fmt, uint8_t* q,
+                                     float* scales, cudaStream_t stream);
+
+// Copy the device status word to out[0] (device memory), clearing it if asked.
+cudaError_t launch_device_status(unsigned int* out, int clear, cudaStream_t stream);
+
+// A single-thread kernel whose bounded wait can only time out (sets the
+// wait-timeout status bit after limit_ns).
+cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
 // Any block shape, any cols (ragged right edge), element-wise accesses.
 cudaError_t launch_quant_block_general(const void* x, int dtype, int64_t rows, int64_t cols,
                                        int block_rows, int block_cols, int fmt,

@@ -9,116 +9,77 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "lane_vec.cuh"
 
 namespace fp8q {
 namespace {
 
 constexpr int kThreads = 256;
 
-// Widen one 16-byte vector of T (8 bf16 or 4 fp32) and fold |x| into amax.
-template <typename T>
-struct Vec16;
-
-template <>
-struct Vec16<uint16_t> {  // bf16 bit patterns
-    static constexpr int kElems = 8;
-    static __device__ __forceinline__ float amax(const uint4& v) {
-        uint32_t m = absmax_bf16x2(0u, v.x);
-        m = absmax_bf16x2(m, v.y);
-        m = absmax_bf16x2(m, v.z);
-        m = absmax_bf16x2(m, v.w);
-        return bf16x2_hmax(m);
-    }
-    // 8 codes -> 8 bytes
-    template <int FMT>
-    static __device__ __forceinline__ uint2 cast(const uint4& v, float s) {
-        const uint32_t c0 = cvt_fp8x2<FMT>(__fmul_rn(bf16_lo(v.x), s), __fmul_rn(bf16_hi(v.x), s));
-        const uint32_t c1 = cvt_fp8x2<FMT>(__fmul_rn(bf16_lo(v.y), s), __fmul_rn(bf16_hi(v.y), s));
-        const uint32_t c2 = cvt_fp8x2<FMT>(__fmul_rn(bf16_lo(v.z), s), __fmul_rn(bf16_hi(v.z), s));
-        const uint32_t c3 = cvt_fp8x2<FMT>(__fmul_rn(bf16_lo(v.w), s), __fmul_rn(bf16_hi(v.w), s));
-        return make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
-    }
-    using Out = uint2;
-};
-
-template <>
-struct Vec16<float> {
-    static constexpr int kElems = 4;
-    static __device__ __forceinline__ float amax(const uint4& v) {
-        const float a = fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y)));
-        const float b = fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)));
-        return fmaxf(a, b);
-    }
-    // 4 codes -> 4 bytes
-    template <int FMT>
-    static __device__ __forceinline__ uint32_t cast(const uint4& v, float s) {
-        const uint32_t c0 = cvt_fp8x2<FMT>(__fmul_rn(__uint_as_float(v.x), s), __fmul_rn(__uint_as_float(v.y), s));
-        const uint32_t c1 = cvt_fp8x2<FMT>(__fmul_rn(__uint_as_float(v.z), s), __fmul_rn(__uint_as_float(v.w), s));
-        return c0 | (c1 << 16);
-    }
-    using Out = uint32_t;
-};
+// Warp-loads per warp in the 1x128 kernel (each CTA covers 8 x LOADS
+// warp-loads = 32 KiB of bf16 with 32-byte lanes and LOADS = 4).
+#ifndef FP8Q_Q1X128_LOADS
+#define FP8Q_Q1X128_LOADS 4
+#endif
 
 // ---------------------------------------------------------------------------
-// 1x128: a block is 128 consecutive elements.  With 16-byte lanes a block is
-// 16 lanes (bf16) or 32 lanes (fp32), so one warp-wide load covers 2 (bf16) or
-// 1 (fp32) whole blocks and the block amax is a shuffle reduction inside the
-// lane group -- no shared memory, no block barrier.  Each warp takes UNROLL
-// consecutive warp-loads per trip (UNROLL * 512 contiguous bytes in flight per
-// warp) and the grid strides over the tensor.
+// 1x128: a block is 128 consecutive elements.  One lane holds a 16- or 32-byte
+// slice, so a block spans 128 / kElems lanes (8 lanes for bf16 with 32-byte
+// slices) and one warp-wide load covers 32 / that many whole blocks.  The
+// block amax is a shuffle reduction inside the lane group -- no shared
+// memory, no block barrier.  Each CTA owns one contiguous chunk: every warp
+// issues all LOADS of its warp-loads before it computes, and finished CTAs are
+// replaced by new ones, so each SM keeps its resident CTAs' chunks in flight.
 // ---------------------------------------------------------------------------
-template <typename T, int FMT, int UNROLL>
+template <typename T, int FMT, int BYTES, int LOADS>
 __global__ void __launch_bounds__(kThreads)
-k_quant_1x128(const uint4* __restrict__ x, typename Vec16<T>::Out* __restrict__ q,
+k_quant_1x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
               float* __restrict__ scales, int64_t nblocks) {
-    using V = Vec16<T>;
-    constexpr int kLanesPerBlock = 128 / V::kElems;          // 16 (bf16) or 32 (fp32)
-    constexpr int kBlocksPerLoad = 32 / kLanesPerBlock;       // 2 or 1
+    using V = LaneVec<T, BYTES>;
+    constexpr int kLanesPerBlock = 128 / V::kElems;
+    constexpr int kBlocksPerLoad = 32 / kLanesPerBlock;
     const int lane = threadIdx.x & 31;
     const int sub_block = lane / kLanesPerBlock;
     const int64_t nloads = (nblocks + kBlocksPerLoad - 1) / kBlocksPerLoad;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    const int64_t l0 = (static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5)) * LOADS;
 
-    for (int64_t l0 = warp * UNROLL; l0 < nloads; l0 += nwarps * UNROLL) {
-        uint4 v[UNROLL];
+    typename V::In v[LOADS];
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t l = l0 + u;
-            const int64_t blk = l * kBlocksPerLoad + sub_block;
-            v[u] = (l < nloads && blk < nblocks) ? ld_stream(x + l * 32 + lane) : make_uint4(0, 0, 0, 0);
-        }
+    for (int u = 0; u < LOADS; ++u) {
+        const int64_t l = l0 + u;
+        const int64_t blk = l * kBlocksPerLoad + sub_block;
+        v[u] = (l < nloads && blk < nblocks) ? ld_words_stream(x + l * 32 + lane) : V::zero();
+    }
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t l = l0 + u;
-            const int64_t blk = l * kBlocksPerLoad + sub_block;
-            const float amax = warp_max<kLanesPerBlock>(V::amax(v[u]));
-            const float s = scale_from_amax<FMT>(amax);
-            if (l < nloads && blk < nblocks) {
-                st_stream(q + l * 32 + lane, V::template cast<FMT>(v[u], s));
-                if ((lane % kLanesPerBlock) == 0) scales[blk] = s;
-            }
+    for (int u = 0; u < LOADS; ++u) {
+        const int64_t l = l0 + u;
+        const int64_t blk = l * kBlocksPerLoad + sub_block;
+        const float amax = warp_max<kLanesPerBlock>(V::amax(v[u]));
+        const float s = scale_from_amax<FMT>(amax);
+        if (l < nloads && blk < nblocks) {
+            st_stream(q + l * 32 + lane, V::template cast<FMT>(v[u], f32x2(s, s)));
+            if ((lane % kLanesPerBlock) == 0) scales[blk] = s;
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// 128x128: one CTA per tile, 8 warps, each warp owns 16 rows of the tile.  A
-// row of the tile is 256 B (bf16) or 512 B (fp32); one warp-wide 16-byte load
-// covers 2 rows (bf16) or 1 row (fp32).  The whole tile stays in registers
-// (128 B/thread bf16, 256 B/thread fp32) between the amax and the cast, so x
-// is read from HBM exactly once.  Tile amax: shuffle within the warp, then
+// 128x128, register-resident tile: one CTA per tile, 8 warps, each warp owns
+// 16 rows of the tile.  One warp-wide load covers 32 / (128 / kElems) tile
+// rows.  The whole tile stays in registers between the amax and the cast, so
+// x is read from HBM exactly once.  Tile amax: shuffle within the warp, then
 // the 8 warp maxima through shared memory.  Rows past the end (ragged bottom
-// edge) are masked; they do not count toward the amax.
+// edge) are masked and do not count toward the amax.  Used for fp32 input and
+// whenever the TMA path is unavailable.
 // ---------------------------------------------------------------------------
-template <typename T, int FMT>
+template <typename T, int FMT, int BYTES>
 __global__ void __launch_bounds__(kThreads)
-k_quant_128x128(const uint4* __restrict__ x, typename Vec16<T>::Out* __restrict__ q,
+k_quant_128x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
                 float* __restrict__ scales, int64_t rows, int64_t cols) {
-    using V = Vec16<T>;
-    constexpr int kVecPerRow = 128 / V::kElems;               // 16 (bf16) or 32 (fp32) vectors per tile row
-    constexpr int kRowsPerLoad = 32 / kVecPerRow;              // 2 or 1
-    constexpr int kLoads = 16 / kRowsPerLoad;                  // 8 or 16 loads per thread
+    using V = LaneVec<T, BYTES>;
+    constexpr int kVecPerRow = 128 / V::kElems;                // lane slices per tile row
+    constexpr int kRowsPerLoad = 32 / kVecPerRow;
+    constexpr int kLoads = 16 / kRowsPerLoad;                  // loads per thread
     __shared__ float warp_amax[kThreads / 32];
 
     const int lane = threadIdx.x & 31;
@@ -128,16 +89,16 @@ k_quant_128x128(const uint4* __restrict__ x, typename Vec16<T>::Out* __restrict_
     const int64_t tc = blockIdx.x - tr * tiles_c;
     const int row_in_load = lane / kVecPerRow;
     const int vec_in_row = lane % kVecPerRow;
-    const int64_t vec_cols = cols / V::kElems;                 // 16-byte vectors per tensor row
+    const int64_t vec_cols = cols / V::kElems;                 // lane slices per tensor row
     const int64_t r_base = tr * 128 + warp * 16 + row_in_load;
     const int64_t v_base = r_base * vec_cols + tc * kVecPerRow + vec_in_row;
 
-    uint4 v[kLoads];
+    typename V::In v[kLoads];
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < kLoads; ++i) {
         const int64_t r = r_base + i * kRowsPerLoad;
-        v[i] = (r < rows) ? ld_stream(x + v_base + i * kRowsPerLoad * vec_cols) : make_uint4(0, 0, 0, 0);
+        v[i] = (r < rows) ? ld_words_stream(x + v_base + i * kRowsPerLoad * vec_cols) : V::zero();
     }
 #pragma unroll
     for (int i = 0; i < kLoads; ++i) amax = fmaxf(amax, V::amax(v[i]));
@@ -148,10 +109,11 @@ k_quant_128x128(const uint4* __restrict__ x, typename Vec16<T>::Out* __restrict_
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w) tile_amax = fmaxf(tile_amax, warp_amax[w]);
     const float s = scale_from_amax<FMT>(tile_amax);
+    const uint64_t s2 = f32x2(s, s);
 #pragma unroll
     for (int i = 0; i < kLoads; ++i) {
         const int64_t r = r_base + i * kRowsPerLoad;
-        if (r < rows) st_stream(q + v_base + i * kRowsPerLoad * vec_cols, V::template cast<FMT>(v[i], s));
+        if (r < rows) st_stream(q + v_base + i * kRowsPerLoad * vec_cols, V::template cast<FMT>(v[i], s2));
     }
     if (threadIdx.x == 0) scales[blockIdx.x] = s;
 }
@@ -206,30 +168,31 @@ k_quant_block_general(const T* __restrict__ x, uint8_t* __restrict__ q, float* _
     }
 }
 
-template <typename T, int FMT, int UNROLL>
+template <typename T, int FMT, int BYTES, int LOADS>
 cudaError_t launch_1x128_typed(const void* x, int64_t nblocks, uint8_t* q, float* scales, cudaStream_t st) {
-    constexpr int kBlocksPerLoad = (sizeof(T) == 2) ? 2 : 1;
+    using V = LaneVec<T, BYTES>;
+    constexpr int kBlocksPerLoad = 32 / (128 / V::kElems);
     const int64_t nloads = (nblocks + kBlocksPerLoad - 1) / kBlocksPerLoad;
-    const int64_t warps_needed = (nloads + UNROLL - 1) / UNROLL;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_1x128<T, FMT, UNROLL>, kThreads, 0);
-    if (e != cudaSuccess) return e;
-    const int64_t full = static_cast<int64_t>(device_sm_count()) * (per_sm > 0 ? per_sm : 1);
-    const int64_t grid = std::min<int64_t>(full, (warps_needed + kThreads / 32 - 1) / (kThreads / 32));
-    k_quant_1x128<T, FMT, UNROLL><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
-        static_cast<const uint4*>(x), reinterpret_cast<typename Vec16<T>::Out*>(q), scales, nblocks);
+    const int64_t per_cta = static_cast<int64_t>(kThreads / 32) * LOADS;
+    const int64_t grid = (nloads + per_cta - 1) / per_cta;
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    k_quant_1x128<T, FMT, BYTES, LOADS><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
+        static_cast<const typename V::In*>(x), reinterpret_cast<typename V::Out*>(q), scales, nblocks);
     return cudaGetLastError();
 }
 
-template <typename T, int FMT>
+template <typename T, int FMT, int BYTES>
 cudaError_t launch_128x128_typed(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
                                  cudaStream_t st) {
+    using V = LaneVec<T, BYTES>;
     const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
     if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    k_quant_128x128<T, FMT><<<static_cast<unsigned>(tiles), kThreads, 0, st>>>(
-        static_cast<const uint4*>(x), reinterpret_cast<typename Vec16<T>::Out*>(q), scales, rows, cols);
+    k_quant_128x128<T, FMT, BYTES><<<static_cast<unsigned>(tiles), kThreads, 0, st>>>(
+        static_cast<const typename V::In*>(x), reinterpret_cast<typename V::Out*>(q), scales, rows, cols);
     return cudaGetLastError();
 }
+
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 template <typename T, int FMT>
 cudaError_t launch_general_typed(const void* x, int64_t rows, int64_t cols, int br, int bc, uint8_t* q,
@@ -245,22 +208,36 @@ cudaError_t launch_general_typed(const void* x, int64_t rows, int64_t cols, int 
 
 cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fmt, uint8_t* q, float* scales,
                                cudaStream_t st) {
+    const bool w32 = aligned32(x);
     if (dtype == 1) {
-        return fmt == kE4M3 ? launch_1x128_typed<uint16_t, kE4M3, 4>(x, nblocks, q, scales, st)
-                            : launch_1x128_typed<uint16_t, kE5M2, 4>(x, nblocks, q, scales, st);
+        if (w32)
+            return fmt == kE4M3 ? launch_1x128_typed<uint16_t, kE4M3, 32, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st)
+                                : launch_1x128_typed<uint16_t, kE5M2, 32, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st);
+        return fmt == kE4M3 ? launch_1x128_typed<uint16_t, kE4M3, 16, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st)
+                            : launch_1x128_typed<uint16_t, kE5M2, 16, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st);
     }
-    return fmt == kE4M3 ? launch_1x128_typed<float, kE4M3, 4>(x, nblocks, q, scales, st)
-                        : launch_1x128_typed<float, kE5M2, 4>(x, nblocks, q, scales, st);
+    if (w32)
+        return fmt == kE4M3 ? launch_1x128_typed<float, kE4M3, 32, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st)
+                            : launch_1x128_typed<float, kE5M2, 32, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st);
+    return fmt == kE4M3 ? launch_1x128_typed<float, kE4M3, 16, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st)
+                        : launch_1x128_typed<float, kE5M2, 16, FP8Q_Q1X128_LOADS>(x, nblocks, q, scales, st);
 }
 
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt, uint8_t* q,
                                  float* scales, cudaStream_t st) {
+    const bool w32 = aligned32(x);
     if (dtype == 1) {
-        return fmt == kE4M3 ? launch_128x128_typed<uint16_t, kE4M3>(x, rows, cols, q, scales, st)
-                            : launch_128x128_typed<uint16_t, kE5M2>(x, rows, cols, q, scales, st);
+        if (w32)
+            return fmt == kE4M3 ? launch_128x128_typed<uint16_t, kE4M3, 32>(x, rows, cols, q, scales, st)
+                                : launch_128x128_typed<uint16_t, kE5M2, 32>(x, rows, cols, q, scales, st);
+        return fmt == kE4M3 ? launch_128x128_typed<uint16_t, kE4M3, 16>(x, rows, cols, q, scales, st)
+                            : launch_128x128_typed<uint16_t, kE5M2, 16>(x, rows, cols, q, scales, st);
     }
-    return fmt == kE4M3 ? launch_128x128_typed<float, kE4M3>(x, rows, cols, q, scales, st)
-                        : launch_128x128_typed<float, kE5M2>(x, rows, cols, q, scales, st);
+    if (w32)
+        return fmt == kE4M3 ? launch_128x128_typed<float, kE4M3, 32>(x, rows, cols, q, scales, st)
+                            : launch_128x128_typed<float, kE5M2, 32>(x, rows, cols, q, scales, st);
+    return fmt == kE4M3 ? launch_128x128_typed<float, kE4M3, 16>(x, rows, cols, q, scales, st)
+                        : launch_128x128_typed<float, kE5M2, 16>(x, rows, cols, q, scales, st);
 }
 
 cudaError_t launch_quant_block_general(const void* x, int dtype, int64_t rows, int64_t cols, int br, int bc,

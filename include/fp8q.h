@@ -159,6 +159,32 @@ int fp8_amax_history_update(float *history, int32_t *state, int window,
 /* Static, human-readable text for a status code (never NULL). */
 const char *fp8_status_string(int status);
 
+/* ---- Diagnostics (no counterpart on the pages) ---------------------------
+ * Kernels that wait on a tile copy (the TMA pipelines) never wait forever:
+ * each wait gives up after about a second, the kernel leaves its loop, and
+ * it records the event in a device status word.  Results of that launch are
+ * then incomplete.
+ *
+ * Device status bits: */
+#define FP8_DEVICE_STATUS_WAIT_TIMEOUT 0x1u
+
+/*
+ * Enqueue a copy of the device status word of the current device into
+ * *status (a DEVICE pointer to one uint32), resetting the word to 0 when
+ * `clear` is nonzero.  Read *status after synchronizing the stream.
+ * Errors: FP8_ERR_NULL, FP8_ERR_ALIGN (status not 4-byte aligned),
+ * FP8_ERR_CUDA.
+ */
+int fp8_device_status(uint32_t *status, int clear, void *stream);
+
+/*
+ * Self-test of the bounded wait: launch one thread that waits on a barrier
+ * nothing will complete; after timeout_us microseconds it gives up and sets
+ * FP8_DEVICE_STATUS_WAIT_TIMEOUT.  The device stays usable.
+ * Errors: FP8_ERR_ARG (timeout_us == 0 or > 10 s), FP8_ERR_CUDA.
+ */
+int fp8_selftest_wait_timeout(uint32_t timeout_us, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,7 +30,8 @@ def L():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(["fp8_quantize_per_tensor", "fp8_quantize_blockwise", "fp8_dequantize",
-                                           "fp8_amax_history_update", "fp8_status_string"])
+                                           "fp8_amax_history_update", "fp8_status_string", "fp8_device_status",
+                                           "fp8_selftest_wait_timeout"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -122,6 +123,13 @@ def test_history_validation(L):
     assert f(A16, A16, 16, A16, 1, None, None) == ERR_NULL
     assert f(A1, A16, 16, A16, 1, A16, None) == ERR_ALIGN
     assert f(A16, A16 + 2, 16, A16, 1, A16, None) == ERR_ALIGN
+
+
+def test_diagnostics_validation(L):
+    assert L.fp8_device_status(None, 0, None) == ERR_NULL
+    assert L.fp8_device_status(A1, 0, None) == ERR_ALIGN
+    assert L.fp8_selftest_wait_timeout(0, None) == ERR_ARG
+    assert L.fp8_selftest_wait_timeout(20_000_000, None) == ERR_ARG
 
 
 def test_binding_refuses_cpu_tensors():

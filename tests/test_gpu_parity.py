@@ -222,6 +222,11 @@ def test_dequant_every_code_with_extreme_scales(fmt):
     scales[5, 0] = 1.4e-45   # subnormal scale
     scales[6, 1] = 3.4e38
     scales[7, 0] = 448.0 / 1e-12
+    scales[8:16] *= -1       # negative scales: the sign of zero quotients must follow IEEE
+    scales[16, 0] = 2.0 ** -100
+    scales[16, 1] = 2.0 ** -101
+    scales[17, 0] = 2.0 ** 100
+    scales[17, 1] = 2.0 ** 101
     qg = to_cuda(torch.from_numpy(q))
     sg = to_cuda(torch.from_numpy(scales))
     for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
