@@ -146,9 +146,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------
 
 KERNEL_SOURCES = {
-    "k_quant_128x128_tma": ["fine_grained_block_b200/csrc/quant_block_tma.cu",
-                            "fine_grained_block_b200/csrc/fp8q_device.cuh", "fine_grained_block_b200/csrc/fp8q_tma.cuh"],
-    "k_dequant_128x128": ["fine_grained_block_b200/csrc/dequant.cu", "fine_grained_block_b200/csrc/fp8q_device.cuh"],
+    "k_quant_128x128": ["fine_grained_block_b200/csrc/quant_block.cu", "fine_grained_block_b200/csrc/fp8q_device.cuh",
+                        "fine_grained_block_b200/csrc/lane_vec.cuh"],
+    "k_dequant_128x128": ["fine_grained_block_b200/csrc/dequant.cu", "fine_grained_block_b200/csrc/fp8q_device.cuh",
+                          "fine_grained_block_b200/csrc/lane_vec.cuh"],
 }
 
 
@@ -495,7 +496,7 @@ def run_ours(args):
 
     line = None
     if rank == 0:
-        dom = "k_quant_128x128_tma" if tq >= td else "k_dequant_128x128"
+        dom = "k_quant_128x128" if tq >= td else "k_dequant_128x128"
         dom_bytes = qb if tq >= td else db
         dom_ms = max(tq, td)
         achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -512,7 +513,7 @@ def run_ours(args):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic, "alg_bytes_per_launch": dom_bytes,
                          "us_per_launch": round(dom_ms * 1e3, 3)},
-            "kernels_us": {"k_quant_128x128_tma": round(tq * 1e3, 3), "k_dequant_128x128": round(td * 1e3, 3)},
+            "kernels_us": {"k_quant_128x128": round(tq * 1e3, 3), "k_dequant_128x128": round(td * 1e3, 3)},
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": hx.numel() * 2,
                     "d2h_bytes_per_step": hq.numel() + hs.numel() * 4 + hy.numel() * 2, "steps": e2e_steps},
             "gpu_launches": 2 * args.steps,
