@@ -68,6 +68,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def max_over_ranks(values, world: int, device="cuda"):
+    """Element-wise max of a list of floats over all ranks (all-reduce MAX); the identity at world == 1."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def step_bytes(rows=ROWS, cols=COLS, br=128, bc=128):
     """Algorithmic bytes of one step: quantize (read bf16, write codes + scales) + dequant (read codes +
     scales, write bf16)."""
@@ -315,7 +325,33 @@ def modes_breakdown(dev, stream, peak):
     wl = "bf16 activations 16384x7168, 8 channels x1e3, seed 2"
     put("1x128_e4m3_quant", wl, 3 * n + 4 * (n // 128), tq)
     put("1x128_dequant_bf16", wl, 3 * n + 4 * (n // 128), td)
+    # fused fake quant (quantize -> dequantize in one pass, bf16 in and out, no codes written)
+    fqa = lambda r: raw.check(L.fp8_fake_quantize(a.data_ptr(), 1, a.shape[0], a.shape[1], 1, 128, 0, None,
+                                                  y.data_ptr(), None, st), "fake quant")
+    (tf,) = time_per_launch([fqa], 30, 5, stream, flush)
+    put("1x128_fake_quant_bf16", wl + " (one pass, bf16 -> bf16, no codes written)", 4 * n, tf)
     del a, q, s, y
+
+    # per-tensor current scaling on small tensors: two passes vs the one-pass cooperative kernel
+    ws = torch.zeros(4, dtype=torch.int32, device=dev)
+    so1 = torch.empty(1, dtype=torch.float32, device=dev)
+    ao1 = torch.empty(1, dtype=torch.float32, device=dev)
+    for label, x_small, dt, esz in (
+            ("fp32 256x1024 outliers x1e4, seed 0 (the handbook's experiment tensor)",
+             inputs.relerr_outlier_tensors()[1][1].to(dev), 0, 4),
+            ("bf16 randn 2^22 as [1024, 4096], 0.1% x1e3, seed 4", inputs.sweep_tensor(22, device=dev), 1, 2)):
+        nn = x_small.numel()
+        qs_ = torch.empty(x_small.shape, dtype=torch.uint8, device=dev)
+        two = lambda r: raw.check(L.fp8_quantize_per_tensor(x_small.data_ptr(), dt, nn, 0, None, qs_.data_ptr(),
+                                                            so1.data_ptr(), ao1.data_ptr(), st), "per-tensor")
+        one = lambda r: raw.check(L.fp8_quantize_per_tensor_fused(x_small.data_ptr(), dt, nn, 0, qs_.data_ptr(),
+                                                                  so1.data_ptr(), ao1.data_ptr(), ws.data_ptr(), st),
+                                  "fused per-tensor")
+        t2, t1 = time_per_launch([two, one], 30, 5, stream, flush)
+        key = "fp32_1MiB" if dt == 0 else "bf16_2^22"
+        put(f"per_tensor_current_e4m3_{key}_two_pass", label, (esz + 1) * nn, t2)
+        put(f"per_tensor_current_e4m3_{key}_one_pass", label + " (cooperative one-pass kernel)", (esz + 1) * nn, t1)
+        del x_small, qs_
 
     # size sweep point 2^28 (512 MiB bf16): 1x128, 128x128, per-tensor current E5M2
     x = inputs.sweep_tensor(28, device=dev)
@@ -454,10 +490,7 @@ def run_ours(args):
     all_evs = [e for _, evs in chunks for e in evs]
     tq = statistics.fmean(e[0].elapsed_time(e[1]) for e in all_evs)
     td = statistics.fmean(e[1].elapsed_time(e[2]) for e in all_evs)
-    t = torch.tensor([total_ms, tq, td], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, tq, td = t.tolist()
+    total_ms, tq, td = max_over_ranks([total_ms, tq, td], world, device=dev)
     value = (qb + db) * args.steps * world / (total_ms * 1e-3) / 1e9
 
     # end to end through the same C ABI with host buffers: H2D of the input from pinned memory, both
@@ -489,10 +522,8 @@ def run_ours(args):
         e2e_step(r)
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = (qb + db) * e2e_steps * world / (te.item() * 1e-3) / 1e9
+    (te,) = max_over_ranks([e0.elapsed_time(e1)], world, device=dev)
+    e2e_value = (qb + db) * e2e_steps * world / (te * 1e-3) / 1e9
 
     line = None
     if rank == 0:

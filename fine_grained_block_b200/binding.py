@@ -34,11 +34,16 @@ SIGNATURES = {
     "fp8_quantize_blockwise": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "fp8_dequantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _c_int, _vp]),
     "fp8_amax_history_update": (_c_int, [_vp, _vp, _c_int, _vp, _c_int, _vp, _vp]),
+    "fp8_quantize_per_tensor_fused": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _vp, _vp]),
+    "fp8_amax": (_c_int, [_vp, _c_int, _i64, _vp, _vp]),
+    "fp8_scale_from_amax": (_c_int, [_vp, _c_int, _vp, _vp]),
+    "fp8_fake_quantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_c_int]),
     "fp8_device_status": (_c_int, [_vp, _c_int, _vp]),
     "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
 }
 DEVICE_STATUS_WAIT_TIMEOUT = 0x1
+FUSED_WORKSPACE_BYTES = 16
 
 
 class FP8Error(RuntimeError):
@@ -128,6 +133,49 @@ def fp8_quantize_per_tensor(x: torch.Tensor, fmt: int = E4M3, scale_in: torch.Te
     return q, scale_out, amax_out
 
 
+def fused_workspace(device="cuda") -> torch.Tensor:
+    """A zeroed workspace for fp8_quantize_per_tensor_fused (one per stream)."""
+    return torch.zeros(FUSED_WORKSPACE_BYTES // 4, dtype=torch.int32, device=device)
+
+
+def fp8_quantize_per_tensor_fused(x: torch.Tensor, fmt: int = E4M3, workspace: torch.Tensor | None = None,
+                                  q: torch.Tensor | None = None, scale_out: torch.Tensor | None = None,
+                                  amax_out: torch.Tensor | None = None, stream=None):
+    """Per-tensor current scaling in one pass when x fits on chip (else the two-pass path).
+
+    Returns (q, scale_out [1], amax_out [1])."""
+    _need_cuda(x, workspace, q, scale_out, amax_out)
+    dev = x.device
+    workspace = fused_workspace(dev) if workspace is None else workspace
+    q = torch.empty(x.shape, dtype=torch.uint8, device=dev) if q is None else q
+    scale_out = torch.empty(1, dtype=torch.float32, device=dev) if scale_out is None else scale_out
+    amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
+    st = load_library().fp8_quantize_per_tensor_fused(_ptr(x), _DTYPE_CODE[x.dtype], x.numel(), fmt, _ptr(q),
+                                                      _ptr(scale_out), _ptr(amax_out), _ptr(workspace),
+                                                      _stream(stream))
+    _check("fp8_quantize_per_tensor_fused", st)
+    return q, scale_out, amax_out
+
+
+def fp8_amax(x: torch.Tensor, amax_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """max |x| into a 1-element fp32 CUDA tensor."""
+    _need_cuda(x, amax_out)
+    amax_out = torch.empty(1, dtype=torch.float32, device=x.device) if amax_out is None else amax_out
+    _check("fp8_amax", load_library().fp8_amax(_ptr(x), _DTYPE_CODE[x.dtype], x.numel(), _ptr(amax_out),
+                                               _stream(stream)))
+    return amax_out
+
+
+def fp8_scale_from_amax(amax: torch.Tensor, fmt: int = E4M3, scale_out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """MAX / max(amax, 1e-12) into a 1-element fp32 CUDA tensor."""
+    _need_cuda(amax, scale_out)
+    scale_out = torch.empty(1, dtype=torch.float32, device=amax.device) if scale_out is None else scale_out
+    _check("fp8_scale_from_amax", load_library().fp8_scale_from_amax(_ptr(amax), fmt, _ptr(scale_out),
+                                                                     _stream(stream)))
+    return scale_out
+
+
 def fp8_quantize_blockwise(x: torch.Tensor, block=(1, 128), fmt: int = E4M3, q: torch.Tensor | None = None,
                            scales: torch.Tensor | None = None, stream=None):
     """Blockwise quantize of a 2-D tensor with (1, 128) or (128, 128) blocks.  Returns (q, scales)."""
@@ -159,6 +207,23 @@ def fp8_dequantize(q: torch.Tensor, scales: torch.Tensor, block=(0, 0), fmt: int
     st = load_library().fp8_dequantize(_ptr(q), fmt, R, C, block[0], block[1], _ptr(scales), _ptr(y),
                                        _DTYPE_CODE[y.dtype], _stream(stream))
     _check("fp8_dequantize", st)
+    return y
+
+
+def fp8_fake_quantize(x: torch.Tensor, block=(1, 128), fmt: int = E4M3, scale_in: torch.Tensor | None = None,
+                      y: torch.Tensor | None = None, scales_out: torch.Tensor | None = None, stream=None):
+    """Quantize -> dequantize round trip in x's dtype (block (0, 0) = per tensor with scale_in).  Returns y."""
+    _need_cuda(x, scale_in, y, scales_out)
+    if x.dim() == 1:
+        R, C = 1, x.shape[0]
+    elif x.dim() == 2:
+        R, C = x.shape
+    else:
+        raise ValueError("fake quantize takes a 1-D or 2-D tensor")
+    y = torch.empty_like(x) if y is None else y
+    st = load_library().fp8_fake_quantize(_ptr(x), _DTYPE_CODE[x.dtype], R, C, block[0], block[1], fmt,
+                                          _ptr(scale_in), _ptr(y), _ptr(scales_out), _stream(stream))
+    _check("fp8_fake_quantize", st)
     return y
 
 

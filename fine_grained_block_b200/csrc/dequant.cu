@@ -26,6 +26,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "dequant_math.cuh"
 #include "lane_vec.cuh"
 
 namespace fp8q {
@@ -37,39 +38,6 @@ constexpr int kThreads = 256;
 #define FP8Q_DEQ_UNROLL 4
 #endif
 constexpr int kUnroll = FP8Q_DEQ_UNROLL;
-
-// |s| in [2^-100, 2^101): r, q * r, the residual and the result all stay normal.
-__device__ __forceinline__ bool scale_fast_ok(float s) {
-    const uint32_t ex = (__float_as_uint(s) >> 23) & 0xFFu;
-    return ex >= 27u && ex <= 227u;
-}
-
-// True when any of the 4 codes in w is an E5M2 Inf/NaN code (exponent field all ones).
-__device__ __forceinline__ bool e5m2_has_special(uint32_t w) {
-    return (((w & 0x7C7C7C7Cu) + 0x04040404u) & 0x80808080u) != 0u;
-}
-
-// Two codes (low 16 bits of c2) -> two exact quotients RN(q / s), from
-// r2 = {RN(1/s)} x2 and ns2 = {-s} x2:
-//   y0 = q * r;  e = q - s * y0 (fma);  y = y0 + e * r (fma)
-// For q = +-0 the last fma would give +0 for -0, so the sign is taken from
-// y0, which carries the quotient's sign for every q.
-template <int FMT>
-__device__ __forceinline__ float2 dequant2_fast(uint32_t c2, uint64_t r2, uint64_t ns2) {
-    const float2 a = fp8x2_to_float2<FMT>(c2);
-    const uint64_t q2 = f32x2(a.x, a.y);
-    const uint64_t y0 = mul_f32x2(q2, r2);
-    const uint64_t e = fma_f32x2(y0, ns2, q2);
-    const float2 y = f32x2_split(fma_f32x2(e, r2, y0));
-    const float2 z = f32x2_split(y0);
-    return make_float2(copysignf(y.x, z.x), copysignf(y.y, z.y));
-}
-
-template <int FMT>
-__device__ __forceinline__ float2 dequant2_div(uint32_t c2, float s) {
-    const float2 a = fp8x2_to_float2<FMT>(c2);
-    return make_float2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s));
-}
 
 template <int NW>
 __device__ __forceinline__ void unpack_codes(const typename CodeWords<NW>::T& c, uint32_t* w);

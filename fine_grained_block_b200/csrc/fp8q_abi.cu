@@ -80,6 +80,44 @@ int fp8_quantize_per_tensor(const void* x, int dtype, int64_t n, int fmt, const 
                                               scale_in ? amax_out : nullptr, st));
 }
 
+int fp8_quantize_per_tensor_fused(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
+                                  float* amax_out, void* workspace, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (scale_out == nullptr || amax_out == nullptr || workspace == nullptr) return FP8_ERR_NULL;
+    if (n > 0 && (x == nullptr || q == nullptr)) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale_out, 4) || !aligned(amax_out, 4) ||
+        !aligned(workspace, 16))
+        return FP8_ERR_ALIGN;
+    if (n > 0) {
+        bool launched = false;
+        const cudaError_t e = fp8q::launch_tensor_fused(x, dtype, n, fmt, q, scale_out, amax_out, workspace,
+                                                        static_cast<cudaStream_t>(stream), &launched);
+        if (e != cudaSuccess) return FP8_ERR_CUDA;
+        if (launched) return FP8_OK;
+    }
+    return fp8_quantize_per_tensor(x, dtype, n, fmt, nullptr, q, scale_out, amax_out, stream);
+}
+
+int fp8_amax(const void* x, int dtype, int64_t n, float* amax_out, void* stream) {
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (amax_out == nullptr || (n > 0 && x == nullptr)) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(amax_out, 4)) return FP8_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax_out, 0, sizeof(float), st) != cudaSuccess) return FP8_ERR_CUDA;
+    if (n == 0) return FP8_OK;
+    return status_of(fp8q::launch_tensor_amax(x, dtype, n, amax_out, st));
+}
+
+int fp8_scale_from_amax(const float* amax_in, int fmt, float* scale_out, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (amax_in == nullptr || scale_out == nullptr) return FP8_ERR_NULL;
+    if (!aligned(amax_in, 4) || !aligned(scale_out, 4)) return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_scale_from_amax(amax_in, fmt, scale_out, static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_quantize_blockwise(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows, int block_cols,
                            int fmt, uint8_t* q, float* scales, void* stream) {
     if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
@@ -122,6 +160,27 @@ int fp8_dequantize(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int bl
     if (!aligned(q, 16) || !aligned(y, 16) || !aligned(scales, 4)) return FP8_ERR_ALIGN;
     return status_of(fp8q::launch_dequant(q, fmt, rows, cols, mode, scales, y, out_dtype,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_fake_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows, int block_cols, int fmt,
+                      const float* scale_in, void* y, float* scales_out, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    const bool per_tensor = (block_rows == 0 && block_cols == 0);
+    if (!per_tensor && !((block_rows == 1 || block_rows == 128) && block_cols == 128)) return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (per_tensor && scale_in == nullptr) return FP8_ERR_NULL;
+    if (n == 0) return FP8_OK;
+    if (x == nullptr || y == nullptr) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(scale_in, 4) || !aligned(scales_out, 4)) return FP8_ERR_ALIGN;
+    const size_t esize = dtype == FP8_F32 ? 4 : 2;
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t bytes = static_cast<uintptr_t>(n) * esize;
+    if (xb != yb && xb < yb + bytes && yb < xb + bytes) return FP8_ERR_ARG;  // partial overlap
+    return status_of(fp8q::launch_fake_quant(x, dtype, rows, cols, per_tensor ? 0 : block_rows, fmt, scale_in, y,
+                                             per_tensor ? nullptr : scales_out, static_cast<cudaStream_t>(stream)));
 }
 
 int fp8_amax_history_update(float* history, int32_t* state, int window, const float* amax, int fmt, float* scale,

@@ -29,6 +29,15 @@ bool tma_128x128_supported(int dtype, int64_t rows, int64_t cols);
 cudaError_t launch_quant_128x128_tma(const void* x, int64_t rows, int64_t cols, int fmt, uint8_t* q,
                                      float* scales, cudaStream_t stream);
 
+// Device address of the status word of the current device (nullptr on failure).
+unsigned int* device_status_word();
+
+// One-pass per-tensor current scaling (cooperative launch, 16-byte workspace).
+// Sets *launched = false (and enqueues nothing) when x is too large for one
+// pass; the caller then takes the two-pass path.
+cudaError_t launch_tensor_fused(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
+                                float* amax_out, void* workspace, cudaStream_t stream, bool* launched);
+
 // Copy the device status word to out[0] (device memory), clearing it if asked.
 cudaError_t launch_device_status(unsigned int* out, int clear, cudaStream_t stream);
 
@@ -45,6 +54,9 @@ cudaError_t launch_quant_block_general(const void* x, int dtype, int64_t rows, i
 cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_out,
                                cudaStream_t stream);
 
+// *scale_out = MAX / max(*amax_in, eps) (one thread).
+cudaError_t launch_scale_from_amax(const float* amax_in, int fmt, float* scale_out, cudaStream_t stream);
+
 // Per-tensor cast.  scale_in == nullptr: s from *amax_in (current scaling);
 // else s = *scale_in (delayed), and amax_out (if non-null, zeroed by the
 // caller) receives amax(x) from the same pass.  *scale_out = s.
@@ -52,6 +64,12 @@ cudaError_t launch_tensor_cast(const void* x, int dtype, int64_t n, int fmt,
                                const float* scale_in, const float* amax_in,
                                uint8_t* q, float* scale_out, float* amax_out,
                                cudaStream_t stream);
+
+// Fused quantize -> dequantize round trip in x's dtype.  block_rows 0: per
+// tensor with *scale_in; 1 or 128: block scales (written to `scales` if it is
+// non-null).
+cudaError_t launch_fake_quant(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows, int fmt,
+                              const float* scale_in, void* y, float* scales, cudaStream_t stream);
 
 // Dequantize.  mode 0: per-tensor; 1: 1x128; 2: 128x128.
 cudaError_t launch_dequant(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int mode,

@@ -1,5 +1,4 @@
-// quant_block_tma.cu -- 128x128 block quantization with TMA-staged tiles, and
-// the library's device status word.
+// quant_block_tma.cu -- 128x128 block quantization with TMA-staged tiles.
 //
 // Mixed-precision handbook, section "FP8 training", per_block with 128x128
 // blocks (the weight layout): one scale per 128x128 tile.
@@ -28,9 +27,6 @@
 
 namespace fp8q {
 
-// Bits of kStatus*; set by kernels whose bounded waits ran out.
-__device__ unsigned int g_device_status = 0u;
-
 namespace {
 
 constexpr int kTmaThreads = 256;
@@ -44,14 +40,12 @@ constexpr int kTileBytes = 128 * 128 * 2;  // one bf16 tile
 constexpr int kStages = FP8Q_TMA_STAGES;   // tiles in flight per CTA
 constexpr int kCtasPerSm = FP8Q_TMA_CTAS;  // independent pipelines per SM
 
-__device__ __forceinline__ void record_status(unsigned int bit) { atomicOr(&g_device_status, bit); }
-
 using TileVec = LaneVec<uint16_t, 16>;  // 16 bytes of a tile row per lane
 
 template <int FMT, int STAGES>
 __global__ void __launch_bounds__(kTmaThreads, kCtasPerSm)
 k_quant_128x128_tma(const __grid_constant__ CUtensorMap tmap, uint2* __restrict__ q, float* __restrict__ scales,
-                    int64_t rows, int64_t cols, int64_t ntiles) {
+                    int64_t rows, int64_t cols, int64_t ntiles, unsigned int* status) {
     extern __shared__ uint8_t smem_raw[];
     // tiles first (128-byte aligned for the copy engine), then the barriers
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -116,7 +110,7 @@ k_quant_128x128_tma(const __grid_constant__ CUtensorMap tmap, uint2* __restrict_
         // may be refilled) and its maximum in red[]; red[] alternates by tile
         // parity, so the next tile's writes cannot race these reads.
         if (__syncthreads_or(!ok)) {
-            if (tid == 0) record_status(kStatusWaitTimeout);
+            if (tid == 0) atomicOr(status, kStatusWaitTimeout);
             break;
         }
         if (tid == 0) {
@@ -150,19 +144,6 @@ k_quant_128x128_tma(const __grid_constant__ CUtensorMap tmap, uint2* __restrict_
     }
 }
 
-// Diagnostics: copy (and optionally clear) the status word; and a wait that
-// nothing will ever complete, to exercise the timeout path.
-__global__ void k_device_status(unsigned int* out, int clear) {
-    out[0] = clear ? atomicExch(&g_device_status, 0u) : atomicOr(&g_device_status, 0u);
-}
-
-__global__ void k_selftest_wait_timeout(uint64_t limit_ns) {
-    __shared__ uint64_t bar;
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-    if (!mbar_wait_bounded(&bar, 0, limit_ns)) record_status(kStatusWaitTimeout);
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -185,8 +166,10 @@ cudaError_t launch_tma_typed(const CUtensorMap& map, uint8_t* q, float* scales, 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(ntiles, static_cast<int64_t>(device_sm_count()) * kCtasPerSm);
+    unsigned int* status = device_status_word();
+    if (status == nullptr) return cudaErrorInvalidValue;
     kern<<<static_cast<unsigned>(grid), kTmaThreads, smem, st>>>(map, reinterpret_cast<uint2*>(q), scales, rows,
-                                                                 cols, ntiles);
+                                                                 cols, ntiles, status);
     return cudaGetLastError();
 }
 
@@ -212,16 +195,6 @@ cudaError_t launch_quant_128x128_tma(const void* x, int64_t rows, int64_t cols, 
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     return fmt == kE4M3 ? launch_tma_typed<kE4M3>(map, q, scales, rows, cols, st)
                         : launch_tma_typed<kE5M2>(map, q, scales, rows, cols, st);
-}
-
-cudaError_t launch_device_status(unsigned int* out, int clear, cudaStream_t st) {
-    k_device_status<<<1, 1, 0, st>>>(out, clear);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st) {
-    k_selftest_wait_timeout<<<1, 1, 0, st>>>(limit_ns);
-    return cudaGetLastError();
 }
 
 }  // namespace fp8q

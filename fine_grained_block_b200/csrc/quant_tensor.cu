@@ -115,6 +115,11 @@ k_tensor_cast(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
 }
 
+template <int FMT>
+__global__ void k_scale_from_amax(const float* amax_in, float* scale_out) {
+    *scale_out = scale_from_amax<FMT>(*amax_in);
+}
+
 int64_t chunk_grid(int64_t nvec) {
     const int64_t per_cta = static_cast<int64_t>(kThreads) * kUnroll;
     return std::max<int64_t>(1, (nvec + per_cta - 1) / per_cta);
@@ -175,6 +180,12 @@ cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_
     if (dtype == 1)
         return aligned32(x) ? amax_typed<uint16_t, 32>(x, n, amax_out, st) : amax_typed<uint16_t, 16>(x, n, amax_out, st);
     return aligned32(x) ? amax_typed<float, 32>(x, n, amax_out, st) : amax_typed<float, 16>(x, n, amax_out, st);
+}
+
+cudaError_t launch_scale_from_amax(const float* amax_in, int fmt, float* scale_out, cudaStream_t st) {
+    if (fmt == kE4M3) k_scale_from_amax<kE4M3><<<1, 1, 0, st>>>(amax_in, scale_out);
+    else k_scale_from_amax<kE5M2><<<1, 1, 0, st>>>(amax_in, scale_out);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_tensor_cast(const void* x, int dtype, int64_t n, int fmt, const float* scale_in,

@@ -1,0 +1,201 @@
+// quant_tensor_fused.cu -- per-tensor current scaling in ONE pass over x, for
+// tensors that fit in the registers of the CTAs that can be resident at once.
+//
+// PyTorch-FP8 page s4.1 (scale = max_val / amax) and mixed-precision handbook
+// "FP8 training" per_tensor: the scale needs the amax of the whole tensor
+// before any element is cast, which normally costs a second read of x.  Here
+// every CTA loads its slice of x into registers, folds its amax into a small
+// workspace, and waits at a grid-wide barrier; the last CTA to arrive writes
+// amax_out and scale_out and resets the workspace; then every CTA casts the
+// slice it still holds.  x is read once and the three launches of the
+// two-pass path (memset, amax, cast) become one.
+//
+// The launch is cooperative, so all CTAs are co-resident and the barrier
+// cannot deadlock.  The barrier wait is still bounded (about a second); if it
+// runs out the CTA records the wait-timeout bit in the device status word and
+// returns without writing its codes.
+//
+// Workspace (16 bytes of device memory, zero before the first use, left zero
+// after every call): {arrivals, generation, amax bits, unused}.  Calls that
+// share a workspace must not overlap on the device.
+
+#include <algorithm>
+
+#include "fp8q_device.cuh"
+#include "fp8q_launch.h"
+#include "fp8q_tma.cuh"
+#include "lane_vec.cuh"
+
+namespace fp8q {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kLoads = 4;  // lane vectors per thread held in registers
+
+struct Workspace {
+    unsigned int arrivals;
+    unsigned int generation;
+    unsigned int amax_bits;
+    unsigned int unused;
+};
+static_assert(sizeof(Workspace) == 16, "workspace layout");
+
+__device__ __forceinline__ unsigned int ld_volatile(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.volatile.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_volatile(const float* p) {
+    float v;
+    asm volatile("ld.volatile.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+
+template <typename T>
+__device__ __forceinline__ float load_scalar(const T* p, int i);
+template <>
+__device__ __forceinline__ float load_scalar<uint16_t>(const uint16_t* p, int i) {
+    return __uint_as_float(static_cast<uint32_t>(p[i]) << 16);
+}
+template <>
+__device__ __forceinline__ float load_scalar<float>(const float* p, int i) { return p[i]; }
+
+template <typename T, int FMT, int BYTES>
+__global__ void __launch_bounds__(kThreads)
+k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec, const T* __restrict__ tail,
+               int tail_n, typename LaneVec<T, BYTES>::Out* __restrict__ q, uint8_t* __restrict__ q_tail,
+               float* scale_out, float* amax_out, Workspace* ws, unsigned int* status) {
+    using V = LaneVec<T, BYTES>;
+    __shared__ float warp_amax[kThreads / 32];
+    __shared__ float cta_result;
+    __shared__ int cta_ok;
+
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kLoads + threadIdx.x;
+    typename V::In v[kLoads];
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+        const int64_t i = base + u * kThreads;
+        v[u] = (i < nvec) ? ld_words_stream(x + i) : V::zero();
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) a = fmaxf(a, V::amax(v[u]));
+    float xt = 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x < tail_n) {
+        xt = load_scalar(tail, threadIdx.x);
+        a = fmaxf(a, fabsf(xt));
+    }
+    a = warp_max<32>(a);
+    if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = a;
+    __syncthreads();
+
+    if (threadIdx.x == 0) {
+        float m = warp_amax[0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_amax[w]);
+        // contribute this CTA's amax (skipped when the running maximum is already as large)
+        if (__float_as_uint(m) > ld_volatile(&ws->amax_bits)) atomicMax(&ws->amax_bits, __float_as_uint(m));
+        const unsigned int gen = ld_volatile(&ws->generation);  // read before arriving
+        __threadfence();
+        const unsigned int arrived = atomicAdd(&ws->arrivals, 1u);
+        bool ok = true;
+        float amax;
+        if (arrived == gridDim.x - 1) {
+            // last to arrive: every other CTA's atomicMax is ordered before its arrival
+            __threadfence();
+            amax = __uint_as_float(atomicOr(&ws->amax_bits, 0u));
+            *amax_out = amax;
+            *scale_out = scale_from_amax<FMT>(amax);
+            ws->amax_bits = 0u;
+            ws->arrivals = 0u;
+            __threadfence();
+            atomicAdd(&ws->generation, 1u);  // releases the waiting CTAs
+        } else {
+            const uint64_t start = global_timer_ns();
+            while (ld_volatile(&ws->generation) == gen) {
+                if (global_timer_ns() - start > kWaitLimitNs) {
+                    ok = false;
+                    break;
+                }
+            }
+            __threadfence();
+            amax = ld_volatile(amax_out);
+        }
+        if (!ok) atomicOr(status, kStatusWaitTimeout);
+        cta_result = amax;
+        cta_ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (!cta_ok) return;
+
+    const float s = scale_from_amax<FMT>(cta_result);
+    const uint64_t s2 = f32x2(s, s);
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+        const int64_t i = base + u * kThreads;
+        if (i < nvec) st_stream(q + i, V::template cast<FMT>(v[u], s2));
+    }
+    if (blockIdx.x == 0 && threadIdx.x < tail_n)
+        q_tail[threadIdx.x] = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(xt, s), 0.0f) & 0xFFu);
+}
+
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+// Largest grid that can be co-resident, or 0 when cooperative launch is unavailable.
+template <typename Kernel>
+int64_t resident_ctas(Kernel k) {
+    int dev = 0, coop = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, 0) != cudaSuccess) return 0;
+    return static_cast<int64_t>(per_sm) * device_sm_count();
+}
+
+template <typename T, int FMT, int BYTES>
+cudaError_t fused_typed(const void* x, int64_t n, uint8_t* q, float* scale_out, float* amax_out, void* ws,
+                        cudaStream_t st, bool* launched) {
+    using V = LaneVec<T, BYTES>;
+    auto kern = k_tensor_fused<T, FMT, BYTES>;
+    const int64_t nvec = n / V::kElems;
+    const int tail_n = static_cast<int>(n - nvec * V::kElems);
+    const int64_t per_cta = static_cast<int64_t>(kThreads) * kLoads;
+    const int64_t grid = std::max<int64_t>(1, (nvec + per_cta - 1) / per_cta);
+    *launched = false;
+    if (grid > resident_ctas(kern)) return cudaSuccess;  // too large for one pass: caller falls back
+    const typename V::In* xv = static_cast<const typename V::In*>(x);
+    const T* tail = static_cast<const T*>(x) + nvec * V::kElems;
+    typename V::Out* qv = reinterpret_cast<typename V::Out*>(q);
+    uint8_t* q_tail = q + nvec * V::kElems;
+    Workspace* w = static_cast<Workspace*>(ws);
+    unsigned int* status = device_status_word();
+    if (status == nullptr) return cudaErrorInvalidValue;
+    int64_t nvec_arg = nvec;
+    int tail_arg = tail_n;
+    void* args[] = {&xv, &nvec_arg, &tail, &tail_arg, &qv, &q_tail, &scale_out, &amax_out, &w, &status};
+    cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(static_cast<unsigned>(grid)),
+                                                dim3(kThreads), args, 0, st);
+    if (e == cudaSuccess) *launched = true;
+    return e;
+}
+
+template <typename T, int FMT>
+cudaError_t fused_width(const void* x, int64_t n, uint8_t* q, float* scale_out, float* amax_out, void* ws,
+                        cudaStream_t st, bool* launched) {
+    if (aligned32(x)) return fused_typed<T, FMT, 32>(x, n, q, scale_out, amax_out, ws, st, launched);
+    return fused_typed<T, FMT, 16>(x, n, q, scale_out, amax_out, ws, st, launched);
+}
+
+}  // namespace
+
+cudaError_t launch_tensor_fused(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
+                                float* amax_out, void* workspace, cudaStream_t st, bool* launched) {
+    if (dtype == 1) {
+        return fmt == kE4M3 ? fused_width<uint16_t, kE4M3>(x, n, q, scale_out, amax_out, workspace, st, launched)
+                            : fused_width<uint16_t, kE5M2>(x, n, q, scale_out, amax_out, workspace, st, launched);
+    }
+    return fmt == kE4M3 ? fused_width<float, kE4M3>(x, n, q, scale_out, amax_out, workspace, st, launched)
+                        : fused_width<float, kE5M2>(x, n, q, scale_out, amax_out, workspace, st, launched);
+}
+
+}  // namespace fp8q

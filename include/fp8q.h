@@ -88,6 +88,51 @@ int fp8_quantize_per_tensor(const void *x, int dtype, int64_t n, int fmt,
                             float *scale_out, float *amax_out, void *stream);
 
 /*
+ * Per-tensor CURRENT scaling in one pass over x, for tensors small enough to
+ * be held on chip by the CTAs that fit on the GPU at once (about 8-9 MiB of
+ * input on a B200; larger tensors transparently take the two-pass path of
+ * fp8_quantize_per_tensor and do not touch the workspace).  Same results as
+ * fp8_quantize_per_tensor with scale_in == NULL.
+ *
+ *   x, dtype, n, fmt, q, scale_out, amax_out   as fp8_quantize_per_tensor
+ *              (scale_out and amax_out both required)
+ *   workspace  FP8_FUSED_WORKSPACE_BYTES of caller-owned device memory,
+ *              16-byte aligned, zeroed once before its first use; every call
+ *              leaves it zeroed again.  Calls that share a workspace must not
+ *              overlap on the device (use one workspace per stream).
+ * The one-pass kernel holds its slice of x in registers, meets the other CTAs
+ * at a grid-wide barrier (a cooperative launch, so every CTA is resident),
+ * and then casts.  The barrier wait gives up after about a second, sets
+ * FP8_DEVICE_STATUS_WAIT_TIMEOUT and leaves the codes unwritten.
+ * Errors: those of fp8_quantize_per_tensor; FP8_ERR_NULL or FP8_ERR_ALIGN
+ * for the workspace.
+ */
+#define FP8_FUSED_WORKSPACE_BYTES 16
+int fp8_quantize_per_tensor_fused(const void *x, int dtype, int64_t n, int fmt,
+                                  uint8_t *q, float *scale_out, float *amax_out,
+                                  void *workspace, void *stream);
+
+/*
+ * amax of a tensor: *amax_out = max |x| (0 for n == 0).  [FP8-native] s4.1.
+ * The first step of per-tensor current scaling, exposed on its own so that a
+ * tensor sharded over several GPUs can all-reduce (MAX) the shards' amax
+ * before the scale is formed.
+ *   x          [n], FP8_F32 or FP8_BF16
+ *   amax_out   [1] fp32 output (device)
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_DTYPE,
+ * FP8_ERR_CUDA.
+ */
+int fp8_amax(const void *x, int dtype, int64_t n, float *amax_out, void *stream);
+
+/*
+ * The scale from an amax: *scale_out = fp32(MAX / max(*amax_in, 1e-12f)).
+ * [FP8-native] s4.1.  Both pointers are device pointers (one fp32 each) and
+ * may be equal.
+ * Errors: FP8_ERR_NULL, FP8_ERR_ALIGN, FP8_ERR_FORMAT, FP8_ERR_CUDA.
+ */
+int fp8_scale_from_amax(const float *amax_in, int fmt, float *scale_out, void *stream);
+
+/*
  * Fine-grained (blockwise) quantization: one scale per block_rows x
  * block_cols block, in one fused pass (amax, scale, cast, scale store).
  * Follows [MP-handbook] "FP8 training" per_block: 1x128 blocks for
@@ -130,6 +175,29 @@ int fp8_quantize_blockwise(const void *x, int dtype, int64_t rows, int64_t cols,
 int fp8_dequantize(const uint8_t *q, int fmt, int64_t rows, int64_t cols,
                    int block_rows, int block_cols, const float *scales,
                    void *y, int out_dtype, void *stream);
+
+/*
+ * Fake quantization: the quantize -> dequantize round trip in one pass,
+ *   y = RN_dtype( RN_f32( decode(q) / s ) ),  q = fp8( RN_f32(x * s) ),
+ * in x's own dtype.  No codes are written.  Follows [FP8-native] s3.2
+ * (FP8QuantizeFunction forward: scale, cast to FP8, cast back) and s4.2
+ * DelayedScaler.quantize(), and [MP-handbook] "FP8 training" quant().
+ *
+ *   x, y       [rows, cols] of dtype (FP8_F32 or FP8_BF16); y may be x
+ *              (in place) but must not otherwise overlap it
+ *   block_rows, block_cols   (1, 128) or (128, 128): s from each block's
+ *              amax, as in fp8_quantize_blockwise (ragged edges allowed);
+ *              (0, 0): one scale for the tensor, given by scale_in
+ *   scale_in   (0, 0) only: device pointer to the fp32 scale (required)
+ *   scales_out block modes only: where to write the block scales (layout of
+ *              fp8_quantize_blockwise), or NULL to not write them
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN, FP8_ERR_FORMAT,
+ * FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_fake_quantize(const void *x, int dtype, int64_t rows, int64_t cols,
+                      int block_rows, int block_cols, int fmt,
+                      const float *scale_in, void *y, float *scales_out,
+                      void *stream);
 
 /*
  * Delayed scaling: push one amax into the amax history and refresh the scale.

@@ -176,6 +176,23 @@ def dequantize(q: np.ndarray, fmt: int, scales: np.ndarray, br: int = 0, bc: int
     return y
 
 
+def fake_quantize(x: np.ndarray, fmt: int, br: int = 1, bc: int = 128, scale: float | None = None):
+    """Quantize -> dequantize round trip in x's dtype: the composition of the two oracle steps.
+
+    br = bc = 0 is per tensor with the given scale.  Returns (y, scales) -- scales is the block
+    scales, or the one-element scale array for per tensor."""
+    x, dt = _as_input(x)
+    if br == 0 and bc == 0:
+        if scale is None:
+            raise ValueError("per-tensor fake quantize needs a scale")
+        q, s, _ = quantize_per_tensor(x, fmt, scale=scale)
+        scales = np.array([s], dtype=np.float32)
+    else:
+        q, scales = quantize_blockwise(x if x.ndim == 2 else x.reshape(1, -1), br, bc, fmt)
+    y = dequantize(q.reshape(x.shape) if x.ndim == 2 else q.reshape(1, -1), fmt, scales, br, bc, out_dtype=dt)
+    return y.reshape(x.shape), scales
+
+
 class AmaxHistory:
     """Delayed-scaling state: a window of past amax values and the current scale."""
 

@@ -99,18 +99,32 @@ def oracle_dequant(q: np.ndarray, fmt: int, scales: np.ndarray, br: int, bc: int
     return np.concatenate(parts)
 
 
+def _nan_mask(bits: np.ndarray, kind: str) -> np.ndarray:
+    if kind == "f32":
+        return ((bits & 0x7F800000) == 0x7F800000) & ((bits & 0x007FFFFF) != 0)
+    return ((bits & 0x7F80) == 0x7F80) & ((bits & 0x007F) != 0)
+
+
 def assert_bytes_equal(got: torch.Tensor, want: np.ndarray, what: str):
+    """Bit-for-bit equality.  For fp32 / bf16 values, two NaNs count as equal whatever their payload
+    (the contract fixes NaN-ness, not the NaN bit pattern)."""
     g = got.detach().cpu().contiguous()
+    kind = None
     if g.dtype == torch.bfloat16:
         g = g.view(torch.int16).numpy().view(np.uint16)
+        kind = "bf16"
     elif g.dtype == torch.float32:
         g = g.numpy().view(np.uint32)
         want = want.view(np.uint32) if want.dtype == np.float32 else want
+        kind = "f32"
     else:
         g = g.numpy()
     want = np.asarray(want).reshape(g.shape)
-    if not np.array_equal(g, want):
-        bad = np.argwhere(g != want)
+    diff = g != want
+    if kind is not None:
+        diff &= ~(_nan_mask(g, kind) & _nan_mask(want, kind))
+    if diff.any():
+        bad = np.argwhere(diff)
         i = tuple(bad[0])
         raise AssertionError(f"{what}: {len(bad)} mismatches; first at {i}: got {g[i]!r} want {want[i]!r}")
 

@@ -31,6 +31,8 @@ def L():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(["fp8_quantize_per_tensor", "fp8_quantize_blockwise", "fp8_dequantize",
                                            "fp8_amax_history_update", "fp8_status_string", "fp8_device_status",
+                                           "fp8_fake_quantize", "fp8_amax", "fp8_scale_from_amax",
+                                           "fp8_quantize_per_tensor_fused",
                                            "fp8_selftest_wait_timeout"])
 
 
@@ -110,6 +112,47 @@ def test_per_tensor_validation(L):
     assert f(A16, 1, 16, 0, A1, A16, A16, A16, None) == ERR_ALIGN
     assert f(A16, 1, 16, 0, None, A16, A1, A16, None) == ERR_ALIGN
     assert f(A16, 1, 16, 0, None, A16, A16, A1, None) == ERR_ALIGN
+
+
+def test_fake_quant_validation(L):
+    f = L.fp8_fake_quantize
+    assert f(A16, 1, 4, 256, 1, 128, 3, None, A16, None, None) == ERR_FORMAT
+    assert f(A16, 4, 4, 256, 1, 128, 0, None, A16, None, None) == ERR_DTYPE
+    assert f(A16, 1, 4, 256, 1, 64, 0, None, A16, None, None) == ERR_SHAPE
+    assert f(A16, 1, -4, 256, 1, 128, 0, None, A16, None, None) == ERR_SHAPE
+    assert f(A16, 1, 4, 256, 0, 0, 0, None, A16, None, None) == ERR_NULL   # per tensor needs scale_in
+    assert f(None, 1, 4, 256, 1, 128, 0, None, A16, None, None) == ERR_NULL
+    assert f(A16, 1, 4, 256, 1, 128, 0, None, None, None, None) == ERR_NULL
+    assert f(A1, 1, 4, 256, 1, 128, 0, None, A16, None, None) == ERR_ALIGN
+    assert f(A16, 1, 4, 256, 1, 128, 0, None, A16 + 8, None, None) == ERR_ALIGN
+    assert f(A16, 1, 4, 256, 1, 128, 0, None, A16 + 16, None, None) == ERR_ARG  # partial overlap
+    assert f(None, 1, 0, 256, 1, 128, 0, None, None, None, None) == OK
+
+
+def test_fused_per_tensor_validation(L):
+    f = L.fp8_quantize_per_tensor_fused
+    assert f(A16, 1, 16, 9, A16, A16, A16, A16, None) == ERR_FORMAT
+    assert f(A16, 5, 16, 0, A16, A16, A16, A16, None) == ERR_DTYPE
+    assert f(A16, 1, -1, 0, A16, A16, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 16, 0, A16, A16, A16, None, None) == ERR_NULL   # workspace
+    assert f(A16, 1, 16, 0, A16, None, A16, A16, None) == ERR_NULL
+    assert f(A16, 1, 16, 0, A16, A16, None, A16, None) == ERR_NULL
+    assert f(None, 1, 16, 0, A16, A16, A16, A16, None) == ERR_NULL
+    assert f(A16, 1, 16, 0, A16, A16, A16, A16 + 8, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, A4, A16, A16, A16, None) == ERR_ALIGN
+
+
+def test_amax_and_scale_validation(L):
+    assert L.fp8_amax(A16, 7, 16, A16, None) == ERR_DTYPE
+    assert L.fp8_amax(A16, 1, -1, A16, None) == ERR_SHAPE
+    assert L.fp8_amax(A16, 1, 16, None, None) == ERR_NULL
+    assert L.fp8_amax(None, 1, 16, A16, None) == ERR_NULL
+    assert L.fp8_amax(A1, 1, 16, A16, None) == ERR_ALIGN
+    assert L.fp8_amax(A16, 1, 16, A16 + 2, None) == ERR_ALIGN
+    assert L.fp8_scale_from_amax(A16, 2, A16, None) == ERR_FORMAT
+    assert L.fp8_scale_from_amax(None, 0, A16, None) == ERR_NULL
+    assert L.fp8_scale_from_amax(A16, 0, None, None) == ERR_NULL
+    assert L.fp8_scale_from_amax(A16 + 1, 0, A16, None) == ERR_ALIGN
 
 
 def test_history_validation(L):

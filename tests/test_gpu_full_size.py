@@ -122,3 +122,17 @@ def test_sweep_2pow30_sampled():
     for r in rows[:64]:
         oq, _, _ = oracle.quantize_per_tensor(xh[r], oracle.E5M2, scale=float(os_))
         assert_bytes_equal(q[r], oq, f"per-tensor row {r}")
+
+
+def test_fake_quant_activations_16384x7168():
+    a = inputs.activation_outlier_channels()
+    xh = host_input(a)
+    from parity_util import oracle_dequant
+    oq, os_ = oracle_blockwise(xh, 1, 128, oracle.E4M3)
+    oy = oracle_dequant(oq, oracle.E4M3, os_, 1, 128, oracle.BF16)
+    x = to_cuda(a)
+    y = B.fp8_fake_quantize(x, (1, 128), B.E4M3)
+    assert_bytes_equal(y, oy, "fake quant 1x128")
+    del y
+    B.fp8_fake_quantize(x, (1, 128), B.E4M3, y=x)  # in place
+    assert_bytes_equal(x, oy, "fake quant 1x128 in place")

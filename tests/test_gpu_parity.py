@@ -317,3 +317,116 @@ def test_runs_on_a_side_stream():
     oq, os_ = oracle_blockwise(host_input(x.cpu()), 1, 128, oracle.E4M3)
     assert_bytes_equal(q, oq, "side-stream codes")
     assert_bytes_equal(s, fp32_bits(os_), "side-stream scales")
+
+
+# -- fake quantization (fused round trip) ---------------------------------------------
+
+def check_fake_quant(x_cpu, block, fmt, what, scale=None, in_place=False, want_scales=True):
+    br, bc = block
+    xh = host_input(x_cpu)
+    oy, os_ = oracle.fake_quantize(xh, fmt, br, bc, scale=scale)
+    x = to_cuda(x_cpu)
+    s_in = None if scale is None else torch.tensor([scale], dtype=torch.float32, device="cuda")
+    gs = None
+    if want_scales and br != 0:
+        R, C = x.shape
+        gs = Guarded((math.ceil(R / br), math.ceil(C / bc)), torch.float32)
+    if in_place:
+        y = B.fp8_fake_quantize(x, block, fmt, scale_in=s_in, y=x, scales_out=None if gs is None else gs.t)
+        assert y.data_ptr() == x.data_ptr()
+    else:
+        gy = Guarded(tuple(x.shape), x.dtype)
+        y = B.fp8_fake_quantize(x, block, fmt, scale_in=s_in, y=gy.t, scales_out=None if gs is None else gs.t)
+    torch.cuda.synchronize()
+    if not in_place:
+        gy.check()
+    assert_bytes_equal(y, oy, f"{what} fake-quant values")
+    if gs is not None:
+        gs.check()
+        assert_bytes_equal(gs.t, fp32_bits(os_), f"{what} fake-quant scales")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("block", [(1, 128), (128, 128)])
+def test_fake_quant_blockwise(fmt, dtype, block):
+    for i, (R, C) in enumerate(SHAPES):
+        x = inputs.random_matrix(R, C, seed=3000 + i, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        check_fake_quant(x, block, fmt, f"{block} {R}x{C} {dtype}", want_scales=(i % 2 == 0))
+        check_fake_quant(x, block, fmt, f"{block} {R}x{C} {dtype} in place", in_place=True)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_fake_quant_per_tensor(fmt, dtype):
+    for i, n in enumerate([1, 7, 8, 17, 4096, 4097, (1 << 20) + 3]):
+        x = inputs.random_matrix(1, n, seed=4000 + i, dtype=dtype, outlier_frac=0.001, factor=1e3).reshape(-1)
+        for scale in (1.0, 37.5, 1e-30, 3e30):
+            check_fake_quant(x, (0, 0), fmt, f"per-tensor n={n} s={scale}", scale=scale)
+        check_fake_quant(x, (0, 0), fmt, f"per-tensor n={n} in place", scale=2.5, in_place=True)
+
+
+def test_fake_quant_edge_values():
+    x = special_values().repeat(8)[:256].reshape(2, 128).contiguous()
+    for fmt in FMTS:
+        check_fake_quant(x, (1, 128), fmt, "special values 1x128")
+        check_fake_quant(x, (0, 0), fmt, "special values per tensor", scale=1.0)
+
+
+# -- amax and scale entry points (the pieces of sharded per-tensor scaling) -----------
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_amax_and_scale_entry_points(dtype):
+    for i, n in enumerate([0, 1, 9, 4097, (1 << 20) + 5]):
+        x = inputs.random_matrix(1, max(n, 1), seed=5000 + i, dtype=dtype, outlier_frac=0.01, factor=1e3).reshape(-1)[:n]
+        a = B.fp8_amax(to_cuda(x))
+        oa = oracle.amax(host_input(x)) if n else np.float32(0)
+        for fmt in FMTS:
+            s = B.fp8_scale_from_amax(a, fmt)
+            torch.cuda.synchronize()
+            assert_bytes_equal(a, fp32_bits([oa]), f"amax n={n}")
+            assert_bytes_equal(s, fp32_bits([oracle.scale_from_amax(oa, fmt)]), f"scale n={n}")
+
+
+def test_sharded_per_tensor_single_rank_matches_unsharded():
+    from fine_grained_block_b200 import sharded
+    x = inputs.random_matrix(512, 1024, seed=91, dtype=torch.bfloat16, outlier_frac=0.001, factor=1e3)
+    q, s, a = sharded.quantize_per_tensor_sharded(to_cuda(x), B.E5M2)
+    oq, os_, oa = oracle_per_tensor(host_input(x), oracle.E5M2)
+    torch.cuda.synchronize()
+    assert_bytes_equal(q, oq, "sharded codes")
+    assert_bytes_equal(s, fp32_bits([os_]), "sharded scale")
+    assert_bytes_equal(a, fp32_bits([oa]), "sharded amax")
+
+
+# -- one-pass per-tensor current scaling --------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_fused_per_tensor_matches_two_pass_and_oracle(fmt, dtype):
+    ws = B.fused_workspace()
+    for i, n in enumerate([1, 7, 8, 9, 1000, 4097, 1 << 16, (1 << 20) + 3, 1 << 22, 3 << 22, 1 << 24]):
+        x_cpu = inputs.random_matrix(1, n, seed=6000 + i, dtype=dtype, outlier_frac=0.001, factor=1e3).reshape(-1)
+        x = to_cuda(x_cpu)
+        for rep in range(2):  # the workspace must come back clean for the next call
+            gq = Guarded((n,), torch.uint8)
+            q, s, a = B.fp8_quantize_per_tensor_fused(x, fmt, workspace=ws, q=gq.t)
+            torch.cuda.synchronize()
+            gq.check()
+            oq, os_, oa = oracle_per_tensor(host_input(x_cpu), fmt)
+            assert_bytes_equal(a, fp32_bits([oa]), f"fused amax n={n}")
+            assert_bytes_equal(s, fp32_bits([os_]), f"fused scale n={n}")
+            assert_bytes_equal(q, oq, f"fused codes n={n}")
+            # arrivals and amax are back to zero (the generation counter may have moved)
+            assert ws[0].item() == 0 and ws[2].item() == 0
+    assert B.fp8_device_status() == 0
+
+
+def test_fused_per_tensor_outlier_tensors():
+    ws = B.fused_workspace()
+    for factor, a_cpu in inputs.relerr_outlier_tensors():
+        q, s, a = B.fp8_quantize_per_tensor_fused(to_cuda(a_cpu), B.E4M3, workspace=ws)
+        oq, os_, oa = oracle.quantize_per_tensor(a_cpu.numpy(), oracle.E4M3)
+        torch.cuda.synchronize()
+        assert_bytes_equal(q, oq, f"fused x{factor}")
+        assert_bytes_equal(s, fp32_bits([os_]), f"fused scale x{factor}")

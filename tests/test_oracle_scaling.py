@@ -280,3 +280,26 @@ def test_product_rounded_to_fp32_before_cast():
         if found >= 60:
             break
     assert found >= 20 and differs >= 5
+
+
+# -- fake quantization (quantize -> dequantize round trip) -------------------------
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_fake_quantize_vs_torch_handbook_quant(fmt, dtype):
+    """The handbook's quant(): scale, clamp, cast to FP8, cast back and undo the scale, in x's dtype."""
+    MAX = oracle.MAX[fmt]
+    for br, bc in ((1, 128), (128, 128)):
+        x = inputs.random_matrix(256, 384, seed=71, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        y, s = oracle.fake_quantize(as_oracle_input(x), fmt, br, bc)
+        xf = x.float()
+        b = xf.reshape(256 // br, br, 3, 128)
+        st = torch.tensor(MAX) / b.abs().amax(dim=(1, 3), keepdim=True).clamp(min=1e-12)
+        ref = ((b * st).clamp(-MAX, MAX).to(TORCH_FP8[fmt]).to(torch.float32) / st).reshape(256, 384).to(dtype)
+        assert np.array_equal(s, st.reshape(256 // br, 3).numpy())
+        assert np.array_equal(y, as_oracle_input(ref))
+    x = inputs.random_matrix(1, 1000, seed=72, dtype=dtype).reshape(-1)
+    y, _ = oracle.fake_quantize(as_oracle_input(x), fmt, 0, 0, scale=123.0)
+    s = torch.tensor(123.0)
+    ref = ((x.float() * s).clamp(-MAX, MAX).to(TORCH_FP8[fmt]).to(torch.float32) / s).to(dtype)
+    assert np.array_equal(y, as_oracle_input(ref))
