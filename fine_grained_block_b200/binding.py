@@ -35,6 +35,7 @@ SIGNATURES = {
     "fp8_dequantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _c_int, _vp]),
     "fp8_amax_history_update": (_c_int, [_vp, _vp, _c_int, _vp, _c_int, _vp, _vp]),
     "fp8_quantize_per_tensor_fused": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _vp, _vp]),
+    "fp8_quantize_per_tensor_fused_noalloc": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _vp]),
     "fp8_amax": (_c_int, [_vp, _c_int, _i64, _vp, _vp]),
     "fp8_scale_from_amax": (_c_int, [_vp, _c_int, _vp, _vp]),
     "fp8_fake_quantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]),

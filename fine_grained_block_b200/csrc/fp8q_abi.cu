@@ -100,6 +100,20 @@ int fp8_quantize_per_tensor_fused(const void* x, int dtype, int64_t n, int fmt, 
     return fp8_quantize_per_tensor(x, dtype, n, fmt, nullptr, q, scale_out, amax_out, stream);
 }
 
+int fp8_quantize_per_tensor_fused_noalloc(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
+                                          float* amax_out, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (scale_out == nullptr || amax_out == nullptr) return FP8_ERR_NULL;
+    if (n > 0 && (x == nullptr || q == nullptr)) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale_out, 4) || !aligned(amax_out, 4)) return FP8_ERR_ALIGN;
+    if (n == 0) return fp8_quantize_per_tensor(x, dtype, n, fmt, nullptr, q, scale_out, amax_out, stream);
+    if (!fp8q::tensor_fused_fits(x, dtype, n, fmt)) return FP8_ERR_TOO_LARGE;
+    return status_of(fp8q::launch_tensor_fused_noalloc(x, dtype, n, fmt, q, scale_out, amax_out,
+                                                       static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_amax(const void* x, int dtype, int64_t n, float* amax_out, void* stream) {
     if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
     if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
@@ -215,6 +229,7 @@ const char* fp8_status_string(int status) {
         case FP8_ERR_DTYPE: return "dtype is not FP8_F32 or FP8_BF16";
         case FP8_ERR_CUDA: return "a CUDA call or kernel launch failed";
         case FP8_ERR_ARG: return "invalid argument";
+        case FP8_ERR_TOO_LARGE: return "tensor too large for the one-pass kernel of the no-allocation entry point";
         default: return "unknown status";
     }
 }

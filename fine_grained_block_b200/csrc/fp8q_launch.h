@@ -38,6 +38,15 @@ unsigned int* device_status_word();
 cudaError_t launch_tensor_fused(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
                                 float* amax_out, void* workspace, cudaStream_t stream, bool* launched);
 
+// Whether x (n elements) is small enough for the one-pass kernel.
+bool tensor_fused_fits(const void* x, int dtype, int64_t n, int fmt);
+
+// The one-pass kernel with its workspace in a fixed array of this module's
+// device memory instead of caller memory (see quant_tensor_fused.cu).  The
+// caller has checked tensor_fused_fits first.
+cudaError_t launch_tensor_fused_noalloc(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
+                                        float* amax_out, cudaStream_t stream);
+
 // Copy the device status word to out[0] (device memory), clearing it if asked.
 cudaError_t launch_device_status(unsigned int* out, int clear, cudaStream_t stream);
 

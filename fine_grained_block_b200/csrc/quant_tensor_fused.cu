@@ -20,6 +20,7 @@
 // share a workspace must not overlap on the device.
 
 #include <algorithm>
+#include <atomic>
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
@@ -186,7 +187,64 @@ cudaError_t fused_width(const void* x, int64_t n, uint8_t* q, float* scale_out, 
     return fused_typed<T, FMT, 16>(x, n, q, scale_out, amax_out, ws, st, launched);
 }
 
+template <typename T, int FMT, int BYTES>
+bool fused_fits_typed(int64_t n) {
+    using V = LaneVec<T, BYTES>;
+    const int64_t per_cta = static_cast<int64_t>(kThreads) * kLoads;
+    const int64_t grid = std::max<int64_t>(1, (n / V::kElems + per_cta - 1) / per_cta);
+    return grid <= resident_ctas(k_tensor_fused<T, FMT, BYTES>);
+}
+
+// ---------------------------------------------------------------------------
+// Scratch for callers that cannot allocate device memory: a fixed array in
+// this module's device memory, which every GPU that loads the library keeps
+// until the process exits.  Its maximum size is kNoAllocScratchBytes; the
+// one-pass kernel uses the first sizeof(Workspace) bytes of it as its
+// workspace.  Host code cannot use the array's name as a device address, so
+// the address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = 256;
+static_assert(sizeof(Workspace) <= kNoAllocScratchBytes, "the workspace must fit the fixed scratch");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch for the current device (looked up on
+// the first call on that device), or nullptr if the lookup failed.
+void* noalloc_scratch_address() {
+    static std::atomic<void*> cache[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+    void* p = cache[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        cache[dev].store(p, std::memory_order_release);
+    }
+    return p;
+}
+
 }  // namespace
+
+bool tensor_fused_fits(const void* x, int dtype, int64_t n, int fmt) {
+    const bool w32 = aligned32(x);
+    if (dtype == 1) {
+        if (fmt == kE4M3) return w32 ? fused_fits_typed<uint16_t, kE4M3, 32>(n) : fused_fits_typed<uint16_t, kE4M3, 16>(n);
+        return w32 ? fused_fits_typed<uint16_t, kE5M2, 32>(n) : fused_fits_typed<uint16_t, kE5M2, 16>(n);
+    }
+    if (fmt == kE4M3) return w32 ? fused_fits_typed<float, kE4M3, 32>(n) : fused_fits_typed<float, kE4M3, 16>(n);
+    return w32 ? fused_fits_typed<float, kE5M2, 32>(n) : fused_fits_typed<float, kE5M2, 16>(n);
+}
+
+cudaError_t launch_tensor_fused_noalloc(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
+                                        float* amax_out, cudaStream_t st) {
+    void* ws = noalloc_scratch_address();
+    if (ws == nullptr) return cudaErrorInvalidSymbol;
+    // The array keeps whatever the last call left; the workspace must start at zero.
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(Workspace), st);
+    if (e != cudaSuccess) return e;
+    bool launched = false;
+    e = launch_tensor_fused(x, dtype, n, fmt, q, scale_out, amax_out, ws, st, &launched);
+    if (e == cudaSuccess && !launched) return cudaErrorInvalidValue;  // the caller checks the size first
+    return e;
+}
 
 cudaError_t launch_tensor_fused(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
                                 float* amax_out, void* workspace, cudaStream_t st, bool* launched) {

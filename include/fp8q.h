@@ -61,7 +61,8 @@ enum fp8_status {
     FP8_ERR_FORMAT = -4,        /* fmt is not an fp8_format */
     FP8_ERR_DTYPE = -5,         /* dtype is not an fp8_dtype */
     FP8_ERR_CUDA = -6,          /* a CUDA call or launch failed */
-    FP8_ERR_ARG = -7            /* any other invalid argument (e.g. window <= 0) */
+    FP8_ERR_ARG = -7,           /* any other invalid argument (e.g. window <= 0) */
+    FP8_ERR_TOO_LARGE = -8      /* larger than fp8_quantize_per_tensor_fused_noalloc can take */
 };
 
 /*
@@ -111,6 +112,39 @@ int fp8_quantize_per_tensor(const void *x, int dtype, int64_t n, int fmt,
 int fp8_quantize_per_tensor_fused(const void *x, int dtype, int64_t n, int fmt,
                                   uint8_t *q, float *scale_out, float *amax_out,
                                   void *workspace, void *stream);
+
+/*
+ * fp8_quantize_per_tensor_fused without a workspace argument, for callers that
+ * cannot allocate device memory: code that runs where cudaMalloc is not
+ * allowed or not safe (it synchronizes the device and can fail under memory
+ * pressure), such as a plugin called by an inference runtime that offers no
+ * workspace, or a C caller whose device memory is all owned by another
+ * framework's allocator.  (The pages have no counterpart: this is an
+ * interface convenience, not part of the method.)
+ *
+ * Same arguments and results as fp8_quantize_per_tensor_fused minus the
+ * workspace.  Instead, the workspace lives in a fixed 256-byte array in the
+ * library's own device memory (16 bytes of it are used), which every GPU that
+ * loads the library keeps until the process exits.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - The first call on each device looks up that array's device address
+ *     (cudaGetSymbolAddress) with the device current; make that first call
+ *     before any stream capture.
+ *   - Every call clears the workspace (cudaMemsetAsync) before its launch.
+ *   - All calls share the one array: calls that can overlap on the GPU
+ *     (different streams without ordering between them) race and give wrong
+ *     results.  Order such calls, or use fp8_quantize_per_tensor_fused with
+ *     one workspace per stream.
+ *   - Limit: only tensors that fit the one-pass kernel (fp8_quantize_per_
+ *     tensor_fused's on-chip capacity, about 8 MiB of bf16 on a B200) are
+ *     accepted; larger ones return FP8_ERR_TOO_LARGE with nothing enqueued.
+ *     n == 0 writes amax 0 and its scale, as the other per-tensor calls do.
+ * Errors: those of fp8_quantize_per_tensor_fused (without the workspace
+ * ones), FP8_ERR_TOO_LARGE.
+ */
+int fp8_quantize_per_tensor_fused_noalloc(const void *x, int dtype, int64_t n, int fmt,
+                                          uint8_t *q, float *scale_out, float *amax_out,
+                                          void *stream);
 
 /*
  * amax of a tensor: *amax_out = max |x| (0 for n == 0).  [FP8-native] s4.1.

@@ -33,6 +33,7 @@ def test_header_declares_the_boundary():
                                            "fp8_amax_history_update", "fp8_status_string", "fp8_device_status",
                                            "fp8_fake_quantize", "fp8_amax", "fp8_scale_from_amax",
                                            "fp8_quantize_per_tensor_fused",
+                                           "fp8_quantize_per_tensor_fused_noalloc",
                                            "fp8_selftest_wait_timeout"])
 
 
