@@ -26,6 +26,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "launch_util.h"
 #include "dequant_math.cuh"
 #include "lane_vec.cuh"
 
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(kThreads)
 k_dequant_flat(const typename DOut<OUT, OB>::In* __restrict__ q, int64_t ngroups,
                const uint8_t* __restrict__ q_tail, int tail_n, const float* __restrict__ scales,
                typename DOut<OUT, OB>::Out* __restrict__ y, void* __restrict__ y_tail) {
+    pdl_enter();
     using D = DOut<OUT, OB>;
     constexpr int kGroupsPerBlock = 128 / D::kCodes;
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x;
@@ -159,6 +161,7 @@ template <int FMT, int OUT, int OB>
 __global__ void __launch_bounds__(kThreads)
 k_dequant_128x128(const typename DOut<OUT, OB>::In* __restrict__ q, const float* __restrict__ scales,
                   typename DOut<OUT, OB>::Out* __restrict__ y, int64_t rows, int64_t cols) {
+    pdl_enter();
     using D = DOut<OUT, OB>;
     constexpr int kGroupsPerRow = 128 / D::kCodes;
     constexpr int kRowsPerPass = kThreads / kGroupsPerRow;
@@ -196,6 +199,7 @@ template <int FMT, int OUT>
 __global__ void __launch_bounds__(kThreads)
 k_dequant_general(const uint8_t* __restrict__ q, int64_t rows, int64_t cols, int mode,
                   const float* __restrict__ scales, void* __restrict__ y) {
+    pdl_enter();
     const int64_t n = rows * cols;
     const int64_t nbc = (cols + 127) / 128;
     const int br = (mode == 2) ? 128 : 1;
@@ -217,8 +221,10 @@ cudaError_t dequant_fast(const uint8_t* q, int64_t rows, int64_t cols, int mode,
     if (mode == 2) {
         const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
         if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-        k_dequant_128x128<FMT, OUT, OB><<<static_cast<unsigned>(tiles), kThreads, 0, st>>>(
-            reinterpret_cast<const typename D::In*>(q), scales, static_cast<typename D::Out*>(y), rows, cols);
+        {
+        const cudaError_t e_ = launch_kernel(k_dequant_128x128<FMT, OUT, OB>, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), 0, st, reinterpret_cast<const typename D::In*>(q), scales, static_cast<typename D::Out*>(y), rows, cols);
+        if (e_ != cudaSuccess) return e_;
+    }
         return cudaGetLastError();
     }
     const int64_t ngroups = n / D::kCodes;
@@ -227,14 +233,13 @@ cudaError_t dequant_fast(const uint8_t* q, int64_t rows, int64_t cols, int mode,
     const int64_t per_cta = static_cast<int64_t>(kThreads) * kUnroll;
     const int64_t grid = std::max<int64_t>(1, (ngroups + per_cta - 1) / per_cta);
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    auto launch = [&](auto kern) {
-        kern<<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
-            reinterpret_cast<const typename D::In*>(q), ngroups, q + ngroups * D::kCodes, tail_n, scales,
-            static_cast<typename D::Out*>(y), static_cast<char*>(y) + ngroups * D::kCodes * osz);
+    auto launch = [&](auto kern) -> cudaError_t {
+        return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st,
+                             reinterpret_cast<const typename D::In*>(q), ngroups, q + ngroups * D::kCodes, tail_n,
+                             scales, static_cast<typename D::Out*>(y), static_cast<char*>(y) + ngroups * D::kCodes * osz);
     };
-    if (mode == 0) launch(k_dequant_flat<FMT, OUT, OB, 0>);
-    else launch(k_dequant_flat<FMT, OUT, OB, 1>);
-    return cudaGetLastError();
+    if (mode == 0) return launch(k_dequant_flat<FMT, OUT, OB, 0>);
+    return launch(k_dequant_flat<FMT, OUT, OB, 1>);
 }
 
 template <int FMT, int OUT>
@@ -247,7 +252,10 @@ cudaError_t dequant_typed(const uint8_t* q, int64_t rows, int64_t cols, int mode
     }
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((n + kThreads - 1) / kThreads,
                                                                 static_cast<int64_t>(device_sm_count()) * 8));
-    k_dequant_general<FMT, OUT><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(q, rows, cols, mode, scales, y);
+    {
+        const cudaError_t e_ = launch_kernel(k_dequant_general<FMT, OUT>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st, q, rows, cols, mode, scales, y);
+        if (e_ != cudaSuccess) return e_;
+    }
     return cudaGetLastError();
 }
 

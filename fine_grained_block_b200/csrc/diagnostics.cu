@@ -1,6 +1,6 @@
 // diagnostics.cu -- the library's device status word.
 //
-// Kernels that wait (on a tile copy, or at a grid-wide barrier) never wait
+// Kernels that wait (at the one-pass kernel's grid-wide barrier) never wait
 // forever: a wait that runs out sets a bit here and the kernel returns.  The
 // word lives in this file; other kernels receive its device address as an
 // argument (device_status_word()), so no relocatable device code is needed.
@@ -9,7 +9,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
-#include "fp8q_tma.cuh"
+#include "fp8q_wait.cuh"
 
 namespace fp8q {
 namespace {
@@ -20,12 +20,12 @@ __global__ void k_device_status(unsigned int* out, int clear) {
     out[0] = clear ? atomicExch(&g_device_status, 0u) : atomicOr(&g_device_status, 0u);
 }
 
-// A wait that nothing will ever complete, to exercise the timeout path.
+// A word that nothing ever changes: the same bounded wait the one-pass kernel
+// uses at its grid barrier must give up on it.
+__device__ unsigned int g_never_changes = 0u;
+
 __global__ void k_selftest_wait_timeout(uint64_t limit_ns) {
-    __shared__ uint64_t bar;
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-    if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(&g_device_status, kStatusWaitTimeout);
+    if (!wait_for_change(&g_never_changes, 0u, limit_ns)) atomicOr(&g_device_status, kStatusWaitTimeout);
 }
 
 }  // namespace

@@ -15,6 +15,7 @@
 #include "dequant_math.cuh"
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "launch_util.h"
 #include "lane_vec.cuh"
 
 namespace fp8q {
@@ -106,6 +107,7 @@ struct RoundTrip<float, BYTES, FMT> {
 template <typename T, int FMT, int BYTES>
 __global__ void __launch_bounds__(kThreads)
 k_fake_quant_1x128(const Words<BYTES / 4>* x, Words<BYTES / 4>* y, float* __restrict__ scales, int64_t nblocks) {
+    pdl_enter();
     using V = LaneVec<T, BYTES>;
     using R = RoundTrip<T, BYTES, FMT>;
     constexpr int kLanesPerBlock = 128 / V::kElems;
@@ -138,6 +140,7 @@ template <typename T, int FMT, int BYTES>
 __global__ void __launch_bounds__(kThreads)
 k_fake_quant_128x128(const Words<BYTES / 4>* x, Words<BYTES / 4>* y, float* __restrict__ scales, int64_t rows,
                      int64_t cols) {
+    pdl_enter();
     using V = LaneVec<T, BYTES>;
     using R = RoundTrip<T, BYTES, FMT>;
     constexpr int kVecPerRow = 128 / V::kElems;
@@ -207,6 +210,7 @@ template <typename T, int FMT, int BYTES>
 __global__ void __launch_bounds__(kThreads)
 k_fake_quant_tensor(const Words<BYTES / 4>* x, Words<BYTES / 4>* y, int64_t nvec, const T* x_tail, T* y_tail,
                     int tail_n, const float* scale_in) {
+    pdl_enter();
     using R = RoundTrip<T, BYTES, FMT>;
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kLoads + threadIdx.x;
     Words<BYTES / 4> v[kLoads];
@@ -233,6 +237,7 @@ template <typename T, int FMT>
 __global__ void __launch_bounds__(kGeneralThreads)
 k_fake_quant_general(const T* x, T* y, float* __restrict__ scales, int64_t rows, int64_t cols, int br,
                      int64_t nblocks) {
+    pdl_enter();
     __shared__ float warp_amax[kGeneralThreads / 32];
     const int64_t nbc = (cols + 127) / 128;
     for (int64_t b = blockIdx.x; b < nblocks; b += gridDim.x) {
@@ -273,9 +278,11 @@ cudaError_t launch_fq_fast(const void* x, void* y, int64_t rows, int64_t cols, i
         const int64_t per_cta = static_cast<int64_t>(kThreads) * kLoads;
         const int64_t grid = std::max<int64_t>(1, (nvec + per_cta - 1) / per_cta);
         if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-        k_fake_quant_tensor<T, FMT, BYTES><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
-            static_cast<const W*>(x), static_cast<W*>(y), nvec, static_cast<const T*>(x) + nvec * V::kElems,
+        {
+        const cudaError_t e_ = launch_kernel(k_fake_quant_tensor<T, FMT, BYTES>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st, static_cast<const W*>(x), static_cast<W*>(y), nvec, static_cast<const T*>(x) + nvec * V::kElems,
             static_cast<T*>(y) + nvec * V::kElems, tail_n, scale_in);
+        if (e_ != cudaSuccess) return e_;
+    }
     } else if (br == 1) {
         const int64_t nblocks = n / 128;
         constexpr int kBlocksPerLoad = 32 / (128 / V::kElems);
@@ -283,13 +290,17 @@ cudaError_t launch_fq_fast(const void* x, void* y, int64_t rows, int64_t cols, i
         const int64_t per_cta = static_cast<int64_t>(kThreads / 32) * kLoads;
         const int64_t grid = (nloads + per_cta - 1) / per_cta;
         if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-        k_fake_quant_1x128<T, FMT, BYTES><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
-            static_cast<const W*>(x), static_cast<W*>(y), scales, nblocks);
+        {
+        const cudaError_t e_ = launch_kernel(k_fake_quant_1x128<T, FMT, BYTES>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st, static_cast<const W*>(x), static_cast<W*>(y), scales, nblocks);
+        if (e_ != cudaSuccess) return e_;
+    }
     } else {
         const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
         if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-        k_fake_quant_128x128<T, FMT, BYTES><<<static_cast<unsigned>(tiles), kThreads, 0, st>>>(
-            static_cast<const W*>(x), static_cast<W*>(y), scales, rows, cols);
+        {
+        const cudaError_t e_ = launch_kernel(k_fake_quant_128x128<T, FMT, BYTES>, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), 0, st, static_cast<const W*>(x), static_cast<W*>(y), scales, rows, cols);
+        if (e_ != cudaSuccess) return e_;
+    }
     }
     return cudaGetLastError();
 }
@@ -304,8 +315,10 @@ cudaError_t launch_fq_typed(const void* x, void* y, int64_t rows, int64_t cols, 
     }
     const int64_t nblocks = ((rows + br - 1) / br) * ((cols + 127) / 128);
     const int64_t grid = std::min<int64_t>(nblocks, static_cast<int64_t>(device_sm_count()) * 16);
-    k_fake_quant_general<T, FMT><<<static_cast<unsigned>(grid), kGeneralThreads, 0, st>>>(
-        static_cast<const T*>(x), static_cast<T*>(y), scales, rows, cols, br, nblocks);
+    {
+        const cudaError_t e_ = launch_kernel(k_fake_quant_general<T, FMT>, dim3(static_cast<unsigned>(grid)), dim3(kGeneralThreads), 0, st, static_cast<const T*>(x), static_cast<T*>(y), scales, rows, cols, br, nblocks);
+        if (e_ != cudaSuccess) return e_;
+    }
     return cudaGetLastError();
 }
 

@@ -13,13 +13,6 @@
 #include "fp8q.h"
 #include "fp8q_launch.h"
 
-// 128x128 bf16 blocks: TMA-staged tile pipeline (1) or register-resident tiles
-// (0).  Measured on B200 at 2^28 elements: register tiles 6446 GB/s, TMA ring
-// 5461 GB/s (the register kernel keeps 4 tiles per SM both in flight and in
-// process), so register tiles are the default.
-#ifndef FP8Q_USE_TMA_128
-#define FP8Q_USE_TMA_128 0
-#endif
 
 namespace fp8q {
 
@@ -149,8 +142,6 @@ int fp8_quantize_blockwise(const void* x, int dtype, int64_t rows, int64_t cols,
         e = fp8q::launch_quant_block_general(x, dtype, rows, cols, block_rows, block_cols, fmt, q, scales, st);
     } else if (block_rows == 1) {
         e = fp8q::launch_quant_1x128(x, dtype, n / 128, fmt, q, scales, st);
-    } else if (FP8Q_USE_TMA_128 && fp8q::tma_128x128_supported(dtype, rows, cols)) {
-        e = fp8q::launch_quant_128x128_tma(x, rows, cols, fmt, q, scales, st);
     } else {
         e = fp8q::launch_quant_128x128(x, dtype, rows, cols, fmt, q, scales, st);
     }

@@ -23,12 +23,6 @@ cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fm
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                  uint8_t* q, float* scales, cudaStream_t stream);
 
-// 128x128 blocks with TMA-staged tiles (bf16, cols % 128 == 0, rows and cols
-// below 2^31, and a driver that provides the tensor-map encoder).
-bool tma_128x128_supported(int dtype, int64_t rows, int64_t cols);
-cudaError_t launch_quant_128x128_tma(const void* x, int64_t rows, int64_t cols, int fmt, uint8_t* q,
-                                     float* scales, cudaStream_t stream);
-
 // Device address of the status word of the current device (nullptr on failure).
 unsigned int* device_status_word();
 

@@ -11,6 +11,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "launch_util.h"
 
 namespace fp8q {
 namespace {
@@ -19,6 +20,7 @@ template <int FMT>
 __global__ void __launch_bounds__(32)
 k_amax_history_update(float* __restrict__ history, int32_t* __restrict__ state, int window,
                       const float* __restrict__ amax, float* __restrict__ scale) {
+    pdl_enter();
     const int lane = threadIdx.x;
     // Out-of-range state is brought into range instead of indexing outside
     // the ring: pos modulo window, count clamped to [0, window].
@@ -45,9 +47,9 @@ k_amax_history_update(float* __restrict__ history, int32_t* __restrict__ state, 
 
 cudaError_t launch_amax_history_update(float* history, int32_t* state, int window, const float* amax, int fmt,
                                        float* scale, cudaStream_t st) {
-    if (fmt == kE4M3) k_amax_history_update<kE4M3><<<1, 32, 0, st>>>(history, state, window, amax, scale);
-    else k_amax_history_update<kE5M2><<<1, 32, 0, st>>>(history, state, window, amax, scale);
-    return cudaGetLastError();
+    if (fmt == kE4M3)
+        return launch_kernel(k_amax_history_update<kE4M3>, dim3(1), dim3(32), 0, st, history, state, window, amax, scale);
+    return launch_kernel(k_amax_history_update<kE5M2>, dim3(1), dim3(32), 0, st, history, state, window, amax, scale);
 }
 
 }  // namespace fp8q

@@ -17,6 +17,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "launch_util.h"
 #include "lane_vec.cuh"
 
 namespace fp8q {
@@ -62,6 +63,7 @@ template <typename T, int BYTES>
 __global__ void __launch_bounds__(kThreads)
 k_tensor_amax(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec, const T* __restrict__ tail,
               int tail_n, float* __restrict__ amax_out) {
+    pdl_enter();
     using V = LaneVec<T, BYTES>;
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x;
     typename V::In v[kUnroll];
@@ -86,6 +88,7 @@ k_tensor_cast(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec
               int tail_n, const float* scale_in, const float* __restrict__ amax_in,
               typename LaneVec<T, BYTES>::Out* __restrict__ q, uint8_t* __restrict__ q_tail, float* scale_out,
               float* __restrict__ amax_out) {
+    pdl_enter();
     using V = LaneVec<T, BYTES>;
     const int64_t chunk = static_cast<int64_t>(gridDim.x) - 1 - blockIdx.x;
     const int64_t base = chunk * kThreads * kUnroll + threadIdx.x;
@@ -117,6 +120,7 @@ k_tensor_cast(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec
 
 template <int FMT>
 __global__ void k_scale_from_amax(const float* amax_in, float* scale_out) {
+    pdl_enter();
     *scale_out = scale_from_amax<FMT>(*amax_in);
 }
 
@@ -136,8 +140,11 @@ cudaError_t amax_typed(const void* x, int64_t n, float* amax_out, cudaStream_t s
     auto kern = k_tensor_amax<T, BYTES>;
     const int64_t grid = chunk_grid(nvec);
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    kern<<<static_cast<unsigned>(grid), kThreads, 0, st>>>(static_cast<const typename V::In*>(x), nvec, tail,
+    {
+        const cudaError_t e_ = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st, static_cast<const typename V::In*>(x), nvec, tail,
                                                            tail_n, amax_out);
+        if (e_ != cudaSuccess) return e_;
+    }
     return cudaGetLastError();
 }
 
@@ -151,9 +158,11 @@ cudaError_t cast_typed(const void* x, int64_t n, const float* scale_in, const fl
     auto kern = k_tensor_cast<T, FMT, BYTES, DELAYED, WITH_AMAX>;
     const int64_t grid = chunk_grid(nvec);
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    kern<<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
-        static_cast<const typename V::In*>(x), nvec, tail, tail_n, scale_in, amax_in,
+    {
+        const cudaError_t e_ = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st, static_cast<const typename V::In*>(x), nvec, tail, tail_n, scale_in, amax_in,
         reinterpret_cast<typename V::Out*>(q), q + nvec * V::kElems, scale_out, amax_out);
+        if (e_ != cudaSuccess) return e_;
+    }
     return cudaGetLastError();
 }
 
@@ -183,9 +192,8 @@ cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_
 }
 
 cudaError_t launch_scale_from_amax(const float* amax_in, int fmt, float* scale_out, cudaStream_t st) {
-    if (fmt == kE4M3) k_scale_from_amax<kE4M3><<<1, 1, 0, st>>>(amax_in, scale_out);
-    else k_scale_from_amax<kE5M2><<<1, 1, 0, st>>>(amax_in, scale_out);
-    return cudaGetLastError();
+    if (fmt == kE4M3) return launch_kernel(k_scale_from_amax<kE4M3>, dim3(1), dim3(1), 0, st, amax_in, scale_out);
+    return launch_kernel(k_scale_from_amax<kE5M2>, dim3(1), dim3(1), 0, st, amax_in, scale_out);
 }
 
 cudaError_t launch_tensor_cast(const void* x, int dtype, int64_t n, int fmt, const float* scale_in,

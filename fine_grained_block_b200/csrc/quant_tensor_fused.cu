@@ -24,7 +24,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
-#include "fp8q_tma.cuh"
+#include "fp8q_wait.cuh"
 #include "lane_vec.cuh"
 
 namespace fp8q {
@@ -113,13 +113,7 @@ k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nve
             __threadfence();
             atomicAdd(&ws->generation, 1u);  // releases the waiting CTAs
         } else {
-            const uint64_t start = global_timer_ns();
-            while (ld_volatile(&ws->generation) == gen) {
-                if (global_timer_ns() - start > kWaitLimitNs) {
-                    ok = false;
-                    break;
-                }
-            }
+            ok = wait_for_change(&ws->generation, gen, kWaitLimitNs);
             __threadfence();
             amax = ld_volatile(amax_out);
         }

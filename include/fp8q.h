@@ -262,10 +262,10 @@ int fp8_amax_history_update(float *history, int32_t *state, int window,
 const char *fp8_status_string(int status);
 
 /* ---- Diagnostics (no counterpart on the pages) ---------------------------
- * Kernels that wait on a tile copy (the TMA pipelines) never wait forever:
- * each wait gives up after about a second, the kernel leaves its loop, and
- * it records the event in a device status word.  Results of that launch are
- * then incomplete.
+ * Kernels that wait (the grid-wide barrier of the one-pass per-tensor kernel)
+ * never wait forever: each wait gives up after about a second, the kernel
+ * returns, and it records the event in a device status word.  Results of
+ * that launch are then incomplete.
  *
  * Device status bits: */
 #define FP8_DEVICE_STATUS_WAIT_TIMEOUT 0x1u
@@ -280,8 +280,9 @@ const char *fp8_status_string(int status);
 int fp8_device_status(uint32_t *status, int clear, void *stream);
 
 /*
- * Self-test of the bounded wait: launch one thread that waits on a barrier
- * nothing will complete; after timeout_us microseconds it gives up and sets
+ * Self-test of the bounded wait: launch one thread that runs the same wait as
+ * the one-pass kernel's barrier on a word that nothing changes; after
+ * timeout_us microseconds it gives up and sets
  * FP8_DEVICE_STATUS_WAIT_TIMEOUT.  The device stays usable.
  * Errors: FP8_ERR_ARG (timeout_us == 0 or > 10 s), FP8_ERR_CUDA.
  */

@@ -1,9 +1,9 @@
 """Bounded waits and the device status word (no GPU fault involved).
 
-The TMA pipelines never wait forever: a wait that runs out sets a bit in the
-library's device status word and the kernel returns.  The self-test kernel
-waits on a barrier that nothing completes, so its wait must run out; the real
-pipelines must never set the bit."""
+The one-pass per-tensor kernel's grid barrier never waits forever: a wait that
+runs out sets a bit in the library's device status word and the kernel
+returns.  The self-test kernel runs the same wait on a word that nothing
+changes, so its wait must run out; real calls must never set the bit."""
 import pytest
 import torch
 
@@ -26,11 +26,13 @@ def test_selftest_wait_times_out_and_is_reported():
     assert bool((q == 0x7E).all()) and bool((s == 448.0).all())
 
 
-def test_tile_pipeline_never_times_out():
+def test_one_pass_barrier_never_times_out():
     B.fp8_device_status(clear=True)
-    for rows, cols in ((128, 128), (4096, 4096), (130, 384), (1, 128), (16384, 7168)):
-        x = inputs.random_matrix(rows, cols, seed=rows + cols, device="cuda")
+    ws = B.fused_workspace()
+    for n in (1, 4096, 1 << 20, 3 << 21):
+        x = inputs.random_matrix(1, n, seed=n, device="cuda").reshape(-1)
         for fmt in (B.E4M3, B.E5M2):
-            B.fp8_quantize_blockwise(x, (128, 128), fmt)
+            for _ in range(3):
+                B.fp8_quantize_per_tensor_fused(x, fmt, workspace=ws)
     torch.cuda.synchronize()
     assert B.fp8_device_status() == 0
