@@ -34,6 +34,8 @@ SIGNATURES = {
     "fp8_quantize_blockwise": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "fp8_dequantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _c_int, _vp]),
     "fp8_amax_history_update": (_c_int, [_vp, _vp, _c_int, _vp, _c_int, _vp, _vp]),
+    "fp8_amax_history_update_ex": (_c_int, [_vp, _vp, _c_int, _vp, _c_int, _vp, _c_int, ctypes.c_float,
+                                            ctypes.c_float, _vp]),
     "fp8_quantize_per_tensor_fused": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _vp, _vp]),
     "fp8_quantize_per_tensor_fused_noalloc": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _vp]),
     "fp8_amax": (_c_int, [_vp, _c_int, _i64, _vp, _vp]),
@@ -44,6 +46,7 @@ SIGNATURES = {
     "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
 }
 DEVICE_STATUS_WAIT_TIMEOUT = 0x1
+AMAX_WINDOW_MAX, AMAX_EMA = 0, 1
 FUSED_WORKSPACE_BYTES = 16
 
 
@@ -250,13 +253,26 @@ def fp8_selftest_wait_timeout(timeout_us: int = 1000, stream=None):
     _check("fp8_selftest_wait_timeout", load_library().fp8_selftest_wait_timeout(int(timeout_us), _stream(stream)))
 
 
+def fp8_amax_history_update_ex(history: torch.Tensor, state: torch.Tensor, amax: torch.Tensor, scale: torch.Tensor,
+                               fmt: int = E4M3, algo: int = AMAX_WINDOW_MAX, alpha: float = 1.0,
+                               margin: float = 1.0, stream=None):
+    """Delayed-scaling update with a margin and window-max or EMA smoothing (PyTorch-FP8 page s4.3)."""
+    _need_cuda(history, state, amax, scale)
+    st = load_library().fp8_amax_history_update_ex(_ptr(history), _ptr(state), history.numel(), _ptr(amax), fmt,
+                                                   _ptr(scale), algo, float(alpha), float(margin), _stream(stream))
+    _check("fp8_amax_history_update_ex", st)
+    return scale
+
+
 class DelayedScaler:
     """Device-resident delayed-scaling state (history ring, {pos, count}, scale), after the
     PyTorch-FP8 page's DelayedScaler (s4.2).  step(x) quantizes x with the current scale, then
     pushes amax(x) into the history -- all on the device, no host round trip."""
 
-    def __init__(self, window: int = 16, fmt: int = E5M2, device="cuda"):
+    def __init__(self, window: int = 16, fmt: int = E5M2, device="cuda", algo: int = AMAX_WINDOW_MAX,
+                 alpha: float = 1.0, margin: float = 1.0):
         self.fmt = fmt
+        self.algo, self.alpha, self.margin = algo, alpha, margin
         self.history = torch.zeros(window, dtype=torch.float32, device=device)
         self.state = torch.zeros(2, dtype=torch.int32, device=device)
         self.scale = torch.ones(1, dtype=torch.float32, device=device)
@@ -266,5 +282,9 @@ class DelayedScaler:
     def step(self, x: torch.Tensor, q: torch.Tensor | None = None, stream=None):
         q, s, _ = fp8_quantize_per_tensor(x, self.fmt, scale_in=self.scale, q=q, scale_out=self.scale_used,
                                           amax_out=self.amax, stream=stream)
-        fp8_amax_history_update(self.history, self.state, self.amax, self.scale, self.fmt, stream=stream)
+        if self.algo == AMAX_WINDOW_MAX and self.margin == 1.0:
+            fp8_amax_history_update(self.history, self.state, self.amax, self.scale, self.fmt, stream=stream)
+        else:
+            fp8_amax_history_update_ex(self.history, self.state, self.amax, self.scale, self.fmt, self.algo,
+                                       self.alpha, self.margin, stream=stream)
         return q, self.scale_used

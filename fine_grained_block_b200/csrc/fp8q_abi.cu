@@ -198,6 +198,18 @@ int fp8_amax_history_update(float* history, int32_t* state, int window, const fl
                                                       static_cast<cudaStream_t>(stream)));
 }
 
+int fp8_amax_history_update_ex(float* history, int32_t* state, int window, const float* amax, int fmt, float* scale,
+                               int algo, float alpha, float margin, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (window <= 0 || window > 65536) return FP8_ERR_ARG;
+    if (algo != FP8_AMAX_WINDOW_MAX && algo != FP8_AMAX_EMA) return FP8_ERR_ARG;
+    if (!(alpha >= 0.0f && alpha <= 1.0f) || !(margin > 0.0f)) return FP8_ERR_ARG;
+    if (history == nullptr || state == nullptr || amax == nullptr || scale == nullptr) return FP8_ERR_NULL;
+    if (!aligned(history, 4) || !aligned(state, 4) || !aligned(amax, 4) || !aligned(scale, 4)) return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_amax_history_update_ex(history, state, window, amax, fmt, scale, algo, alpha, margin,
+                                                         static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_device_status(uint32_t* status, int clear, void* stream) {
     if (status == nullptr) return FP8_ERR_NULL;
     if (!aligned(status, 4)) return FP8_ERR_ALIGN;

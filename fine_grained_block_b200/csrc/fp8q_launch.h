@@ -23,6 +23,10 @@ cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fm
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                  uint8_t* q, float* scales, cudaStream_t stream);
 
+// Delayed scaling with a margin and a choice of window max (algo 0) or EMA (algo 1).
+cudaError_t launch_amax_history_update_ex(float* history, int32_t* state, int window, const float* amax, int fmt,
+                                          float* scale, int algo, float alpha, float margin, cudaStream_t stream);
+
 // Device address of the status word of the current device (nullptr on failure).
 unsigned int* device_status_word();
 

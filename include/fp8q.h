@@ -258,6 +258,33 @@ int fp8_amax_history_update(float *history, int32_t *state, int window,
                             const float *amax, int fmt, float *scale,
                             void *stream);
 
+/*
+ * Delayed scaling with the refinements of [FP8-native] s4.3 (keep a margin,
+ * smooth the amax) -- the same state and call pattern as
+ * fp8_amax_history_update.
+ *
+ *   algo       FP8_AMAX_WINDOW_MAX: the window of fp8_amax_history_update;
+ *              once full, scale = MAX / RN(max(max(window), eps) * margin).
+ *              FP8_AMAX_EMA: history[0] holds a moving average m of amax
+ *              (s4.2 names this smoothing): the first update sets m = amax,
+ *              later ones m = RN(RN(alpha*amax) + RN(RN(1-alpha) * m)), all
+ *              in fp32.  state[1] counts updates up to `window` (a warm-up);
+ *              from then on every update sets
+ *              scale = MAX / RN(max(m, eps) * margin).  state[0] is unused and
+ *              history needs only 1 element (window is still the warm-up).
+ *   alpha      EMA weight of the new amax, in [0, 1] (ignored by WINDOW_MAX)
+ *   margin     > 0; 1.0 keeps the plain scale (the page's example is 1.1)
+ * With algo = FP8_AMAX_WINDOW_MAX and margin = 1 the results equal
+ * fp8_amax_history_update's.  Initialise history and state to zero and
+ * *scale to 1.0f as there.
+ * Errors: those of fp8_amax_history_update; FP8_ERR_ARG for an unknown
+ * algo, alpha outside [0, 1] or margin <= 0 (NaN included).
+ */
+enum fp8_amax_algo { FP8_AMAX_WINDOW_MAX = 0, FP8_AMAX_EMA = 1 };
+int fp8_amax_history_update_ex(float *history, int32_t *state, int window,
+                               const float *amax, int fmt, float *scale,
+                               int algo, float alpha, float margin, void *stream);
+
 /* Static, human-readable text for a status code (never NULL). */
 const char *fp8_status_string(int status);
 

@@ -59,6 +59,15 @@ def lib() -> ctypes.CDLL:
         L.orc_dequantize.restype = c_int
         L.orc_amax_history_update.argtypes = [c_void, c_void, c_int, ctypes.c_float, c_int, c_void]
         L.orc_amax_history_update.restype = c_int
+        L.orc_amax_history_update_ex.argtypes = [c_void, c_void, c_int, ctypes.c_float, c_int, c_void, c_int,
+                                                 ctypes.c_float, ctypes.c_float]
+        L.orc_amax_history_update_ex.restype = c_int
+        L.orc_mx_exponent.argtypes = [ctypes.c_float, c_int, c_int]
+        L.orc_mx_exponent.restype = c_int
+        L.orc_quantize_mx.argtypes = [c_void, c_int, c_i64, c_i64, c_int, c_int, c_void, c_void]
+        L.orc_quantize_mx.restype = c_int
+        L.orc_dequantize_mx.argtypes = [c_void, c_int, c_i64, c_i64, c_void, c_void, c_int]
+        L.orc_dequantize_mx.restype = c_int
         if L.orc_selfcheck() != 0:
             raise RuntimeError("oracle self-check failed: decoded table disagrees with the format table")
         _lib = L
@@ -193,17 +202,60 @@ def fake_quantize(x: np.ndarray, fmt: int, br: int = 1, bc: int = 128, scale: fl
     return y.reshape(x.shape), scales
 
 
-class AmaxHistory:
-    """Delayed-scaling state: a window of past amax values and the current scale."""
+MX_FIT, MX_OCP = 0, 1
 
-    def __init__(self, window: int, fmt: int):
+
+def mx_exponent(amax: float, fmt: int, rule: int = MX_FIT) -> int:
+    """k of the power-of-two scale 2^k of an MX block with this amax."""
+    return lib().orc_mx_exponent(float(amax), fmt, rule)
+
+
+def quantize_mx(x: np.ndarray, fmt: int, rule: int = MX_FIT):
+    """MX quantize of a 2-D array: (codes, e8m0 [R, ceil(C/32)] uint8)."""
+    x, dt = _as_input(x)
+    if x.ndim != 2:
+        raise ValueError("MX quantize takes a 2-D array")
+    R, C = x.shape
+    q = np.empty((R, C), dtype=np.uint8)
+    e = np.empty((R, math.ceil(C / 32)), dtype=np.uint8)
+    _check(lib().orc_quantize_mx(_ptr(x), dt, R, C, fmt, rule, _ptr(q), _ptr(e)))
+    return q, e
+
+
+def dequantize_mx(q: np.ndarray, fmt: int, e8m0: np.ndarray, out_dtype: int = F32) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    e8m0 = np.ascontiguousarray(e8m0, dtype=np.uint8)
+    R, C = q.shape
+    y = np.empty(q.shape, dtype=np.float32 if out_dtype == F32 else np.uint16)
+    _check(lib().orc_dequantize_mx(_ptr(q), fmt, R, C, _ptr(e8m0), _ptr(y), out_dtype))
+    return y
+
+
+WINDOW_MAX, EMA = 0, 1
+
+
+class AmaxHistory:
+    """Delayed-scaling state: a window of past amax values (or their moving average) and the scale.
+
+    algo WINDOW_MAX with margin 1.0 is the plain window of the PyTorch-FP8 page's DelayedScaler;
+    margin and EMA are its s4.3 refinements."""
+
+    def __init__(self, window: int, fmt: int, algo: int = WINDOW_MAX, alpha: float = 1.0, margin: float = 1.0):
         self.window = window
         self.fmt = fmt
+        self.algo = algo
+        self.alpha = alpha
+        self.margin = margin
         self.history = np.zeros(window, dtype=np.float32)
         self.state = np.zeros(2, dtype=np.int32)
         self.scale = np.ones(1, dtype=np.float32)
 
     def update(self, amax_value: float) -> np.float32:
-        _check(lib().orc_amax_history_update(_ptr(self.history), _ptr(self.state), self.window,
-                                             float(amax_value), self.fmt, _ptr(self.scale)))
+        if self.algo == WINDOW_MAX and self.margin == 1.0:
+            _check(lib().orc_amax_history_update(_ptr(self.history), _ptr(self.state), self.window,
+                                                 float(amax_value), self.fmt, _ptr(self.scale)))
+        else:
+            _check(lib().orc_amax_history_update_ex(_ptr(self.history), _ptr(self.state), self.window,
+                                                    float(amax_value), self.fmt, _ptr(self.scale), self.algo,
+                                                    float(self.alpha), float(self.margin)))
         return self.scale[0]

@@ -35,6 +35,13 @@
  *   R6  Blocks at a ragged edge hold only the elements inside the tensor.
  *   R7  bf16 input is widened to fp32 exactly; bf16 output is the fp32
  *       result rounded once more to bf16, nearest-even.
+ *   R14 The delayed-scaling margin divides: s = MAX / (max(amax, eps) * m),
+ *       each operation rounded to fp32 ([FP8-native] s4.3).
+ *   R15 The moving-average amax: first update m = amax, later ones
+ *       m = alpha * amax + (1 - alpha) * m, each product and the sum rounded
+ *       to fp32; the scale follows from m once `window` updates are in.
+ *   R16 MX blocks: scale 2^k, k by the fit rule or the OCP MX rule (below).
+ *   R17 An MX block with an infinite amax gets the NaN scale byte.
  */
 #include <math.h>
 #include <stdint.h>
@@ -333,6 +340,17 @@ int orc_dequantize(const uint8_t *q, int fmt, int64_t rows, int64_t cols,
 /* Delayed scaling: the amax history                                   */
 /* ------------------------------------------------------------------ */
 
+/* [FP8-native] s4.3: the scale may keep a margin, max_val / (amax * margin)
+ * (the page's example margin is 1.1).  Reading R14: both steps in fp32,
+ * s = RN(MAX / RN(max(amax, eps) * margin)); margin 1 gives
+ * orc_scale_from_amax exactly. */
+static float scale_with_margin(float amax, float margin, int fmt)
+{
+    const float m = (amax > AMAX_EPS) ? amax : AMAX_EPS;
+    const float d = (float)((double)m * (double)margin); /* exact product, one rounding */
+    return (float)(MAX_FINITE[fmt] / (double)d);        /* correctly rounded fp32 quotient */
+}
+
 /* [FP8-native] s4.2 DelayedScaler.update: append this step's amax to a
  * window of the last `window` amax values; once the window is full, the
  * scale becomes max_val / max(max(window), eps).  Until then it keeps its
@@ -355,5 +373,141 @@ int orc_amax_history_update(float *history, int32_t *state, int window,
     }
     state[0] = pos;
     state[1] = count;
+    return ORC_OK;
+}
+
+/* Delayed scaling with the [FP8-native] s4.3 refinements.
+ *   algo 0 (window max): as orc_amax_history_update, but the refreshed scale
+ *          keeps the margin: MAX / (max(max(window), eps) * margin).
+ *   algo 1 (EMA): the amax is smoothed instead of windowed (s4.2 names an
+ *          exponential moving average as Transformer Engine's smoothing).
+ *          history[0] holds the average m: the first update sets m = amax,
+ *          later ones m = RN(RN(alpha*amax) + RN(RN(1 - alpha) * m)) in fp32
+ *          (reading R15).  state[1] counts updates (saturating at window);
+ *          once it reaches window the scale becomes MAX / (max(m, eps) *
+ *          margin) at every update -- window acts as the warm-up length.
+ *          state[0] is unused. */
+int orc_amax_history_update_ex(float *history, int32_t *state, int window, float amax, int fmt,
+                               float *scale, int algo, float alpha, float margin)
+{
+    if (!fmt_ok(fmt) || window <= 0 || (algo != 0 && algo != 1)) return ORC_EBADARG;
+    if (!(margin > 0.0f) || !(alpha >= 0.0f && alpha <= 1.0f)) return ORC_EBADARG;
+    int32_t pos = state[0], count = state[1];
+    if (count < 0 || count > window) return ORC_EBADARG;
+    if (algo == 0) {
+        if (pos < 0 || pos >= window) return ORC_EBADARG;
+        history[pos] = amax;
+        pos = (pos + 1) % window;
+        if (count < window) count += 1;
+        if (count == window) {
+            float m = 0.0f;
+            for (int i = 0; i < window; ++i)
+                if (history[i] > m) m = history[i];
+            *scale = scale_with_margin(m, margin, fmt);
+        }
+    } else {
+        if (count == 0) {
+            history[0] = amax;
+        } else {
+            const float beta = (float)(1.0 - (double)alpha);
+            const float a_part = (float)((double)alpha * (double)amax);
+            const float m_part = (float)((double)beta * (double)history[0]);
+            history[0] = (float)((double)a_part + (double)m_part);
+        }
+        if (count < window) count += 1;
+        if (count == window) *scale = scale_with_margin(history[0], margin, fmt);
+    }
+    state[0] = pos;
+    state[1] = count;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* MX blocks: 1x32 with a power-of-two scale                           */
+/* ------------------------------------------------------------------ */
+
+/* [MP-handbook] "FP8 training", last notes: Blackwell's MX formats (MXFP8)
+ * let every 32 consecutive elements share one scale factor, in hardware.  That
+ * scale is a power of two, s = 2^k, stored as the E8M0 byte of the dequant
+ * multiplier 2^-k (byte = 127 - k; E8M0 is an unsigned exponent with bias 127
+ * whose byte 0xFF means NaN).
+ * Reading R16: which k --
+ *   rule 0 (fit): the largest k with max(amax, eps) * 2^k <= MAX, i.e. the
+ *                 pages' s = MAX / amax restricted to a power of two; no
+ *                 element of the block saturates.
+ *   rule 1 (OCP MX): k = emax_elem - floor(log2(max(amax, eps))), emax_elem
+ *                 the exponent of the format's largest normal (8 for E4M3, 15
+ *                 for E5M2); the top of a binade can saturate.
+ * Reading R17: a block holding +-Inf has an infinite amax and no power of two
+ * that fits; it gets k = 0 for its elements and the NaN byte 0xFF, so its
+ * dequantized values are all NaN.  (NaN elements are skipped by amax, as in
+ * every other mode.)
+ * Elements: q = fp8(fp32(x * 2^k)), as in every other mode. */
+static int mx_exponent(float amax, int fmt, int rule)
+{
+    if (isinf(amax)) return 0;
+    const double a = (double)((amax > AMAX_EPS) ? amax : AMAX_EPS);
+    const int emax_elem = (fmt == ORC_E4M3) ? 8 : 15;
+    int e; /* frexp: a = f * 2^e with f in [0.5, 1), so floor(log2 a) = e - 1 */
+    (void)frexp(a, &e);
+    int k = emax_elem - (e - 1);
+    if (rule == 1) return k;
+    /* fit: the OCP exponent is at most one too large; step down until
+     * a * 2^k <= MAX holds (exact in double) */
+    while (ldexp(a, k) > MAX_FINITE[fmt]) --k;
+    return k;
+}
+
+static uint8_t mx_byte(float amax, int k)
+{
+    return isinf(amax) ? (uint8_t)0xFF : (uint8_t)(127 - k);
+}
+
+int orc_mx_exponent(float amax, int fmt, int rule)
+{
+    if (!fmt_ok(fmt) || (rule != 0 && rule != 1)) return -1000;
+    return mx_exponent(amax, fmt, rule);
+}
+
+/* x [rows, cols]; blocks of 32 consecutive elements of a row (the last one in
+ * a row may be short); e8m0 [rows, ceil(cols / 32)]. */
+int orc_quantize_mx(const void *x, int dtype, int64_t rows, int64_t cols, int fmt, int rule,
+                    uint8_t *q, uint8_t *e8m0)
+{
+    if (!fmt_ok(fmt) || !dtype_ok(dtype) || rows < 0 || cols < 0 || (rule != 0 && rule != 1))
+        return ORC_EBADARG;
+    const int64_t nbc = (cols + 31) / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t bj = 0; bj < nbc; ++bj) {
+            const int64_t c0 = bj * 32, c1 = (c0 + 32 < cols) ? c0 + 32 : cols;
+            const float amax = amax_of(x, dtype, r * cols + c0, r * cols + c1);
+            const int k = mx_exponent(amax, fmt, rule);
+            const float s = (float)ldexp(1.0, k);
+            e8m0[r * nbc + bj] = mx_byte(amax, k);
+            for (int64_t c = c0; c < c1; ++c)
+                q[r * cols + c] = scaled_code(load_elem(x, dtype, r * cols + c), s, fmt);
+        }
+    }
+    return ORC_OK;
+}
+
+/* MX dequant: y = fp32(decode(q) * 2^(byte - 127)), the MX value being the
+ * element times the shared scale; for a byte made by the quantizer that is
+ * the real number decode(q) / 2^k.  Byte 0xFF (NaN) gives NaN. */
+int orc_dequantize_mx(const uint8_t *q, int fmt, int64_t rows, int64_t cols, const uint8_t *e8m0,
+                      void *y, int out_dtype)
+{
+    if (!fmt_ok(fmt) || !dtype_ok(out_dtype) || rows < 0 || cols < 0) return ORC_EBADARG;
+    const int64_t nbc = (cols + 31) / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            const int64_t i = r * cols + c;
+            const uint8_t b = e8m0[r * nbc + c / 32];
+            const double xs = (b == 0xFF) ? NAN : ldexp(1.0, (int)b - 127);
+            const float out = (float)(orc_fp8_decode(q[i], fmt) * xs);
+            if (out_dtype == ORC_F32) ((float *)y)[i] = out;
+            else ((uint16_t *)y)[i] = orc_f32_to_bf16(out);
+        }
+    }
     return ORC_OK;
 }

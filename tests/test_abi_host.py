@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
                                            "fp8_amax_history_update", "fp8_status_string", "fp8_device_status",
                                            "fp8_fake_quantize", "fp8_amax", "fp8_scale_from_amax",
                                            "fp8_quantize_per_tensor_fused",
-                                           "fp8_quantize_per_tensor_fused_noalloc",
+                                           "fp8_quantize_per_tensor_fused_noalloc", "fp8_amax_history_update_ex",
                                            "fp8_selftest_wait_timeout"])
 
 
@@ -167,6 +167,19 @@ def test_history_validation(L):
     assert f(A16, A16, 16, A16, 1, None, None) == ERR_NULL
     assert f(A1, A16, 16, A16, 1, A16, None) == ERR_ALIGN
     assert f(A16, A16 + 2, 16, A16, 1, A16, None) == ERR_ALIGN
+
+
+def test_history_ex_validation(L):
+    f = L.fp8_amax_history_update_ex
+    assert f(A16, A16, 16, A16, 3, A16, 0, 1.0, 1.0, None) == ERR_FORMAT
+    assert f(A16, A16, 16, A16, 0, A16, 2, 1.0, 1.0, None) == ERR_ARG
+    assert f(A16, A16, 16, A16, 0, A16, 1, 1.5, 1.0, None) == ERR_ARG
+    assert f(A16, A16, 16, A16, 0, A16, 1, -0.1, 1.0, None) == ERR_ARG
+    assert f(A16, A16, 16, A16, 0, A16, 0, 1.0, 0.0, None) == ERR_ARG
+    assert f(A16, A16, 16, A16, 0, A16, 0, 1.0, float("nan"), None) == ERR_ARG
+    assert f(A16, A16, 0, A16, 0, A16, 0, 1.0, 1.0, None) == ERR_ARG
+    assert f(None, A16, 16, A16, 0, A16, 0, 1.0, 1.0, None) == ERR_NULL
+    assert f(A16, A16, 16, A16, 0, A1, 0, 1.0, 1.0, None) == ERR_ALIGN
 
 
 def test_diagnostics_validation(L):

@@ -430,3 +430,34 @@ def test_fused_per_tensor_outlier_tensors():
         torch.cuda.synchronize()
         assert_bytes_equal(q, oq, f"fused x{factor}")
         assert_bytes_equal(s, fp32_bits([os_]), f"fused scale x{factor}")
+
+
+# -- delayed scaling refinements: margin and moving average ------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("algo,alpha,margin,window", [(0, 1.0, 1.1, 16), (0, 1.0, 1.0, 5), (0, 1.0, 2.5, 33),
+                                                      (1, 0.1, 1.0, 1), (1, 0.25, 1.1, 8), (1, 1.0, 1.0, 3),
+                                                      (1, 0.0, 1.3, 2)])
+def test_history_update_ex_matches_oracle(fmt, algo, alpha, margin, window):
+    rng = np.random.default_rng(17 + window)
+    amaxes = np.exp(rng.uniform(np.log(1e-14), np.log(1e4), size=3 * window + 10)).astype(np.float32)
+    amaxes[2] = 0.0
+    h = torch.zeros(window, dtype=torch.float32, device="cuda")
+    st = torch.zeros(2, dtype=torch.int32, device="cuda")
+    sc = torch.ones(1, dtype=torch.float32, device="cuda")
+    am = torch.empty(1, dtype=torch.float32, device="cuda")
+    ref = oracle.AmaxHistory(window, fmt, algo=algo, alpha=alpha, margin=margin)
+    for k, a in enumerate(amaxes):
+        am.fill_(float(a))
+        B.fp8_amax_history_update_ex(h, st, am, sc, fmt, algo, alpha, margin)
+        lib = oracle.lib()
+        assert lib.orc_amax_history_update_ex(ref.history.ctypes.data, ref.state.ctypes.data, window, float(a), fmt,
+                                              ref.scale.ctypes.data, algo, float(alpha), float(margin)) == 0
+        torch.cuda.synchronize()
+        assert_bytes_equal(sc, fp32_bits(ref.scale), f"scale step {k}")
+        assert st.cpu().tolist()[1] == int(ref.state[1])
+        if algo == 0:
+            assert st.cpu().tolist()[0] == int(ref.state[0])
+            assert_bytes_equal(h, fp32_bits(ref.history), f"history step {k}")
+        else:
+            assert_bytes_equal(h[:1], fp32_bits(ref.history[:1]), f"ema step {k}")

@@ -303,3 +303,75 @@ def test_fake_quantize_vs_torch_handbook_quant(fmt, dtype):
     s = torch.tensor(123.0)
     ref = ((x.float() * s).clamp(-MAX, MAX).to(TORCH_FP8[fmt]).to(torch.float32) / s).to(dtype)
     assert np.array_equal(y, as_oracle_input(ref))
+
+
+# -- delayed scaling refinements (PyTorch-FP8 page s4.3: margin, moving average) ---------
+
+def _amax_sequence(seed, steps):
+    rng = np.random.default_rng(seed)
+    return np.exp(rng.uniform(np.log(1e-6), np.log(1e4), size=steps)).astype(np.float32)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_window_max_with_margin_one_is_the_plain_window(fmt):
+    seq = _amax_sequence(1, 40)
+    plain = oracle.AmaxHistory(16, fmt)
+    ex = oracle.AmaxHistory(16, fmt, algo=oracle.WINDOW_MAX, margin=1.0)
+    for a in seq:  # the extended entry point, called directly with margin exactly 1
+        s1 = plain.update(a)
+        lib = oracle.lib()
+        assert lib.orc_amax_history_update_ex(ex.history.ctypes.data, ex.state.ctypes.data, 16, float(a), fmt,
+                                              ex.scale.ctypes.data, 0, 1.0, 1.0) == 0
+        assert ex.scale[0] == s1 and np.array_equal(ex.history, plain.history)
+        assert np.array_equal(ex.state, plain.state)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_margin_keeps_the_window_max_below_max(fmt):
+    MAX = oracle.MAX[fmt]
+    seq = _amax_sequence(2, 40)
+    h = oracle.AmaxHistory(8, fmt, algo=oracle.WINDOW_MAX, margin=1.1)
+    plain = oracle.AmaxHistory(8, fmt)
+    for k, a in enumerate(seq):
+        s = h.update(a)
+        s0 = plain.update(a)
+        if k >= 7:
+            m = float(max(seq[k - 7:k + 1]))
+            # the window max lands at MAX / 1.1, never at MAX: within fp32 rounding of the two steps
+            assert abs(m * float(s) * 1.1 / MAX - 1.0) < 4e-7
+            # and the margin divides the plain scale (up to one rounding each)
+            assert abs(float(s) * 1.1 / float(s0) - 1.0) < 4e-7
+            # quantizing that max element gives a code below the format's top code
+            code = oracle.encode(np.float32(np.float32(m) * s), fmt)
+            assert (code & 0x7F) < oracle.top_code(fmt)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_ema_alpha_one_is_the_latest_amax_and_alpha_zero_the_first(fmt):
+    seq = _amax_sequence(3, 30)
+    h1 = oracle.AmaxHistory(4, fmt, algo=oracle.EMA, alpha=1.0)
+    h0 = oracle.AmaxHistory(4, fmt, algo=oracle.EMA, alpha=0.0)
+    for k, a in enumerate(seq):
+        s1 = h1.update(a)
+        s0 = h0.update(a)
+        if k >= 3:
+            assert s1 == oracle.scale_from_amax(a, fmt)
+            assert s0 == oracle.scale_from_amax(seq[0], fmt)
+        else:
+            assert s1 == 1.0 and s0 == 1.0  # warm-up: the scale keeps its initial value
+
+
+@pytest.mark.parametrize("alpha", [0.01, 0.1, 0.5, 0.9])
+def test_ema_stays_inside_the_seen_range(alpha):
+    seq = _amax_sequence(4, 200)
+    h = oracle.AmaxHistory(1, oracle.E4M3, algo=oracle.EMA, alpha=alpha)
+    for k, a in enumerate(seq):
+        h.update(a)
+        m = float(h.history[0])
+        lo, hi = float(seq[:k + 1].min()), float(seq[:k + 1].max())
+        assert lo * (1 - 1e-6) <= m <= hi * (1 + 1e-6)
+    # a constant amax is (to fp32 rounding) a fixed point
+    h = oracle.AmaxHistory(1, oracle.E4M3, algo=oracle.EMA, alpha=alpha)
+    for _ in range(50):
+        h.update(3.25)
+    assert abs(float(h.history[0]) / 3.25 - 1) < 1e-6
