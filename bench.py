@@ -350,7 +350,27 @@ def modes_breakdown(dev, stream, peak):
     put("1x128_fake_quant_bf16", wl + " (one pass, bf16 -> bf16, no codes written)", 4 * n, time_in_graph([
         lambda r, st: raw.check(L.fp8_fake_quantize(a.data_ptr(), 1, R_, C_, 1, 128, 0, None, y.data_ptr(), None,
                                                     st), "fake quant")], 20, dev))
-    del a, q, s, y
+    # MX (1x32 blocks, E8M0 byte scales, fit rule) on the same activations
+    e8 = torch.empty(R_, C_ // 32, dtype=torch.uint8, device=dev)
+    put("mx1x32_e4m3_quant", wl, 3 * n + n // 32, time_in_graph([lambda r, st: raw.check(
+        L.fp8_quantize_mx(a.data_ptr(), 1, R_, C_, 0, 0, q.data_ptr(), e8.data_ptr(), st), "mx")], 20, dev))
+    put("mx1x32_dequant_bf16", wl, 3 * n + n // 32, time_in_graph([lambda r, st: raw.check(
+        L.fp8_dequantize_mx(q.data_ptr(), 0, R_, C_, e8.data_ptr(), y.data_ptr(), 1, st), "mx dequant")], 20, dev))
+    # per-tensor with a transposed copy (q and qt), delayed scale (one pass: 2 B read + 2 B written per element)
+    # and current scaling (amax pass first)
+    qt = torch.empty(C_, R_, dtype=torch.uint8, device=dev)
+    sc = torch.full((1,), 0.25, dtype=torch.float32, device=dev)
+    so_ = torch.empty(1, dtype=torch.float32, device=dev)
+    ao_ = torch.empty(1, dtype=torch.float32, device=dev)
+    put("per_tensor_transpose_delayed_e4m3", wl + " (q and qt, one pass with amax)", 4 * n, time_in_graph([
+        lambda r, st: raw.check(L.fp8_quantize_per_tensor_transpose(a.data_ptr(), 1, R_, C_, 0, sc.data_ptr(),
+                                                                    q.data_ptr(), qt.data_ptr(), so_.data_ptr(),
+                                                                    ao_.data_ptr(), st), "transpose")], 20, dev))
+    put("per_tensor_transpose_current_e4m3", wl + " (amax pass, then q and qt; alg bytes 4/elem)", 4 * n,
+        time_in_graph([lambda r, st: raw.check(L.fp8_quantize_per_tensor_transpose(
+            a.data_ptr(), 1, R_, C_, 0, None, q.data_ptr(), qt.data_ptr(), so_.data_ptr(), ao_.data_ptr(), st),
+            "transpose")], 20, dev))
+    del a, q, s, y, e8, qt
 
     # size sweep point 2^28 (512 MiB bf16): 1x128, 128x128, per-tensor current E5M2, dequant
     x = inputs.sweep_tensor(28, device=dev)
@@ -402,6 +422,38 @@ def modes_breakdown(dev, stream, peak):
         "(cast + amax in one pass, then the history update)", 3 * n, t_step)
     out["delayed_e5m2_history_update_us"] = round(t_hist * 1e3, 2)
     del gs, q
+
+    # the consumer: blockwise-scaled FP8 GEMM on the tensor cores, 1x128 activations x 128x128 weights
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16_peak, peak_kind = float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2 (nominal fp8/bf16)"
+    except (OSError, KeyError, ValueError):
+        bf16_peak, peak_kind = 1590.0, "fallback bf16 x 2 (nominal fp8/bf16)"
+    fp8_peak = 2.0 * bf16_peak
+    st0 = stream.cuda_stream
+    for (Mg, Ng, Kg) in ((4096, 4096, 4096), (16384, 4096, 7168)):
+        xg = inputs.random_matrix(Mg, Kg, seed=6, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e2, device=dev)
+        wg = inputs.random_matrix(Ng, Kg, seed=7, dtype=torch.bfloat16, scale=0.02, device=dev)
+        qa = torch.empty(Mg, Kg, dtype=torch.uint8, device=dev)
+        sa = torch.empty(Mg, Kg // 128, dtype=torch.float32, device=dev)
+        qb = torch.empty(Ng, Kg, dtype=torch.uint8, device=dev)
+        sb = torch.empty(Ng // 128, Kg // 128, dtype=torch.float32, device=dev)
+        raw.check(L.fp8_quantize_blockwise(xg.data_ptr(), 1, Mg, Kg, 1, 128, 0, qa.data_ptr(), sa.data_ptr(), st0),
+                  "1x128")
+        raw.check(L.fp8_quantize_blockwise(wg.data_ptr(), 1, Ng, Kg, 128, 128, 0, qb.data_ptr(), sb.data_ptr(), st0),
+                  "128x128")
+        cg = torch.empty(Mg, Ng, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        del xg, wg
+        ms = time_in_graph([lambda r, st: raw.check(L.fp8_gemm_blockwise(
+            qa.data_ptr(), sa.data_ptr(), 0, qb.data_ptr(), sb.data_ptr(), 0, Mg, Ng, Kg, cg.data_ptr(), 1, st),
+            "gemm")], 10, dev)
+        tflops = 2.0 * Mg * Ng * Kg / (ms * 1e-3) / 1e12
+        out[f"gemm_blockwise_e4m3_{Mg}x{Ng}x{Kg}"] = {
+            "workload": f"A [{Mg}, {Kg}] 1x128-scaled E4M3 x B [{Ng}, {Kg}] 128x128-scaled E4M3 -> bf16",
+            "TFLOP_s": round(tflops, 1), "frac_of_peak": round(tflops / fp8_peak, 4), "peak_TFLOP_s": fp8_peak,
+            "peak_kind": peak_kind, "us": round(ms * 1e3, 2)}
+        del qa, sa, qb, sb, cg
 
     # per-tensor current scaling on small tensors (latency-bound): two passes vs the one-pass kernel, each
     # launch timed alone after an untimed L2 flush

@@ -4,8 +4,9 @@ Two layers with the C names:
 
 * ``lib()`` returns the loaded ``ctypes.CDLL`` whose functions take the exact
   C arguments (device pointers as ints, sizes, enums, a stream handle).
-* ``fp8_quantize_per_tensor``, ``fp8_quantize_blockwise``, ``fp8_dequantize``
-  and ``fp8_amax_history_update`` below take torch CUDA tensors, allocate any
+* ``fp8_quantize_per_tensor``, ``fp8_quantize_blockwise``, ``fp8_dequantize``,
+  ``fp8_quantize_mx``, ``fp8_dequantize_mx``, ``fp8_amax_history_update`` and
+  the other wrappers below take torch CUDA tensors, allocate any
   output the caller did not pass (``torch.empty`` on the input's device), pass
   pointers and the current stream to the C function, and raise ``FP8Error`` on
   a nonzero status.  All computation happens in the library's kernels; there
@@ -41,12 +42,17 @@ SIGNATURES = {
     "fp8_amax": (_c_int, [_vp, _c_int, _i64, _vp, _vp]),
     "fp8_scale_from_amax": (_c_int, [_vp, _c_int, _vp, _vp]),
     "fp8_fake_quantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]),
+    "fp8_quantize_per_tensor_transpose": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fp8_quantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _vp]),
+    "fp8_dequantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _vp, _vp, _c_int, _vp]),
+    "fp8_gemm_blockwise": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _i64, _i64, _i64, _vp, _c_int, _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_c_int]),
     "fp8_device_status": (_c_int, [_vp, _c_int, _vp]),
     "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
 }
 DEVICE_STATUS_WAIT_TIMEOUT = 0x1
 AMAX_WINDOW_MAX, AMAX_EMA = 0, 1
+MX_FIT, MX_OCP = 0, 1
 FUSED_WORKSPACE_BYTES = 16
 
 
@@ -137,6 +143,28 @@ def fp8_quantize_per_tensor(x: torch.Tensor, fmt: int = E4M3, scale_in: torch.Te
     return q, scale_out, amax_out
 
 
+def fp8_quantize_per_tensor_transpose(x: torch.Tensor, fmt: int = E4M3, scale_in: torch.Tensor | None = None,
+                                      with_q: bool = True, q: torch.Tensor | None = None,
+                                      qt: torch.Tensor | None = None, scale_out: torch.Tensor | None = None,
+                                      amax_out: torch.Tensor | None = None, stream=None):
+    """Per-tensor quantize of a 2-D tensor with a transposed copy.  Returns (q or None, qt [C, R], scale, amax)."""
+    _need_cuda(x, scale_in, q, qt, scale_out, amax_out)
+    if x.dim() != 2:
+        raise ValueError("the transposing quantize takes a 2-D tensor")
+    R, C = x.shape
+    dev = x.device
+    if q is None and with_q:
+        q = torch.empty((R, C), dtype=torch.uint8, device=dev)
+    qt = torch.empty((C, R), dtype=torch.uint8, device=dev) if qt is None else qt
+    scale_out = torch.empty(1, dtype=torch.float32, device=dev) if scale_out is None else scale_out
+    amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
+    st = load_library().fp8_quantize_per_tensor_transpose(_ptr(x), _DTYPE_CODE[x.dtype], R, C, fmt, _ptr(scale_in),
+                                                          _ptr(q), _ptr(qt), _ptr(scale_out), _ptr(amax_out),
+                                                          _stream(stream))
+    _check("fp8_quantize_per_tensor_transpose", st)
+    return q, qt, scale_out, amax_out
+
+
 def fused_workspace(device="cuda") -> torch.Tensor:
     """A zeroed workspace for fp8_quantize_per_tensor_fused (one per stream)."""
     return torch.zeros(FUSED_WORKSPACE_BYTES // 4, dtype=torch.int32, device=device)
@@ -195,6 +223,52 @@ def fp8_quantize_blockwise(x: torch.Tensor, block=(1, 128), fmt: int = E4M3, q: 
                                                _ptr(scales), _stream(stream))
     _check("fp8_quantize_blockwise", st)
     return q, scales
+
+
+def fp8_quantize_mx(x: torch.Tensor, fmt: int = E4M3, rule: int = MX_FIT, q: torch.Tensor | None = None,
+                    e8m0: torch.Tensor | None = None, stream=None):
+    """MX quantize of a 2-D tensor: 1x32 blocks, power-of-two scales.  Returns (q, e8m0 uint8 [R, ceil(C/32)])."""
+    _need_cuda(x, q, e8m0)
+    if x.dim() != 2:
+        raise ValueError("MX quantize takes a 2-D tensor")
+    R, C = x.shape
+    q = torch.empty((R, C), dtype=torch.uint8, device=x.device) if q is None else q
+    if e8m0 is None:
+        e8m0 = torch.empty((R, math.ceil(C / 32)), dtype=torch.uint8, device=x.device)
+    st = load_library().fp8_quantize_mx(_ptr(x), _DTYPE_CODE[x.dtype], R, C, fmt, rule, _ptr(q), _ptr(e8m0),
+                                        _stream(stream))
+    _check("fp8_quantize_mx", st)
+    return q, e8m0
+
+
+def fp8_dequantize_mx(q: torch.Tensor, e8m0: torch.Tensor, fmt: int = E4M3, out_dtype=torch.float32,
+                      y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """MX dequantize: y = decode(q) * 2^(e8m0 - 127) per 1x32 block."""
+    _need_cuda(q, e8m0, y)
+    if q.dim() != 2:
+        raise ValueError("MX dequantize takes a 2-D tensor")
+    R, C = q.shape
+    y = torch.empty((R, C), dtype=out_dtype, device=q.device) if y is None else y
+    st = load_library().fp8_dequantize_mx(_ptr(q), fmt, R, C, _ptr(e8m0), _ptr(y), _DTYPE_CODE[y.dtype],
+                                          _stream(stream))
+    _check("fp8_dequantize_mx", st)
+    return y
+
+
+def fp8_gemm_blockwise(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, a_fmt: int = E4M3,
+                       b_fmt: int = E4M3, out_dtype=torch.bfloat16, c: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """C [M, N] = A [M, K] (1x128 scales sa) x B [N, K]^T (128x128 scales sb), FP8 tensor cores."""
+    _need_cuda(a, sa, b, sb, c)
+    if a.dim() != 2 or b.dim() != 2 or a.shape[1] != b.shape[1]:
+        raise ValueError("fp8_gemm_blockwise takes a [M, K] and b [N, K]")
+    M, K = a.shape
+    N = b.shape[0]
+    c = torch.empty((M, N), dtype=out_dtype, device=a.device) if c is None else c
+    st = load_library().fp8_gemm_blockwise(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_fmt, M, N, K, _ptr(c),
+                                           _DTYPE_CODE[c.dtype], _stream(stream))
+    _check("fp8_gemm_blockwise", st)
+    return c
 
 
 def fp8_dequantize(q: torch.Tensor, scales: torch.Tensor, block=(0, 0), fmt: int = E4M3,

@@ -108,6 +108,27 @@ struct DOut {
         }
         return o;
     }
+
+    // MX: y = RN(decode(q) * m), m = 2^(byte - 127).  The product of an FP8
+    // value and a power of two is exact unless it leaves the fp32 normal
+    // range, where the one rounding of mul.rn (no flush to zero) is the
+    // rounding of the real product.
+    template <int FMT>
+    static __device__ __forceinline__ Out multiply(const In& cin, float m) {
+        uint32_t cw[kCodeWords];
+        unpack_codes<kCodeWords>(cin, cw);
+        const uint64_t m2 = f32x2(m, m);
+        Out o;
+#pragma unroll
+        for (int k = 0; k < kCodeWords; ++k) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 a = fp8x2_to_float2<FMT>(h ? (cw[k] >> 16) : (cw[k] & 0xFFFFu));
+                put<FMT>(o, 2 * k + h, f32x2_split(mul_f32x2(f32x2(a.x, a.y), m2)));
+            }
+        }
+        return o;
+    }
 };
 
 __device__ __forceinline__ uint32_t ld_codes(const uint32_t* p) {
@@ -213,6 +234,78 @@ k_dequant_general(const uint8_t* __restrict__ q, int64_t rows, int64_t cols, int
     }
 }
 
+// MX (1x32 blocks, E8M0 scales) with cols % 32 == 0: a row's blocks are the
+// consecutive 32-code runs of the flat array, so group g's block is
+// g / (32 / kCodes).  Each CTA owns kThreads x kUnroll consecutive groups.
+template <int FMT, int OUT, int OB>
+__global__ void __launch_bounds__(kThreads)
+k_dequant_mx(const typename DOut<OUT, OB>::In* __restrict__ q, int64_t ngroups, const uint8_t* __restrict__ e8m0,
+             typename DOut<OUT, OB>::Out* __restrict__ y) {
+    pdl_enter();
+    using D = DOut<OUT, OB>;
+    constexpr int kGroupsPerBlock = 32 / D::kCodes;
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x;
+    typename D::In c[kUnroll];
+    uint32_t b[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t g = base + u * kThreads;
+        const bool ok = g < ngroups;
+        c[u] = ok ? ld_codes(q + g) : typename D::In{};
+        b[u] = ok ? static_cast<uint32_t>(__ldcs(e8m0 + g / kGroupsPerBlock)) : 127u;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t g = base + u * kThreads;
+        if (g < ngroups) store_words(y + g, D::template multiply<FMT>(c[u], e8m0_to_float(b[u])));
+    }
+}
+
+// MX over any cols (ragged right edge), element by element.
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(kThreads)
+k_dequant_mx_general(const uint8_t* __restrict__ q, int64_t rows, int64_t cols, const uint8_t* __restrict__ e8m0,
+                     void* __restrict__ y) {
+    pdl_enter();
+    const int64_t n = rows * cols;
+    const int64_t nbc = (cols + 31) / 32;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * kThreads) {
+        const int64_t r = i / cols, c = i - (i / cols) * cols;
+        const float v = __fmul_rn(decode1<FMT>(q[i]), e8m0_to_float(e8m0[r * nbc + c / 32]));
+        if (OUT == 0) static_cast<float*>(y)[i] = v;
+        else static_cast<uint16_t*>(y)[i] = static_cast<uint16_t>(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+    }
+}
+
+template <int FMT, int OUT, int OB>
+cudaError_t dequant_mx_fast(const uint8_t* q, int64_t n, const uint8_t* e8m0, void* y, cudaStream_t st) {
+    using D = DOut<OUT, OB>;
+    const int64_t ngroups = n / D::kCodes;  // n is a multiple of 32, so of kCodes
+    const int64_t per_cta = static_cast<int64_t>(kThreads) * kUnroll;
+    const int64_t grid = std::max<int64_t>(1, (ngroups + per_cta - 1) / per_cta);
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const cudaError_t e = launch_kernel(k_dequant_mx<FMT, OUT, OB>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+                                        0, st, reinterpret_cast<const typename D::In*>(q), ngroups, e8m0,
+                                        static_cast<typename D::Out*>(y));
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int FMT, int OUT>
+cudaError_t dequant_mx_typed(const uint8_t* q, int64_t rows, int64_t cols, const uint8_t* e8m0, void* y,
+                             cudaStream_t st) {
+    const int64_t n = rows * cols;
+    if (cols % 32 == 0) {
+        if ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) return dequant_mx_fast<FMT, OUT, 32>(q, n, e8m0, y, st);
+        return dequant_mx_fast<FMT, OUT, 16>(q, n, e8m0, y, st);
+    }
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((n + kThreads - 1) / kThreads,
+                                                                static_cast<int64_t>(device_sm_count()) * 8));
+    const cudaError_t e = launch_kernel(k_dequant_mx_general<FMT, OUT>, dim3(static_cast<unsigned>(grid)),
+                                        dim3(kThreads), 0, st, q, rows, cols, e8m0, y);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int FMT, int OUT, int OB>
 cudaError_t dequant_fast(const uint8_t* q, int64_t rows, int64_t cols, int mode, const float* scales, void* y,
                          cudaStream_t st) {
@@ -260,6 +353,16 @@ cudaError_t dequant_typed(const uint8_t* q, int64_t rows, int64_t cols, int mode
 }
 
 }  // namespace
+
+cudaError_t launch_dequant_mx(const uint8_t* q, int fmt, int64_t rows, int64_t cols, const uint8_t* e8m0, void* y,
+                              int out_dtype, cudaStream_t st) {
+    if (fmt == kE4M3) {
+        return out_dtype == 0 ? dequant_mx_typed<kE4M3, 0>(q, rows, cols, e8m0, y, st)
+                              : dequant_mx_typed<kE4M3, 1>(q, rows, cols, e8m0, y, st);
+    }
+    return out_dtype == 0 ? dequant_mx_typed<kE5M2, 0>(q, rows, cols, e8m0, y, st)
+                          : dequant_mx_typed<kE5M2, 1>(q, rows, cols, e8m0, y, st);
+}
 
 cudaError_t launch_dequant(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int mode, const float* scales,
                            void* y, int out_dtype, cudaStream_t st) {

@@ -107,6 +107,34 @@ int fp8_quantize_per_tensor_fused_noalloc(const void* x, int dtype, int64_t n, i
                                                        static_cast<cudaStream_t>(stream)));
 }
 
+int fp8_quantize_per_tensor_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
+                                      const float* scale_in, uint8_t* q, uint8_t* qt, float* scale_out,
+                                      float* amax_out, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (scale_out == nullptr) return FP8_ERR_NULL;
+    if (scale_in == nullptr && amax_out == nullptr) return FP8_ERR_NULL;
+    if (n > 0 && (x == nullptr || qt == nullptr)) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(qt, 16) || !aligned(scale_out, 4) || !aligned(scale_in, 4) ||
+        !aligned(amax_out, 4))
+        return FP8_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (amax_out != nullptr && cudaMemsetAsync(amax_out, 0, sizeof(float), st) != cudaSuccess) return FP8_ERR_CUDA;
+    if (n == 0) {
+        // no element: the scale of an empty tensor, as fp8_quantize_per_tensor gives it
+        return fp8_quantize_per_tensor(x, dtype, 0, fmt, scale_in, q, scale_out, amax_out, stream);
+    }
+    if (scale_in == nullptr) {
+        const cudaError_t e = fp8q::launch_tensor_amax(x, dtype, n, amax_out, st);
+        if (e != cudaSuccess) return FP8_ERR_CUDA;
+    }
+    return status_of(fp8q::launch_tensor_cast_transpose(x, dtype, rows, cols, fmt, scale_in, amax_out, q, qt, scale_out,
+                                                        scale_in ? amax_out : nullptr, st));
+}
+
 int fp8_amax(const void* x, int dtype, int64_t n, float* amax_out, void* stream) {
     if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
     if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
@@ -186,6 +214,53 @@ int fp8_fake_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int 
     if (xb != yb && xb < yb + bytes && yb < xb + bytes) return FP8_ERR_ARG;  // partial overlap
     return status_of(fp8q::launch_fake_quant(x, dtype, rows, cols, per_tensor ? 0 : block_rows, fmt, scale_in, y,
                                              per_tensor ? nullptr : scales_out, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_quantize_mx(const void* x, int dtype, int64_t rows, int64_t cols, int fmt, int rule, uint8_t* q,
+                    uint8_t* e8m0, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (rule != FP8_MX_FIT && rule != FP8_MX_OCP) return FP8_ERR_ARG;
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (n == 0) return FP8_OK;
+    if (x == nullptr || q == nullptr || e8m0 == nullptr) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16)) return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_quant_mx(x, dtype, rows, cols, fmt, rule, q, e8m0, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_dequantize_mx(const uint8_t* q, int fmt, int64_t rows, int64_t cols, const uint8_t* e8m0, void* y,
+                      int out_dtype, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(out_dtype)) return FP8_ERR_DTYPE;
+    if (rows < 0 || cols < 0) return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (n == 0) return FP8_OK;
+    if (q == nullptr || e8m0 == nullptr || y == nullptr) return FP8_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(y, 16)) return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_dequant_mx(q, fmt, rows, cols, e8m0, y, out_dtype, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb, int b_fmt,
+                       int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream) {
+    if (!fmt_ok(a_fmt) || !fmt_ok(b_fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(c_dtype)) return FP8_ERR_DTYPE;
+    if (M < 0 || N < 0 || K < 0 || N % 256 != 0 || K % 128 != 0) return FP8_ERR_SHAPE;
+    if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || checked_count(M, N) < 0) return FP8_ERR_SHAPE;
+    if (M == 0 || N == 0) return FP8_OK;
+    if (c == nullptr) return FP8_ERR_NULL;
+    if (!aligned(c, 16)) return FP8_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {  // an empty sum
+        const size_t bytes = static_cast<size_t>(M) * static_cast<size_t>(N) * (c_dtype == FP8_F32 ? 4u : 2u);
+        return status_of(cudaMemsetAsync(c, 0, bytes, st));
+    }
+    if (a == nullptr || sa == nullptr || b == nullptr || sb == nullptr) return FP8_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(sa, 4) || !aligned(sb, 4)) return FP8_ERR_ALIGN;
+    if (!fp8q::gemm_blockwise_supported()) return FP8_ERR_CUDA;
+    return status_of(fp8q::launch_gemm_blockwise(a, sa, a_fmt, b, sb, b_fmt, M, N, K, c, c_dtype, st));
 }
 
 int fp8_amax_history_update(float* history, int32_t* state, int window, const float* amax, int fmt, float* scale,

@@ -35,6 +35,38 @@ __device__ __forceinline__ float scale_from_amax(float amax) {
     return __fdiv_rn(fmt_max<FMT>(), fmaxf(amax, kAmaxEps));
 }
 
+// MX block scale (handbook, FP8 training notes: Blackwell's MX formats give
+// every 32 elements one shared power-of-two scale).  Returns s = 2^k and sets
+// `byte` to its E8M0 encoding 127 - k (the exponent of the dequant multiplier
+// 2^-k; E8M0 byte 0xFF is NaN).
+//   rule 0 (fit): the largest k with max(amax, eps) * 2^k <= MAX;
+//   rule 1 (OCP MX): k = emax - floor(log2(max(amax, eps))).
+// MAX is 1.75 * 2^emax in both formats (emax 8 and 15), so for
+// a = m * 2^e with m in [1, 2), rule 1 is k = emax - e and rule 0 takes one
+// less when m > 1.75 -- integer work on the bits of a.  The eps clamp keeps a
+// normal, so k lies in [-120, 55] and 2^k is a normal fp32.  An infinite amax
+// has no fitting power of two: s = 1 and the NaN byte.
+template <int FMT>
+__device__ __forceinline__ float mx_scale(float amax, int rule, uint8_t& byte) {
+    constexpr int kEmax = FMT == kE4M3 ? 8 : 15;
+    const uint32_t b = __float_as_uint(fmaxf(amax, kAmaxEps));
+    const int e = static_cast<int>(b >> 23) - 127;
+    if (e == 128) {
+        byte = 0xFFu;
+        return 1.0f;
+    }
+    const int k = kEmax - e - ((rule == 0 && (b & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
+    byte = static_cast<uint8_t>(127 - k);
+    return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+}
+
+// The dequant multiplier of an E8M0 byte: 2^(byte - 127) as an fp32 (byte 0
+// is the subnormal 2^-127), NaN for byte 0xFF.
+__device__ __forceinline__ float e8m0_to_float(uint32_t byte) {
+    if (byte == 0xFFu) return __uint_as_float(0x7FC00000u);
+    return byte == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(byte << 23);
+}
+
 // ---------------------------------------------------------------------------
 // casts
 // ---------------------------------------------------------------------------

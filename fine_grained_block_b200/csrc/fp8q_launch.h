@@ -23,9 +23,25 @@ cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fm
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                  uint8_t* q, float* scales, cudaStream_t stream);
 
+// MX: 1x32 blocks with power-of-two scales stored as E8M0 bytes
+// [rows, ceil(cols / 32)]; rule 0 = fit, 1 = OCP MX.
+cudaError_t launch_quant_mx(const void* x, int dtype, int64_t rows, int64_t cols, int fmt, int rule, uint8_t* q,
+                            uint8_t* e8m0, cudaStream_t stream);
+cudaError_t launch_dequant_mx(const uint8_t* q, int fmt, int64_t rows, int64_t cols, const uint8_t* e8m0, void* y,
+                              int out_dtype, cudaStream_t stream);
+
 // Delayed scaling with a margin and a choice of window max (algo 0) or EMA (algo 1).
 cudaError_t launch_amax_history_update_ex(float* history, int32_t* state, int window, const float* amax, int fmt,
                                           float* scale, int algo, float alpha, float margin, cudaStream_t stream);
+
+// FP8 GEMM with blockwise scales on the tcgen05 tensor cores:
+// C[M, N] = sum over 128-wide K chunks of (A_c B_c^T) / (sa * sb), A [M, K]
+// codes with 1x128 scales sa [M, K/128], B [N, K] codes with 128x128 scales
+// sb [N/128, K/128].  Needs N % 256 == 0, K % 128 == 0, K > 0.
+bool gemm_blockwise_supported();
+cudaError_t launch_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb,
+                                  int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
+                                  cudaStream_t stream);
 
 // Device address of the status word of the current device (nullptr on failure).
 unsigned int* device_status_word();
@@ -71,6 +87,12 @@ cudaError_t launch_tensor_cast(const void* x, int dtype, int64_t n, int fmt,
                                const float* scale_in, const float* amax_in,
                                uint8_t* q, float* scale_out, float* amax_out,
                                cudaStream_t stream);
+
+// Per-tensor cast with a transposed second output qt [cols, rows] (q [rows,
+// cols] optional).  Scale arguments as in launch_tensor_cast.
+cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
+                                         const float* scale_in, const float* amax_in, uint8_t* q, uint8_t* qt,
+                                         float* scale_out, float* amax_out, cudaStream_t stream);
 
 // Fused quantize -> dequantize round trip in x's dtype.  block_rows 0: per
 // tensor with *scale_in; 1 or 128: block scales (written to `scales` if it is

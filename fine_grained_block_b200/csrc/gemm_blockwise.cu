@@ -1,0 +1,285 @@
+// gemm_blockwise.cu -- the consumer of the blockwise codes: an FP8 GEMM on
+// the tcgen05 tensor cores with per-block scales applied in fp32.
+//
+// Mixed-precision handbook, section "FP8 training", closing notes: the
+// matrix products take FP8 inputs with fp32 accumulation, and because an FP8
+// tensor-core accumulator holds limited precision, every 128 products the
+// partial sum is promoted to CUDA cores and accumulated there in fp32; the
+// fine-grained scales (1x128 activations, 128x128 weights) are applied at that
+// promotion.  Here
+//     C[m][n] = sum over 128-wide K chunks c of
+//               P_c[m][n] / (sa[m][c] * sb[n/128][c]),
+//     P_c[m][n] = sum_{k in c} decode(A[m][k]) * decode(B[n][k]),
+// with A [M, K] the 1x128-scaled codes (scales sa [M, K/128]) and B [N, K]
+// the 128x128-scaled codes of a weight stored [out, in] (scales
+// sb [N/128, K/128]); both scales are the quantizers' multipliers, so each
+// promotion divides by them.
+//
+// One CTA computes a 128 x 256 tile of C (10 warps):
+//   warp 0    TMA producer: per K chunk, one 128x128-byte box of A and one
+//             256x128-byte box of B into a ring of kStages shared-memory
+//             stages (128-byte swizzle, the layout the MMA descriptors name);
+//   warp 1    allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
+//             issues the MMAs: per chunk, 4 x tcgen05.mma (M 128, N 256,
+//             K 32) into a fresh accumulator, then commits to the stage's
+//             "empty" barrier and the accumulator's "full" barrier;
+//   warps 2-9 the promotion: each thread owns one row (its TMEM lane) and 128
+//             columns; per chunk it loads its partial sums from TMEM, frees
+//             the accumulator, and adds partial * 1/(sa * sb) into 128 fp32
+//             registers.  The two accumulators alternate, so the MMAs of
+//             chunk c+1 run while chunk c is promoted.
+// At the end each promotion thread writes its 128 results (fp32 or bf16).
+// Rows past M arrive as zeros from the copy engine and are not stored.
+//
+// Every barrier wait is bounded (1 s); a wait that runs out sets the
+// wait-timeout bit of the device status word, and the CTA still waits
+// (bounded) for its MMAs before it frees its tensor memory.
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "fp8q_device.cuh"
+#include "fp8q_launch.h"
+#include "launch_util.h"
+#include "umma.cuh"
+
+namespace fp8q {
+namespace {
+
+constexpr int kBM = 128;                  // tile rows (MMA M)
+constexpr int kBN = 256;                  // tile columns (MMA N)
+constexpr int kBK = 128;                  // K chunk = one promotion = one stage
+constexpr int kMmaK = 32;                 // K of one kind::f8f6f4 instruction
+constexpr int kStages = 4;
+constexpr int kWarps = 10;
+constexpr int kThreads = kWarps * 32;
+constexpr int kABytes = kBM * kBK;        // 16 KiB
+constexpr int kBBytes = kBN * kBK;        // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTmemCols = 2 * kBN;   // two accumulators
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
+
+struct Barriers {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+};
+
+template <int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const float* __restrict__ sa, const float* __restrict__ sb, void* __restrict__ c, int64_t M,
+                 int64_t N, int64_t K, uint32_t idesc, unsigned int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Barriers* bars = reinterpret_cast<Barriers*>(tiles + kStages * kStageBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kBN;
+    const int nchunks = static_cast<int>(K / kBK);
+    const int64_t kc_stride = K / kBK;  // scales per row of sa / sb
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            umma::mbar_init(&bars->full[s], 1);
+            umma::mbar_init(&bars->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            umma::mbar_init(&bars->acc_full[b], 1);
+            umma::mbar_init(&bars->acc_empty[b], 8);  // one arrival per promotion warp
+        }
+        umma::mbar_init(&bars->mma_done, 1);
+        umma::fence_mbar_init();
+    }
+    if (warp == 1) umma::tmem_alloc(&bars->tmem_base, kTmemCols);
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+    pdl_enter();  // A, B and the scales may come from the previous kernel
+
+    bool timed_out = false;
+    if (warp == 0) {
+        // ---- TMA producer ----------------------------------------------------
+        if (lane == 0) {
+            for (int kc = 0; kc < nchunks; ++kc) {
+                const int s = kc % kStages;
+                const uint32_t phase = static_cast<uint32_t>(kc / kStages) & 1u;
+                if (!umma::mbar_wait(&bars->empty[s], phase ^ 1u, kWaitLimitNs)) {
+                    timed_out = true;
+                    break;
+                }
+                uint8_t* sa_tile = tiles + s * kStageBytes;
+                umma::mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
+                umma::tma_load_2d(sa_tile, &map_a, &bars->full[s], kc * kBK, static_cast<int>(m0));
+                umma::tma_load_2d(sa_tile + kABytes, &map_b, &bars->full[s], kc * kBK, static_cast<int>(n0));
+            }
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer ------------------------------------------------------
+        if (lane == 0) {
+            for (int kc = 0; kc < nchunks; ++kc) {
+                const int s = kc % kStages;
+                const uint32_t phase = static_cast<uint32_t>(kc / kStages) & 1u;
+                const int buf = kc & 1;
+                const uint32_t acc_phase = static_cast<uint32_t>(kc >> 1) & 1u;
+                if (!umma::mbar_wait(&bars->acc_empty[buf], acc_phase ^ 1u, kWaitLimitNs) ||
+                    !umma::mbar_wait(&bars->full[s], phase, kWaitLimitNs)) {
+                    timed_out = true;
+                    break;
+                }
+                umma::fence_after_sync();
+                const uint32_t a_addr = umma::smem_u32(tiles + s * kStageBytes);
+                const uint64_t a_desc = umma::smem_desc_kmajor_sw128(a_addr);
+                const uint64_t b_desc = umma::smem_desc_kmajor_sw128(a_addr + kABytes);
+                const uint32_t d = tmem + static_cast<uint32_t>(buf * kBN);
+#pragma unroll
+                for (int k = 0; k < kBK / kMmaK; ++k) {
+                    // the next 32 bytes of K: start address + 32 bytes (2 in 16-byte units)
+                    umma::mma_f8f6f4(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
+                }
+                umma::commit(&bars->empty[s]);
+                umma::commit(&bars->acc_full[buf]);
+            }
+            umma::commit(&bars->mma_done);
+            if (!umma::mbar_wait(&bars->mma_done, 0, kWaitLimitNs)) timed_out = true;
+        }
+    } else {
+        // ---- promotion warps -------------------------------------------------
+        const int quarter = warp & 3;            // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;        // column half of the tile
+        const int row = quarter * 32 + lane;     // tile row = TMEM lane
+        const int64_t m = m0 + row;
+        const float* sa_row = sa + (m < M ? m : 0) * kc_stride;
+        const float* sb_row = sb + ((n0 >> 7) + half) * kc_stride;
+        float acc[128];
+#pragma unroll
+        for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
+        for (int kc = 0; kc < nchunks; ++kc) {
+            const int buf = kc & 1;
+            const uint32_t acc_phase = static_cast<uint32_t>(kc >> 1) & 1u;
+            // 1 / (sa * sb): the dequant factor of this chunk for this row and column half
+            const float f = (m < M) ? __frcp_rn(__fmul_rn(__ldg(sa_row + kc), __ldg(sb_row + kc))) : 0.0f;
+            if (!umma::mbar_wait(&bars->acc_full[buf], acc_phase, kWaitLimitNs)) {
+                timed_out = true;
+                break;
+            }
+            umma::fence_after_sync();
+            const uint32_t t = t_lane + static_cast<uint32_t>(buf * kBN);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float p[32];
+                umma::tmem_ld32(t + h * 32, p);
+                umma::wait_ld(p);
+                if (h == 3) {
+                    // every partial sum of this buffer is in registers: hand it back
+                    umma::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) umma::mbar_arrive(&bars->acc_empty[buf]);
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc[h * 32 + j] = __fmaf_rn(p[j], f, acc[h * 32 + j]);
+            }
+        }
+        if (!timed_out && m < M) {
+            const int64_t col0 = n0 + half * 128;
+            if (OUT == 0) {
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(c) + m * N + col0);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(c) + m * N + col0);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    dst[j] = make_uint4(pack_bf16x2(acc[8 * j], acc[8 * j + 1]), pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
+                                        pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
+                                        pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+            }
+        }
+    }
+    if (timed_out) atomicOr(status, kStatusWaitTimeout);
+    umma::fence_before_sync();
+    if (__syncthreads_or(timed_out)) {
+        // A wait ran out: give copies that may still be landing in this
+        // CTA's shared memory time to finish (bounded) before it goes away.
+        if (threadIdx.x == 0) {
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 1000000ull) {
+            }
+        }
+        __syncthreads();
+    }
+    if (warp == 1) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult res;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &res) == cudaSuccess &&
+            res == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [rows, K] bytes, K-major, boxes of box_rows x 128 bytes with the 128-byte
+// swizzle; rows past the end read as zeros.
+bool make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+    auto encode = tensor_map_encoder();
+    if (encode == nullptr) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool gemm_blockwise_supported() { return tensor_map_encoder() != nullptr; }
+
+cudaError_t launch_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb,
+                                  int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
+                                  cudaStream_t st) {
+    CUtensorMap map_a, map_b;
+    if (!make_kmajor_map(&map_a, a, M, K, kBM) || !make_kmajor_map(&map_b, b, N, K, kBN))
+        return cudaErrorInvalidValue;
+    unsigned int* status = device_status_word();
+    if (status == nullptr) return cudaErrorInvalidValue;
+    const uint32_t idesc = umma::instr_desc_f8f6f4(a_fmt, b_fmt, kBM, kBN);
+    const dim3 grid(static_cast<unsigned>((M + kBM - 1) / kBM), static_cast<unsigned>(N / kBN));
+    auto kern = c_dtype == 0 ? k_gemm_blockwise<0> : k_gemm_blockwise<1>;
+    // The shared-memory opt-in, once per device and output type (not inside
+    // a stream capture on later calls).
+    static std::atomic<bool> opted[128][2];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    if (!opted[dev][c_dtype ? 1 : 0].load(std::memory_order_acquire)) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        opted[dev][c_dtype ? 1 : 0].store(true, std::memory_order_release);
+    }
+    return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, st, map_a, map_b, sa, sb, c, M, N, K, idesc,
+                         status);
+}
+
+}  // namespace fp8q

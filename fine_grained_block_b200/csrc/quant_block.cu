@@ -22,24 +22,49 @@ constexpr int kThreads = 256;
 #ifndef FP8Q_Q1X128_LOADS
 #define FP8Q_Q1X128_LOADS 4
 #endif
+// The same for the 1x32 MX kernel.
+#ifndef FP8Q_QMX_LOADS
+#define FP8Q_QMX_LOADS 4
+#endif
+
+// Scale rules of the row-block kernel: how a block's amax becomes its scale
+// and what is stored for it.
+template <int FMT>
+struct RatioScale {  // handbook per_block: s = MAX / max(amax, eps), stored as fp32
+    using Stored = float;
+    static __device__ __forceinline__ float scale(float amax, int, Stored& stored) {
+        const float s = scale_from_amax<FMT>(amax);
+        stored = s;
+        return s;
+    }
+};
+template <int FMT>
+struct Pow2Scale {  // MX: s = 2^k, stored as the E8M0 byte of 2^-k
+    using Stored = uint8_t;
+    static __device__ __forceinline__ float scale(float amax, int rule, Stored& stored) {
+        return mx_scale<FMT>(amax, rule, stored);
+    }
+};
 
 // ---------------------------------------------------------------------------
-// 1x128: a block is 128 consecutive elements.  One lane holds a 16- or 32-byte
-// slice, so a block spans 128 / kElems lanes (8 lanes for bf16 with 32-byte
-// slices) and one warp-wide load covers 32 / that many whole blocks.  The
-// block amax is a shuffle reduction inside the lane group -- no shared
-// memory, no block barrier.  Each CTA owns one contiguous chunk: every warp
-// issues all LOADS of its warp-loads before it computes, and finished CTAs are
-// replaced by new ones, so each SM keeps its resident CTAs' chunks in flight.
+// Row blocks (1x128, and the 1x32 MX blocks): a block is BW consecutive
+// elements.  One lane holds a 16- or 32-byte slice, so a block spans
+// BW / kElems lanes (8 lanes for bf16 1x128 with 32-byte slices, 2 for MX) and
+// one warp-wide load covers 32 / that many whole blocks.  The block amax is a
+// shuffle reduction inside the lane group -- no shared memory, no block
+// barrier.  Each CTA owns one contiguous chunk: every warp issues all LOADS of
+// its warp-loads before it computes, and finished CTAs are replaced by new
+// ones, so each SM keeps its resident CTAs' chunks in flight.
 // ---------------------------------------------------------------------------
-template <typename T, int FMT, int BYTES, int LOADS>
+template <typename T, int FMT, int BYTES, int LOADS, int BW, typename SCALE>
 __global__ void __launch_bounds__(kThreads)
-k_quant_1x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
-              float* __restrict__ scales, int64_t nblocks) {
+k_quant_rowblocks(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
+                  typename SCALE::Stored* __restrict__ scales, int64_t nblocks, int rule) {
     pdl_enter();
     using V = LaneVec<T, BYTES>;
-    constexpr int kLanesPerBlock = 128 / V::kElems;
+    constexpr int kLanesPerBlock = BW / V::kElems;
     constexpr int kBlocksPerLoad = 32 / kLanesPerBlock;
+    static_assert(kLanesPerBlock >= 1 && kLanesPerBlock <= 32, "a block spans 1..32 lanes");
     const int lane = threadIdx.x & 31;
     const int sub_block = lane / kLanesPerBlock;
     const int64_t nloads = (nblocks + kBlocksPerLoad - 1) / kBlocksPerLoad;
@@ -57,10 +82,11 @@ k_quant_1x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename Lan
         const int64_t l = l0 + u;
         const int64_t blk = l * kBlocksPerLoad + sub_block;
         const float amax = warp_max<kLanesPerBlock>(V::amax(v[u]));
-        const float s = scale_from_amax<FMT>(amax);
+        typename SCALE::Stored stored;
+        const float s = SCALE::scale(amax, rule, stored);
         if (l < nloads && blk < nblocks) {
             st_stream(q + l * 32 + lane, V::template cast<FMT>(v[u], f32x2(s, s)));
-            if ((lane % kLanesPerBlock) == 0) scales[blk] = s;
+            if ((lane % kLanesPerBlock) == 0) scales[blk] = stored;
         }
     }
 }
@@ -174,19 +200,54 @@ k_quant_block_general(const T* __restrict__ x, uint8_t* __restrict__ q, float* _
     }
 }
 
-template <typename T, int FMT, int BYTES, int LOADS>
-cudaError_t launch_1x128_typed(const void* x, int64_t nblocks, uint8_t* q, float* scales, cudaStream_t st) {
+// MX blocks over any cols (ragged right edge): one warp per 1x32 block, lane
+// i holding element i of the block; blocks are taken warp-stride.
+template <typename T, int FMT>
+__global__ void __launch_bounds__(kGeneralThreads)
+k_quant_mx_general(const T* __restrict__ x, uint8_t* __restrict__ q, uint8_t* __restrict__ e8m0, int64_t rows,
+                   int64_t cols, int64_t nblocks, int rule) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const int64_t nbc = (cols + 31) / 32;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kGeneralThreads / 32);
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * (kGeneralThreads / 32) + (threadIdx.x >> 5); b < nblocks;
+         b += warps) {
+        const int64_t r = b / nbc, c = (b - r * nbc) * 32 + lane;
+        const bool in = c < cols;
+        const float v = in ? load_elem(x, r * cols + c) : 0.0f;
+        const float amax = warp_max<32>(fabsf(v));
+        uint8_t byte;
+        const float s = mx_scale<FMT>(amax, rule, byte);
+        if (in) q[r * cols + c] = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(v, s), 0.0f) & 0xFFu);
+        if (lane == 0) e8m0[b] = byte;
+    }
+}
+
+template <typename T, int FMT, int BYTES, int LOADS, int BW, typename SCALE>
+cudaError_t launch_rowblocks_typed(const void* x, int64_t nblocks, uint8_t* q, typename SCALE::Stored* scales,
+                                   int rule, cudaStream_t st) {
     using V = LaneVec<T, BYTES>;
-    constexpr int kBlocksPerLoad = 32 / (128 / V::kElems);
+    constexpr int kBlocksPerLoad = 32 / (BW / V::kElems);
     const int64_t nloads = (nblocks + kBlocksPerLoad - 1) / kBlocksPerLoad;
     const int64_t per_cta = static_cast<int64_t>(kThreads / 32) * LOADS;
     const int64_t grid = (nloads + per_cta - 1) / per_cta;
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    {
-        const cudaError_t e_ = launch_kernel(k_quant_1x128<T, FMT, BYTES, LOADS>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st, static_cast<const typename V::In*>(x), reinterpret_cast<typename V::Out*>(q), scales, nblocks);
-        if (e_ != cudaSuccess) return e_;
-    }
+    const cudaError_t e = launch_kernel(k_quant_rowblocks<T, FMT, BYTES, LOADS, BW, SCALE>,
+                                        dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, st,
+                                        static_cast<const typename V::In*>(x), reinterpret_cast<typename V::Out*>(q),
+                                        scales, nblocks, rule);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+template <typename T, int FMT, int BYTES, int LOADS>
+cudaError_t launch_1x128_typed(const void* x, int64_t nblocks, uint8_t* q, float* scales, cudaStream_t st) {
+    return launch_rowblocks_typed<T, FMT, BYTES, LOADS, 128, RatioScale<FMT>>(x, nblocks, q, scales, 0, st);
+}
+
+template <typename T, int FMT, int BYTES>
+cudaError_t launch_mx_typed(const void* x, int64_t nblocks, uint8_t* q, uint8_t* e8m0, int rule, cudaStream_t st) {
+    return launch_rowblocks_typed<T, FMT, BYTES, FP8Q_QMX_LOADS, 32, Pow2Scale<FMT>>(x, nblocks, q, e8m0, rule, st);
 }
 
 template <typename T, int FMT, int BYTES>
@@ -260,6 +321,41 @@ cudaError_t launch_quant_block_general(const void* x, int dtype, int64_t rows, i
     }
     return fmt == kE4M3 ? launch_general_typed<float, kE4M3>(x, rows, cols, br, bc, q, scales, st)
                         : launch_general_typed<float, kE5M2>(x, rows, cols, br, bc, q, scales, st);
+}
+
+cudaError_t launch_quant_mx(const void* x, int dtype, int64_t rows, int64_t cols, int fmt, int rule, uint8_t* q,
+                            uint8_t* e8m0, cudaStream_t st) {
+    if (cols % 32 != 0) {
+        const int64_t nblocks = rows * ((cols + 31) / 32);
+        const int64_t grid = std::max<int64_t>(
+            1, std::min<int64_t>((nblocks + kGeneralThreads / 32 - 1) / (kGeneralThreads / 32),
+                                 static_cast<int64_t>(device_sm_count()) * 16));
+        auto go = [&](auto kern, auto* xt) -> cudaError_t {
+            const cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kGeneralThreads), 0, st,
+                                                xt, q, e8m0, rows, cols, nblocks, rule);
+            return e != cudaSuccess ? e : cudaGetLastError();
+        };
+        if (dtype == 1) {
+            const auto* xt = static_cast<const uint16_t*>(x);
+            return fmt == kE4M3 ? go(k_quant_mx_general<uint16_t, kE4M3>, xt) : go(k_quant_mx_general<uint16_t, kE5M2>, xt);
+        }
+        const auto* xt = static_cast<const float*>(x);
+        return fmt == kE4M3 ? go(k_quant_mx_general<float, kE4M3>, xt) : go(k_quant_mx_general<float, kE5M2>, xt);
+    }
+    const int64_t nblocks = rows * (cols / 32);
+    const bool w32 = aligned32(x);
+    if (dtype == 1) {
+        if (w32)
+            return fmt == kE4M3 ? launch_mx_typed<uint16_t, kE4M3, 32>(x, nblocks, q, e8m0, rule, st)
+                                : launch_mx_typed<uint16_t, kE5M2, 32>(x, nblocks, q, e8m0, rule, st);
+        return fmt == kE4M3 ? launch_mx_typed<uint16_t, kE4M3, 16>(x, nblocks, q, e8m0, rule, st)
+                            : launch_mx_typed<uint16_t, kE5M2, 16>(x, nblocks, q, e8m0, rule, st);
+    }
+    if (w32)
+        return fmt == kE4M3 ? launch_mx_typed<float, kE4M3, 32>(x, nblocks, q, e8m0, rule, st)
+                            : launch_mx_typed<float, kE5M2, 32>(x, nblocks, q, e8m0, rule, st);
+    return fmt == kE4M3 ? launch_mx_typed<float, kE4M3, 16>(x, nblocks, q, e8m0, rule, st)
+                        : launch_mx_typed<float, kE5M2, 16>(x, nblocks, q, e8m0, rule, st);
 }
 
 }  // namespace fp8q

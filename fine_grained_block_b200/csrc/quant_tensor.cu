@@ -118,6 +118,100 @@ k_tensor_cast(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
 }
 
+// ---------------------------------------------------------------------------
+// Per-tensor cast with a second, transposed output: q [R, C] (optional) and
+// qt [C, R] with qt[c][r] = q[r][c] -- the copy a weight-gradient GEMM reads
+// along the other dimension.  One CTA per 128x128 tile: the tile's codes go
+// through shared memory so that both outputs are written row by row.
+// DELAYED / WITH_AMAX as in k_tensor_cast.
+//
+// Full tiles with vector-friendly strides (FAST) load one lane vector per
+// slice, 16 rows per warp, as the 128x128 block kernel does; each lane then
+// builds 32 consecutive codes of one qt row from one byte per tile row (the
+// 32 lanes of a warp read 32 consecutive bytes of a smem row: no bank
+// conflicts).  Edge tiles and other strides take an element-wise path.
+// ---------------------------------------------------------------------------
+constexpr int kTT = 128;           // tile side
+constexpr int kTStride = kTT + 16;  // smem row pitch in bytes (16-byte aligned rows)
+
+template <typename T, int FMT, int BYTES, bool DELAYED, bool WITH_AMAX>
+__global__ void __launch_bounds__(kThreads)
+k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, const float* scale_in,
+                        const float* __restrict__ amax_in, uint8_t* __restrict__ q, uint8_t* __restrict__ qt,
+                        float* scale_out, float* __restrict__ amax_out, int vector_ok) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    __shared__ __align__(16) uint8_t tile[kTT * kTStride];
+    const int64_t tiles_c = (cols + kTT - 1) / kTT;
+    const int64_t tr = blockIdx.x / tiles_c;
+    const int64_t tc = blockIdx.x - tr * tiles_c;
+    const int64_t r0 = tr * kTT, c0 = tc * kTT;
+    const int h = static_cast<int>(min(static_cast<int64_t>(kTT), rows - r0));
+    const int w = static_cast<int>(min(static_cast<int64_t>(kTT), cols - c0));
+    const float s = DELAYED ? *scale_in : scale_from_amax<FMT>(*amax_in);
+    const uint64_t s2 = f32x2(s, s);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float a = 0.0f;
+
+    if (vector_ok && h == kTT && w == kTT) {
+        constexpr int kVecPerRow = kTT / V::kElems;
+        constexpr int kRowsPerLoad = 32 / kVecPerRow;
+        constexpr int kLoads = 16 / kRowsPerLoad;
+        const int row_in_load = lane / kVecPerRow, vec_in_row = lane % kVecPerRow;
+        const int lr0 = warp * 16 + row_in_load;
+        const auto* xv = reinterpret_cast<const typename V::In*>(x + (r0 + lr0) * cols + c0) + vec_in_row;
+        const int64_t vstride = cols / V::kElems * kRowsPerLoad;  // lane vectors between this lane's rows
+        typename V::In v[kLoads];
+#pragma unroll
+        for (int i = 0; i < kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
+#pragma unroll
+        for (int i = 0; i < kLoads; ++i) {
+            if (WITH_AMAX) a = fmaxf(a, V::amax(v[i]));
+            const typename V::Out c = V::template cast<FMT>(v[i], s2);
+            const int lr = lr0 + i * kRowsPerLoad;
+            if (q != nullptr)
+                st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row, c);
+            *reinterpret_cast<typename V::Out*>(tile + lr * kTStride + vec_in_row * V::kElems) = c;
+        }
+        __syncthreads();
+        // qt: 128 rows (tile columns) x 4 runs of 32 codes; 2 runs per thread
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int task = p * kThreads + threadIdx.x;
+            const int c = task % kTT, run = task / kTT;
+            uint32_t wd[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint8_t* col = tile + (run * 32 + 4 * k) * kTStride + c;
+                wd[k] = static_cast<uint32_t>(col[0]) | (static_cast<uint32_t>(col[kTStride]) << 8) |
+                        (static_cast<uint32_t>(col[2 * kTStride]) << 16) |
+                        (static_cast<uint32_t>(col[3 * kTStride]) << 24);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(qt + (c0 + c) * rows + r0 + run * 32);
+            st_stream(dst, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+            st_stream(dst + 1, make_uint4(wd[4], wd[5], wd[6], wd[7]));
+        }
+    } else {
+        for (int i = threadIdx.x; i < kTT * kTT; i += kThreads) {
+            const int r = i / kTT, c = i % kTT;
+            if (r < h && c < w) {
+                const float xv = load_scalar(x + (r0 + r) * cols + c0, c);
+                if (WITH_AMAX) a = fmaxf(a, fabsf(xv));
+                const uint8_t code = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(xv, s), 0.0f) & 0xFFu);
+                if (q != nullptr) q[(r0 + r) * cols + c0 + c] = code;
+                tile[r * kTStride + c] = code;
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < kTT * kTT; i += kThreads) {
+            const int c = i / kTT, r = i % kTT;
+            if (r < h && c < w) qt[(c0 + c) * rows + r0 + r] = tile[r * kTStride + c];
+        }
+    }
+    if (WITH_AMAX) cta_amax_to_global(a, amax_out);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+}
+
 template <int FMT>
 __global__ void k_scale_from_amax(const float* amax_in, float* scale_out) {
     pdl_enter();
@@ -183,7 +277,62 @@ cudaError_t cast_width(const void* x, int64_t n, const float* scale_in, const fl
     return cast_dispatch<T, FMT, 16>(x, n, scale_in, amax_in, q, scale_out, amax_out, st);
 }
 
+template <typename T, int FMT, int BYTES, bool DELAYED, bool WITH_AMAX>
+cudaError_t cast_transpose_typed(const void* x, int64_t rows, int64_t cols, const float* scale_in,
+                                 const float* amax_in, uint8_t* q, uint8_t* qt, float* scale_out, float* amax_out,
+                                 int vector_ok, cudaStream_t st) {
+    const int64_t tiles = ((rows + kTT - 1) / kTT) * ((cols + kTT - 1) / kTT);
+    if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const cudaError_t e = launch_kernel(k_tensor_cast_transpose<T, FMT, BYTES, DELAYED, WITH_AMAX>,
+                                        dim3(static_cast<unsigned>(tiles)), dim3(kThreads), 0, st,
+                                        static_cast<const T*>(x), rows, cols, scale_in, amax_in, q, qt, scale_out,
+                                        amax_out, vector_ok);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <typename T, int FMT, int BYTES>
+cudaError_t cast_transpose_mode(const void* x, int64_t rows, int64_t cols, const float* scale_in,
+                                const float* amax_in, uint8_t* q, uint8_t* qt, float* scale_out, float* amax_out,
+                                int vector_ok, cudaStream_t st) {
+    if (scale_in == nullptr)
+        return cast_transpose_typed<T, FMT, BYTES, false, false>(x, rows, cols, nullptr, amax_in, q, qt, scale_out,
+                                                                 nullptr, vector_ok, st);
+    if (amax_out != nullptr)
+        return cast_transpose_typed<T, FMT, BYTES, true, true>(x, rows, cols, scale_in, nullptr, q, qt, scale_out,
+                                                               amax_out, vector_ok, st);
+    return cast_transpose_typed<T, FMT, BYTES, true, false>(x, rows, cols, scale_in, nullptr, q, qt, scale_out,
+                                                            nullptr, vector_ok, st);
+}
+
+template <typename T, int FMT>
+cudaError_t cast_transpose_width(const void* x, int64_t rows, int64_t cols, const float* scale_in,
+                                 const float* amax_in, uint8_t* q, uint8_t* qt, float* scale_out, float* amax_out,
+                                 cudaStream_t st) {
+    // Vector path: every tile row starts on a 32-byte (else 16-byte) boundary
+    // of x and a 16-byte boundary of q, and every qt run of 32 codes on a
+    // 16-byte boundary.
+    const int64_t rb = cols * static_cast<int64_t>(sizeof(T));
+    const bool ok16 = (rb % 16 == 0) && (cols % 16 == 0) && (rows % 16 == 0);
+    if (ok16 && aligned32(x) && rb % 32 == 0)
+        return cast_transpose_mode<T, FMT, 32>(x, rows, cols, scale_in, amax_in, q, qt, scale_out, amax_out, 1, st);
+    return cast_transpose_mode<T, FMT, 16>(x, rows, cols, scale_in, amax_in, q, qt, scale_out, amax_out,
+                                           ok16 ? 1 : 0, st);
+}
+
 }  // namespace
+
+cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
+                                         const float* scale_in, const float* amax_in, uint8_t* q, uint8_t* qt,
+                                         float* scale_out, float* amax_out, cudaStream_t st) {
+    if (dtype == 1) {
+        return fmt == kE4M3
+                   ? cast_transpose_width<uint16_t, kE4M3>(x, rows, cols, scale_in, amax_in, q, qt, scale_out, amax_out, st)
+                   : cast_transpose_width<uint16_t, kE5M2>(x, rows, cols, scale_in, amax_in, q, qt, scale_out, amax_out, st);
+    }
+    return fmt == kE4M3
+               ? cast_transpose_width<float, kE4M3>(x, rows, cols, scale_in, amax_in, q, qt, scale_out, amax_out, st)
+               : cast_transpose_width<float, kE5M2>(x, rows, cols, scale_in, amax_in, q, qt, scale_out, amax_out, st);
+}
 
 cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_out, cudaStream_t st) {
     if (dtype == 1)

@@ -234,6 +234,103 @@ int fp8_fake_quantize(const void *x, int dtype, int64_t rows, int64_t cols,
                       void *stream);
 
 /*
+ * Per-tensor quantization with a second, transposed copy of the codes:
+ * qt[c][r] = q[r][c], for a consumer that reads the tensor along its other
+ * dimension (the weight-gradient GEMM reads activations and output gradients
+ * transposed).  Scaling exactly as fp8_quantize_per_tensor ([MP-handbook]
+ * per_tensor; [FP8-native] s4.1-4.2, current or delayed): with one scale for
+ * the whole tensor the transposed codes are the same codes, moved.
+ *
+ *   x          [rows, cols] input, FP8_F32 or FP8_BF16
+ *   scale_in   NULL: current scaling (amax pass, then the cast); else the
+ *              delayed scale (device fp32), one pass
+ *   q          [rows, cols] codes, or NULL to write only qt
+ *   qt         [cols, rows] codes (required)
+ *   scale_out, amax_out   as in fp8_quantize_per_tensor
+ * Tiles of 128x128 go through shared memory; rows % 16 == 0 and
+ * cols % 16 == 0 take the vectorised path for full tiles, everything else an
+ * element-wise path with the same results.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN (x, q, qt: 16 bytes),
+ * FP8_ERR_FORMAT, FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_quantize_per_tensor_transpose(const void *x, int dtype, int64_t rows, int64_t cols,
+                                      int fmt, const float *scale_in, uint8_t *q,
+                                      uint8_t *qt, float *scale_out, float *amax_out,
+                                      void *stream);
+
+/*
+ * MX quantization: blocks of 32 consecutive elements of a row share one
+ * power-of-two scale.  Follows [MP-handbook] "FP8 training", closing notes
+ * (Blackwell's MX formats, MXFP8: every 32 elements share a scale factor in
+ * hardware).  For each block, s = 2^k and q = fp8(RN_f32(x * s)); the scale
+ * is stored as the E8M0 byte 127 - k, i.e. the exponent of the dequant
+ * multiplier 2^-k (the MX shared-scale encoding, bias 127, 0xFF = NaN).
+ *
+ *   x          [rows, cols] input, FP8_F32 or FP8_BF16
+ *   rule       FP8_MX_FIT: the largest k with max(amax, 1e-12f) * 2^k <= MAX
+ *              (the pages' MAX / amax rounded down to a power of two; no
+ *              element saturates).  FP8_MX_OCP: k = emax - floor(log2(
+ *              max(amax, 1e-12f))) with emax 8 (E4M3) or 15 (E5M2), the OCP
+ *              MX rule; elements in the top of a binade may saturate.
+ *   q          [rows, cols] output codes
+ *   e8m0       [rows, ceil(cols / 32)] uint8, row-major (no alignment rule)
+ * A block holding +-Inf gets the byte 0xFF and k = 0 for its elements.  NaN
+ * elements do not count toward amax.  Ragged right edge: the last block of
+ * a row holds cols % 32 elements.  cols % 32 == 0 takes the vectorised
+ * kernel; other widths a slower kernel with the same results.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN (x, q: 16 bytes),
+ * FP8_ERR_FORMAT, FP8_ERR_DTYPE, FP8_ERR_ARG (unknown rule), FP8_ERR_CUDA.
+ */
+enum fp8_mx_rule { FP8_MX_FIT = 0, FP8_MX_OCP = 1 };
+int fp8_quantize_mx(const void *x, int dtype, int64_t rows, int64_t cols,
+                    int fmt, int rule, uint8_t *q, uint8_t *e8m0, void *stream);
+
+/*
+ * MX dequantization: y = RN_f32(decode(q) * 2^(e8m0 - 127)) with the byte of
+ * q's block (the layout of fp8_quantize_mx); byte 0xFF gives NaN.  For bytes
+ * made by fp8_quantize_mx this is the real quotient decode(q) / s, so it is
+ * exact except where it leaves the fp32 range.  bf16 output is that fp32
+ * rounded to nearest-even.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN (q, y: 16 bytes),
+ * FP8_ERR_FORMAT, FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_dequantize_mx(const uint8_t *q, int fmt, int64_t rows, int64_t cols,
+                      const uint8_t *e8m0, void *y, int out_dtype, void *stream);
+
+/*
+ * The consumer of the blockwise codes: an FP8 GEMM on the tensor cores with
+ * the fine-grained scales applied in fp32 every 128 products.  Follows
+ * [MP-handbook] "FP8 training", closing notes (FP8 inputs, fp32 accumulation;
+ * the FP8 accumulator is promoted to CUDA cores every 128 elements, where the
+ * 1x128 / 128x128 scales are applied):
+ *     C[m][n] = sum over K chunks c of 128:
+ *               (sum_{k in c} decode(a[m][k]) * decode(b[n][k])) / (sa[m][c] * sb[n/128][c])
+ *
+ *   a, a_fmt   [M, K] codes, row-major (K contiguous): an activation
+ *              quantized with 1x128 blocks (fp8_quantize_blockwise)
+ *   sa         [M, K/128] fp32 scales of a (the quantizer's multipliers)
+ *   b, b_fmt   [N, K] codes, row-major: a weight stored [out, in], quantized
+ *              with 128x128 blocks
+ *   sb         [N/128, K/128] fp32 scales of b
+ *   c, c_dtype [M, N] output, FP8_F32 or FP8_BF16 (the fp32 sum rounded to
+ *              nearest-even)
+ * The per-chunk products run on tcgen05 tensor cores (kind::f8f6f4, fp32
+ * accumulator in tensor memory); each chunk's partial sum is multiplied by
+ * RN(1 / RN(sa * sb)) and added in fp32 (fma).  Results agree with the exact
+ * sum within the accumulation error of that arithmetic (not bit-exact: the
+ * tensor cores' summation order is theirs).
+ * Shapes: N % 256 == 0 and K % 128 == 0 (else FP8_ERR_SHAPE); any M.  K == 0
+ * writes zeros.  M, N, K < 2^31.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE, FP8_ERR_ALIGN (a, b, c: 16 bytes;
+ * sa, sb: 4), FP8_ERR_FORMAT, FP8_ERR_DTYPE, FP8_ERR_CUDA (also when the
+ * driver offers no tensor-map encoder).
+ */
+int fp8_gemm_blockwise(const uint8_t *a, const float *sa, int a_fmt,
+                       const uint8_t *b, const float *sb, int b_fmt,
+                       int64_t M, int64_t N, int64_t K,
+                       void *c, int c_dtype, void *stream);
+
+/*
  * Delayed scaling: push one amax into the amax history and refresh the scale.
  * Follows [FP8-native] s4.2 DelayedScaler.update: the last `window` amax
  * values are kept; once `window` of them have been seen, the scale becomes

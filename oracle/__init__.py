@@ -62,6 +62,11 @@ def lib() -> ctypes.CDLL:
         L.orc_amax_history_update_ex.argtypes = [c_void, c_void, c_int, ctypes.c_float, c_int, c_void, c_int,
                                                  ctypes.c_float, ctypes.c_float]
         L.orc_amax_history_update_ex.restype = c_int
+        L.orc_quantize_per_tensor_transpose.argtypes = [c_void, c_int, c_i64, c_i64, c_int, c_void, c_void, c_void,
+                                                        c_void, c_void]
+        L.orc_quantize_per_tensor_transpose.restype = c_int
+        L.orc_gemm_blockwise.argtypes = [c_void, c_void, c_int, c_void, c_void, c_int, c_i64, c_i64, c_i64, c_void]
+        L.orc_gemm_blockwise.restype = c_int
         L.orc_mx_exponent.argtypes = [ctypes.c_float, c_int, c_int]
         L.orc_mx_exponent.restype = c_int
         L.orc_quantize_mx.argtypes = [c_void, c_int, c_i64, c_i64, c_int, c_int, c_void, c_void]
@@ -154,6 +159,22 @@ def quantize_per_tensor(x: np.ndarray, fmt: int, scale: float | None = None):
     return q, s_out[0], a_out[0]
 
 
+def quantize_per_tensor_transpose(x: np.ndarray, fmt: int, scale: float | None = None):
+    """Per-tensor quantize of a 2-D array with a transposed copy: (q [R, C], qt [C, R], scale, amax)."""
+    x, dt = _as_input(x)
+    if x.ndim != 2:
+        raise ValueError("the transposing quantize takes a 2-D array")
+    R, C = x.shape
+    q = np.empty((R, C), dtype=np.uint8)
+    qt = np.empty((C, R), dtype=np.uint8)
+    s_out = np.zeros(1, dtype=np.float32)
+    a_out = np.zeros(1, dtype=np.float32)
+    s_in = None if scale is None else np.array([scale], dtype=np.float32)
+    _check(lib().orc_quantize_per_tensor_transpose(_ptr(x), dt, R, C, fmt, None if s_in is None else _ptr(s_in),
+                                                   _ptr(q), _ptr(qt), _ptr(s_out), _ptr(a_out)))
+    return q, qt, s_out[0], a_out[0]
+
+
 def quantize_blockwise(x: np.ndarray, br: int, bc: int, fmt: int):
     """Blockwise quantize of a 2-D array.  Returns (codes, scales [ceil(R/br), ceil(C/bc)])."""
     x, dt = _as_input(x)
@@ -200,6 +221,22 @@ def fake_quantize(x: np.ndarray, fmt: int, br: int = 1, bc: int = 128, scale: fl
         q, scales = quantize_blockwise(x if x.ndim == 2 else x.reshape(1, -1), br, bc, fmt)
     y = dequantize(q.reshape(x.shape) if x.ndim == 2 else q.reshape(1, -1), fmt, scales, br, bc, out_dtype=dt)
     return y.reshape(x.shape), scales
+
+
+def gemm_blockwise(a: np.ndarray, sa: np.ndarray, a_fmt: int, b: np.ndarray, sb: np.ndarray, b_fmt: int):
+    """C [M, N] (float64) = sum over 128-wide K chunks of (dec(a) dec(b)^T) / (sa * sb)."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    M, K = a.shape
+    N = b.shape[0]
+    nkc = math.ceil(K / 128)
+    if b.shape[1] != K or sa.shape != (M, nkc) or sb.shape != (math.ceil(N / 128), nkc):
+        raise ValueError("gemm_blockwise: inconsistent shapes")
+    c = np.empty((M, N), dtype=np.float64)
+    _check(lib().orc_gemm_blockwise(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_fmt, M, N, K, _ptr(c)))
+    return c
 
 
 MX_FIT, MX_OCP = 0, 1

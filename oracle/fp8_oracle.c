@@ -42,6 +42,9 @@
  *       to fp32; the scale follows from m once `window` updates are in.
  *   R16 MX blocks: scale 2^k, k by the fit rule or the OCP MX rule (below).
  *   R17 An MX block with an infinite amax gets the NaN scale byte.
+ *   R18 The transposed per-tensor output holds the same codes as q.
+ *   R19 The consumer GEMM divides each 128-chunk partial sum by the two
+ *       block scales (the quantizers' multipliers).
  */
 #include <math.h>
 #include <stdint.h>
@@ -272,6 +275,22 @@ int orc_quantize_per_tensor(const void *x, int dtype, int64_t n, int fmt,
     for (int64_t i = 0; i < n; ++i) q[i] = scaled_code(load_elem(x, dtype, i), s, fmt);
     if (scale_out) *scale_out = s;
     if (amax_out) *amax_out = amax;
+    return ORC_OK;
+}
+
+/* Per-tensor scaling with a transposed second output: qt[c][r] = q[r][c]
+ * (x is [rows, cols] row-major, qt is [cols, rows] row-major).  One scale for
+ * the whole tensor, so the transposed codes are the same codes in the other
+ * order; reading R18: nothing else changes. */
+int orc_quantize_per_tensor_transpose(const void *x, int dtype, int64_t rows, int64_t cols, int fmt,
+                                      const float *scale_in, uint8_t *q, uint8_t *qt,
+                                      float *scale_out, float *amax_out)
+{
+    if (rows < 0 || cols < 0) return ORC_EBADARG;
+    const int rc = orc_quantize_per_tensor(x, dtype, rows * cols, fmt, scale_in, q, scale_out, amax_out);
+    if (rc != ORC_OK) return rc;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) qt[c * rows + r] = q[r * cols + c];
     return ORC_OK;
 }
 
@@ -507,6 +526,41 @@ int orc_dequantize_mx(const uint8_t *q, int fmt, int64_t rows, int64_t cols, con
             const float out = (float)(orc_fp8_decode(q[i], fmt) * xs);
             if (out_dtype == ORC_F32) ((float *)y)[i] = out;
             else ((uint16_t *)y)[i] = orc_f32_to_bf16(out);
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Consumer: blockwise-scaled FP8 GEMM                                 */
+/* ------------------------------------------------------------------ */
+
+/* [MP-handbook] "FP8 training", closing notes: FP8 inputs with fp32
+ * accumulation; the tensor-core partial sum is promoted every 128 elements,
+ * where the 1x128 (activation) and 128x128 (weight) scales are applied.
+ * Reading R19: with the quantizers' multiplier scales,
+ *   C[m][n] = sum over chunks c of (sum_{k in c} decode(a[m][k]) *
+ *             decode(b[n][k])) / (sa[m][c] * sb[n/128][c]).
+ * a [M, K], b [N, K] row-major codes; sa [M, ceil(K/128)],
+ * sb [ceil(N/128), ceil(K/128)]; c [M, N] in double.  Each product of two
+ * FP8 values is exact in double, the chunk sums and the quotient are rounded
+ * in double only: the result is the real value to within a few double ulps. */
+int orc_gemm_blockwise(const uint8_t *a, const float *sa, int a_fmt, const uint8_t *b, const float *sb,
+                       int b_fmt, int64_t M, int64_t N, int64_t K, double *c)
+{
+    if (!fmt_ok(a_fmt) || !fmt_ok(b_fmt) || M < 0 || N < 0 || K < 0) return ORC_EBADARG;
+    const int64_t nkc = (K + 127) / 128;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t kc = 0; kc < nkc; ++kc) {
+                const int64_t k0 = kc * 128, k1 = (k0 + 128 < K) ? k0 + 128 : K;
+                double p = 0.0;
+                for (int64_t k = k0; k < k1; ++k)
+                    p += orc_fp8_decode(a[m * K + k], a_fmt) * orc_fp8_decode(b[n * K + k], b_fmt);
+                acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / 128) * nkc + kc]);
+            }
+            c[m * N + n] = acc;
         }
     }
     return ORC_OK;

@@ -99,6 +99,23 @@ def oracle_dequant(q: np.ndarray, fmt: int, scales: np.ndarray, br: int, bc: int
     return np.concatenate(parts)
 
 
+def oracle_mx(x: np.ndarray, fmt: int, rule: int):
+    """oracle.quantize_mx in row chunks: (codes, e8m0)."""
+    R, C = x.shape
+    chunks = _row_chunks(R, 1)
+    parts = list(_pool.map(lambda rc: oracle.quantize_mx(x[rc[0]:rc[1]], fmt, rule), chunks))
+    if not parts:
+        return np.zeros((R, C), np.uint8), np.zeros((0, math.ceil(C / 32)), np.uint8)
+    return np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts])
+
+
+def oracle_dequant_mx(q: np.ndarray, fmt: int, e8m0: np.ndarray, out_dtype: int):
+    chunks = _row_chunks(q.shape[0], 1)
+    parts = list(_pool.map(lambda rc: oracle.dequantize_mx(q[rc[0]:rc[1]], fmt, e8m0[rc[0]:rc[1]], out_dtype),
+                           chunks))
+    return np.concatenate(parts)
+
+
 def _nan_mask(bits: np.ndarray, kind: str) -> np.ndarray:
     if kind == "f32":
         return ((bits & 0x7F800000) == 0x7F800000) & ((bits & 0x007FFFFF) != 0)

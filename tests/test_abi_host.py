@@ -34,7 +34,8 @@ def test_header_declares_the_boundary():
                                            "fp8_fake_quantize", "fp8_amax", "fp8_scale_from_amax",
                                            "fp8_quantize_per_tensor_fused",
                                            "fp8_quantize_per_tensor_fused_noalloc", "fp8_amax_history_update_ex",
-                                           "fp8_selftest_wait_timeout"])
+                                           "fp8_selftest_wait_timeout", "fp8_quantize_mx", "fp8_dequantize_mx",
+                                           "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -180,6 +181,50 @@ def test_history_ex_validation(L):
     assert f(A16, A16, 0, A16, 0, A16, 0, 1.0, 1.0, None) == ERR_ARG
     assert f(None, A16, 16, A16, 0, A16, 0, 1.0, 1.0, None) == ERR_NULL
     assert f(A16, A16, 16, A16, 0, A1, 0, 1.0, 1.0, None) == ERR_ALIGN
+
+
+def test_transpose_validation(L):
+    f = L.fp8_quantize_per_tensor_transpose
+    assert f(A16, 1, 4, 64, 9, None, A16, A16, A16, A16, None) == ERR_FORMAT
+    assert f(A16, 7, 4, 64, 0, None, A16, A16, A16, A16, None) == ERR_DTYPE
+    assert f(A16, 1, -4, 64, 0, None, A16, A16, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 4, 64, 0, None, A16, A16, None, A16, None) == ERR_NULL      # scale_out
+    assert f(A16, 1, 4, 64, 0, None, A16, A16, A16, None, None) == ERR_NULL      # current scaling needs amax_out
+    assert f(A16, 1, 4, 64, 0, A16, A16, None, A16, None, None) == ERR_NULL      # qt
+    assert f(A16, 1, 4, 64, 0, A16, A16, A1, A16, None, None) == ERR_ALIGN
+    assert f(A16, 1, 4, 64, 0, A16, A1, A16, A16, None, None) == ERR_ALIGN
+
+
+def test_gemm_validation(L):
+    g = L.fp8_gemm_blockwise
+    assert g(A16, A16, 2, A16, A16, 0, 128, 256, 128, A16, 1, None) == ERR_FORMAT
+    assert g(A16, A16, 0, A16, A16, 0, 128, 256, 128, A16, 3, None) == ERR_DTYPE
+    assert g(A16, A16, 0, A16, A16, 0, 128, 128, 128, A16, 1, None) == ERR_SHAPE   # N % 256
+    assert g(A16, A16, 0, A16, A16, 0, 128, 256, 100, A16, 1, None) == ERR_SHAPE   # K % 128
+    assert g(A16, A16, 0, A16, A16, 0, -1, 256, 128, A16, 1, None) == ERR_SHAPE
+    assert g(None, None, 0, None, None, 0, 0, 256, 128, None, 1, None) == OK        # M = 0: nothing to do
+    assert g(A16, A16, 0, A16, A16, 0, 128, 256, 128, None, 1, None) == ERR_NULL
+    assert g(A16, None, 0, A16, A16, 0, 128, 256, 128, A16, 1, None) == ERR_NULL
+    assert g(A1, A16, 0, A16, A16, 0, 128, 256, 128, A16, 1, None) == ERR_ALIGN
+    assert g(A16, A16, 0, A16, A16, 0, 128, 256, 128, A1, 1, None) == ERR_ALIGN
+
+
+def test_mx_validation(L):
+    q = L.fp8_quantize_mx
+    assert q(A16, 1, 4, 64, 2, 0, A16, A16, None) == ERR_FORMAT
+    assert q(A16, 2, 4, 64, 0, 0, A16, A16, None) == ERR_DTYPE
+    assert q(A16, 1, 4, 64, 0, 2, A16, A16, None) == ERR_ARG
+    assert q(A16, 1, -1, 64, 0, 0, A16, A16, None) == ERR_SHAPE
+    assert q(A16, 1, 1 << 40, 1 << 40, 0, 0, A16, A16, None) == ERR_SHAPE
+    assert q(None, 1, 0, 64, 0, 0, None, None, None) == OK  # empty: nothing to do
+    assert q(A16, 1, 4, 64, 0, 0, A16, None, None) == ERR_NULL
+    assert q(A1, 1, 4, 64, 0, 0, A16, A1, None) == ERR_ALIGN
+    d = L.fp8_dequantize_mx
+    assert d(A16, 0, 4, 64, A16, A16, 2, None) == ERR_DTYPE
+    assert d(A16, 5, 4, 64, A16, A16, 0, None) == ERR_FORMAT
+    assert d(A16, 0, 4, -3, A16, A16, 0, None) == ERR_SHAPE
+    assert d(A16, 0, 4, 64, None, A16, 0, None) == ERR_NULL
+    assert d(A16, 0, 4, 64, A1, A1, 0, None) == ERR_ALIGN
 
 
 def test_diagnostics_validation(L):

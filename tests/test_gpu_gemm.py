@@ -1,0 +1,102 @@
+"""GPU parity of the consumer GEMM (fp8_gemm_blockwise) against the oracle.
+
+The tensor cores sum each 128-product chunk in an order of their own, so this
+is not bit-exact.  The bound is derived from the arithmetic: every FP8 product
+is exact in fp32; a chunk sum of 128 products carries at most a relative
+2^-14 of the chunk's absolute sum (allowing an accumulator narrower than fp32,
+the limitation the handbook's promotion works around); the factor
+RN(1/RN(sa*sb)) adds 2^-23; the fp32 fma accumulation over K/128 chunks adds
+(K/128) * 2^-24.  With S[m][n] the same GEMM over absolute values,
+    |C_gpu - C_exact| <= (2^-14 + 2^-23 + (K/128) 2^-24) * S    (+ half a bf16
+ulp of |C| for bf16 output).  The test uses 2^-12 * S, well inside which a
+wrong block, scale or index (an O(1) relative error) cannot hide.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fine_grained_block_b200 import binding as B
+from fine_grained_block_b200 import inputs
+from parity_util import host_input, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_codes(M, N, K, a_fmt, b_fmt, seed):
+    x = inputs.random_matrix(M, K, seed=seed, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e2)
+    w = inputs.random_matrix(N, K, seed=seed + 1, dtype=torch.bfloat16, scale=0.02)
+    qa, sa = oracle.quantize_blockwise(host_input(x), 1, 128, a_fmt)
+    qb, sb = oracle.quantize_blockwise(host_input(w), 128, 128, b_fmt)
+    return qa, sa, qb, sb
+
+
+def check_gemm(qa, sa, a_fmt, qb, sb, b_fmt, c_gpu, what, rows=None):
+    """Compare c_gpu (torch, [M, N]) with the oracle on the given rows (all by default)."""
+    if rows is not None:
+        qa, sa = qa[rows], sa[rows]
+        c_gpu = c_gpu[torch.as_tensor(rows, device=c_gpu.device)]
+    want = oracle.gemm_blockwise(qa, sa, a_fmt, qb, sb, b_fmt)
+    mag = oracle.gemm_blockwise(qa & 0x7F, sa, a_fmt, qb & 0x7F, sb, b_fmt)
+    got = c_gpu.float().cpu().numpy().astype(np.float64)
+    tol = 2.0 ** -12 * mag
+    if c_gpu.dtype == torch.bfloat16:
+        tol = tol + 2.0 ** -8 * np.abs(want)
+    err = np.abs(got - want)
+    bad = err > tol
+    assert not np.isnan(got).any(), what
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outside the bound; worst "
+                           f"{float((err / np.maximum(mag, 1e-30)).max()):.3g} of S")
+    return float((err / np.maximum(mag, 1e-30)).max())
+
+
+SHAPES = [(128, 256, 128), (256, 512, 1024), (200, 256, 384), (1, 256, 128), (130, 768, 640)]
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_matches_oracle(out_dtype):
+    for i, (M, N, K) in enumerate(SHAPES):
+        qa, sa, qb, sb = oracle_codes(M, N, K, B.E4M3, B.E4M3, seed=5000 + i)
+        c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
+                                 to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        check_gemm(qa, sa, B.E4M3, qb, sb, B.E4M3, c, f"{M}x{N}x{K} {out_dtype}")
+
+
+def test_gemm_consumes_the_gpu_quantizers_output():
+    """x (bf16) -> 1x128 codes, w (bf16) -> 128x128 codes, both on the GPU, then the GEMM."""
+    M, N, K = 512, 1024, 2048
+    x = inputs.random_matrix(M, K, seed=5100, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e2, device="cuda")
+    w = (inputs.random_matrix(N, K, seed=5101, dtype=torch.float32, device="cuda") * 0.02).to(torch.bfloat16)
+    qa, sa = B.fp8_quantize_blockwise(x, (1, 128), B.E4M3)
+    qb, sb = B.fp8_quantize_blockwise(w, (128, 128), B.E4M3)
+    c = B.fp8_gemm_blockwise(qa, sa, qb, sb, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    check_gemm(qa.cpu().numpy(), sa.cpu().numpy(), B.E4M3, qb.cpu().numpy(), sb.cpu().numpy(), B.E4M3, c,
+               "quantize -> gemm")
+    # against the unquantized product: within the quantization error of both operands
+    ref = x.double() @ w.double().T
+    mag = x.double().abs() @ w.double().abs().T
+    assert bool(((c.double() - ref).abs() <= 0.15 * mag).all())
+
+
+def test_gemm_large_sampled_rows():
+    M, N, K = 4096, 4096, 4096
+    qa, sa, qb, sb = oracle_codes(M, N, K, B.E4M3, B.E4M3, seed=5200)
+    c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
+                             to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rows = [0, 1, 127, 128, 2047, 2900, 4094, 4095]
+    check_gemm(qa, sa, B.E4M3, qb, sb, B.E4M3, c, "4096^3 sampled rows", rows=rows)
+
+
+def test_gemm_k_zero_and_empty():
+    a = torch.zeros(64, 0, dtype=torch.uint8, device="cuda")
+    b = torch.zeros(256, 0, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(1, dtype=torch.float32, device="cuda")
+    c = torch.full((64, 256), 7.0, dtype=torch.float32, device="cuda")
+    B.fp8_gemm_blockwise(a, s, b, s, c=c)
+    torch.cuda.synchronize()
+    assert bool((c == 0).all())

@@ -14,7 +14,7 @@ import oracle
 from fine_grained_block_b200 import binding as B
 from fine_grained_block_b200 import inputs
 from parity_util import (Guarded, assert_bytes_equal, fp32_bits, host_input, oracle_blockwise, oracle_dequant,
-                         oracle_per_tensor, to_cuda)
+                         oracle_dequant_mx, oracle_mx, oracle_per_tensor, to_cuda)
 
 pytestmark = pytest.mark.gpu
 
@@ -461,3 +461,180 @@ def test_history_update_ex_matches_oracle(fmt, algo, alpha, margin, window):
             assert_bytes_equal(h, fp32_bits(ref.history), f"history step {k}")
         else:
             assert_bytes_equal(h[:1], fp32_bits(ref.history[:1]), f"ema step {k}")
+
+
+# -- MX: 1x32 blocks, power-of-two scales as E8M0 bytes ----------------------------------
+
+def run_mx(x_cpu: torch.Tensor, fmt, rule):
+    R, C = x_cpu.shape
+    x = to_cuda(x_cpu)
+    gq = Guarded((R, C), torch.uint8)
+    ge = Guarded((R, math.ceil(C / 32)), torch.uint8)
+    B.fp8_quantize_mx(x, fmt, rule, q=gq.t, e8m0=ge.t)
+    torch.cuda.synchronize()
+    gq.check()
+    ge.check()
+    return gq.t, ge.t
+
+
+def check_mx(x_cpu, fmt, rule, what, nan_positions=None):
+    xh = host_input(x_cpu)
+    q, e = run_mx(x_cpu, fmt, rule)
+    oq, oe = oracle_mx(xh, fmt, rule)
+    assert_bytes_equal(e, oe, f"{what} e8m0")
+    if nan_positions is not None:
+        # a NaN element has several valid NaN codes: require a NaN code there,
+        # exact bytes everywhere else
+        qc = q.cpu().numpy()
+        nan_codes = {oracle.E4M3: (0x7F,), oracle.E5M2: (0x7D, 0x7E, 0x7F)}[fmt]
+        assert all((int(qc[i]) & 0x7F) in nan_codes for i in nan_positions), what
+        for i in nan_positions:
+            qc[i] = oq[i]
+        q = torch.from_numpy(qc)
+    assert_bytes_equal(q, oq, f"{what} codes")
+    for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
+        gy = Guarded(tuple(oq.shape), out_dtype)
+        B.fp8_dequantize_mx(to_cuda(torch.from_numpy(oq)), e, fmt, out_dtype, y=gy.t)
+        torch.cuda.synchronize()
+        gy.check()
+        assert_bytes_equal(gy.t, oracle_dequant_mx(oq, fmt, oe, oc), f"{what} dequant {out_dtype}")
+
+
+MX_SHAPES = SHAPES + [(3, 32), (5, 33), (7, 95), (9, 64), (33, 160), (2, 31)]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("rule", [B.MX_FIT, B.MX_OCP])
+def test_mx_ragged(fmt, dtype, rule):
+    for i, (R, C) in enumerate(MX_SHAPES):
+        x = inputs.random_matrix(R, C, seed=3000 + i, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        check_mx(x, fmt, rule, f"mx rule {rule} {R}x{C} {dtype}")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("rule", [B.MX_FIT, B.MX_OCP])
+def test_mx_edge_values(fmt, rule):
+    R, C = 16, 256
+    x = inputs.random_matrix(R, C, seed=78, dtype=torch.float32)
+    x[0, :32] = 0.0                          # all-zero block
+    x[1, :32] = -0.0
+    x[2, :32] = 1e-42                        # fp32 subnormals only
+    x[3, :64] = torch.linspace(-1e-30, 1e-30, 64)
+    x[4, 32:64] = 3.0e38                     # near fp32 max: k = -120 or so
+    x[4, 64:96] = torch.finfo(torch.float32).max  # fp32 max: its dequant overflows to Inf
+    x[5, :128] = torch.tensor([2.0 ** k for k in range(-64, 64)])
+    x[6, :] = 1.0                            # every element hits the top of its binade
+    x[7, :32] = 1.75 * 2.0 ** -8             # amax * 2^k exactly MAX under the fit rule
+    x[7, 32:64] = 1.7500001
+    x[8, 3] = float("inf")                   # blocks holding Inf: the NaN byte
+    x[9, 40] = float("-inf")
+    x[10, :32] = torch.linspace(-3.0, 3.0, 32) * 2.0 ** 100
+    for dtype in (torch.float32, torch.bfloat16):
+        check_mx(x.to(dtype), fmt, rule, f"mx edge {dtype}")
+    x[11, 7] = float("nan")                  # NaN does not count toward amax
+    check_mx(x, fmt, rule, "mx edge NaN", nan_positions=[(11, 7)])
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_mx_dequant_every_byte(fmt):
+    """Every finite code against every E8M0 byte, 0 (the subnormal multiplier 2^-127) to 0xFF (NaN)."""
+    top = oracle.top_code(fmt)
+    codes = np.array([c for c in range(256) if (c & 0x7F) <= top], dtype=np.uint8)
+    q = np.ascontiguousarray(np.tile(codes, (256, 1))[:, :224])   # 224 codes = 7 blocks per row
+    e = np.tile(np.arange(256, dtype=np.uint8).reshape(256, 1), (1, 7))
+    e[:, 3] = e[::-1, 0]
+    qg, eg = to_cuda(torch.from_numpy(q)), to_cuda(torch.from_numpy(np.ascontiguousarray(e)))
+    for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
+        y = B.fp8_dequantize_mx(qg, eg, fmt, out_dtype)
+        torch.cuda.synchronize()
+        assert_bytes_equal(y, oracle.dequantize_mx(q, fmt, e, oc), f"mx dequant bytes {out_dtype}")
+        y2 = B.fp8_dequantize_mx(qg[:, :200].contiguous(), eg, fmt, out_dtype)  # ragged: 200 = 6 blocks + 8
+        torch.cuda.synchronize()
+        assert_bytes_equal(y2, oracle.dequantize_mx(np.ascontiguousarray(q[:, :200]), fmt, e, oc),
+                           f"mx dequant ragged {out_dtype}")
+
+
+def test_mx_empty():
+    q, e = B.fp8_quantize_mx(torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda"))
+    assert q.numel() == 0 and e.numel() == 0
+    y = B.fp8_dequantize_mx(torch.zeros(4, 0, dtype=torch.uint8, device="cuda"),
+                            torch.zeros(4, 0, dtype=torch.uint8, device="cuda"))
+    assert y.numel() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_mx_16_byte_aligned_buffers(fmt, dtype):
+    """Input and output 16- but not 32-byte aligned: the 16-byte lane kernels."""
+    R, C = 67, 320
+    x_cpu = inputs.random_matrix(R, C, seed=3100, dtype=dtype, outlier_frac=0.01, factor=1e3)
+    off = 16 // x_cpu.element_size()
+    buf = torch.empty(R * C + off, dtype=dtype, device="cuda")
+    x = buf[off:].view(R, C)
+    x.copy_(x_cpu.to("cuda"))
+    assert x.data_ptr() % 32 == 16
+    q, e = B.fp8_quantize_mx(x, fmt, B.MX_FIT)
+    torch.cuda.synchronize()
+    oq, oe = oracle_mx(host_input(x_cpu), fmt, B.MX_FIT)
+    assert_bytes_equal(e, oe, "e8m0")
+    assert_bytes_equal(q, oq, "codes")
+    for out_dtype, oc in ((torch.float32, oracle.F32), (torch.bfloat16, oracle.BF16)):
+        esz = torch.empty(0, dtype=out_dtype).element_size()
+        ybuf = torch.empty(R * C + 16 // esz, dtype=out_dtype, device="cuda")
+        y = ybuf[16 // esz:].view(R, C)
+        assert y.data_ptr() % 32 == 16
+        B.fp8_dequantize_mx(q, e, fmt, out_dtype, y=y)
+        torch.cuda.synchronize()
+        assert_bytes_equal(y, oracle_dequant_mx(oq, fmt, oe, oc), f"dequant {out_dtype}")
+
+
+# -- per-tensor with a transposed copy ---------------------------------------------------
+
+def check_transpose(x_cpu, fmt, what, scale=None, with_q=True):
+    R, C = x_cpu.shape
+    x = to_cuda(x_cpu)
+    gq = Guarded((R, C), torch.uint8) if with_q else None
+    gt = Guarded((C, R), torch.uint8)
+    s_in = None if scale is None else torch.tensor([scale], dtype=torch.float32, device="cuda")
+    _, _, s, a = B.fp8_quantize_per_tensor_transpose(x, fmt, s_in, with_q=with_q, q=None if gq is None else gq.t,
+                                                     qt=gt.t)
+    torch.cuda.synchronize()
+    gt.check()
+    oq, oqt, os_, oa = oracle.quantize_per_tensor_transpose(host_input(x_cpu), fmt, scale)
+    assert_bytes_equal(s, fp32_bits([os_]), f"{what} scale")
+    assert_bytes_equal(a, fp32_bits([oa]), f"{what} amax")
+    assert_bytes_equal(gt.t, oqt, f"{what} qt")
+    if gq is not None:
+        gq.check()
+        assert_bytes_equal(gq.t, oq, f"{what} q")
+
+
+TRANSPOSE_SHAPES = [(128, 128), (256, 384), (1024, 4096), (130, 384), (257, 640), (64, 100), (200, 77), (5, 1),
+                    (1, 8), (16, 4096), (4096, 16), (48, 96)]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_per_tensor_transpose(fmt, dtype):
+    for i, (R, C) in enumerate(TRANSPOSE_SHAPES):
+        x = inputs.random_matrix(R, C, seed=4000 + i, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        check_transpose(x, fmt, f"transpose {R}x{C} {dtype}")
+        check_transpose(x, fmt, f"transpose delayed {R}x{C} {dtype}", scale=3.25)
+    x = inputs.random_matrix(512, 256, seed=4100, dtype=dtype)
+    check_transpose(x, fmt, "transpose qt only", with_q=False)
+    check_transpose(x, fmt, "transpose qt only delayed", scale=0.5, with_q=False)
+
+
+def test_per_tensor_transpose_16_byte_aligned_input():
+    R, C = 256, 512
+    x_cpu = inputs.random_matrix(R, C, seed=4200, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e3)
+    buf = torch.empty(R * C + 8, dtype=torch.bfloat16, device="cuda")
+    x = buf[8:].view(R, C)
+    x.copy_(x_cpu.to("cuda"))
+    assert x.data_ptr() % 32 == 16
+    q, qt, s, a = B.fp8_quantize_per_tensor_transpose(x, B.E4M3)
+    torch.cuda.synchronize()
+    oq, oqt, os_, oa = oracle.quantize_per_tensor_transpose(host_input(x_cpu), B.E4M3)
+    assert_bytes_equal(qt, oqt, "qt")
+    assert_bytes_equal(q, oq, "q")

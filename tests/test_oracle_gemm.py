@@ -1,0 +1,54 @@
+"""Pins of the oracle's blockwise-scaled GEMM (the consumer of the codes).
+
+Mixed-precision handbook, "FP8 training", closing notes: FP8 products with
+fp32 accumulation, the partial sum promoted every 128 elements where the
+1x128 / 128x128 scales are applied.  The oracle sums exact FP8 products per
+128-chunk and divides by the two scales; here it is checked against a hand
+example and against the other order of the same mathematics (dequantize each
+operand first, then one float64 matrix product).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import E4M3, E5M2
+
+
+def test_hand_example_two_chunks():
+    # K = 256: two chunks.  Every code 0x38 (= 1.0 in E4M3), so each chunk's
+    # partial sum is 128.  sa = [2, 4], sb = [1, 0.5]:
+    # C = 128 / (2 * 1) + 128 / (4 * 0.5) = 64 + 64 = 128.
+    a = np.full((1, 256), 0x38, dtype=np.uint8)
+    b = np.full((1, 256), 0x38, dtype=np.uint8)
+    c = oracle.gemm_blockwise(a, np.array([[2.0, 4.0]], np.float32), E4M3, b, np.array([[1.0, 0.5]], np.float32),
+                              E4M3)
+    assert c.shape == (1, 1) and c[0, 0] == 128.0
+    # sign: 0xB8 = -1.0 in one operand flips the chunk it sits in
+    a[0, :128] = 0xB8
+    c = oracle.gemm_blockwise(a, np.array([[2.0, 4.0]], np.float32), E4M3, b, np.array([[1.0, 0.5]], np.float32),
+                              E4M3)
+    assert c[0, 0] == 0.0
+
+
+@pytest.mark.parametrize("a_fmt,b_fmt", [(E4M3, E4M3), (E5M2, E4M3), (E4M3, E5M2)])
+@pytest.mark.parametrize("M,N,K", [(3, 130, 384), (17, 256, 256), (5, 7, 200)])
+def test_equals_dequantize_then_matmul(a_fmt, b_fmt, M, N, K):
+    rng = np.random.default_rng(M * 1000 + N + K)
+    x = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-3, 3, (M, 1)))).astype(np.float32)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    qa, sa = oracle.quantize_blockwise(x, 1, 128, a_fmt)
+    qb, sb = oracle.quantize_blockwise(w, 128, 128, b_fmt)
+    c = oracle.gemm_blockwise(qa, sa, a_fmt, qb, sb, b_fmt)
+    # the other order: dequantize in float64 with the scales broadcast over
+    # their blocks, then a single library matrix product
+    da = oracle.decode_table(a_fmt)[qa].astype(np.float64) / np.repeat(sa.astype(np.float64), 128, axis=1)[:, :K]
+    sbx = np.repeat(np.repeat(sb.astype(np.float64), 128, axis=0), 128, axis=1)[:N, :K]
+    db = oracle.decode_table(b_fmt)[qb].astype(np.float64) / sbx
+    ref = da @ db.T
+    mag = np.abs(da) @ np.abs(db).T
+    assert np.all(np.abs(c - ref) <= 1e-13 * mag + 1e-300)
+    # and the product approximates x w^T within the quantization error
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    assert np.all(np.abs(c - exact) <= 0.25 * (np.abs(x) @ np.abs(w).T) + 1e-30)

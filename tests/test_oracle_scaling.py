@@ -375,3 +375,27 @@ def test_ema_stays_inside_the_seen_range(alpha):
     for _ in range(50):
         h.update(3.25)
     assert abs(float(h.history[0]) / 3.25 - 1) < 1e-6
+
+
+def test_transposed_per_tensor_output_hand_example():
+    """2x3 example worked by hand from the E4M3 bit layout (bias 7): 1 = 0x38,
+    2 = 0x40, 448 = 0x7E, -1 = 0xB8, 0.5 = 0x30, 0 = 0x00.  amax 448 gives
+    s = 1 under current scaling, the same as a delayed scale of 1."""
+    x = np.array([[1.0, 2.0, 448.0], [-1.0, 0.5, 0.0]], dtype=np.float32)
+    want_q = np.array([[0x38, 0x40, 0x7E], [0xB8, 0x30, 0x00]], dtype=np.uint8)
+    want_qt = np.array([[0x38, 0xB8], [0x40, 0x30], [0x7E, 0x00]], dtype=np.uint8)
+    for scale in (None, 1.0):
+        q, qt, s, a = oracle.quantize_per_tensor_transpose(x, oracle.E4M3, scale)
+        assert np.array_equal(q, want_q) and np.array_equal(qt, want_qt)
+        assert s == 1.0 and a == 448.0
+
+
+def test_transposed_output_is_the_per_tensor_codes():
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((37, 53)) * 10).astype(np.float32)
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        q, qt, s, a = oracle.quantize_per_tensor_transpose(x, fmt)
+        q1, s1, a1 = oracle.quantize_per_tensor(x, fmt)
+        assert np.array_equal(q, q1) and s == s1 and a == a1
+        assert qt.shape == (53, 37)
+        assert all(qt[c, r] == q1[r, c] for r in range(37) for c in range(53))
