@@ -15,21 +15,37 @@
 // sb [N/128, K/128]); both scales are the quantizers' multipliers, so each
 // promotion divides by them.
 //
-// One CTA computes a 128 x 256 tile of C (10 warps):
-//   warp 0    TMA producer: per K chunk, one 128x128-byte box of A and one
-//             256x128-byte box of B into a ring of kStages shared-memory
-//             stages (128-byte swizzle, the layout the MMA descriptors name);
-//   warp 1    allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
-//             issues the MMAs: per chunk, 4 x tcgen05.mma (M 128, N 256,
-//             K 32) into a fresh accumulator, then commits to the stage's
-//             "empty" barrier and the accumulator's "full" barrier;
-//   warps 2-9 the promotion: each thread owns one row (its TMEM lane) and 128
-//             columns; per chunk it loads its partial sums from TMEM, frees
-//             the accumulator, and adds partial * 1/(sa * sb) into 128 fp32
-//             registers.  The two accumulators alternate, so the MMAs of
-//             chunk c+1 run while chunk c is promoted.
+// Each CTA owns 128 rows x 256 columns of C (12 warps):
+//   warp 0     TMA producer: per K chunk, a 128x128-byte box of A and the
+//              box of B this CTA holds, into a ring of shared-memory stages
+//              (128-byte swizzle, the layout the MMA descriptors name);
+//   warp 1     allocates 512 TMEM columns (two 128x256 fp32 accumulators)
+//              and issues the MMAs: per chunk, 4 x tcgen05.mma (K 32) into a
+//              fresh accumulator, then commits to the stage's "empty" barrier
+//              and the accumulator's "full" barrier;
+//   warps 4-11 the promotion: each thread owns one row (its TMEM lane) and
+//              128 columns; per chunk it loads its partial sums from TMEM,
+//              frees the accumulator, and adds partial * 1/(sa * sb) into
+//              128 fp32 registers.  The two accumulators alternate, so the
+//              MMAs of chunk c+1 run while chunk c is promoted;
+//   warps 2-3  idle (they complete the first warpgroup, whose registers go
+//              to the promotion warpgroups).
 // At the end each promotion thread writes its 128 results (fp32 or bf16).
 // Rows past M arrive as zeros from the copy engine and are not stored.
+//
+// Two variants:
+//   single CTA (M 128 x N 256 per MMA): the CTA loads A (16 KiB) and all of
+//              B (32 KiB) per chunk, 4 stages;
+//   CTA pair   (a cluster of 2, M 256 x N 256 per MMA): each CTA loads its
+//              own 128 rows of A and one 128-row half of B (32 KiB per
+//              chunk), and the tensor cores of the pair read the other half
+//              from the peer -- a third less operand traffic per CTA for the
+//              same work, and 6 stages.  The even CTA issues the MMAs; its
+//              "full" barriers count both CTAs' copies, and both CTAs'
+//              promotion warps release the accumulators to it.
+// The operand traffic is what bounds the single-CTA kernel on B200: its TMA
+// loads alone, with no MMA or promotion, already take as long as the whole
+// kernel.
 //
 // Every barrier wait is bounded (1 s); a wait that runs out sets the
 // wait-timeout bit of the device status word, and the CTA still waits
@@ -50,86 +66,123 @@
 namespace fp8q {
 namespace {
 
-constexpr int kBM = 128;                  // tile rows (MMA M)
-constexpr int kBN = 256;                  // tile columns (MMA N)
+constexpr int kBM = 128;                  // rows of C per CTA (TMEM lanes)
+constexpr int kBN = 256;                  // columns of C per CTA (MMA N)
 constexpr int kBK = 128;                  // K chunk = one promotion = one stage
 constexpr int kMmaK = 32;                 // K of one kind::f8f6f4 instruction
-constexpr int kStages = 4;
-constexpr int kWarps = 10;
+constexpr int kWarps = 12;                // 3 warpgroups: control, promotion x2
 constexpr int kThreads = kWarps * 32;
 constexpr int kABytes = kBM * kBK;        // 16 KiB
-constexpr int kBBytes = kBN * kBK;        // 32 KiB
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 2 * kBN;   // two accumulators
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
+// Register split (setmaxnreg): the kernel launches at kLaunchRegs per thread;
+// the control warpgroup gives registers back, the two promotion warpgroups
+// take them.  The per-thread counts must add up to the launch total exactly
+// (and per SM sub-partition: each holds one warp of every warpgroup), or an
+// increase would never be granted.
+constexpr int kLaunchRegs = 168;          // 65536 / 384 rounded down to a multiple of 8
+constexpr int kControlRegs = 40;
+constexpr int kPromoteRegs = 232;
+static_assert(kControlRegs + 2 * kPromoteRegs == 3 * kLaunchRegs, "register split must equal the launch total");
+static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the register file");
 
+template <bool PAIR>
+struct Cfg {
+    static constexpr int kBRows = PAIR ? kBN / 2 : kBN;      // rows of B this CTA loads
+    static constexpr int kBBytes = kBRows * kBK;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = PAIR ? 6 : 4;
+    static constexpr int kAccEmptyArrivals = PAIR ? 16 : 8;  // promotion warps releasing an accumulator
+    static constexpr uint32_t kFullTx = PAIR ? 2 * kStageBytes : kStageBytes;  // bytes per "full" phase
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
+};
+
+template <int STAGES>
 struct Barriers {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
 };
 
-template <int OUT>
+template <int OUT, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const float* __restrict__ sa, const float* __restrict__ sb, void* __restrict__ c, int64_t M,
                  int64_t N, int64_t K, uint32_t idesc, unsigned int* status) {
+    using C = Cfg<PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Barriers* bars = reinterpret_cast<Barriers*>(tiles + kStages * kStageBytes);
+    auto* bars = reinterpret_cast<Barriers<C::kStages>*>(tiles + C::kStages * C::kStageBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? umma::cluster_ctarank() : 0u;  // 0: this CTA issues the MMAs
     const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kBN;
     const int nchunks = static_cast<int>(K / kBK);
     const int64_t kc_stride = K / kBK;  // scales per row of sa / sb
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             umma::mbar_init(&bars->full[s], 1);
             umma::mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             umma::mbar_init(&bars->acc_full[b], 1);
-            umma::mbar_init(&bars->acc_empty[b], 8);  // one arrival per promotion warp
+            umma::mbar_init(&bars->acc_empty[b], C::kAccEmptyArrivals);
         }
         umma::mbar_init(&bars->mma_done, 1);
         umma::fence_mbar_init();
     }
-    if (warp == 1) umma::tmem_alloc(&bars->tmem_base, kTmemCols);
+    if (warp == 1) {
+        if (PAIR) umma::tmem_alloc_pair(&bars->tmem_base, kTmemCols);
+        else umma::tmem_alloc(&bars->tmem_base, kTmemCols);
+    }
     umma::fence_before_sync();
     __syncthreads();
+    if (PAIR) umma::cluster_sync();  // the peer's barriers are initialised before any remote arrival
     umma::fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
     pdl_enter();  // A, B and the scales may come from the previous kernel
 
     bool timed_out = false;
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
     if (warp == 0) {
         // ---- TMA producer ----------------------------------------------------
         if (lane == 0) {
             for (int kc = 0; kc < nchunks; ++kc) {
-                const int s = kc % kStages;
-                const uint32_t phase = static_cast<uint32_t>(kc / kStages) & 1u;
+                const int s = kc % C::kStages;
+                const uint32_t phase = static_cast<uint32_t>(kc / C::kStages) & 1u;
                 if (!umma::mbar_wait(&bars->empty[s], phase ^ 1u, kWaitLimitNs)) {
                     timed_out = true;
                     break;
                 }
-                uint8_t* sa_tile = tiles + s * kStageBytes;
-                umma::mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
-                umma::tma_load_2d(sa_tile, &map_a, &bars->full[s], kc * kBK, static_cast<int>(m0));
-                umma::tma_load_2d(sa_tile + kABytes, &map_b, &bars->full[s], kc * kBK, static_cast<int>(n0));
+                uint8_t* stage = tiles + s * C::kStageBytes;
+                if (PAIR) {
+                    // both CTAs' copies complete on the even CTA's barrier, which
+                    // expects the bytes of both
+                    const uint32_t full0 = umma::mapa(umma::smem_u32(&bars->full[s]), 0);
+                    if (rank == 0) umma::mbar_arrive_expect_tx(&bars->full[s], C::kFullTx);
+                    umma::tma_load_2d_pair(stage, &map_a, full0, kc * kBK, static_cast<int>(m0));
+                    umma::tma_load_2d_pair(stage + kABytes, &map_b, full0, kc * kBK,
+                                           static_cast<int>(n0 + rank * C::kBRows));
+                } else {
+                    umma::mbar_arrive_expect_tx(&bars->full[s], C::kFullTx);
+                    umma::tma_load_2d(stage, &map_a, &bars->full[s], kc * kBK, static_cast<int>(m0));
+                    umma::tma_load_2d(stage + kABytes, &map_b, &bars->full[s], kc * kBK, static_cast<int>(n0));
+                }
             }
         }
     } else if (warp == 1) {
-        // ---- MMA issuer ------------------------------------------------------
-        if (lane == 0) {
+        // ---- MMA issuer (the even CTA of a pair) -------------------------------
+        if (lane == 0 && rank == 0) {
+            const uint32_t peer_empty0 = PAIR ? umma::mapa(umma::smem_u32(&bars->empty[0]), 1) : 0u;
+            const uint32_t peer_accf0 = PAIR ? umma::mapa(umma::smem_u32(&bars->acc_full[0]), 1) : 0u;
             for (int kc = 0; kc < nchunks; ++kc) {
-                const int s = kc % kStages;
-                const uint32_t phase = static_cast<uint32_t>(kc / kStages) & 1u;
+                const int s = kc % C::kStages;
+                const uint32_t phase = static_cast<uint32_t>(kc / C::kStages) & 1u;
                 const int buf = kc & 1;
                 const uint32_t acc_phase = static_cast<uint32_t>(kc >> 1) & 1u;
                 if (!umma::mbar_wait(&bars->acc_empty[buf], acc_phase ^ 1u, kWaitLimitNs) ||
@@ -138,29 +191,41 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     break;
                 }
                 umma::fence_after_sync();
-                const uint32_t a_addr = umma::smem_u32(tiles + s * kStageBytes);
+                const uint32_t a_addr = umma::smem_u32(tiles + s * C::kStageBytes);
                 const uint64_t a_desc = umma::smem_desc_kmajor_sw128(a_addr);
                 const uint64_t b_desc = umma::smem_desc_kmajor_sw128(a_addr + kABytes);
                 const uint32_t d = tmem + static_cast<uint32_t>(buf * kBN);
 #pragma unroll
                 for (int k = 0; k < kBK / kMmaK; ++k) {
                     // the next 32 bytes of K: start address + 32 bytes (2 in 16-byte units)
-                    umma::mma_f8f6f4(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
+                    if (PAIR) umma::mma_f8f6f4_pair(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
+                    else umma::mma_f8f6f4(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
                 }
-                umma::commit(&bars->empty[s]);
-                umma::commit(&bars->acc_full[buf]);
+                if (PAIR) {
+                    umma::commit_pair(umma::smem_u32(&bars->empty[s]));
+                    umma::commit_pair(peer_empty0 + static_cast<uint32_t>(s * sizeof(uint64_t)));
+                    umma::commit_pair(umma::smem_u32(&bars->acc_full[buf]));
+                    umma::commit_pair(peer_accf0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
+                } else {
+                    umma::commit(&bars->empty[s]);
+                    umma::commit(&bars->acc_full[buf]);
+                }
             }
-            umma::commit(&bars->mma_done);
+            if (PAIR) umma::commit_pair(umma::smem_u32(&bars->mma_done));
+            else umma::commit(&bars->mma_done);
             if (!umma::mbar_wait(&bars->mma_done, 0, kWaitLimitNs)) timed_out = true;
         }
-    } else {
+    } else if (warp >= 4) {
         // ---- promotion warps -------------------------------------------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPromoteRegs));
         const int quarter = warp & 3;            // TMEM lanes this warp may access
-        const int half = (warp - 2) >> 2;        // column half of the tile
+        const int half = (warp - 4) >> 2;        // column half of the tile
         const int row = quarter * 32 + lane;     // tile row = TMEM lane
         const int64_t m = m0 + row;
         const float* sa_row = sa + (m < M ? m : 0) * kc_stride;
         const float* sb_row = sb + ((n0 >> 7) + half) * kc_stride;
+        const uint32_t acc_empty0 = PAIR ? umma::mapa(umma::smem_u32(&bars->acc_empty[0]), 0)
+                                         : umma::smem_u32(&bars->acc_empty[0]);
         float acc[128];
 #pragma unroll
         for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
@@ -177,18 +242,21 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             umma::fence_after_sync();
             const uint32_t t = t_lane + static_cast<uint32_t>(buf * kBN);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                float p[32];
-                umma::tmem_ld32(t + h * 32, p);
+            for (int h = 0; h < 2; ++h) {
+                float p[64];
+                umma::tmem_ld32(t + h * 64, p);
+                umma::tmem_ld32(t + h * 64 + 32, p + 32);
                 umma::wait_ld(p);
-                if (h == 3) {
+                umma::hold_after_wait(p + 32);
+                if (h == 1) {
                     // every partial sum of this buffer is in registers: hand it back
                     umma::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) umma::mbar_arrive(&bars->acc_empty[buf]);
+                    if (lane == 0)
+                        umma::mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
                 }
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc[h * 32 + j] = __fmaf_rn(p[j], f, acc[h * 32 + j]);
+                for (int j = 0; j < 64; ++j) acc[h * 64 + j] = __fmaf_rn(p[j], f, acc[h * 64 + j]);
             }
         }
         if (!timed_out && m < M) {
@@ -220,9 +288,13 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
         __syncthreads();
     }
+    // The even CTA's MMAs read the odd CTA's shared memory and write its
+    // tensor memory: neither CTA frees or leaves before both are done.
+    if (PAIR) umma::cluster_sync();
     if (warp == 1) {
         umma::fence_after_sync();
-        umma::tmem_dealloc(tmem, kTmemCols);
+        if (PAIR) umma::tmem_dealloc_pair(tmem, kTmemCols);
+        else umma::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -253,6 +325,49 @@ bool make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int OUT, bool PAIR>
+cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, const float* sa, const float* sb,
+                         void* c, int64_t M, int64_t N, int64_t K, uint32_t idesc, unsigned int* status,
+                         cudaStream_t st) {
+    using C = Cfg<PAIR>;
+    auto kern = k_gemm_blockwise<OUT, PAIR>;
+    // The shared-memory opt-in, once per device (not inside a stream capture
+    // on later calls).
+    static std::atomic<bool> opted[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    if (!opted[dev].load(std::memory_order_acquire)) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        opted[dev].store(true, std::memory_order_release);
+    }
+    int64_t mt = (M + kBM - 1) / kBM;
+    if (PAIR) mt = (mt + 1) & ~int64_t(1);  // whole pairs; rows past M are zeros and not stored
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(mt), static_cast<unsigned>(N / kBN));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+#if FP8Q_PDL
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+#endif
+    if (PAIR) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, sa, sb, c, M, N, K, idesc, status);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 }  // namespace
 
 bool gemm_blockwise_supported() { return tensor_map_encoder() != nullptr; }
@@ -260,26 +375,19 @@ bool gemm_blockwise_supported() { return tensor_map_encoder() != nullptr; }
 cudaError_t launch_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb,
                                   int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
                                   cudaStream_t st) {
+    // A pair pays off once there are two row tiles to share B between.
+    const bool pair = M > kBM;
     CUtensorMap map_a, map_b;
-    if (!make_kmajor_map(&map_a, a, M, K, kBM) || !make_kmajor_map(&map_b, b, N, K, kBN))
+    if (!make_kmajor_map(&map_a, a, M, K, kBM) || !make_kmajor_map(&map_b, b, N, K, pair ? kBN / 2 : kBN))
         return cudaErrorInvalidValue;
     unsigned int* status = device_status_word();
     if (status == nullptr) return cudaErrorInvalidValue;
-    const uint32_t idesc = umma::instr_desc_f8f6f4(a_fmt, b_fmt, kBM, kBN);
-    const dim3 grid(static_cast<unsigned>((M + kBM - 1) / kBM), static_cast<unsigned>(N / kBN));
-    auto kern = c_dtype == 0 ? k_gemm_blockwise<0> : k_gemm_blockwise<1>;
-    // The shared-memory opt-in, once per device and output type (not inside
-    // a stream capture on later calls).
-    static std::atomic<bool> opted[128][2];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-    if (!opted[dev][c_dtype ? 1 : 0].load(std::memory_order_acquire)) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        opted[dev][c_dtype ? 1 : 0].store(true, std::memory_order_release);
-    }
-    return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, st, map_a, map_b, sa, sb, c, M, N, K, idesc,
-                         status);
+    const uint32_t idesc = umma::instr_desc_f8f6f4(a_fmt, b_fmt, pair ? 2 * kBM : kBM, kBN);
+    if (pair)
+        return c_dtype == 0 ? launch_typed<0, true>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st)
+                            : launch_typed<1, true>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st);
+    return c_dtype == 0 ? launch_typed<0, false>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st)
+                        : launch_typed<1, false>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st);
 }
 
 }  // namespace fp8q
