@@ -125,17 +125,23 @@ k_tensor_cast(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec
 // through shared memory so that both outputs are written row by row.
 // DELAYED / WITH_AMAX as in k_tensor_cast.
 //
-// Full tiles with vector-friendly strides (FAST) load one lane vector per
-// slice, 16 rows per warp, as the 128x128 block kernel does; each lane then
-// builds 32 consecutive codes of one qt row from one byte per tile row (the
-// 32 lanes of a warp read 32 consecutive bytes of a smem row: no bank
-// conflicts).  Edge tiles and other strides take an element-wise path.
+// Full tiles with vector-friendly strides load one lane vector per slice, 16
+// rows per warp, as the 128x128 block kernel does; the read-out transposes
+// 4x4-byte blocks in registers (byte permutes) so that each lane writes 16
+// consecutive codes into 4 qt rows.  Edge tiles and other strides take an
+// element-wise path.
 // ---------------------------------------------------------------------------
 constexpr int kTT = 128;           // tile side
 constexpr int kTStride = kTT + 16;  // smem row pitch in bytes (16-byte aligned rows)
 
+// Resident CTAs per SM the transposing cast is compiled for (register cap):
+// each CTA keeps one 32 KiB input tile in flight.
+#ifndef FP8Q_TRANSPOSE_MIN_CTAS
+#define FP8Q_TRANSPOSE_MIN_CTAS 4
+#endif
+
 template <typename T, int FMT, int BYTES, bool DELAYED, bool WITH_AMAX>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, FP8Q_TRANSPOSE_MIN_CTAS)
 k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, const float* scale_in,
                         const float* __restrict__ amax_in, uint8_t* __restrict__ q, uint8_t* __restrict__ qt,
                         float* scale_out, float* __restrict__ amax_out, int vector_ok) {
@@ -174,22 +180,32 @@ k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, con
             *reinterpret_cast<typename V::Out*>(tile + lr * kTStride + vec_in_row * V::kElems) = c;
         }
         __syncthreads();
-        // qt: 128 rows (tile columns) x 4 runs of 32 codes; 2 runs per thread
+        // qt: lane l takes tile columns 4l..4l+3, warp w tile rows 16w..16w+15.
+        // It reads 16 words (4 codes of one tile row each; the warp reads
+        // 128 consecutive bytes of a row: no bank conflicts), transposes
+        // them in 4x4-byte blocks with byte permutes, and writes 16
+        // consecutive codes into each of its 4 qt rows.
+        {
+            const int cq = lane * 4, rq = warp * 16;
+            uint32_t wv[16];
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const int task = p * kThreads + threadIdx.x;
-            const int c = task % kTT, run = task / kTT;
-            uint32_t wd[8];
+            for (int i = 0; i < 16; ++i)
+                wv[i] = *reinterpret_cast<const uint32_t*>(tile + (rq + i) * kTStride + cq);
+            uint32_t o[4][4];  // o[j][g]: column cq+j, rows rq+4g..rq+4g+3
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint8_t* col = tile + (run * 32 + 4 * k) * kTStride + c;
-                wd[k] = static_cast<uint32_t>(col[0]) | (static_cast<uint32_t>(col[kTStride]) << 8) |
-                        (static_cast<uint32_t>(col[2 * kTStride]) << 16) |
-                        (static_cast<uint32_t>(col[3 * kTStride]) << 24);
+            for (int g = 0; g < 4; ++g) {
+                const uint32_t w0 = wv[4 * g], w1 = wv[4 * g + 1], w2 = wv[4 * g + 2], w3 = wv[4 * g + 3];
+                const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), lo23 = __byte_perm(w2, w3, 0x5140);
+                const uint32_t hi01 = __byte_perm(w0, w1, 0x7362), hi23 = __byte_perm(w2, w3, 0x7362);
+                o[0][g] = __byte_perm(lo01, lo23, 0x5410);
+                o[1][g] = __byte_perm(lo01, lo23, 0x7632);
+                o[2][g] = __byte_perm(hi01, hi23, 0x5410);
+                o[3][g] = __byte_perm(hi01, hi23, 0x7632);
             }
-            uint4* dst = reinterpret_cast<uint4*>(qt + (c0 + c) * rows + r0 + run * 32);
-            st_stream(dst, make_uint4(wd[0], wd[1], wd[2], wd[3]));
-            st_stream(dst + 1, make_uint4(wd[4], wd[5], wd[6], wd[7]));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                st_stream(reinterpret_cast<uint4*>(qt + (c0 + cq + j) * rows + r0 + rq),
+                          make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]));
         }
     } else {
         for (int i = threadIdx.x; i < kTT * kTT; i += kThreads) {

@@ -25,6 +25,15 @@ from parity_util import host_input, to_cuda
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(scope="module", autouse=True)
+def _clear_device_status():
+    """Start this module with a clear device status word (other tests set its bits on purpose)."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert B.load_library().fp8_device_status(st.data_ptr(), 1, torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    yield
+
+
 def oracle_codes(M, N, K, a_fmt, b_fmt, seed):
     x = inputs.random_matrix(M, K, seed=seed, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e2)
     w = inputs.random_matrix(N, K, seed=seed + 1, dtype=torch.bfloat16, scale=0.02)
@@ -100,3 +109,24 @@ def test_gemm_k_zero_and_empty():
     B.fp8_gemm_blockwise(a, s, b, s, c=c)
     torch.cuda.synchronize()
     assert bool((c == 0).all())
+
+
+@pytest.mark.parametrize("a_fmt,b_fmt", [(B.E5M2, B.E4M3), (B.E4M3, B.E5M2), (B.E5M2, B.E5M2)])
+def test_gemm_mixed_formats(a_fmt, b_fmt):
+    """kind::f8f6f4 takes each operand's format separately: E5M2 gradients against E4M3 activations."""
+    for i, (M, N, K) in enumerate([(128, 256, 256), (384, 512, 768)]):
+        qa, sa, qb, sb = oracle_codes(M, N, K, a_fmt, b_fmt, seed=5300 + 10 * i + 3 * a_fmt + b_fmt)
+        c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
+                                 to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), a_fmt=a_fmt,
+                                 b_fmt=b_fmt, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        check_gemm(qa, sa, a_fmt, qb, sb, b_fmt, c, f"{M}x{N}x{K} fmts {a_fmt},{b_fmt}")
+
+
+def test_gemm_reports_no_wait_timeout():
+    """After every GEMM above, the device status word has no wait-timeout bit."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = B.load_library().fp8_device_status(st.data_ptr(), 0, torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) & B.DEVICE_STATUS_WAIT_TIMEOUT == 0
