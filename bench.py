@@ -421,6 +421,12 @@ def modes_breakdown(dev, stream, peak):
     put("delayed_e5m2_step", "bf16 gradients 8192x8192, |g| log-uniform [1e-6,1e-2], seed 3, W=16 "
         "(cast + amax in one pass, then the history update)", 3 * n, t_step)
     out["delayed_e5m2_history_update_us"] = round(t_hist * 1e3, 2)
+    ws = torch.zeros(4, dtype=torch.int32, device=dev)
+    fs = lambda r, st: raw.check(L.fp8_quantize_delayed_step(
+        gs[r % 2].data_ptr(), 1, n, 1, scale.data_ptr(), hist.data_ptr(), state.data_ptr(), 16, 0, 1.0, 1.0,
+        q.data_ptr(), used.data_ptr(), amax.data_ptr(), ws.data_ptr(), st), "delayed step")
+    put("delayed_e5m2_step_one_launch", "bf16 gradients 8192x8192, |g| log-uniform [1e-6,1e-2], seed 3, W=16 "
+        "(cast + amax + history update in one launch: the last CTA updates)", 3 * n, time_in_graph([fs], 32, dev))
     del gs, q
 
     # the consumer: blockwise-scaled FP8 GEMM on the tensor cores, 1x128 activations x 128x128 weights

@@ -46,6 +46,8 @@ SIGNATURES = {
     "fp8_quantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _vp]),
     "fp8_dequantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _vp, _vp, _c_int, _vp]),
     "fp8_gemm_blockwise": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _i64, _i64, _i64, _vp, _c_int, _vp]),
+    "fp8_quantize_delayed_step": (_c_int, [_vp, _c_int, _i64, _c_int, _vp, _vp, _vp, _c_int, _c_int, ctypes.c_float,
+                                           ctypes.c_float, _vp, _vp, _vp, _vp, _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_c_int]),
     "fp8_device_status": (_c_int, [_vp, _c_int, _vp]),
     "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
@@ -338,14 +340,37 @@ def fp8_amax_history_update_ex(history: torch.Tensor, state: torch.Tensor, amax:
     return scale
 
 
+def fp8_quantize_delayed_step(x: torch.Tensor, scale: torch.Tensor, history: torch.Tensor, state: torch.Tensor,
+                              fmt: int = E5M2, algo: int = AMAX_WINDOW_MAX, alpha: float = 1.0, margin: float = 1.0,
+                              q: torch.Tensor | None = None, scale_used: torch.Tensor | None = None,
+                              amax_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                              stream=None) -> torch.Tensor:
+    """Cast x with *scale, then (same launch) push amax(x) into the history and rewrite *scale."""
+    _need_cuda(x, scale, history, state, q, scale_used, amax_out, workspace)
+    dev = x.device
+    q = torch.empty(x.shape, dtype=torch.uint8, device=dev) if q is None else q
+    scale_used = torch.empty(1, dtype=torch.float32, device=dev) if scale_used is None else scale_used
+    amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
+    workspace = fused_workspace(dev) if workspace is None else workspace
+    st = load_library().fp8_quantize_delayed_step(_ptr(x), _DTYPE_CODE[x.dtype], x.numel(), fmt, _ptr(scale),
+                                                  _ptr(history), _ptr(state), history.numel(), algo, alpha, margin,
+                                                  _ptr(q), _ptr(scale_used), _ptr(amax_out), _ptr(workspace),
+                                                  _stream(stream))
+    _check("fp8_quantize_delayed_step", st)
+    return q
+
+
 class DelayedScaler:
     """Device-resident delayed-scaling state (history ring, {pos, count}, scale), after the
     PyTorch-FP8 page's DelayedScaler (s4.2).  step(x) quantizes x with the current scale, then
-    pushes amax(x) into the history -- all on the device, no host round trip."""
+    pushes amax(x) into the history -- all on the device, no host round trip.  fused=True (the
+    default) does both in one launch (fp8_quantize_delayed_step); fused=False uses the two calls."""
 
     def __init__(self, window: int = 16, fmt: int = E5M2, device="cuda", algo: int = AMAX_WINDOW_MAX,
-                 alpha: float = 1.0, margin: float = 1.0):
+                 alpha: float = 1.0, margin: float = 1.0, fused: bool = True):
         self.fmt = fmt
+        self.fused = fused
+        self.workspace = fused_workspace(device) if fused else None
         self.algo, self.alpha, self.margin = algo, alpha, margin
         self.history = torch.zeros(window, dtype=torch.float32, device=device)
         self.state = torch.zeros(2, dtype=torch.int32, device=device)
@@ -354,6 +379,11 @@ class DelayedScaler:
         self.scale_used = torch.ones(1, dtype=torch.float32, device=device)
 
     def step(self, x: torch.Tensor, q: torch.Tensor | None = None, stream=None):
+        if self.fused:
+            q = fp8_quantize_delayed_step(x, self.scale, self.history, self.state, self.fmt, self.algo, self.alpha,
+                                          self.margin, q=q, scale_used=self.scale_used, amax_out=self.amax,
+                                          workspace=self.workspace, stream=stream)
+            return q, self.scale_used
         q, s, _ = fp8_quantize_per_tensor(x, self.fmt, scale_in=self.scale, q=q, scale_out=self.scale_used,
                                           amax_out=self.amax, stream=stream)
         if self.algo == AMAX_WINDOW_MAX and self.margin == 1.0:

@@ -285,6 +285,28 @@ int fp8_amax_history_update_ex(float* history, int32_t* state, int window, const
                                                          static_cast<cudaStream_t>(stream)));
 }
 
+int fp8_quantize_delayed_step(const void* x, int dtype, int64_t n, int fmt, float* scale, float* history,
+                              int32_t* state, int window, int algo, float alpha, float margin, uint8_t* q,
+                              float* scale_used, float* amax_out, void* workspace, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (window <= 0 || window > 65536) return FP8_ERR_ARG;
+    if (algo != FP8_AMAX_WINDOW_MAX && algo != FP8_AMAX_EMA) return FP8_ERR_ARG;
+    if (!(alpha >= 0.0f && alpha <= 1.0f) || !(margin > 0.0f)) return FP8_ERR_ARG;
+    if (scale == nullptr || history == nullptr || state == nullptr || scale_used == nullptr || amax_out == nullptr ||
+        workspace == nullptr)
+        return FP8_ERR_NULL;
+    if (n > 0 && (x == nullptr || q == nullptr)) return FP8_ERR_NULL;
+    if (scale_used == scale) return FP8_ERR_ARG;  // the scale is rewritten in place
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4) || !aligned(history, 4) || !aligned(state, 4) ||
+        !aligned(scale_used, 4) || !aligned(amax_out, 4) || !aligned(workspace, 16))
+        return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_tensor_delayed_step(x, dtype, n, fmt, scale, q, scale_used, amax_out, history,
+                                                      state, window, algo, alpha, margin, workspace,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_device_status(uint32_t* status, int clear, void* stream) {
     if (status == nullptr) return FP8_ERR_NULL;
     if (!aligned(status, 4)) return FP8_ERR_ALIGN;

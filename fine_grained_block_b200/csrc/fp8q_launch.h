@@ -94,6 +94,14 @@ cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows,
                                          const float* scale_in, const float* amax_in, uint8_t* q, uint8_t* qt,
                                          float* scale_out, float* amax_out, cudaStream_t stream);
 
+// One delayed-scaling step in one launch: cast with *scale, amax(x), then (in
+// the last CTA) the history update that rewrites *scale.  16-byte workspace,
+// zero before the first call and left zero.
+cudaError_t launch_tensor_delayed_step(const void* x, int dtype, int64_t n, int fmt, float* scale, uint8_t* q,
+                                       float* scale_used, float* amax_out, float* history, int32_t* state,
+                                       int window, int algo, float alpha, float margin, void* workspace,
+                                       cudaStream_t stream);
+
 // Fused quantize -> dequantize round trip in x's dtype.  block_rows 0: per
 // tensor with *scale_in; 1 or 128: block scales (written to `scales` if it is
 // non-null).

@@ -11,6 +11,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "history_update.cuh"
 #include "launch_util.h"
 
 namespace fp8q {
@@ -43,52 +44,13 @@ k_amax_history_update(float* __restrict__ history, int32_t* __restrict__ state, 
     }
 }
 
-// PyTorch-FP8 page s4.3: the refreshed scale keeps a margin,
-// MAX / (max(amax, eps) * margin), both steps rounded in fp32.
-template <int FMT>
-__device__ __forceinline__ float scale_with_margin(float amax, float margin) {
-    return __fdiv_rn(fmt_max<FMT>(), __fmul_rn(fmaxf(amax, kAmaxEps), margin));
-}
-
-// The s4.3 refinements of delayed scaling.  algo 0: window max as above, with
-// the margin.  algo 1: exponential moving average of amax in history[0]
-// (first update m = amax, then m = RN(RN(alpha*amax) + RN(RN(1-alpha)*m)));
-// state[1] counts updates up to `window`, after which every update refreshes
-// the scale from m with the margin.
 template <int FMT>
 __global__ void __launch_bounds__(32)
 k_amax_history_update_ex(float* __restrict__ history, int32_t* __restrict__ state, int window,
                          const float* __restrict__ amax, float* __restrict__ scale, int algo, float alpha,
                          float margin) {
     pdl_enter();
-    const int lane = threadIdx.x;
-    const float a = *amax;
-    int count = min(max(state[1], 0), window);
-    if (algo == 1) {
-        if (lane == 0) {
-            const float m = (count == 0)
-                ? a
-                : __fadd_rn(__fmul_rn(alpha, a), __fmul_rn(__fsub_rn(1.0f, alpha), history[0]));
-            history[0] = m;
-            count = min(count + 1, window);
-            state[1] = count;
-            if (count == window) *scale = scale_with_margin<FMT>(m, margin);
-        }
-        return;
-    }
-    int pos = state[0] % window;
-    if (pos < 0) pos += window;
-    count = min(count + 1, window);
-    float m = 0.0f;
-    for (int i = lane; i < window; i += 32) m = fmaxf(m, (i == pos) ? a : history[i]);
-    m = warp_max<32>(m);
-    __syncwarp();  // every lane has read history[] before lane 0 writes it
-    if (lane == 0) {
-        history[pos] = a;
-        state[0] = (pos + 1 == window) ? 0 : pos + 1;
-        state[1] = count;
-        if (count == window) *scale = scale_with_margin<FMT>(m, margin);
-    }
+    history_update_warp<FMT>(history, state, window, *amax, scale, algo, alpha, margin);
 }
 
 }  // namespace

@@ -17,6 +17,7 @@
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
+#include "history_update.cuh"
 #include "launch_util.h"
 #include "lane_vec.cuh"
 
@@ -116,6 +117,84 @@ k_tensor_cast(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec
     // Written after every read of *scale_in in this CTA (the caller may pass
     // the same pointer for both; other CTAs read the same value either way).
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+}
+
+// ---------------------------------------------------------------------------
+// One step of delayed scaling in one launch: the cast with the given scale,
+// amax(x) from the same registers, and -- in whichever CTA finishes last --
+// the amax-history update that produces the next step's scale.  The same
+// result as the delayed cast followed by the history update kernel.
+//
+// Every CTA folds its amax into ws->amax_bits, then counts itself in
+// ws->arrivals (fence first); the CTA that takes the count to gridDim.x is
+// last, so it sees every CTA's amax.  It writes amax_out and scale_used, runs
+// the history update (one warp), and puts the workspace back to zero.  No CTA
+// waits for another.  *scale is read by every CTA before it counts itself and
+// written only by the last one, so it is updated in place.
+// ---------------------------------------------------------------------------
+struct StepWorkspace {
+    unsigned int arrivals;
+    unsigned int amax_bits;
+    unsigned int unused[2];
+};
+static_assert(sizeof(StepWorkspace) == 16, "workspace layout");
+
+template <typename T, int FMT, int BYTES>
+__global__ void __launch_bounds__(kThreads)
+k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec,
+                           const T* __restrict__ tail, int tail_n, float* scale,
+                           typename LaneVec<T, BYTES>::Out* __restrict__ q, uint8_t* __restrict__ q_tail,
+                           float* __restrict__ scale_used, float* __restrict__ amax_out, float* history,
+                           int32_t* state, int window, int algo, float alpha, float margin, StepWorkspace* ws) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    __shared__ float warp_amax[kThreads / 32];
+    __shared__ int last;
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x;
+    typename V::In v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * kThreads;
+        v[u] = (i < nvec) ? ld_words_stream(x + i) : V::zero();
+    }
+    const float s = *scale;
+    const uint64_t s2 = f32x2(s, s);
+    float a = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * kThreads;
+        a = fmaxf(a, V::amax(v[u]));
+        if (i < nvec) st_stream(q + i, V::template cast<FMT>(v[u], s2));
+    }
+    if (blockIdx.x == 0 && threadIdx.x < tail_n) {
+        const float xv = load_scalar(tail, threadIdx.x);
+        a = fmaxf(a, fabsf(xv));
+        q_tail[threadIdx.x] = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(xv, s), 0.0f) & 0xFFu);
+    }
+    a = warp_max<32>(a);
+    if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = a;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = warp_amax[0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_amax[w]);
+        atomicMax(&ws->amax_bits, __float_as_uint(m));  // non-negative floats order as their bits
+        __threadfence();
+        last = (atomicAdd(&ws->arrivals, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!last || threadIdx.x >= 32) return;
+    __threadfence();
+    const float amax = __uint_as_float(atomicAdd(&ws->amax_bits, 0u));
+    if (threadIdx.x == 0) {
+        *amax_out = amax;
+        *scale_used = s;
+    }
+    history_update_warp<FMT>(history, state, window, amax, scale, algo, alpha, margin);
+    if (threadIdx.x == 0) {
+        ws->amax_bits = 0u;
+        ws->arrivals = 0u;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -335,7 +414,52 @@ cudaError_t cast_transpose_width(const void* x, int64_t rows, int64_t cols, cons
                                            ok16 ? 1 : 0, st);
 }
 
+template <typename T, int FMT, int BYTES>
+cudaError_t delayed_step_typed(const void* x, int64_t n, float* scale, uint8_t* q, float* scale_used,
+                               float* amax_out, float* history, int32_t* state, int window, int algo, float alpha,
+                               float margin, void* workspace, cudaStream_t st) {
+    using V = LaneVec<T, BYTES>;
+    const int64_t nvec = n / V::kElems;
+    const int tail_n = static_cast<int>(n - nvec * V::kElems);
+    const T* tail = static_cast<const T*>(x) + nvec * V::kElems;
+    const int64_t grid = chunk_grid(nvec);
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const cudaError_t e = launch_kernel(k_tensor_cast_delayed_step<T, FMT, BYTES>, dim3(static_cast<unsigned>(grid)),
+                                        dim3(kThreads), 0, st, static_cast<const typename V::In*>(x), nvec, tail,
+                                        tail_n, scale, reinterpret_cast<typename V::Out*>(q), q + nvec * V::kElems,
+                                        scale_used, amax_out, history, state, window, algo, alpha, margin,
+                                        static_cast<StepWorkspace*>(workspace));
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <typename T, int FMT>
+cudaError_t delayed_step_width(const void* x, int64_t n, float* scale, uint8_t* q, float* scale_used,
+                               float* amax_out, float* history, int32_t* state, int window, int algo, float alpha,
+                               float margin, void* workspace, cudaStream_t st) {
+    if (aligned32(x))
+        return delayed_step_typed<T, FMT, 32>(x, n, scale, q, scale_used, amax_out, history, state, window, algo,
+                                              alpha, margin, workspace, st);
+    return delayed_step_typed<T, FMT, 16>(x, n, scale, q, scale_used, amax_out, history, state, window, algo, alpha,
+                                          margin, workspace, st);
+}
+
 }  // namespace
+
+cudaError_t launch_tensor_delayed_step(const void* x, int dtype, int64_t n, int fmt, float* scale, uint8_t* q,
+                                       float* scale_used, float* amax_out, float* history, int32_t* state,
+                                       int window, int algo, float alpha, float margin, void* workspace,
+                                       cudaStream_t st) {
+    if (dtype == 1) {
+        return fmt == kE4M3 ? delayed_step_width<uint16_t, kE4M3>(x, n, scale, q, scale_used, amax_out, history,
+                                                                  state, window, algo, alpha, margin, workspace, st)
+                            : delayed_step_width<uint16_t, kE5M2>(x, n, scale, q, scale_used, amax_out, history,
+                                                                  state, window, algo, alpha, margin, workspace, st);
+    }
+    return fmt == kE4M3 ? delayed_step_width<float, kE4M3>(x, n, scale, q, scale_used, amax_out, history, state,
+                                                           window, algo, alpha, margin, workspace, st)
+                        : delayed_step_width<float, kE5M2>(x, n, scale, q, scale_used, amax_out, history, state,
+                                                           window, algo, alpha, margin, workspace, st);
+}
 
 cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                          const float* scale_in, const float* amax_in, uint8_t* q, uint8_t* qt,

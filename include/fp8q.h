@@ -382,6 +382,32 @@ int fp8_amax_history_update_ex(float *history, int32_t *state, int window,
                                const float *amax, int fmt, float *scale,
                                int algo, float alpha, float margin, void *stream);
 
+/*
+ * One delayed-scaling step in one launch: exactly fp8_quantize_per_tensor with
+ * scale_in = scale (the delayed scale of [FP8-native] s4.2) followed by
+ * fp8_amax_history_update_ex (s4.2-4.3) on this step's amax, which rewrites
+ * *scale for the next step.  The CTA that finishes last performs the
+ * update, so no second launch and no host round trip is needed.
+ *
+ *   x, dtype, n, fmt, q   as in fp8_quantize_per_tensor
+ *   scale      [1] fp32 (device), in: this step's scale; out: the next one
+ *   history, state, window, algo, alpha, margin   as in
+ *              fp8_amax_history_update_ex
+ *   scale_used [1] fp32 (device): the scale this step used (must not be
+ *              `scale`)
+ *   amax_out   [1] fp32 (device): amax(x)
+ *   workspace  FP8_FUSED_WORKSPACE_BYTES of device memory, zero before the
+ *              first call and left zero by every call; calls that share it
+ *              must not overlap on the device
+ * Errors: those of the two calls it replaces; FP8_ERR_ARG also when
+ * scale_used == scale.
+ */
+int fp8_quantize_delayed_step(const void *x, int dtype, int64_t n, int fmt,
+                              float *scale, float *history, int32_t *state, int window,
+                              int algo, float alpha, float margin,
+                              uint8_t *q, float *scale_used, float *amax_out,
+                              void *workspace, void *stream);
+
 /* Static, human-readable text for a status code (never NULL). */
 const char *fp8_status_string(int status);
 

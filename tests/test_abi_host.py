@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
                                            "fp8_quantize_per_tensor_fused",
                                            "fp8_quantize_per_tensor_fused_noalloc", "fp8_amax_history_update_ex",
                                            "fp8_selftest_wait_timeout", "fp8_quantize_mx", "fp8_dequantize_mx",
-                                           "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise"])
+                                           "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise",
+                                           "fp8_quantize_delayed_step"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -193,6 +194,30 @@ def test_transpose_validation(L):
     assert f(A16, 1, 4, 64, 0, A16, A16, None, A16, None, None) == ERR_NULL      # qt
     assert f(A16, 1, 4, 64, 0, A16, A16, A1, A16, None, None) == ERR_ALIGN
     assert f(A16, 1, 4, 64, 0, A16, A1, A16, A16, None, None) == ERR_ALIGN
+
+
+def test_delayed_step_validation(L):
+    f = L.fp8_quantize_delayed_step
+    ok = (A16, 1, 64, 0, A16, A16, A16, 16, 0, 1.0, 1.0, A16, A16 + 16, A16, A16, None)
+    def call(**kw):
+        args = list(ok)
+        names = ["x", "dtype", "n", "fmt", "scale", "history", "state", "window", "algo", "alpha", "margin", "q",
+                 "scale_used", "amax_out", "workspace", "stream"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+    assert call(fmt=5) == ERR_FORMAT
+    assert call(dtype=4) == ERR_DTYPE
+    assert call(n=-1) == ERR_SHAPE
+    assert call(window=0) == ERR_ARG
+    assert call(algo=3) == ERR_ARG
+    assert call(alpha=2.0) == ERR_ARG
+    assert call(margin=0.0) == ERR_ARG
+    assert call(scale_used=A16) == ERR_ARG          # the same pointer as scale
+    assert call(workspace=None) == ERR_NULL
+    assert call(q=None) == ERR_NULL
+    assert call(history=A1) == ERR_ALIGN
+    assert call(workspace=A16 + 4) == ERR_ALIGN
 
 
 def test_gemm_validation(L):

@@ -638,3 +638,37 @@ def test_per_tensor_transpose_16_byte_aligned_input():
     oq, oqt, os_, oa = oracle.quantize_per_tensor_transpose(host_input(x_cpu), B.E4M3)
     assert_bytes_equal(qt, oqt, "qt")
     assert_bytes_equal(q, oq, "q")
+
+
+# -- one delayed-scaling step in one launch ---------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("algo,alpha,margin,window", [(0, 1.0, 1.0, 4), (0, 1.0, 1.1, 3), (1, 0.25, 1.0, 2)])
+def test_delayed_step_matches_oracle_and_two_calls(fmt, dtype, algo, alpha, margin, window):
+    """fp8_quantize_delayed_step == delayed cast + history update: codes, scale used, amax, next scale,
+    history and state, step after step, against the oracle and against the two separate calls."""
+    sizes = [0, 7, 4097, (1 << 20) + 3, 1 << 22]
+    fused = B.DelayedScaler(window=window, fmt=fmt, algo=algo, alpha=alpha, margin=margin, fused=True)
+    split = B.DelayedScaler(window=window, fmt=fmt, algo=algo, alpha=alpha, margin=margin, fused=False)
+    ref = oracle.AmaxHistory(window, fmt, algo=algo, alpha=alpha, margin=margin)
+    for k in range(2 * window + 4):
+        n = sizes[k % len(sizes)]
+        x_cpu = inputs.random_matrix(1, max(n, 1), seed=6000 + k, dtype=dtype, outlier_frac=1e-3,
+                                     factor=10.0 ** (k % 5)).reshape(-1)[:n]
+        x = to_cuda(x_cpu)
+        s_ref = float(ref.scale[0])
+        q1, s1 = fused.step(x)
+        q2, s2 = split.step(x)
+        oq, _, oa = oracle.quantize_per_tensor(host_input(x_cpu), fmt, scale=s_ref)
+        ref.update(oa)
+        torch.cuda.synchronize()
+        assert_bytes_equal(q1, oq, f"step {k} codes")
+        assert_bytes_equal(q1, q2.cpu().numpy(), f"step {k} codes vs two calls")
+        assert_bytes_equal(s1, fp32_bits([s_ref]), f"step {k} scale used")
+        assert_bytes_equal(fused.amax, fp32_bits([oa]), f"step {k} amax")
+        assert_bytes_equal(fused.scale, fp32_bits(ref.scale), f"step {k} next scale")
+        assert_bytes_equal(fused.scale, split.scale.cpu().numpy().view(np.uint32), f"step {k} next scale vs two calls")
+        assert fused.state.cpu().tolist() == split.state.cpu().tolist()
+        assert_bytes_equal(fused.history, split.history.cpu().numpy().view(np.uint32), f"step {k} history")
+    assert int(fused.workspace.abs().sum().item()) == 0  # left zero for the next call
