@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import ctypes
 import math
+import os
 
 import numpy as np
 
@@ -32,7 +33,10 @@ def lib() -> ctypes.CDLL:
     """Load (building first if needed) the oracle shared library."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        # ORACLE_LIB_PATH loads another build of the oracle source instead: the
+        # pin-strength test uses it to run the pins against deliberately broken
+        # copies and check that they fail.
+        path = os.environ.get("ORACLE_LIB_PATH") or _build.build()
         L = ctypes.CDLL(path)
         c_i64, c_int, c_void = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
         L.orc_fp8_decode.argtypes = [c_int, c_int]
