@@ -461,6 +461,51 @@ def modes_breakdown(dev, stream, peak):
             "peak_kind": peak_kind, "us": round(ms * 1e3, 2)}
         del qa, sa, qb, sb, cg
 
+    # size sweep 2^20 .. 2^30 elements (bf16, 0.1% x1e3 outliers, seed 4): GB/s per mode and size.  Sizes
+    # whose buffers fit in L2 rotate over enough copies that every launch reads from HBM.
+    sweep = {}
+    for lg in (20, 22, 24, 26, 28, 30):
+        x0 = inputs.sweep_tensor(lg, device=dev)
+        R, C = x0.shape
+        n = x0.numel()
+        set_bytes = 2 * n + n + 4 * (n // 128) + 2 * n
+        copies = max(1, math.ceil(3 * L2_BYTES / set_bytes))
+        xs_ = [x0] + [x0.clone() for _ in range(copies - 1)]
+        qs_ = [torch.empty(R, C, dtype=torch.uint8, device=dev) for _ in range(copies)]
+        ss_ = [torch.empty(R, C // 128, dtype=torch.float32, device=dev) for _ in range(copies)]
+        st_ = [torch.empty(R // 128 if R >= 128 else 1, C // 128, dtype=torch.float32, device=dev)
+               for _ in range(copies)]
+        ys_ = [torch.empty(R, C, dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+        so_ = torch.empty(1, dtype=torch.float32, device=dev)
+        ao_ = torch.empty(1, dtype=torch.float32, device=dev)
+        reps = max(10, min(200, copies * 4))
+        row = {}
+        t = time_in_graph([lambda r, st: raw.check(L.fp8_quantize_blockwise(
+            xs_[r % copies].data_ptr(), 1, R, C, 1, 128, 0, qs_[r % copies].data_ptr(), ss_[r % copies].data_ptr(),
+            st), "1x128")], reps, dev)
+        row["1x128_e4m3"] = round((3 * n + 4 * (n // 128)) / (t * 1e-3) / 1e9, 1)
+        if R >= 128:
+            t = time_in_graph([lambda r, st: raw.check(L.fp8_quantize_blockwise(
+                xs_[r % copies].data_ptr(), 1, R, C, 128, 128, 0, qs_[r % copies].data_ptr(),
+                st_[r % copies].data_ptr(), st), "128x128")], reps, dev)
+            row["128x128_e4m3"] = round((3 * n + 4 * (n // 16384)) / (t * 1e-3) / 1e9, 1)
+        # per-tensor: at least two inputs, so the reverse cast pass cannot hand the next launch's amax pass
+        # its data in L2
+        xp_ = xs_ if copies >= 2 else [x0, x0.clone()]
+        t = time_in_graph([lambda r, st: raw.check(L.fp8_quantize_per_tensor(
+            xp_[r % len(xp_)].data_ptr(), 1, n, 1, None, qs_[r % copies].data_ptr(), so_.data_ptr(),
+            ao_.data_ptr(), st), "per-tensor")], reps, dev)
+        row["per_tensor_current_e5m2"] = round(3 * n / (t * 1e-3) / 1e9, 1)
+        t = time_in_graph([lambda r, st: raw.check(L.fp8_dequantize(
+            qs_[r % copies].data_ptr(), 0, R, C, 1, 128, ss_[r % copies].data_ptr(), ys_[r % copies].data_ptr(), 1, st),
+            "dequant")], reps, dev)
+        row["1x128_dequant_bf16"] = round((3 * n + 4 * (n // 128)) / (t * 1e-3) / 1e9, 1)
+        row["buffer_sets"] = copies
+        sweep[f"2^{lg}"] = row
+        del x0, xs_, xp_, qs_, ss_, st_, ys_
+        torch.cuda.empty_cache()
+    out["sweep_GB_s"] = sweep
+
     # per-tensor current scaling on small tensors (latency-bound): two passes vs the one-pass kernel, each
     # launch timed alone after an untimed L2 flush
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
