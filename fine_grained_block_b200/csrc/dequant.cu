@@ -17,10 +17,14 @@
 // Inf codes (whose fma residual would be Inf - Inf), take the per-element IEEE
 // division instead.
 //
-// Each thread turns one group of codes into one 16-byte output vector: 8 codes
-// for bf16 output, 4 codes for fp32 output.  Consecutive lanes therefore read
-// consecutive code groups and write consecutive 16-byte vectors, so both the
-// loads and the stores of a warp are contiguous.
+// Each thread turns one group of codes into one 16- or 32-byte output vector
+// (8 or 16 codes for bf16 output, 4 or 8 for fp32).  Consecutive lanes
+// therefore read consecutive code groups and write consecutive vectors, so
+// both the loads and the stores of a warp are contiguous.
+//
+// MX codes (1x32 blocks, E8M0 scale bytes) need no division: the value is
+// decode(q) * 2^(byte - 127), one exact multiplication except at the ends of
+// the fp32 range.
 
 #include <algorithm>
 

@@ -17,7 +17,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Warp-loads per warp in the 1x128 kernel (each CTA covers 8 x LOADS
+// Warp-loads per warp in the row-block kernel for 1x128 blocks (each CTA covers 8 x LOADS
 // warp-loads = 32 KiB of bf16 with 32-byte lanes and LOADS = 4).
 #ifndef FP8Q_Q1X128_LOADS
 #define FP8Q_Q1X128_LOADS 4

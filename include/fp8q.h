@@ -11,17 +11,21 @@
  *                 section "FP8 training": per-tensor vs 1x128 / 128x128
  *                 block scaling (quant, per_tensor, per_block).
  *
- * Arithmetic, identical in every entry point:
+ * Arithmetic of the quantizers:
  *   amax  = max |x| over the scaled group (a block, or the whole tensor)
  *   s     = fp32( MAX / max(amax, 1e-12f) ),  MAX = 448 (E4M3), 57344 (E5M2)
+ *           (per tensor, per 1x128 or 128x128 block; MX blocks of 1x32 use
+ *           a power of two instead, see fp8_quantize_mx)
  *   q     = fp8_rne_satfinite( fp32(x * s) )   x widened to fp32 exactly
  *   y     = fp32( decode(q) / s ),  bf16 output = bf16_rne(y)
  * The stored scale is the multiplier s (not its reciprocal).  Casts round to
  * nearest-even and saturate: no Inf is ever produced, and E4M3 has no Inf.
+ * fp8_gemm_blockwise consumes 1x128 and 128x128 codes on the tensor cores.
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the
- *     library never allocates, frees or keeps them.
+ *     library never allocates, frees or keeps them (the no-allocation entry
+ *     point uses a fixed array of the library's own device memory).
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
  *     void*; NULL = the legacy default stream), never synchronizes, and is
  *     safe to call from several host threads.  Calls that touch the same
