@@ -14,6 +14,7 @@
 // contiguous chunk and issues all its loads before computing.
 
 #include <algorithm>
+#include <atomic>
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
@@ -213,6 +214,62 @@ k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x,
 constexpr int kTT = 128;           // tile side
 constexpr int kTStride = kTT + 16;  // smem row pitch in bytes (16-byte aligned rows)
 
+// Lane geometry of a full 128x128 tile: one lane vector (16 or 32 bytes of
+// x) per slice, 16 tile rows per warp.
+template <typename T, int BYTES>
+struct TileGeom {
+    static constexpr int kVecPerRow = kTT / LaneVec<T, BYTES>::kElems;  // lane slices per tile row
+    static constexpr int kRowsPerLoad = 32 / kVecPerRow;               // tile rows per warp-wide load
+    static constexpr int kLoads = 16 / kRowsPerLoad;                   // lane vectors per thread
+};
+
+// Cast a full tile held in registers (v[i] = tile row lr0 + i*kRowsPerLoad,
+// slice vec_in_row): codes to q (if any) and into the shared code tile.
+template <typename T, int FMT, int BYTES, bool WITH_AMAX>
+__device__ __forceinline__ void tile_cast(const typename LaneVec<T, BYTES>::In (&v)[TileGeom<T, BYTES>::kLoads],
+                                          uint64_t s2, uint8_t* q,
+                                          int64_t cols, int64_t r0, int64_t c0, uint8_t* tile, int lr0,
+                                          int vec_in_row, float& a) {
+    using V = LaneVec<T, BYTES>;
+    using G = TileGeom<T, BYTES>;
+#pragma unroll
+    for (int i = 0; i < G::kLoads; ++i) {
+        if (WITH_AMAX) a = fmaxf(a, V::amax(v[i]));
+        const typename V::Out c = V::template cast<FMT>(v[i], s2);
+        const int lr = lr0 + i * G::kRowsPerLoad;
+        if (q != nullptr) st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row, c);
+        *reinterpret_cast<typename V::Out*>(tile + lr * kTStride + vec_in_row * V::kElems) = c;
+    }
+}
+
+// qt from the shared code tile: lane l takes tile columns 4l..4l+3, warp w
+// tile rows 16w..16w+15.  It reads 16 words (4 codes of one tile row each;
+// the warp reads 128 consecutive bytes of a row: no bank conflicts),
+// transposes them in 4x4-byte blocks with byte permutes, and writes 16
+// consecutive codes into each of its 4 qt rows.
+__device__ __forceinline__ void tile_transpose_out(const uint8_t* tile, uint8_t* qt, int64_t rows, int64_t r0,
+                                                   int64_t c0, int lane, int warp) {
+    const int cq = lane * 4, rq = warp * 16;
+    uint32_t wv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) wv[i] = *reinterpret_cast<const uint32_t*>(tile + (rq + i) * kTStride + cq);
+    uint32_t o[4][4];  // o[j][g]: column cq+j, rows rq+4g..rq+4g+3
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const uint32_t w0 = wv[4 * g], w1 = wv[4 * g + 1], w2 = wv[4 * g + 2], w3 = wv[4 * g + 3];
+        const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), lo23 = __byte_perm(w2, w3, 0x5140);
+        const uint32_t hi01 = __byte_perm(w0, w1, 0x7362), hi23 = __byte_perm(w2, w3, 0x7362);
+        o[0][g] = __byte_perm(lo01, lo23, 0x5410);
+        o[1][g] = __byte_perm(lo01, lo23, 0x7632);
+        o[2][g] = __byte_perm(hi01, hi23, 0x5410);
+        o[3][g] = __byte_perm(hi01, hi23, 0x7632);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        st_stream(reinterpret_cast<uint4*>(qt + (c0 + cq + j) * rows + r0 + rq),
+                  make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]));
+}
+
 // Resident CTAs per SM the transposing cast is compiled for (register cap):
 // each CTA keeps one 32 KiB input tile in flight.
 #ifndef FP8Q_TRANSPOSE_MIN_CTAS
@@ -239,53 +296,16 @@ k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, con
     float a = 0.0f;
 
     if (vector_ok && h == kTT && w == kTT) {
-        constexpr int kVecPerRow = kTT / V::kElems;
-        constexpr int kRowsPerLoad = 32 / kVecPerRow;
-        constexpr int kLoads = 16 / kRowsPerLoad;
-        const int row_in_load = lane / kVecPerRow, vec_in_row = lane % kVecPerRow;
-        const int lr0 = warp * 16 + row_in_load;
+        using G = TileGeom<T, BYTES>;
+        const int lr0 = warp * 16 + lane / G::kVecPerRow, vec_in_row = lane % G::kVecPerRow;
         const auto* xv = reinterpret_cast<const typename V::In*>(x + (r0 + lr0) * cols + c0) + vec_in_row;
-        const int64_t vstride = cols / V::kElems * kRowsPerLoad;  // lane vectors between this lane's rows
-        typename V::In v[kLoads];
+        const int64_t vstride = cols / V::kElems * G::kRowsPerLoad;  // lane vectors between this lane's rows
+        typename V::In v[G::kLoads];
 #pragma unroll
-        for (int i = 0; i < kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
-#pragma unroll
-        for (int i = 0; i < kLoads; ++i) {
-            if (WITH_AMAX) a = fmaxf(a, V::amax(v[i]));
-            const typename V::Out c = V::template cast<FMT>(v[i], s2);
-            const int lr = lr0 + i * kRowsPerLoad;
-            if (q != nullptr)
-                st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row, c);
-            *reinterpret_cast<typename V::Out*>(tile + lr * kTStride + vec_in_row * V::kElems) = c;
-        }
+        for (int i = 0; i < G::kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
+        tile_cast<T, FMT, BYTES, WITH_AMAX>(v, s2, q, cols, r0, c0, tile, lr0, vec_in_row, a);
         __syncthreads();
-        // qt: lane l takes tile columns 4l..4l+3, warp w tile rows 16w..16w+15.
-        // It reads 16 words (4 codes of one tile row each; the warp reads
-        // 128 consecutive bytes of a row: no bank conflicts), transposes
-        // them in 4x4-byte blocks with byte permutes, and writes 16
-        // consecutive codes into each of its 4 qt rows.
-        {
-            const int cq = lane * 4, rq = warp * 16;
-            uint32_t wv[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                wv[i] = *reinterpret_cast<const uint32_t*>(tile + (rq + i) * kTStride + cq);
-            uint32_t o[4][4];  // o[j][g]: column cq+j, rows rq+4g..rq+4g+3
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const uint32_t w0 = wv[4 * g], w1 = wv[4 * g + 1], w2 = wv[4 * g + 2], w3 = wv[4 * g + 3];
-                const uint32_t lo01 = __byte_perm(w0, w1, 0x5140), lo23 = __byte_perm(w2, w3, 0x5140);
-                const uint32_t hi01 = __byte_perm(w0, w1, 0x7362), hi23 = __byte_perm(w2, w3, 0x7362);
-                o[0][g] = __byte_perm(lo01, lo23, 0x5410);
-                o[1][g] = __byte_perm(lo01, lo23, 0x7632);
-                o[2][g] = __byte_perm(hi01, hi23, 0x5410);
-                o[3][g] = __byte_perm(hi01, hi23, 0x7632);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                st_stream(reinterpret_cast<uint4*>(qt + (c0 + cq + j) * rows + r0 + rq),
-                          make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]));
-        }
+        tile_transpose_out(tile, qt, rows, r0, c0, lane, warp);
     } else {
         for (int i = threadIdx.x; i < kTT * kTT; i += kThreads) {
             const int r = i / kTT, c = i % kTT;
