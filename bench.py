@@ -493,6 +493,28 @@ def modes_breakdown(dev, stream, peak):
             "peak_kind": peak_kind, "us": round(ms * 1e3, 2)}
         del qa, sa, qb, sb, cg
 
+    # many small tensors: 128 weights of 1024x1024 bf16 (2^20 elements each, 256 MiB in all), 128x128 E4M3,
+    # one call per tensor against one grouped call
+    from fine_grained_block_b200.binding import FP8BlockTensor
+    ws_ = [inputs.random_matrix(1024, 1024, seed=100 + i, dtype=torch.bfloat16, scale=0.02, device=dev)
+           for i in range(128)]
+    wq_ = [torch.empty(1024, 1024, dtype=torch.uint8, device=dev) for _ in ws_]
+    wsc_ = [torch.empty(8, 8, dtype=torch.float32, device=dev) for _ in ws_]
+    arr = (FP8BlockTensor * len(ws_))(*[FP8BlockTensor(w.data_ptr(), q_.data_ptr(), s_.data_ptr(), 1024, 1024)
+                                        for w, q_, s_ in zip(ws_, wq_, wsc_)])
+    nb = sum(3 * w.numel() + 4 * 64 for w in ws_)
+
+    def one_by_one(r, st):
+        for w, q_, s_ in zip(ws_, wq_, wsc_):
+            raw.check(L.fp8_quantize_blockwise(w.data_ptr(), 1, 1024, 1024, 128, 128, 0, q_.data_ptr(), s_.data_ptr(),
+                                               st), "128x128")
+    put("128_weights_1024x1024_128x128_one_call_each", "128 bf16 weights 1024x1024, N(0,0.02^2), seeds 100..227 "
+        "(128 launches)", nb, time_in_graph([one_by_one], 4, dev))
+    put("128_weights_1024x1024_128x128_grouped", "the same 128 weights in one fp8_quantize_blockwise_grouped call "
+        "(1 launch)", nb, time_in_graph([lambda r, st: raw.check(L.fp8_quantize_blockwise_grouped(
+            arr, len(ws_), 1, 128, 128, 0, st), "grouped")], 16, dev))
+    del ws_, wq_, wsc_, arr
+
     # size sweep 2^20 .. 2^30 elements (bf16, 0.1% x1e3 outliers, seed 4): GB/s per mode and size.  Sizes
     # whose buffers fit in L2 rotate over enough copies that every launch reads from HBM.
     sweep = {}

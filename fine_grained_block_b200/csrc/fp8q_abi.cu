@@ -6,6 +6,7 @@
 // the SM count.
 
 #include <atomic>
+#include <cstddef>
 #include <cstdint>
 
 #include <cuda_runtime.h>
@@ -174,6 +175,35 @@ int fp8_quantize_blockwise(const void* x, int dtype, int64_t rows, int64_t cols,
         e = fp8q::launch_quant_128x128(x, dtype, rows, cols, fmt, q, scales, st);
     }
     return status_of(e);
+}
+
+static_assert(sizeof(fp8_block_tensor) == sizeof(fp8q::GroupTensor) &&
+                  offsetof(fp8_block_tensor, x) == offsetof(fp8q::GroupTensor, x) &&
+                  offsetof(fp8_block_tensor, q) == offsetof(fp8q::GroupTensor, q) &&
+                  offsetof(fp8_block_tensor, scales) == offsetof(fp8q::GroupTensor, scales) &&
+                  offsetof(fp8_block_tensor, rows) == offsetof(fp8q::GroupTensor, rows) &&
+                  offsetof(fp8_block_tensor, cols) == offsetof(fp8q::GroupTensor, cols),
+              "fp8_block_tensor and the launcher's descriptor share one layout");
+
+int fp8_quantize_blockwise_grouped(const fp8_block_tensor* tensors, int count, int dtype, int block_rows,
+                                   int block_cols, int fmt, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (count < 0) return FP8_ERR_ARG;
+    if (!((block_rows == 1 || block_rows == 128) && block_cols == 128)) return FP8_ERR_SHAPE;
+    if (count == 0) return FP8_OK;
+    if (tensors == nullptr) return FP8_ERR_NULL;
+    for (int i = 0; i < count; ++i) {
+        const fp8_block_tensor& t = tensors[i];
+        if (t.rows < 0 || t.cols < 0 || t.cols % 128 != 0) return FP8_ERR_SHAPE;
+        const int64_t n = checked_count(t.rows, t.cols);
+        if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+        if (n == 0) continue;
+        if (t.x == nullptr || t.q == nullptr || t.scales == nullptr) return FP8_ERR_NULL;
+        if (!aligned(t.x, 16) || !aligned(t.q, 16) || !aligned(t.scales, 4)) return FP8_ERR_ALIGN;
+    }
+    return status_of(fp8q::launch_quant_grouped(reinterpret_cast<const fp8q::GroupTensor*>(tensors), count, dtype,
+                                                block_rows, fmt, static_cast<cudaStream_t>(stream)));
 }
 
 int fp8_dequantize(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int block_rows, int block_cols,

@@ -19,6 +19,18 @@ int device_sm_count();
 cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fmt,
                                uint8_t* q, float* scales, cudaStream_t stream);
 
+// Grouped blockwise quantization: `count` tensors (cols % 128 == 0 each) in
+// as few launches as possible (up to 128 tensors per launch).
+struct GroupTensor {
+    const void* x;
+    uint8_t* q;
+    float* scales;
+    int64_t rows;
+    int64_t cols;
+};
+cudaError_t launch_quant_grouped(const GroupTensor* tensors, int count, int dtype, int block_rows, int fmt,
+                                 cudaStream_t stream);
+
 // 128x128 blocks over [rows, cols], cols % 128 == 0, any rows.
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                  uint8_t* q, float* scales, cudaStream_t stream);

@@ -56,11 +56,13 @@ struct Pow2Scale {  // MX: s = 2^k, stored as the E8M0 byte of 2^-k
 // its warp-loads before it computes, and finished CTAs are replaced by new
 // ones, so each SM keeps its resident CTAs' chunks in flight.
 // ---------------------------------------------------------------------------
+// One CTA's chunk `cta` of the row blocks (the body of k_quant_rowblocks, also
+// run by the grouped kernel for each tensor's chunks).
 template <typename T, int FMT, int BYTES, int LOADS, int BW, typename SCALE>
-__global__ void __launch_bounds__(kThreads)
-k_quant_rowblocks(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
-                  typename SCALE::Stored* __restrict__ scales, int64_t nblocks, int rule) {
-    pdl_enter();
+__device__ __forceinline__ void quant_rowblocks_cta(const typename LaneVec<T, BYTES>::In* __restrict__ x,
+                                                    typename LaneVec<T, BYTES>::Out* __restrict__ q,
+                                                    typename SCALE::Stored* __restrict__ scales, int64_t nblocks,
+                                                    int rule, int64_t cta) {
     using V = LaneVec<T, BYTES>;
     constexpr int kLanesPerBlock = BW / V::kElems;
     constexpr int kBlocksPerLoad = 32 / kLanesPerBlock;
@@ -68,7 +70,7 @@ k_quant_rowblocks(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename
     const int lane = threadIdx.x & 31;
     const int sub_block = lane / kLanesPerBlock;
     const int64_t nloads = (nblocks + kBlocksPerLoad - 1) / kBlocksPerLoad;
-    const int64_t l0 = (static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5)) * LOADS;
+    const int64_t l0 = (cta * (kThreads / 32) + (threadIdx.x >> 5)) * LOADS;
 
     typename V::In v[LOADS];
 #pragma unroll
@@ -91,6 +93,14 @@ k_quant_rowblocks(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename
     }
 }
 
+template <typename T, int FMT, int BYTES, int LOADS, int BW, typename SCALE>
+__global__ void __launch_bounds__(kThreads)
+k_quant_rowblocks(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
+                  typename SCALE::Stored* __restrict__ scales, int64_t nblocks, int rule) {
+    pdl_enter();
+    quant_rowblocks_cta<T, FMT, BYTES, LOADS, BW, SCALE>(x, q, scales, nblocks, rule, blockIdx.x);
+}
+
 // ---------------------------------------------------------------------------
 // 128x128, register-resident tile: one CTA per tile, 8 warps, each warp owns
 // 16 rows of the tile.  One warp-wide load covers 32 / (128 / kElems) tile
@@ -102,11 +112,13 @@ k_quant_rowblocks(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename
 // GB/s against 6446 GB/s here, because 4 register-resident CTAs per SM keep 4
 // tiles both in flight and in process.)
 // ---------------------------------------------------------------------------
+// Tile `tile` of a [rows, cols] tensor (the body of k_quant_128x128, also run
+// by the grouped kernel for each tensor's tiles).
 template <typename T, int FMT, int BYTES>
-__global__ void __launch_bounds__(kThreads)
-k_quant_128x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
-                float* __restrict__ scales, int64_t rows, int64_t cols) {
-    pdl_enter();
+__device__ __forceinline__ void quant_tile_128x128(const typename LaneVec<T, BYTES>::In* __restrict__ x,
+                                                   typename LaneVec<T, BYTES>::Out* __restrict__ q,
+                                                   float* __restrict__ scales, int64_t rows, int64_t cols,
+                                                   int64_t tile) {
     using V = LaneVec<T, BYTES>;
     constexpr int kVecPerRow = 128 / V::kElems;                // lane slices per tile row
     constexpr int kRowsPerLoad = 32 / kVecPerRow;
@@ -116,8 +128,8 @@ k_quant_128x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename L
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t tiles_c = cols >> 7;
-    const int64_t tr = blockIdx.x / tiles_c;
-    const int64_t tc = blockIdx.x - tr * tiles_c;
+    const int64_t tr = tile / tiles_c;
+    const int64_t tc = tile - tr * tiles_c;
     const int row_in_load = lane / kVecPerRow;
     const int vec_in_row = lane % kVecPerRow;
     const int64_t vec_cols = cols / V::kElems;                 // lane slices per tensor row
@@ -146,7 +158,15 @@ k_quant_128x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename L
         const int64_t r = r_base + i * kRowsPerLoad;
         if (r < rows) st_stream(q + v_base + i * kRowsPerLoad * vec_cols, V::template cast<FMT>(v[i], s2));
     }
-    if (threadIdx.x == 0) scales[blockIdx.x] = s;
+    if (threadIdx.x == 0) scales[tile] = s;
+}
+
+template <typename T, int FMT, int BYTES>
+__global__ void __launch_bounds__(kThreads)
+k_quant_128x128(const typename LaneVec<T, BYTES>::In* __restrict__ x, typename LaneVec<T, BYTES>::Out* __restrict__ q,
+                float* __restrict__ scales, int64_t rows, int64_t cols) {
+    pdl_enter();
+    quant_tile_128x128<T, FMT, BYTES>(x, q, scales, rows, cols, blockIdx.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -220,6 +240,48 @@ k_quant_mx_general(const T* __restrict__ x, uint8_t* __restrict__ q, uint8_t* __
         const float s = mx_scale<FMT>(amax, rule, byte);
         if (in) q[r * cols + c] = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(v, s), 0.0f) & 0xFFu);
         if (lane == 0) e8m0[b] = byte;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Grouped: many tensors in one launch.  The tensors' work units (128x128
+// tiles, or 1x128 row-block chunks) are numbered consecutively across the
+// group; a CTA finds its tensor by binary search over the units' starting
+// indices, which travel with the tensors' pointers and shapes in the kernel's
+// parameter space.  Many small tensors then cost one launch instead of one
+// each, and their blocks fill the GPU together.
+// ---------------------------------------------------------------------------
+constexpr int kGroupMax = 128;  // tensors per launch (the parameter block stays near 6 KiB)
+
+using GroupEntry = GroupTensor;
+
+struct GroupTable {
+    int count;
+    int64_t start[kGroupMax + 1];  // start[i] = first unit of tensor i; start[count] = all units
+    GroupEntry e[kGroupMax];
+};
+
+template <typename T, int FMT, int BYTES, int MODE>
+__global__ void __launch_bounds__(kThreads)
+k_quant_grouped(const __grid_constant__ GroupTable tab) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    const int64_t b = blockIdx.x;
+    int lo = 0, hi = tab.count;  // start[lo] <= b < start[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tab.start[mid] <= b) lo = mid;
+        else hi = mid;
+    }
+    const GroupEntry& e = tab.e[lo];
+    const int64_t unit = b - tab.start[lo];
+    if (MODE == 2) {
+        quant_tile_128x128<T, FMT, BYTES>(static_cast<const typename V::In*>(e.x),
+                                          reinterpret_cast<typename V::Out*>(e.q), e.scales, e.rows, e.cols, unit);
+    } else {
+        quant_rowblocks_cta<T, FMT, BYTES, FP8Q_Q1X128_LOADS, 128, RatioScale<FMT>>(
+            static_cast<const typename V::In*>(e.x), reinterpret_cast<typename V::Out*>(e.q), e.scales,
+            e.rows * e.cols / 128, 0, unit);
     }
 }
 
@@ -321,6 +383,61 @@ cudaError_t launch_quant_block_general(const void* x, int dtype, int64_t rows, i
     }
     return fmt == kE4M3 ? launch_general_typed<float, kE4M3>(x, rows, cols, br, bc, q, scales, st)
                         : launch_general_typed<float, kE5M2>(x, rows, cols, br, bc, q, scales, st);
+}
+
+namespace {
+
+// Work units of one tensor in the grouped kernel.
+template <typename T, int BYTES>
+int64_t group_units(int64_t rows, int64_t cols, int block_rows) {
+    if (rows == 0 || cols == 0) return 0;
+    if (block_rows == 128) return ((rows + 127) / 128) * (cols / 128);
+    using V = LaneVec<T, BYTES>;
+    constexpr int kBlocksPerLoad = 32 / (128 / V::kElems);
+    const int64_t nblocks = rows * cols / 128;
+    const int64_t nloads = (nblocks + kBlocksPerLoad - 1) / kBlocksPerLoad;
+    const int64_t per_cta = static_cast<int64_t>(kThreads / 32) * FP8Q_Q1X128_LOADS;
+    return (nloads + per_cta - 1) / per_cta;
+}
+
+template <typename T, int FMT, int BYTES>
+cudaError_t launch_grouped_typed(const GroupTensor* t, int count, int block_rows, cudaStream_t st) {
+    GroupTable tab;
+    for (int first = 0; first < count; first += kGroupMax) {
+        tab.count = std::min(kGroupMax, count - first);
+        int64_t units = 0;
+        for (int i = 0; i < tab.count; ++i) {
+            tab.e[i] = t[first + i];
+            tab.start[i] = units;
+            units += group_units<T, BYTES>(t[first + i].rows, t[first + i].cols, block_rows);
+        }
+        tab.start[tab.count] = units;
+        if (units == 0) continue;
+        if (units > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        auto kern = block_rows == 128 ? k_quant_grouped<T, FMT, BYTES, 2> : k_quant_grouped<T, FMT, BYTES, 1>;
+        const cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(units)), dim3(kThreads), 0, st, tab);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T, int FMT>
+cudaError_t launch_grouped_width(const GroupTensor* t, int count, int block_rows, cudaStream_t st) {
+    bool w32 = true;  // 256-bit lanes only when every tensor allows them
+    for (int i = 0; i < count; ++i) w32 = w32 && aligned32(t[i].x);
+    return w32 ? launch_grouped_typed<T, FMT, 32>(t, count, block_rows, st)
+               : launch_grouped_typed<T, FMT, 16>(t, count, block_rows, st);
+}
+
+}  // namespace
+
+cudaError_t launch_quant_grouped(const GroupTensor* t, int count, int dtype, int block_rows, int fmt,
+                                 cudaStream_t st) {
+    if (dtype == 1)
+        return fmt == kE4M3 ? launch_grouped_width<uint16_t, kE4M3>(t, count, block_rows, st)
+                            : launch_grouped_width<uint16_t, kE5M2>(t, count, block_rows, st);
+    return fmt == kE4M3 ? launch_grouped_width<float, kE4M3>(t, count, block_rows, st)
+                        : launch_grouped_width<float, kE5M2>(t, count, block_rows, st);
 }
 
 cudaError_t launch_quant_mx(const void* x, int dtype, int64_t rows, int64_t cols, int fmt, int rule, uint8_t* q,

@@ -195,6 +195,31 @@ int fp8_quantize_blockwise(const void *x, int dtype, int64_t rows, int64_t cols,
                            uint8_t *q, float *scales, void *stream);
 
 /*
+ * Grouped blockwise quantization: fp8_quantize_blockwise over `count`
+ * tensors, with the same codes and scales as one call per tensor, in as few
+ * launches as possible (up to 128 tensors share one).  For the many small
+ * weights and activations of a training step, whose single launches are
+ * dominated by their fixed cost.
+ *
+ *   tensors    host array of `count` descriptors (read during the call; the
+ *              pointers in them are device pointers, as in
+ *              fp8_quantize_blockwise)
+ *   block_rows, block_cols   (1, 128) or (128, 128), for all tensors
+ * Every tensor needs cols % 128 == 0 (FP8_ERR_SHAPE otherwise; ragged
+ * widths go through fp8_quantize_blockwise).  Empty tensors are skipped.
+ * Errors: those of fp8_quantize_blockwise; FP8_ERR_ARG for count < 0.
+ */
+typedef struct fp8_block_tensor {
+    const void *x;      /* [rows, cols] input, dtype */
+    uint8_t *q;         /* [rows, cols] codes */
+    float *scales;      /* block scales, the layout of fp8_quantize_blockwise */
+    int64_t rows;
+    int64_t cols;
+} fp8_block_tensor;
+int fp8_quantize_blockwise_grouped(const fp8_block_tensor *tensors, int count, int dtype,
+                                   int block_rows, int block_cols, int fmt, void *stream);
+
+/*
  * Dequantization: y = fp32(decode(q) / s), with s the scale of q's block.
  * Follows [FP8-native] s4.1 (divide by the scale to restore) and s4.2
  * quantize() (.to(dtype) / scale).

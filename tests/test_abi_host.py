@@ -36,7 +36,7 @@ def test_header_declares_the_boundary():
                                            "fp8_quantize_per_tensor_fused_noalloc", "fp8_amax_history_update_ex",
                                            "fp8_selftest_wait_timeout", "fp8_quantize_mx", "fp8_dequantize_mx",
                                            "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise",
-                                           "fp8_quantize_delayed_step"])
+                                           "fp8_quantize_delayed_step", "fp8_quantize_blockwise_grouped"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -218,6 +218,21 @@ def test_delayed_step_validation(L):
     assert call(q=None) == ERR_NULL
     assert call(history=A1) == ERR_ALIGN
     assert call(workspace=A16 + 4) == ERR_ALIGN
+
+
+def test_grouped_validation(L):
+    T = binding.FP8BlockTensor
+    g = L.fp8_quantize_blockwise_grouped
+    good = (T * 2)(T(A16, A16, A16, 128, 256), T(A16, A16, A16, 3, 128))
+    assert g(good, 2, 1, 1, 128, 9, None) == ERR_FORMAT
+    assert g(good, 2, 3, 1, 128, 0, None) == ERR_DTYPE
+    assert g(good, -1, 1, 1, 128, 0, None) == ERR_ARG
+    assert g(good, 2, 1, 64, 128, 0, None) == ERR_SHAPE
+    assert g(None, 0, 1, 1, 128, 0, None) == OK            # nothing to do
+    assert g(None, 2, 1, 1, 128, 0, None) == ERR_NULL
+    assert g((T * 1)(T(A16, A16, A16, 4, 100)), 1, 1, 1, 128, 0, None) == ERR_SHAPE   # cols % 128
+    assert g((T * 1)(T(A16, None, A16, 4, 128)), 1, 1, 1, 128, 0, None) == ERR_NULL
+    assert g((T * 1)(T(A1, A16, A16, 4, 128)), 1, 1, 1, 128, 0, None) == ERR_ALIGN
 
 
 def test_gemm_validation(L):

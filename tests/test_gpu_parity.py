@@ -672,3 +672,31 @@ def test_delayed_step_matches_oracle_and_two_calls(fmt, dtype, algo, alpha, marg
         assert fused.state.cpu().tolist() == split.state.cpu().tolist()
         assert_bytes_equal(fused.history, split.history.cpu().numpy().view(np.uint32), f"step {k} history")
     assert int(fused.workspace.abs().sum().item()) == 0  # left zero for the next call
+
+
+# -- grouped blockwise quantization ---------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("block", [(1, 128), (128, 128)])
+def test_grouped_matches_oracle(fmt, dtype, block):
+    shapes = [(128, 128), (300, 256), (1, 128), (0, 128), (129, 384), (1024, 1024), (7, 128), (256, 0)]
+    shapes += [(64 + (i % 5), 128 * (1 + i % 3)) for i in range(140)]  # more than one launch's worth
+    xs_cpu = [inputs.random_matrix(max(R, 1), max(C, 1), seed=7000 + i, dtype=dtype, outlier_frac=0.01,
+                                   factor=1e3)[:R, :C].contiguous() for i, (R, C) in enumerate(shapes)]
+    xs = [to_cuda(x) for x in xs_cpu]
+    # one tensor 16- but not 32-byte aligned: the whole group takes 16-byte lanes
+    esz = xs_cpu[1].element_size()
+    buf = torch.empty(xs_cpu[1].numel() + 16 // esz, dtype=dtype, device="cuda")
+    xs[1] = buf[16 // esz:].view(xs_cpu[1].shape)
+    xs[1].copy_(xs_cpu[1].to("cuda"))
+    for lanes in ("16-byte", "32-byte"):
+        group = xs if lanes == "16-byte" else [xs[0], to_cuda(xs_cpu[1])] + xs[2:]
+        qs, ss = B.fp8_quantize_blockwise_grouped(group, block, fmt)
+        torch.cuda.synchronize()
+        for i, (x_cpu, q, s) in enumerate(zip(xs_cpu, qs, ss)):
+            if x_cpu.numel() == 0:
+                continue
+            oq, os_ = oracle.quantize_blockwise(host_input(x_cpu), *block, fmt)
+            assert_bytes_equal(s, fp32_bits(os_), f"{lanes} tensor {i} scales")
+            assert_bytes_equal(q, oq, f"{lanes} tensor {i} codes")
