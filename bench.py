@@ -703,7 +703,7 @@ def run_ours(args):
     value = (qb + db) * args.steps * world / (total_ms * 1e-3) / 1e9
 
     # end to end through the same C ABI with host buffers: H2D of the input from pinned memory, both
-    # kernels, D2H of codes, scales and the dequantized tensor, every step, all on `stream`
+    # kernels, D2H of codes, scales and the dequantized tensor, every step
     hx = w0.cpu().pin_memory()
     hq = torch.empty(ROWS, COLS, dtype=torch.uint8).pin_memory()
     hs = torch.empty(ROWS // 128, COLS // 128, dtype=torch.float32).pin_memory()
