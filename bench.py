@@ -515,6 +515,34 @@ def modes_breakdown(dev, stream, peak):
             arr, len(ws_), 1, 128, 128, 0, st), "grouped")], 16, dev))
     del ws_, wq_, wsc_, arr
 
+    # many small per-tensor delayed steps: 128 bf16 gradients of 2^20 elements, E5M2, W=16; one
+    # fp8_quantize_delayed_step per tensor against one grouped call
+    from fine_grained_block_b200.binding import FP8DelayedTensor
+    gx_ = [inputs.random_matrix(1, 1 << 20, seed=300 + i, dtype=torch.bfloat16, scale=1e-3, device=dev).reshape(-1)
+           for i in range(128)]
+    gq_ = [torch.empty(1 << 20, dtype=torch.uint8, device=dev) for _ in gx_]
+    gst_ = [(torch.ones(1, device=dev), torch.zeros(16, device=dev), torch.zeros(2, dtype=torch.int32, device=dev),
+             torch.empty(1, device=dev), torch.empty(1, device=dev)) for _ in gx_]
+    gws_ = torch.zeros(len(gx_) * 4, dtype=torch.int32, device=dev)
+    garr = (FP8DelayedTensor * len(gx_))(*[FP8DelayedTensor(x_.data_ptr(), q_.data_ptr(), x_.numel(), sc_.data_ptr(),
+                                                            h_.data_ptr(), stt_.data_ptr(), su_.data_ptr(),
+                                                            am_.data_ptr())
+                                           for x_, q_, (sc_, h_, stt_, su_, am_) in zip(gx_, gq_, gst_)])
+    gnb = 3 * sum(x_.numel() for x_ in gx_)
+
+    def steps_one_by_one(r, st):
+        for i, (x_, q_, (sc_, h_, stt_, su_, am_)) in enumerate(zip(gx_, gq_, gst_)):
+            raw.check(L.fp8_quantize_delayed_step(x_.data_ptr(), 1, x_.numel(), 1, sc_.data_ptr(), h_.data_ptr(),
+                                                  stt_.data_ptr(), 16, 0, 1.0, 1.0, q_.data_ptr(), su_.data_ptr(),
+                                                  am_.data_ptr(), gws_[4 * i:4 * i + 4].data_ptr(), st), "step")
+    put("128_gradients_2^20_delayed_e5m2_one_call_each", "128 bf16 tensors of 2^20 elements, N(0,1e-6), seeds "
+        "300..427, W=16 (128 launches)", gnb, time_in_graph([steps_one_by_one], 4, dev))
+    put("128_gradients_2^20_delayed_e5m2_grouped", "the same 128 tensors in one fp8_quantize_delayed_step_grouped "
+        "call (2 launches of up to 96 tensors)", gnb, time_in_graph([lambda r, st: raw.check(
+            L.fp8_quantize_delayed_step_grouped(garr, len(gx_), 1, 1, 16, 0, 1.0, 1.0, gws_.data_ptr(), st),
+            "grouped step")], 16, dev))
+    del gx_, gq_, gst_, gws_, garr
+
     # size sweep 2^20 .. 2^30 elements (bf16, 0.1% x1e3 outliers, seed 4): GB/s per mode and size.  Sizes
     # whose buffers fit in L2 rotate over enough copies that every launch reads from HBM.
     sweep = {}

@@ -34,6 +34,13 @@ class FP8BlockTensor(ctypes.Structure):
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
+class FP8DelayedTensor(ctypes.Structure):
+    """struct fp8_delayed_tensor of include/fp8q.h."""
+    _fields_ = [("x", ctypes.c_void_p), ("q", ctypes.c_void_p), ("n", ctypes.c_int64), ("scale", ctypes.c_void_p),
+                ("history", ctypes.c_void_p), ("state", ctypes.c_void_p), ("scale_used", ctypes.c_void_p),
+                ("amax_out", ctypes.c_void_p)]
+
+
 # Declared in include/fp8q.h: name -> (restype, argtypes)
 _c_int, _i64, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
 SIGNATURES = {
@@ -56,6 +63,8 @@ SIGNATURES = {
                                            ctypes.c_float, _vp, _vp, _vp, _vp, _vp]),
     "fp8_quantize_blockwise_grouped": (_c_int, [ctypes.POINTER(FP8BlockTensor), _c_int, _c_int, _c_int, _c_int,
                                                 _c_int, _vp]),
+    "fp8_quantize_delayed_step_grouped": (_c_int, [ctypes.POINTER(FP8DelayedTensor), _c_int, _c_int, _c_int, _c_int,
+                                                   _c_int, ctypes.c_float, ctypes.c_float, _vp, _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_c_int]),
     "fp8_device_status": (_c_int, [_vp, _c_int, _vp]),
     "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
@@ -390,6 +399,38 @@ def fp8_quantize_delayed_step(x: torch.Tensor, scale: torch.Tensor, history: tor
                                                   _stream(stream))
     _check("fp8_quantize_delayed_step", st)
     return q
+
+
+def fp8_quantize_delayed_step_grouped(xs, scalers, qs=None, workspace: torch.Tensor | None = None, stream=None):
+    """One delayed-scaling step for several tensors in as few launches as possible.
+
+    scalers: one DelayedScaler per tensor (same fmt, window, algo, alpha and margin); each is stepped as
+    scaler.step(x) would step it.  Returns the list of codes."""
+    xs, scalers = list(xs), list(scalers)
+    if len(xs) != len(scalers):
+        raise ValueError("one scaler per tensor")
+    if not xs:
+        return []
+    s0 = scalers[0]
+    if any((s.fmt, s.history.numel(), s.algo, s.alpha, s.margin) !=
+           (s0.fmt, s0.history.numel(), s0.algo, s0.alpha, s0.margin) for s in scalers):
+        raise ValueError("grouped scalers must share fmt, window, algo, alpha and margin")
+    dt = xs[0].dtype
+    qs = [torch.empty(x.shape, dtype=torch.uint8, device=x.device) for x in xs] if qs is None else list(qs)
+    if workspace is None:
+        workspace = torch.zeros(len(xs) * FUSED_WORKSPACE_BYTES // 4, dtype=torch.int32, device=xs[0].device)
+    arr = (FP8DelayedTensor * len(xs))()
+    for i, (x, q, sc) in enumerate(zip(xs, qs, scalers)):
+        _need_cuda(x, q)
+        if x.dtype != dt:
+            raise ValueError("grouped tensors must share one dtype")
+        arr[i] = FP8DelayedTensor(_ptr(x), _ptr(q), x.numel(), _ptr(sc.scale), _ptr(sc.history), _ptr(sc.state),
+                                  _ptr(sc.scale_used), _ptr(sc.amax))
+    st = load_library().fp8_quantize_delayed_step_grouped(arr, len(xs), _DTYPE_CODE[dt], s0.fmt, s0.history.numel(),
+                                                          s0.algo, s0.alpha, s0.margin, _ptr(workspace),
+                                                          _stream(stream))
+    _check("fp8_quantize_delayed_step_grouped", st)
+    return qs
 
 
 class DelayedScaler:

@@ -337,6 +337,45 @@ int fp8_quantize_delayed_step(const void* x, int dtype, int64_t n, int fmt, floa
                                                       static_cast<cudaStream_t>(stream)));
 }
 
+static_assert(sizeof(fp8_delayed_tensor) == sizeof(fp8q::DelayedTensor) &&
+                  offsetof(fp8_delayed_tensor, x) == offsetof(fp8q::DelayedTensor, x) &&
+                  offsetof(fp8_delayed_tensor, q) == offsetof(fp8q::DelayedTensor, q) &&
+                  offsetof(fp8_delayed_tensor, n) == offsetof(fp8q::DelayedTensor, n) &&
+                  offsetof(fp8_delayed_tensor, scale) == offsetof(fp8q::DelayedTensor, scale) &&
+                  offsetof(fp8_delayed_tensor, history) == offsetof(fp8q::DelayedTensor, history) &&
+                  offsetof(fp8_delayed_tensor, state) == offsetof(fp8q::DelayedTensor, state) &&
+                  offsetof(fp8_delayed_tensor, scale_used) == offsetof(fp8q::DelayedTensor, scale_used) &&
+                  offsetof(fp8_delayed_tensor, amax_out) == offsetof(fp8q::DelayedTensor, amax_out),
+              "fp8_delayed_tensor and the launcher's descriptor share one layout");
+
+int fp8_quantize_delayed_step_grouped(const fp8_delayed_tensor* tensors, int count, int dtype, int fmt, int window,
+                                      int algo, float alpha, float margin, void* workspace, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (count < 0) return FP8_ERR_ARG;
+    if (window <= 0 || window > 65536) return FP8_ERR_ARG;
+    if (algo != FP8_AMAX_WINDOW_MAX && algo != FP8_AMAX_EMA) return FP8_ERR_ARG;
+    if (!(alpha >= 0.0f && alpha <= 1.0f) || !(margin > 0.0f)) return FP8_ERR_ARG;
+    if (count == 0) return FP8_OK;
+    if (tensors == nullptr || workspace == nullptr) return FP8_ERR_NULL;
+    if (!aligned(workspace, 16)) return FP8_ERR_ALIGN;
+    for (int i = 0; i < count; ++i) {
+        const fp8_delayed_tensor& t = tensors[i];
+        if (t.n < 0 || t.n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+        if (t.scale == nullptr || t.history == nullptr || t.state == nullptr || t.scale_used == nullptr ||
+            t.amax_out == nullptr)
+            return FP8_ERR_NULL;
+        if (t.n > 0 && (t.x == nullptr || t.q == nullptr)) return FP8_ERR_NULL;
+        if (t.scale_used == t.scale) return FP8_ERR_ARG;
+        if (!aligned(t.x, 16) || !aligned(t.q, 16) || !aligned(t.scale, 4) || !aligned(t.history, 4) ||
+            !aligned(t.state, 4) || !aligned(t.scale_used, 4) || !aligned(t.amax_out, 4))
+            return FP8_ERR_ALIGN;
+    }
+    return status_of(fp8q::launch_tensor_delayed_step_grouped(reinterpret_cast<const fp8q::DelayedTensor*>(tensors),
+                                                              count, dtype, fmt, window, algo, alpha, margin,
+                                                              workspace, static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_device_status(uint32_t* status, int clear, void* stream) {
     if (status == nullptr) return FP8_ERR_NULL;
     if (!aligned(status, 4)) return FP8_ERR_ALIGN;

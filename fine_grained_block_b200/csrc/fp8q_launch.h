@@ -114,6 +114,22 @@ cudaError_t launch_tensor_delayed_step(const void* x, int dtype, int64_t n, int 
                                        int window, int algo, float alpha, float margin, void* workspace,
                                        cudaStream_t stream);
 
+// The same for `count` tensors in as few launches as possible (up to 96 per
+// launch); workspace: one 16-byte slot per tensor, zero before the first call.
+struct DelayedTensor {
+    const void* x;
+    uint8_t* q;
+    int64_t n;
+    float* scale;
+    float* history;
+    int32_t* state;
+    float* scale_used;
+    float* amax_out;
+};
+cudaError_t launch_tensor_delayed_step_grouped(const DelayedTensor* tensors, int count, int dtype, int fmt, int window,
+                                               int algo, float alpha, float margin, void* workspace,
+                                               cudaStream_t stream);
+
 // Fused quantize -> dequantize round trip in x's dtype.  block_rows 0: per
 // tensor with *scale_in; 1 or 128: block scales (written to `scales` if it is
 // non-null).

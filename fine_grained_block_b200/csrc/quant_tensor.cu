@@ -140,18 +140,20 @@ struct StepWorkspace {
 };
 static_assert(sizeof(StepWorkspace) == 16, "workspace layout");
 
+// One CTA's chunk `chunk` of `nchunks` (the body of k_tensor_cast_delayed_step,
+// also run by the grouped kernel for each tensor's chunks).
 template <typename T, int FMT, int BYTES>
-__global__ void __launch_bounds__(kThreads)
-k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec,
-                           const T* __restrict__ tail, int tail_n, float* scale,
-                           typename LaneVec<T, BYTES>::Out* __restrict__ q, uint8_t* __restrict__ q_tail,
-                           float* __restrict__ scale_used, float* __restrict__ amax_out, float* history,
-                           int32_t* state, int window, int algo, float alpha, float margin, StepWorkspace* ws) {
-    pdl_enter();
+__device__ __forceinline__ void delayed_step_cta(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec,
+                                                 const T* __restrict__ tail, int tail_n, float* scale,
+                                                 typename LaneVec<T, BYTES>::Out* __restrict__ q,
+                                                 uint8_t* __restrict__ q_tail, float* __restrict__ scale_used,
+                                                 float* __restrict__ amax_out, float* history, int32_t* state,
+                                                 int window, int algo, float alpha, float margin, StepWorkspace* ws,
+                                                 int64_t chunk, int64_t nchunks) {
     using V = LaneVec<T, BYTES>;
     __shared__ float warp_amax[kThreads / 32];
     __shared__ int last;
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x;
+    const int64_t base = chunk * kThreads * kUnroll + threadIdx.x;
     typename V::In v[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -167,7 +169,7 @@ k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x,
         a = fmaxf(a, V::amax(v[u]));
         if (i < nvec) st_stream(q + i, V::template cast<FMT>(v[u], s2));
     }
-    if (blockIdx.x == 0 && threadIdx.x < tail_n) {
+    if (chunk == 0 && threadIdx.x < tail_n) {
         const float xv = load_scalar(tail, threadIdx.x);
         a = fmaxf(a, fabsf(xv));
         q_tail[threadIdx.x] = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(xv, s), 0.0f) & 0xFFu);
@@ -181,7 +183,7 @@ k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x,
         for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_amax[w]);
         atomicMax(&ws->amax_bits, __float_as_uint(m));  // non-negative floats order as their bits
         __threadfence();
-        last = (atomicAdd(&ws->arrivals, 1u) == gridDim.x - 1);
+        last = (atomicAdd(&ws->arrivals, 1u) == static_cast<unsigned int>(nchunks - 1));
     }
     __syncthreads();
     if (!last || threadIdx.x >= 32) return;
@@ -196,6 +198,55 @@ k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x,
         ws->amax_bits = 0u;
         ws->arrivals = 0u;
     }
+}
+
+template <typename T, int FMT, int BYTES>
+__global__ void __launch_bounds__(kThreads)
+k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nvec,
+                           const T* __restrict__ tail, int tail_n, float* scale,
+                           typename LaneVec<T, BYTES>::Out* __restrict__ q, uint8_t* __restrict__ q_tail,
+                           float* __restrict__ scale_used, float* __restrict__ amax_out, float* history,
+                           int32_t* state, int window, int algo, float alpha, float margin, StepWorkspace* ws) {
+    pdl_enter();
+    delayed_step_cta<T, FMT, BYTES>(x, nvec, tail, tail_n, scale, q, q_tail, scale_used, amax_out, history, state,
+                                    window, algo, alpha, margin, ws, blockIdx.x, gridDim.x);
+}
+
+// Many tensors' delayed steps in one launch: each tensor's chunks are numbered
+// consecutively across the group, a CTA finds its tensor by binary search
+// over the start indices (kernel parameters), and each tensor has its own
+// 16-byte workspace slot, so its last CTA updates its history.
+constexpr int kStepGroupMax = 96;  // tensors per launch (the parameter block stays under 8 KiB)
+
+struct StepTable {
+    int count;
+    int window, algo;
+    float alpha, margin;
+    StepWorkspace* ws;              // slot of this launch's first tensor
+    int64_t start[kStepGroupMax + 1];
+    DelayedTensor e[kStepGroupMax];
+};
+
+template <typename T, int FMT, int BYTES>
+__global__ void __launch_bounds__(kThreads)
+k_tensor_cast_delayed_step_grouped(const __grid_constant__ StepTable tab) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    const int64_t b = blockIdx.x;
+    int lo = 0, hi = tab.count;  // start[lo] <= b < start[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tab.start[mid] <= b) lo = mid;
+        else hi = mid;
+    }
+    const DelayedTensor& e = tab.e[lo];
+    const int64_t nvec = e.n / V::kElems;
+    const int tail_n = static_cast<int>(e.n - nvec * V::kElems);
+    delayed_step_cta<T, FMT, BYTES>(static_cast<const typename V::In*>(e.x), nvec,
+                                    static_cast<const T*>(e.x) + nvec * V::kElems, tail_n, e.scale,
+                                    reinterpret_cast<typename V::Out*>(e.q), e.q + nvec * V::kElems, e.scale_used,
+                                    e.amax_out, e.history, e.state, tab.window, tab.algo, tab.alpha, tab.margin,
+                                    tab.ws + lo, b - tab.start[lo], tab.start[lo + 1] - tab.start[lo]);
 }
 
 // ---------------------------------------------------------------------------
@@ -479,6 +530,57 @@ cudaError_t launch_tensor_delayed_step(const void* x, int dtype, int64_t n, int 
                                                            window, algo, alpha, margin, workspace, st)
                         : delayed_step_width<float, kE5M2>(x, n, scale, q, scale_used, amax_out, history, state,
                                                            window, algo, alpha, margin, workspace, st);
+}
+
+namespace {
+
+template <typename T, int FMT, int BYTES>
+cudaError_t delayed_grouped_typed(const DelayedTensor* t, int count, int window, int algo, float alpha, float margin,
+                                  void* workspace, cudaStream_t st) {
+    using V = LaneVec<T, BYTES>;
+    StepTable tab;
+    tab.window = window;
+    tab.algo = algo;
+    tab.alpha = alpha;
+    tab.margin = margin;
+    for (int first = 0; first < count; first += kStepGroupMax) {
+        tab.count = std::min(kStepGroupMax, count - first);
+        tab.ws = static_cast<StepWorkspace*>(workspace) + first;
+        int64_t units = 0;
+        for (int i = 0; i < tab.count; ++i) {
+            tab.e[i] = t[first + i];
+            tab.start[i] = units;
+            units += chunk_grid(t[first + i].n / V::kElems);  // at least 1: the update runs for empty tensors
+        }
+        tab.start[tab.count] = units;
+        if (units > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        const cudaError_t e = launch_kernel(k_tensor_cast_delayed_step_grouped<T, FMT, BYTES>,
+                                            dim3(static_cast<unsigned>(units)), dim3(kThreads), 0, st, tab);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T, int FMT>
+cudaError_t delayed_grouped_width(const DelayedTensor* t, int count, int window, int algo, float alpha, float margin,
+                                  void* workspace, cudaStream_t st) {
+    bool w32 = true;  // 256-bit lanes only when every tensor allows them
+    for (int i = 0; i < count; ++i) w32 = w32 && aligned32(t[i].x);
+    return w32 ? delayed_grouped_typed<T, FMT, 32>(t, count, window, algo, alpha, margin, workspace, st)
+               : delayed_grouped_typed<T, FMT, 16>(t, count, window, algo, alpha, margin, workspace, st);
+}
+
+}  // namespace
+
+cudaError_t launch_tensor_delayed_step_grouped(const DelayedTensor* t, int count, int dtype, int fmt, int window,
+                                               int algo, float alpha, float margin, void* workspace,
+                                               cudaStream_t st) {
+    if (dtype == 1)
+        return fmt == kE4M3
+                   ? delayed_grouped_width<uint16_t, kE4M3>(t, count, window, algo, alpha, margin, workspace, st)
+                   : delayed_grouped_width<uint16_t, kE5M2>(t, count, window, algo, alpha, margin, workspace, st);
+    return fmt == kE4M3 ? delayed_grouped_width<float, kE4M3>(t, count, window, algo, alpha, margin, workspace, st)
+                        : delayed_grouped_width<float, kE5M2>(t, count, window, algo, alpha, margin, workspace, st);
 }
 
 cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,

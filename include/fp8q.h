@@ -437,6 +437,37 @@ int fp8_quantize_delayed_step(const void *x, int dtype, int64_t n, int fmt,
                               uint8_t *q, float *scale_used, float *amax_out,
                               void *workspace, void *stream);
 
+/*
+ * fp8_quantize_delayed_step for `count` tensors, in as few launches as
+ * possible (up to 96 tensors share one): every tensor's codes, scale, amax,
+ * history and state come out exactly as from its own call.  All tensors share
+ * dtype, fmt, window, algo, alpha and margin.  For the many small activations
+ * and gradients of a training step, whose single launches are dominated by
+ * their fixed cost.
+ *
+ *   tensors    host array of `count` descriptors (read during the call);
+ *              each holds the device pointers of one
+ *              fp8_quantize_delayed_step call and its element count n
+ *   workspace  count * FP8_FUSED_WORKSPACE_BYTES of device memory, zero
+ *              before the first call and left zero; slot i belongs to
+ *              tensors[i]
+ * Errors: those of fp8_quantize_delayed_step, for any tensor; FP8_ERR_ARG
+ * also for count < 0.
+ */
+typedef struct fp8_delayed_tensor {
+    const void *x;      /* [n] input */
+    uint8_t *q;         /* [n] codes */
+    int64_t n;
+    float *scale;       /* [1] in: this step's scale; out: the next one */
+    float *history;     /* [window] */
+    int32_t *state;     /* [2] */
+    float *scale_used;  /* [1] */
+    float *amax_out;    /* [1] */
+} fp8_delayed_tensor;
+int fp8_quantize_delayed_step_grouped(const fp8_delayed_tensor *tensors, int count, int dtype,
+                                      int fmt, int window, int algo, float alpha, float margin,
+                                      void *workspace, void *stream);
+
 /* Static, human-readable text for a status code (never NULL). */
 const char *fp8_status_string(int status);
 

@@ -36,7 +36,8 @@ def test_header_declares_the_boundary():
                                            "fp8_quantize_per_tensor_fused_noalloc", "fp8_amax_history_update_ex",
                                            "fp8_selftest_wait_timeout", "fp8_quantize_mx", "fp8_dequantize_mx",
                                            "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise",
-                                           "fp8_quantize_delayed_step", "fp8_quantize_blockwise_grouped"])
+                                           "fp8_quantize_delayed_step", "fp8_quantize_blockwise_grouped",
+                                           "fp8_quantize_delayed_step_grouped"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -233,6 +234,24 @@ def test_grouped_validation(L):
     assert g((T * 1)(T(A16, A16, A16, 4, 100)), 1, 1, 1, 128, 0, None) == ERR_SHAPE   # cols % 128
     assert g((T * 1)(T(A16, None, A16, 4, 128)), 1, 1, 1, 128, 0, None) == ERR_NULL
     assert g((T * 1)(T(A1, A16, A16, 4, 128)), 1, 1, 1, 128, 0, None) == ERR_ALIGN
+
+
+def test_delayed_grouped_validation(L):
+    T = binding.FP8DelayedTensor
+    g = L.fp8_quantize_delayed_step_grouped
+    one = (T * 1)(T(A16, A16, 64, A16, A16, A16, A16 + 16, A16, ))
+    assert g(one, 1, 1, 7, 16, 0, 1.0, 1.0, A16, None) == ERR_FORMAT
+    assert g(one, 1, 9, 0, 16, 0, 1.0, 1.0, A16, None) == ERR_DTYPE
+    assert g(one, -1, 1, 0, 16, 0, 1.0, 1.0, A16, None) == ERR_ARG
+    assert g(one, 1, 1, 0, 0, 0, 1.0, 1.0, A16, None) == ERR_ARG
+    assert g(one, 1, 1, 0, 16, 0, 1.0, -1.0, A16, None) == ERR_ARG
+    assert g(None, 0, 1, 0, 16, 0, 1.0, 1.0, None, None) == OK
+    assert g(one, 1, 1, 0, 16, 0, 1.0, 1.0, None, None) == ERR_NULL
+    assert g(one, 1, 1, 0, 16, 0, 1.0, 1.0, A16 + 8, None) == ERR_ALIGN
+    same = (T * 1)(T(A16, A16, 64, A16, A16, A16, A16, A16))
+    assert g(same, 1, 1, 0, 16, 0, 1.0, 1.0, A16, None) == ERR_ARG     # scale_used == scale
+    neg = (T * 1)(T(A16, A16, -1, A16, A16, A16, A16 + 16, A16))
+    assert g(neg, 1, 1, 0, 16, 0, 1.0, 1.0, A16, None) == ERR_SHAPE
 
 
 def test_gemm_validation(L):

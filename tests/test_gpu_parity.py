@@ -700,3 +700,35 @@ def test_grouped_matches_oracle(fmt, dtype, block):
             oq, os_ = oracle.quantize_blockwise(host_input(x_cpu), *block, fmt)
             assert_bytes_equal(s, fp32_bits(os_), f"{lanes} tensor {i} scales")
             assert_bytes_equal(q, oq, f"{lanes} tensor {i} codes")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("algo,alpha,margin,window", [(0, 1.0, 1.0, 3), (1, 0.5, 1.1, 2)])
+def test_grouped_delayed_steps_match_single_calls_and_oracle(fmt, dtype, algo, alpha, margin, window):
+    """fp8_quantize_delayed_step_grouped over 110 tensors (more than one launch, with empty and ragged ones)
+    == each tensor's own DelayedScaler, and the oracle, step after step."""
+    sizes = [0, 1, 7, 4097, 1 << 16, (1 << 18) + 3] + [1000 * (i + 1) + (i % 9) for i in range(104)]
+    kw = dict(window=window, fmt=fmt, algo=algo, alpha=alpha, margin=margin)
+    grouped = [B.DelayedScaler(**kw) for _ in sizes]
+    single = [B.DelayedScaler(**kw) for _ in sizes]
+    refs = [oracle.AmaxHistory(window, fmt, algo=algo, alpha=alpha, margin=margin) for _ in sizes]
+    ws = torch.zeros(len(sizes) * B.FUSED_WORKSPACE_BYTES // 4, dtype=torch.int32, device="cuda")
+    for k in range(window + 2):
+        xs_cpu = [inputs.random_matrix(1, max(n, 1), seed=9000 + 131 * k + i, dtype=dtype, outlier_frac=1e-3,
+                                       factor=10.0 ** (i % 4)).reshape(-1)[:n] for i, n in enumerate(sizes)]
+        xs = [to_cuda(x) for x in xs_cpu]
+        s_refs = [float(r.scale[0]) for r in refs]
+        qg = B.fp8_quantize_delayed_step_grouped(xs, grouped, workspace=ws)
+        qs = [sc.step(x)[0] for sc, x in zip(single, xs)]
+        torch.cuda.synchronize()
+        for i, (x_cpu, r) in enumerate(zip(xs_cpu, refs)):
+            oq, _, oa = oracle.quantize_per_tensor(host_input(x_cpu), fmt, scale=s_refs[i])
+            r.update(oa)
+            assert_bytes_equal(qg[i], oq, f"step {k} tensor {i} codes")
+            assert_bytes_equal(qg[i], qs[i].cpu().numpy(), f"step {k} tensor {i} codes vs single")
+            assert_bytes_equal(grouped[i].scale_used, fp32_bits([s_refs[i]]), f"step {k} tensor {i} scale used")
+            assert_bytes_equal(grouped[i].amax, fp32_bits([oa]), f"step {k} tensor {i} amax")
+            assert_bytes_equal(grouped[i].scale, fp32_bits(r.scale), f"step {k} tensor {i} next scale")
+            assert grouped[i].state.cpu().tolist() == single[i].state.cpu().tolist()
+    assert int(ws.abs().sum().item()) == 0
