@@ -152,7 +152,6 @@ __device__ __forceinline__ void delayed_step_cta(const typename LaneVec<T, BYTES
                                                  int64_t chunk, int64_t nchunks) {
     using V = LaneVec<T, BYTES>;
     __shared__ float warp_amax[kThreads / 32];
-    __shared__ int last;
     const int64_t base = chunk * kThreads * kUnroll + threadIdx.x;
     typename V::In v[kUnroll];
 #pragma unroll
@@ -177,16 +176,18 @@ __device__ __forceinline__ void delayed_step_cta(const typename LaneVec<T, BYTES
     a = warp_max<32>(a);
     if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = a;
     __syncthreads();
+    // Only warp 0 goes on: the other warps' slots free up for the next CTAs.
+    if (threadIdx.x >= 32) return;
+    int is_last = 0;
     if (threadIdx.x == 0) {
         float m = warp_amax[0];
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_amax[w]);
         atomicMax(&ws->amax_bits, __float_as_uint(m));  // non-negative floats order as their bits
         __threadfence();
-        last = (atomicAdd(&ws->arrivals, 1u) == static_cast<unsigned int>(nchunks - 1));
+        is_last = (atomicAdd(&ws->arrivals, 1u) == static_cast<unsigned int>(nchunks - 1));
     }
-    __syncthreads();
-    if (!last || threadIdx.x >= 32) return;
+    if (!__shfl_sync(0xFFFFFFFFu, is_last, 0)) return;
     __threadfence();
     const float amax = __uint_as_float(atomicAdd(&ws->amax_bits, 0u));
     if (threadIdx.x == 0) {
