@@ -259,12 +259,19 @@ k_tensor_cast_delayed_step_grouped(const __grid_constant__ StepTable tab) {
 //
 // Full tiles with vector-friendly strides load one lane vector per slice, 16
 // rows per warp, as the 128x128 block kernel does; the read-out transposes
-// 4x4-byte blocks in registers (byte permutes) so that each lane writes 16
-// consecutive codes into 4 qt rows.  Edge tiles and other strides take an
-// element-wise path.
+// 4x4-byte blocks in registers (byte permutes), and each warp writes whole
+// 128-byte qt row segments.  Edge tiles and other strides take an
+// element-wise path.  With current scaling the CTAs take the tiles
+// last-to-first, so the first reads find the end of x that the amax pass
+// left in L2.
 // ---------------------------------------------------------------------------
-constexpr int kTT = 128;           // tile side
-constexpr int kTStride = kTT + 16;  // smem row pitch in bytes (16-byte aligned rows)
+constexpr int kTT = 128;  // tile side; also the smem row pitch in bytes
+
+// Byte offset of code (r, c) in the shared tile.  The 16-byte column group is
+// XORed with tile-row bits 4..6, so the read-out's 32 lanes -- 8 row bands of
+// 16 rows x 4 column words -- hit 32 distinct banks.  16-byte runs stay
+// contiguous, so the cast can store whole lane vectors.
+__device__ __forceinline__ int tile_off(int r, int c) { return r * kTT + (c ^ (((r >> 4) & 7) << 4)); }
 
 // Lane geometry of a full 128x128 tile: one lane vector (16 or 32 bytes of
 // x) per slice, 16 tile rows per warp.
@@ -290,21 +297,22 @@ __device__ __forceinline__ void tile_cast(const typename LaneVec<T, BYTES>::In (
         const typename V::Out c = V::template cast<FMT>(v[i], s2);
         const int lr = lr0 + i * G::kRowsPerLoad;
         if (q != nullptr) st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row, c);
-        *reinterpret_cast<typename V::Out*>(tile + lr * kTStride + vec_in_row * V::kElems) = c;
+        *reinterpret_cast<typename V::Out*>(tile + tile_off(lr, vec_in_row * V::kElems)) = c;
     }
 }
 
-// qt from the shared code tile: lane l takes tile columns 4l..4l+3, warp w
-// tile rows 16w..16w+15.  It reads 16 words (4 codes of one tile row each;
-// the warp reads 128 consecutive bytes of a row: no bank conflicts),
-// transposes them in 4x4-byte blocks with byte permutes, and writes 16
-// consecutive codes into each of its 4 qt rows.
+// qt from the shared code tile.  Warp w writes qt rows c0+16w..c0+16w+15;
+// lane l takes tile rows 16(l&7)..+15 and tile columns 16w+4(l>>3)..+3.  It
+// reads 16 words (4 codes of one tile row each), transposes them in 4x4-byte
+// blocks with byte permutes, and writes 16 codes into each of its 4 qt rows;
+// the 8 lanes that share a qt row cover its 128 bytes, so each store
+// instruction writes 4 whole lines.
 __device__ __forceinline__ void tile_transpose_out(const uint8_t* tile, uint8_t* qt, int64_t rows, int64_t r0,
                                                    int64_t c0, int lane, int warp) {
-    const int cq = lane * 4, rq = warp * 16;
+    const int rq = (lane & 7) * 16, cq = warp * 16 + (lane >> 3) * 4;
     uint32_t wv[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) wv[i] = *reinterpret_cast<const uint32_t*>(tile + (rq + i) * kTStride + cq);
+    for (int i = 0; i < 16; ++i) wv[i] = *reinterpret_cast<const uint32_t*>(tile + tile_off(rq + i, cq));
     uint32_t o[4][4];  // o[j][g]: column cq+j, rows rq+4g..rq+4g+3
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
@@ -335,10 +343,11 @@ k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, con
                         float* scale_out, float* __restrict__ amax_out, int vector_ok) {
     pdl_enter();
     using V = LaneVec<T, BYTES>;
-    __shared__ __align__(16) uint8_t tile[kTT * kTStride];
+    __shared__ __align__(16) uint8_t tile[kTT * kTT];
     const int64_t tiles_c = (cols + kTT - 1) / kTT;
-    const int64_t tr = blockIdx.x / tiles_c;
-    const int64_t tc = blockIdx.x - tr * tiles_c;
+    const int64_t t = DELAYED ? blockIdx.x : gridDim.x - 1 - blockIdx.x;
+    const int64_t tr = t / tiles_c;
+    const int64_t tc = t - tr * tiles_c;
     const int64_t r0 = tr * kTT, c0 = tc * kTT;
     const int h = static_cast<int>(min(static_cast<int64_t>(kTT), rows - r0));
     const int w = static_cast<int>(min(static_cast<int64_t>(kTT), cols - c0));
@@ -366,13 +375,13 @@ k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, con
                 if (WITH_AMAX) a = fmaxf(a, fabsf(xv));
                 const uint8_t code = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(xv, s), 0.0f) & 0xFFu);
                 if (q != nullptr) q[(r0 + r) * cols + c0 + c] = code;
-                tile[r * kTStride + c] = code;
+                tile[tile_off(r, c)] = code;
             }
         }
         __syncthreads();
         for (int i = threadIdx.x; i < kTT * kTT; i += kThreads) {
             const int c = i / kTT, r = i % kTT;
-            if (r < h && c < w) qt[(c0 + c) * rows + r0 + r] = tile[r * kTStride + c];
+            if (r < h && c < w) qt[(c0 + c) * rows + r0 + r] = tile[tile_off(r, c)];
         }
     }
     if (WITH_AMAX) cta_amax_to_global(a, amax_out);
