@@ -15,7 +15,10 @@
 // sb [N/128, K/128]); both scales are the quantizers' multipliers, so each
 // promotion divides by them.
 //
-// Each CTA owns 128 rows x 256 columns of C (12 warps):
+// The kernel is persistent: one CTA (or CTA pair) per SM (pair of SMs) walks
+// the output tiles first, first + step, ..., numbered with the column tile
+// fastest, so the CTAs running at one time share their rows of A and all of
+// B in L2.  Per tile each CTA computes 128 rows x 256 columns of C (12 warps):
 //   warp 0     TMA producer: per K chunk, a 128x128-byte box of A and the
 //              box of B this CTA holds, into a ring of shared-memory stages
 //              (128-byte swizzle, the layout the MMA descriptors name);
@@ -30,7 +33,10 @@
 //              MMAs of chunk c+1 run while chunk c is promoted;
 //   warps 2-3  idle (they complete the first warpgroup, whose registers go
 //              to the promotion warpgroups).
-// At the end each promotion thread writes its 128 results (fp32 or bf16).
+// At the end of a tile each promotion thread writes its 128 results (fp32 or
+// bf16).  Stages and accumulators are taken round-robin by a chunk count that
+// runs on across tiles, so the producer prefetches the next tile and the MMAs
+// start on it while the promotion warps store this one.
 // Rows past M arrive as zeros from the copy engine and are not stored.
 //
 // Two variants:
@@ -91,6 +97,7 @@ static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the regi
 
 template <bool PAIR>
 struct Cfg {
+    static constexpr int kTileM = PAIR ? 2 * kBM : kBM;      // rows of C per tile (per pair)
     static constexpr int kBRows = PAIR ? kBN / 2 : kBN;      // rows of B this CTA loads
     static constexpr int kBBytes = kBRows * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
@@ -117,14 +124,18 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                  int64_t N, int64_t K, uint32_t idesc, unsigned int* status) {
     using C = Cfg<PAIR>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    auto* bars = reinterpret_cast<Barriers<C::kStages>*>(tiles + C::kStages * C::kStageBytes);
+    uint8_t* tiles_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    auto* bars = reinterpret_cast<Barriers<C::kStages>*>(tiles_smem + C::kStages * C::kStageBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = PAIR ? umma::cluster_ctarank() : 0u;  // 0: this CTA issues the MMAs
-    const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
-    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kBN;
+    // Persistent: this CTA (pair) takes tiles first, first + step, ...; a tile is
+    // C::kTileM rows x kBN columns, numbered with the column tile fastest.
+    const int64_t tiles_n = N / kBN;
+    const int64_t tiles = ((M + C::kTileM - 1) / C::kTileM) * tiles_n;
+    const int64_t first = PAIR ? blockIdx.x / 2 : blockIdx.x;
+    const int64_t step = PAIR ? gridDim.x / 2 : gridDim.x;
     const int nchunks = static_cast<int>(K / kBK);
     const int64_t kc_stride = K / kBK;  // scales per row of sa / sb
 
@@ -151,31 +162,39 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const uint32_t tmem = bars->tmem_base;
     pdl_enter();  // A, B and the scales may come from the previous kernel
 
+    // Stages and accumulators are used round-robin by a chunk counter g that
+    // runs on across tiles, so the producer prefetches the next tile and the
+    // MMAs start on it while the promotion warps store this one.
     bool timed_out = false;
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
     if (warp == 0) {
         // ---- TMA producer ----------------------------------------------------
         if (lane == 0) {
-            for (int kc = 0; kc < nchunks; ++kc) {
-                const int s = kc % C::kStages;
-                const uint32_t phase = static_cast<uint32_t>(kc / C::kStages) & 1u;
-                if (!umma::mbar_wait(&bars->empty[s], phase ^ 1u, kWaitLimitNs)) {
-                    timed_out = true;
-                    break;
-                }
-                uint8_t* stage = tiles + s * C::kStageBytes;
-                if (PAIR) {
-                    // both CTAs' copies complete on the even CTA's barrier, which
-                    // expects the bytes of both
-                    const uint32_t full0 = umma::mapa(umma::smem_u32(&bars->full[s]), 0);
-                    if (rank == 0) umma::mbar_arrive_expect_tx(&bars->full[s], C::kFullTx);
-                    umma::tma_load_2d_pair(stage, &map_a, full0, kc * kBK, static_cast<int>(m0));
-                    umma::tma_load_2d_pair(stage + kABytes, &map_b, full0, kc * kBK,
-                                           static_cast<int>(n0 + rank * C::kBRows));
-                } else {
-                    umma::mbar_arrive_expect_tx(&bars->full[s], C::kFullTx);
-                    umma::tma_load_2d(stage, &map_a, &bars->full[s], kc * kBK, static_cast<int>(m0));
-                    umma::tma_load_2d(stage + kABytes, &map_b, &bars->full[s], kc * kBK, static_cast<int>(n0));
+            uint32_t g = 0;
+            for (int64_t t = first; t < tiles && !timed_out; t += step) {
+                const int m0 = static_cast<int>((t / tiles_n) * C::kTileM + rank * kBM);
+                const int n0 = static_cast<int>((t % tiles_n) * kBN);
+                for (int kc = 0; kc < nchunks; ++kc, ++g) {
+                    const uint32_t s = g % C::kStages;
+                    const uint32_t phase = (g / C::kStages) & 1u;
+                    if (!umma::mbar_wait(&bars->empty[s], phase ^ 1u, kWaitLimitNs)) {
+                        timed_out = true;
+                        break;
+                    }
+                    uint8_t* stage = tiles_smem + s * C::kStageBytes;
+                    if (PAIR) {
+                        // both CTAs' copies complete on the even CTA's barrier, which
+                        // expects the bytes of both
+                        const uint32_t full0 = umma::mapa(umma::smem_u32(&bars->full[s]), 0);
+                        if (rank == 0) umma::mbar_arrive_expect_tx(&bars->full[s], C::kFullTx);
+                        umma::tma_load_2d_pair(stage, &map_a, full0, kc * kBK, m0);
+                        umma::tma_load_2d_pair(stage + kABytes, &map_b, full0, kc * kBK,
+                                               n0 + static_cast<int>(rank) * C::kBRows);
+                    } else {
+                        umma::mbar_arrive_expect_tx(&bars->full[s], C::kFullTx);
+                        umma::tma_load_2d(stage, &map_a, &bars->full[s], kc * kBK, m0);
+                        umma::tma_load_2d(stage + kABytes, &map_b, &bars->full[s], kc * kBK, n0);
+                    }
                 }
             }
         }
@@ -184,35 +203,38 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         if (lane == 0 && rank == 0) {
             const uint32_t peer_empty0 = PAIR ? umma::mapa(umma::smem_u32(&bars->empty[0]), 1) : 0u;
             const uint32_t peer_accf0 = PAIR ? umma::mapa(umma::smem_u32(&bars->acc_full[0]), 1) : 0u;
-            for (int kc = 0; kc < nchunks; ++kc) {
-                const int s = kc % C::kStages;
-                const uint32_t phase = static_cast<uint32_t>(kc / C::kStages) & 1u;
-                const int buf = kc & 1;
-                const uint32_t acc_phase = static_cast<uint32_t>(kc >> 1) & 1u;
-                if (!umma::mbar_wait(&bars->acc_empty[buf], acc_phase ^ 1u, kWaitLimitNs) ||
-                    !umma::mbar_wait(&bars->full[s], phase, kWaitLimitNs)) {
-                    timed_out = true;
-                    break;
-                }
-                umma::fence_after_sync();
-                const uint32_t a_addr = umma::smem_u32(tiles + s * C::kStageBytes);
-                const uint64_t a_desc = umma::smem_desc_kmajor_sw128(a_addr);
-                const uint64_t b_desc = umma::smem_desc_kmajor_sw128(a_addr + kABytes);
-                const uint32_t d = tmem + static_cast<uint32_t>(buf * kBN);
+            uint32_t g = 0;
+            for (int64_t t = first; t < tiles && !timed_out; t += step) {
+                for (int kc = 0; kc < nchunks; ++kc, ++g) {
+                    const uint32_t s = g % C::kStages;
+                    const uint32_t phase = (g / C::kStages) & 1u;
+                    const uint32_t buf = g & 1u;
+                    const uint32_t acc_phase = (g >> 1) & 1u;
+                    if (!umma::mbar_wait(&bars->acc_empty[buf], acc_phase ^ 1u, kWaitLimitNs) ||
+                        !umma::mbar_wait(&bars->full[s], phase, kWaitLimitNs)) {
+                        timed_out = true;
+                        break;
+                    }
+                    umma::fence_after_sync();
+                    const uint32_t a_addr = umma::smem_u32(tiles_smem + s * C::kStageBytes);
+                    const uint64_t a_desc = umma::smem_desc_kmajor_sw128(a_addr);
+                    const uint64_t b_desc = umma::smem_desc_kmajor_sw128(a_addr + kABytes);
+                    const uint32_t d = tmem + buf * static_cast<uint32_t>(kBN);
 #pragma unroll
-                for (int k = 0; k < kBK / kMmaK; ++k) {
-                    // the next 32 bytes of K: start address + 32 bytes (2 in 16-byte units)
-                    if (PAIR) umma::mma_f8f6f4_pair(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
-                    else umma::mma_f8f6f4(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
-                }
-                if (PAIR) {
-                    umma::commit_pair(umma::smem_u32(&bars->empty[s]));
-                    umma::commit_pair(peer_empty0 + static_cast<uint32_t>(s * sizeof(uint64_t)));
-                    umma::commit_pair(umma::smem_u32(&bars->acc_full[buf]));
-                    umma::commit_pair(peer_accf0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
-                } else {
-                    umma::commit(&bars->empty[s]);
-                    umma::commit(&bars->acc_full[buf]);
+                    for (int k = 0; k < kBK / kMmaK; ++k) {
+                        // the next 32 bytes of K: start address + 32 bytes (2 in 16-byte units)
+                        if (PAIR) umma::mma_f8f6f4_pair(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
+                        else umma::mma_f8f6f4(d, a_desc + 2 * k, b_desc + 2 * k, idesc, k > 0);
+                    }
+                    if (PAIR) {
+                        umma::commit_pair(umma::smem_u32(&bars->empty[s]));
+                        umma::commit_pair(peer_empty0 + s * static_cast<uint32_t>(sizeof(uint64_t)));
+                        umma::commit_pair(umma::smem_u32(&bars->acc_full[buf]));
+                        umma::commit_pair(peer_accf0 + buf * static_cast<uint32_t>(sizeof(uint64_t)));
+                    } else {
+                        umma::commit(&bars->empty[s]);
+                        umma::commit(&bars->acc_full[buf]);
+                    }
                 }
             }
             if (PAIR) umma::commit_pair(umma::smem_u32(&bars->mma_done));
@@ -224,59 +246,63 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPromoteRegs));
         const int quarter = warp & 3;            // TMEM lanes this warp may access
         const int half = (warp - 4) >> 2;        // column half of the tile
-        const int row = quarter * 32 + lane;     // tile row = TMEM lane
-        const int64_t m = m0 + row;
-        const float* sa_row = sa + (m < M ? m : 0) * kc_stride;
-        const float* sb_row = sb + ((n0 >> 7) + half) * kc_stride;
+        const int row = quarter * 32 + lane;     // row within this CTA's 128 = TMEM lane
         const uint32_t acc_empty0 = PAIR ? umma::mapa(umma::smem_u32(&bars->acc_empty[0]), 0)
                                          : umma::smem_u32(&bars->acc_empty[0]);
-        float acc[128];
-#pragma unroll
-        for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
-        for (int kc = 0; kc < nchunks; ++kc) {
-            const int buf = kc & 1;
-            const uint32_t acc_phase = static_cast<uint32_t>(kc >> 1) & 1u;
-            // 1 / (sa * sb): the dequant factor of this chunk for this row and column half
-            const float f = (m < M) ? __frcp_rn(__fmul_rn(__ldg(sa_row + kc), __ldg(sb_row + kc))) : 0.0f;
-            if (!umma::mbar_wait(&bars->acc_full[buf], acc_phase, kWaitLimitNs)) {
-                timed_out = true;
-                break;
-            }
-            umma::fence_after_sync();
-            const uint32_t t = t_lane + static_cast<uint32_t>(buf * kBN);
+        uint32_t g = 0;
+        for (int64_t t = first; t < tiles && !timed_out; t += step) {
+            const int64_t m = (t / tiles_n) * C::kTileM + rank * kBM + row;
+            const int64_t col0 = (t % tiles_n) * kBN + half * 128;
+            const float* sa_row = sa + (m < M ? m : 0) * kc_stride;
+            const float* sb_row = sb + (col0 >> 7) * kc_stride;
+            float acc[128];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float p[64];
-                umma::tmem_ld32(t + h * 64, p);
-                umma::tmem_ld32(t + h * 64 + 32, p + 32);
-                umma::wait_ld(p);
-                umma::hold_after_wait(p + 32);
-                if (h == 1) {
-                    // every partial sum of this buffer is in registers: hand it back
-                    umma::fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0)
-                        umma::mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
+            for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+            for (int kc = 0; kc < nchunks; ++kc, ++g) {
+                const uint32_t buf = g & 1u;
+                const uint32_t acc_phase = (g >> 1) & 1u;
+                // 1 / (sa * sb): the dequant factor of this chunk for this row and column half
+                const float f = (m < M) ? __frcp_rn(__fmul_rn(__ldg(sa_row + kc), __ldg(sb_row + kc))) : 0.0f;
+                if (!umma::mbar_wait(&bars->acc_full[buf], acc_phase, kWaitLimitNs)) {
+                    timed_out = true;
+                    break;
                 }
+                umma::fence_after_sync();
+                const uint32_t tm = t_lane + buf * static_cast<uint32_t>(kBN);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) acc[h * 64 + j] = __fmaf_rn(p[j], f, acc[h * 64 + j]);
+                for (int h = 0; h < 2; ++h) {
+                    float p[64];
+                    umma::tmem_ld32(tm + h * 64, p);
+                    umma::tmem_ld32(tm + h * 64 + 32, p + 32);
+                    umma::wait_ld(p);
+                    umma::hold_after_wait(p + 32);
+                    if (h == 1) {
+                        // every partial sum of this buffer is in registers: hand it back
+                        umma::fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0)
+                            umma::mbar_arrive_cluster(acc_empty0 + buf * static_cast<uint32_t>(sizeof(uint64_t)));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) acc[h * 64 + j] = __fmaf_rn(p[j], f, acc[h * 64 + j]);
+                }
             }
-        }
-        if (!timed_out && m < M) {
-            const int64_t col0 = n0 + half * 128;
-            if (OUT == 0) {
-                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(c) + m * N + col0);
+            if (!timed_out && m < M) {
+                if (OUT == 0) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(c) + m * N + col0);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
-            } else {
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(c) + m * N + col0);
+                    for (int j = 0; j < 32; ++j)
+                        dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(c) + m * N + col0);
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    dst[j] = make_uint4(pack_bf16x2(acc[8 * j], acc[8 * j + 1]), pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
-                                        pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
-                                        pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+                    for (int j = 0; j < 16; ++j)
+                        dst[j] = make_uint4(pack_bf16x2(acc[8 * j], acc[8 * j + 1]),
+                                            pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
+                                            pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
+                                            pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+                }
             }
         }
     }
@@ -345,10 +371,9 @@ cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, con
         if (e != cudaSuccess) return e;
         opted[dev].store(true, std::memory_order_release);
     }
-    int64_t mt = (M + kBM - 1) / kBM;
-    if (PAIR) mt = (mt + 1) & ~int64_t(1);  // whole pairs; rows past M are zeros and not stored
+    const int64_t tiles = ((M + C::kTileM - 1) / C::kTileM) * (N / kBN);
+    if (tiles == 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(mt), static_cast<unsigned>(N / kBN));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = st;
@@ -368,6 +393,23 @@ cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, con
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
+    // Persistent grid: as many CTAs (pairs) as fit on the device at once (one
+    // per SM), never more than there are tiles.
+    static std::atomic<int> resident[128];
+    int units = resident[dev].load(std::memory_order_acquire);
+    if (units <= 0) {
+        units = PAIR ? device_sm_count() / 2 : device_sm_count();
+        if (PAIR) {
+            int clusters = 0;
+            cfg.gridDim = dim3(2 * static_cast<unsigned>(units));
+            const cudaError_t oe = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+            if (oe != cudaSuccess) (void)cudaGetLastError();  // keep the device-count estimate
+            else if (clusters > 0) units = std::min(units, clusters);
+        }
+        resident[dev].store(std::max(units, 1), std::memory_order_release);
+    }
+    const int64_t ctas = std::min<int64_t>(tiles, units) * (PAIR ? 2 : 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, sa, sb, c, M, N, K, idesc, status);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
