@@ -538,7 +538,7 @@ def modes_breakdown(dev, stream, peak):
     put("128_gradients_2^20_delayed_e5m2_one_call_each", "128 bf16 tensors of 2^20 elements, N(0,1e-6), seeds "
         "300..427, W=16 (128 launches)", gnb, time_in_graph([steps_one_by_one], 4, dev))
     put("128_gradients_2^20_delayed_e5m2_grouped", "the same 128 tensors in one fp8_quantize_delayed_step_grouped "
-        "call (2 launches of up to 96 tensors)", gnb, time_in_graph([lambda r, st: raw.check(
+        "call (1 launch)", gnb, time_in_graph([lambda r, st: raw.check(
             L.fp8_quantize_delayed_step_grouped(garr, len(gx_), 1, 1, 16, 0, 1.0, 1.0, gws_.data_ptr(), st),
             "grouped step")], 16, dev))
     del gx_, gq_, gst_, gws_, garr

@@ -217,7 +217,7 @@ k_tensor_cast_delayed_step(const typename LaneVec<T, BYTES>::In* __restrict__ x,
 // consecutively across the group, a CTA finds its tensor by binary search
 // over the start indices (kernel parameters), and each tensor has its own
 // 16-byte workspace slot, so its last CTA updates its history.
-constexpr int kStepGroupMax = 96;  // tensors per launch (the parameter block stays under 8 KiB)
+constexpr int kStepGroupMax = 128;  // tensors per launch (a 9.3 KiB parameter block; the limit is 32 KiB)
 
 struct StepTable {
     int count;
@@ -227,6 +227,7 @@ struct StepTable {
     int64_t start[kStepGroupMax + 1];
     DelayedTensor e[kStepGroupMax];
 };
+static_assert(sizeof(StepTable) <= 16384, "the grouped step's parameter block must stay well inside 32 KiB");
 
 template <typename T, int FMT, int BYTES>
 __global__ void __launch_bounds__(kThreads)

@@ -439,7 +439,7 @@ int fp8_quantize_delayed_step(const void *x, int dtype, int64_t n, int fmt,
 
 /*
  * fp8_quantize_delayed_step for `count` tensors, in as few launches as
- * possible (up to 96 tensors share one): every tensor's codes, scale, amax,
+ * possible (up to 128 tensors share one): every tensor's codes, scale, amax,
  * history and state come out exactly as from its own call.  All tensors share
  * dtype, fmt, window, algo, alpha and margin.  For the many small activations
  * and gradients of a training step, whose single launches are dominated by

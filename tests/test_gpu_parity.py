@@ -706,9 +706,9 @@ def test_grouped_matches_oracle(fmt, dtype, block):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("algo,alpha,margin,window", [(0, 1.0, 1.0, 3), (1, 0.5, 1.1, 2)])
 def test_grouped_delayed_steps_match_single_calls_and_oracle(fmt, dtype, algo, alpha, margin, window):
-    """fp8_quantize_delayed_step_grouped over 110 tensors (more than one launch, with empty and ragged ones)
-    == each tensor's own DelayedScaler, and the oracle, step after step."""
-    sizes = [0, 1, 7, 4097, 1 << 16, (1 << 18) + 3] + [1000 * (i + 1) + (i % 9) for i in range(104)]
+    """fp8_quantize_delayed_step_grouped over 140 tensors (more than one launch of 128, with empty and ragged
+    ones) == each tensor's own DelayedScaler, and the oracle, step after step."""
+    sizes = [0, 1, 7, 4097, 1 << 16, (1 << 18) + 3] + [1000 * (i + 1) + (i % 9) for i in range(134)]
     kw = dict(window=window, fmt=fmt, algo=algo, alpha=alpha, margin=margin)
     grouped = [B.DelayedScaler(**kw) for _ in sizes]
     single = [B.DelayedScaler(**kw) for _ in sizes]
