@@ -398,10 +398,13 @@ def modes_breakdown(dev, stream, peak):
         lambda r, st: raw.check(L.fp8_quantize_per_tensor_transpose(a.data_ptr(), 1, R_, C_, 0, sc.data_ptr(),
                                                                     q.data_ptr(), qt.data_ptr(), so_.data_ptr(),
                                                                     ao_.data_ptr(), st), "transpose")], 20, dev))
-    put("per_tensor_transpose_current_e4m3", wl + " (amax pass, then q and qt; alg bytes 4/elem)", 4 * n,
-        time_in_graph([lambda r, st: raw.check(L.fp8_quantize_per_tensor_transpose(
-            a.data_ptr(), 1, R_, C_, 0, None, q.data_ptr(), qt.data_ptr(), so_.data_ptr(), ao_.data_ptr(), st),
-            "transpose")], 20, dev))
+    a2 = a.clone()  # alternate two copies: the reverse cast pass ends where the next amax pass starts
+    aa = [a, a2]
+    put("per_tensor_transpose_current_e4m3", wl + " (amax pass, then q and qt; alg bytes 4/elem; two input "
+        "copies alternated)", 4 * n, time_in_graph([lambda r, st: raw.check(L.fp8_quantize_per_tensor_transpose(
+            aa[r % 2].data_ptr(), 1, R_, C_, 0, None, q.data_ptr(), qt.data_ptr(), so_.data_ptr(), ao_.data_ptr(),
+            st), "transpose")], 20, dev))
+    del a2, aa
     del a, q, s, y, e8, qt
 
     # size sweep point 2^28 (512 MiB bf16): 1x128, 128x128, per-tensor current E5M2, dequant
