@@ -53,7 +53,9 @@
 // accumulator to come back from the promotion, and each chunk's MMAs take
 // about 0.6 us from issue to commit, so with two accumulators the chunks run
 // nearly one at a time.  Four 128-column accumulator slots (N 128 MMAs) were
-// slower; spinning waits changed nothing; a timing-only copy that accumulates
+// slower; tiles cut into column halves (N 128) took as long per chunk as
+// whole ones, so the chunk period is the hand-back latency, not the MMA work
+// or the operand bytes; spinning waits changed nothing; a timing-only copy that accumulates
 // all of K in one accumulator (no promotion) reaches about 2.2 PFLOP/s,
 // bound there by the TMA operand delivery.
 //
