@@ -405,6 +405,14 @@ def modes_breakdown(dev, stream, peak):
             aa[r % 2].data_ptr(), 1, R_, C_, 0, None, q.data_ptr(), qt.data_ptr(), so_.data_ptr(), ao_.data_ptr(),
             st), "transpose")], 20, dev))
     del a2, aa
+    # 1x128 blocks of x and of x^T (the operand of the weight-gradient GEMM) from one read: q with row-block
+    # scales, qt with column-block scales
+    sbt = torch.empty(C_, R_ // 128, dtype=torch.float32, device=dev)
+    put("1x128_e4m3_quant_and_transpose", wl + " (q with 1x128 row-block scales and qt = 1x128 blocks of x^T, "
+        "one pass)", 4 * n + 8 * (n // 128), time_in_graph([lambda r, st: raw.check(
+            L.fp8_quantize_blockwise_transpose(a.data_ptr(), 1, R_, C_, 1, 128, 0, q.data_ptr(), s.data_ptr(),
+                                               qt.data_ptr(), sbt.data_ptr(), st), "block transpose")], 20, dev))
+    del sbt
     del a, q, s, y, e8, qt
 
     # size sweep point 2^28 (512 MiB bf16): 1x128, 128x128, per-tensor current E5M2, dequant

@@ -10,7 +10,7 @@ _BINDING_NAMES = (
     "fp8_quantize_per_tensor", "fp8_quantize_blockwise", "fp8_dequantize",
     "fp8_amax_history_update", "fp8_amax_history_update_ex", "fp8_fake_quantize", "fp8_amax", "fp8_scale_from_amax",
     "fp8_quantize_per_tensor_fused", "fused_workspace", "fp8_status_string", "FP8Error", "load_library",
-    "fp8_quantize_mx", "fp8_dequantize_mx", "MX_FIT", "MX_OCP", "fp8_quantize_per_tensor_transpose",
+    "fp8_quantize_mx", "fp8_dequantize_mx", "MX_FIT", "MX_OCP", "fp8_quantize_per_tensor_transpose", "fp8_quantize_blockwise_transpose",
     "fp8_gemm_blockwise", "fp8_quantize_delayed_step", "DelayedScaler",
     "fp8_quantize_blockwise_grouped", "FP8BlockTensor", "fp8_quantize_delayed_step_grouped", "FP8DelayedTensor",
     "E4M3", "E5M2", "F32", "BF16",

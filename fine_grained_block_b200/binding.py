@@ -56,6 +56,8 @@ SIGNATURES = {
     "fp8_scale_from_amax": (_c_int, [_vp, _c_int, _vp, _vp]),
     "fp8_fake_quantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]),
     "fp8_quantize_per_tensor_transpose": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fp8_quantize_blockwise_transpose": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp,
+                                                  _vp, _vp]),
     "fp8_quantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _vp]),
     "fp8_dequantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _vp, _vp, _c_int, _vp]),
     "fp8_gemm_blockwise": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _i64, _i64, _i64, _vp, _c_int, _vp]),
@@ -266,6 +268,29 @@ def fp8_quantize_blockwise_grouped(xs, block=(1, 128), fmt: int = E4M3, qs=None,
     st = load_library().fp8_quantize_blockwise_grouped(arr, len(xs), _DTYPE_CODE[dt], br, bc, fmt, _stream(stream))
     _check("fp8_quantize_blockwise_grouped", st)
     return qs, scales
+
+
+def fp8_quantize_blockwise_transpose(x: torch.Tensor, block=(1, 128), fmt: int = E4M3, q=None, scales=None,
+                                     qt=None, scales_t=None, stream=None):
+    """Blockwise quantize of x and of x^T in one pass (rows, cols multiples of 128).
+
+    Returns (q, scales, qt, scales_t) = fp8_quantize_blockwise(x, block) + fp8_quantize_blockwise(x.T, block)."""
+    _need_cuda(x, q, scales, qt, scales_t)
+    if x.dim() != 2:
+        raise ValueError("the transposing blockwise quantize takes a 2-D tensor")
+    R, C = x.shape
+    br, bc = block
+    dev = x.device
+    q = torch.empty((R, C), dtype=torch.uint8, device=dev) if q is None else q
+    qt = torch.empty((C, R), dtype=torch.uint8, device=dev) if qt is None else qt
+    if scales is None:
+        scales = torch.empty((R // br, C // bc), dtype=torch.float32, device=dev)
+    if scales_t is None:
+        scales_t = torch.empty((C // br, R // bc), dtype=torch.float32, device=dev)
+    st = load_library().fp8_quantize_blockwise_transpose(_ptr(x), _DTYPE_CODE[x.dtype], R, C, br, bc, fmt, _ptr(q),
+                                                         _ptr(scales), _ptr(qt), _ptr(scales_t), _stream(stream))
+    _check("fp8_quantize_blockwise_transpose", st)
+    return q, scales, qt, scales_t
 
 
 def fp8_quantize_mx(x: torch.Tensor, fmt: int = E4M3, rule: int = MX_FIT, q: torch.Tensor | None = None,

@@ -108,6 +108,23 @@ int fp8_quantize_per_tensor_fused_noalloc(const void* x, int dtype, int64_t n, i
                                                        static_cast<cudaStream_t>(stream)));
 }
 
+int fp8_quantize_blockwise_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows,
+                                     int block_cols, int fmt, uint8_t* q, float* scales, uint8_t* qt,
+                                     float* scales_t, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (!((block_rows == 1 || block_rows == 128) && block_cols == 128)) return FP8_ERR_SHAPE;
+    if (rows < 0 || cols < 0 || rows % 128 != 0 || cols % 128 != 0) return FP8_ERR_SHAPE;
+    const int64_t n = checked_count(rows, cols);
+    if (n < 0 || n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+    if (n == 0) return FP8_OK;
+    if (x == nullptr || q == nullptr || scales == nullptr || qt == nullptr || scales_t == nullptr) return FP8_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(qt, 16) || !aligned(scales, 4) || !aligned(scales_t, 4))
+        return FP8_ERR_ALIGN;
+    return status_of(fp8q::launch_quant_block_transpose(x, dtype, rows, cols, block_rows, fmt, q, scales, qt, scales_t,
+                                                        static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_quantize_per_tensor_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                       const float* scale_in, uint8_t* q, uint8_t* qt, float* scale_out,
                                       float* amax_out, void* stream) {

@@ -102,6 +102,11 @@ cudaError_t launch_tensor_cast(const void* x, int dtype, int64_t n, int fmt,
 
 // Per-tensor cast with a transposed second output qt [cols, rows] (q [rows,
 // cols] optional).  Scale arguments as in launch_tensor_cast.
+// Blockwise quantization of x and of x^T in one pass (rows, cols multiples of
+// 128; block_rows 1 for 1x128, 128 for 128x128).
+cudaError_t launch_quant_block_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows,
+                                         int fmt, uint8_t* q, float* scales, uint8_t* qt, float* scales_t,
+                                         cudaStream_t stream);
 cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
                                          const float* scale_in, const float* amax_in, uint8_t* q, uint8_t* qt,
                                          float* scale_out, float* amax_out, cudaStream_t stream);

@@ -1,0 +1,251 @@
+// quant_block_transpose.cu -- blockwise quantization with a transposed second
+// output: q, scales = blockwise(x) and qt, scales_t = blockwise(x^T), from one
+// read of x.
+//
+// Mixed-precision handbook, section "FP8 training", per_block: 1x128 blocks
+// for activations, 128x128 blocks for weights, s = MAX / max(amax, eps) per
+// block.  A weight-gradient (or data-gradient) GEMM reads its operand along
+// the other dimension, so it needs the codes of x^T quantized with the same
+// rule.  For 128x128 blocks x^T has the same blocks as x, transposed: qt is
+// q^T and scales_t is scales^T.  For 1x128 blocks the blocks of x^T are the
+// 128x1 columns of x, with scales of their own.
+//
+// One CTA per 128x128 tile (rows and cols multiples of 128).  The tile stays
+// in registers, loaded as by the 128x128 block kernel (16 tile rows per warp,
+// one lane vector per slice):
+//   128x128  tile amax -> one scale; the codes go to q and into a shared code
+//            tile, which is written out transposed into qt;
+//   1x128    row amax over the lanes of a row (shuffles) -> q with the row
+//            scales; column amax: per lane over its rows, then over the
+//            warp's row groups (shuffles), then over the 8 warps (shared
+//            memory) -> one scale per column, computed once by 128 threads;
+//            the codes of x * column scale go into the shared tile and out
+//            transposed into qt.
+// Both casts are RN_fp32(x * s) then the saturating RNE cast, as everywhere.
+
+#include <algorithm>
+
+#include "fp8q_device.cuh"
+#include "fp8q_launch.h"
+#include "launch_util.h"
+#include "lane_vec.cuh"
+#include "tile_transpose.cuh"
+
+namespace fp8q {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// Cast of one lane vector with a scale per element (column scales): cs[e] is
+// the scale of element e, read from shared memory pair by pair.
+// {cs[2p], cs[2p+1]} as packed fp32 operands (one 8-byte shared load).
+__device__ __forceinline__ uint64_t pair(const float* cs, int p) {
+    const float2 s = reinterpret_cast<const float2*>(cs)[p];
+    return f32x2(s.x, s.y);
+}
+
+template <typename T, int BYTES>
+struct PairCast;
+template <int BYTES>
+struct PairCast<uint16_t, BYTES> {
+    using V = LaneVec<uint16_t, BYTES>;
+    template <int FMT>
+    static __device__ __forceinline__ typename V::Out cast(const typename V::In& v, const float* cs) {
+        uint32_t c[V::kWords / 2];
+#pragma unroll
+        for (int k = 0; k < V::kWords / 2; ++k)
+            c[k] = scale_cast_bf16x2<FMT>(v.w[2 * k], pair(cs, 2 * k)) |
+                   (scale_cast_bf16x2<FMT>(v.w[2 * k + 1], pair(cs, 2 * k + 1)) << 16);
+        return CodeWords<V::kWords / 2>::make(c);
+    }
+};
+template <int BYTES>
+struct PairCast<float, BYTES> {
+    using V = LaneVec<float, BYTES>;
+    template <int FMT>
+    static __device__ __forceinline__ typename V::Out cast(const typename V::In& v, const float* cs) {
+        uint32_t c[V::kWords / 4];
+#pragma unroll
+        for (int k = 0; k < V::kWords / 4; ++k)
+            c[k] = scale_cast_f32x2<FMT>(v.w[4 * k], v.w[4 * k + 1], pair(cs, 2 * k)) |
+                   (scale_cast_f32x2<FMT>(v.w[4 * k + 2], v.w[4 * k + 3], pair(cs, 2 * k + 1)) << 16);
+        return CodeWords<V::kWords / 4>::make(c);
+    }
+};
+
+// |x| maxima of a lane's elements over its kLoads rows, then over the lanes
+// that hold the same columns in the warp's other row groups; written (if
+// `write`) to colmax[e] for element e of this lane's slice.  bf16 pairs reduce packed (exact); a NaN
+// operand yields the other one, as in every amax of the library.
+template <typename T, int BYTES>
+struct ColMax;
+template <int BYTES>
+struct ColMax<uint16_t, BYTES> {
+    using V = LaneVec<uint16_t, BYTES>;
+    using G = TileGeom<uint16_t, BYTES>;
+    static __device__ __forceinline__ void run(const typename V::In (&v)[G::kLoads], bool write, float* colmax) {
+#pragma unroll
+        for (int k = 0; k < V::kWords; ++k) {
+            uint32_t m = v[0].w[k];
+#pragma unroll
+            for (int i = 1; i < G::kLoads; ++i) m = xabsmax_bf16x2(m, v[i].w[k]);
+#pragma unroll
+            for (int off = G::kVecPerRow; off < 32; off <<= 1)
+                m = xabsmax_bf16x2(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+            m &= 0x7FFF7FFFu;
+            if (write) {
+                colmax[2 * k] = __uint_as_float(m << 16);
+                colmax[2 * k + 1] = __uint_as_float(m & 0xFFFF0000u);
+            }
+        }
+    }
+};
+template <int BYTES>
+struct ColMax<float, BYTES> {
+    using V = LaneVec<float, BYTES>;
+    using G = TileGeom<float, BYTES>;
+    static __device__ __forceinline__ void run(const typename V::In (&v)[G::kLoads], bool write, float* colmax) {
+#pragma unroll
+        for (int k = 0; k < V::kWords; ++k) {
+            float m = fabsf(__uint_as_float(v[0].w[k]));
+#pragma unroll
+            for (int i = 1; i < G::kLoads; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i].w[k])));
+#pragma unroll
+            for (int off = G::kVecPerRow; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+            if (write) colmax[k] = m;
+        }
+    }
+};
+
+// MODE 0: 1x128 blocks (row scales for q, column scales for qt);
+// MODE 1: 128x128 blocks (one scale per tile for both).
+// Resident CTAs per SM each mode is compiled for (register cap).  Measured on
+// B200 on the bf16 16384x7168 activations: 128x128 runs at 98.7 % of the copy
+// peak with 3 or 4 and 85 % with 2; 1x128, whose column pass holds more
+// registers, spills under the caps of 3 and 4 (68 % and 58 %) and runs
+// best with 2 (73 %).
+#ifndef FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
+#define FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS 2
+#endif
+#ifndef FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS
+#define FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS 3
+#endif
+
+template <typename T, int FMT, int BYTES, int MODE>
+__global__ void __launch_bounds__(kThreads, MODE == 0 ? FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
+                                                      : FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS)
+k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uint8_t* __restrict__ q,
+                        float* __restrict__ scales, uint8_t* __restrict__ qt, float* __restrict__ scales_t) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    using G = TileGeom<T, BYTES>;
+    __shared__ __align__(16) uint8_t tile[kTT * kTT];
+    __shared__ float part[kWarps][kTT];  // per-warp column maxima (MODE 0); warp maxima (MODE 1)
+    __shared__ __align__(16) float col_scale[kTT];
+
+    const int64_t tiles_c = cols / kTT, tiles_r = rows / kTT;
+    const int64_t tr = blockIdx.x / tiles_c;
+    const int64_t tc = blockIdx.x - tr * tiles_c;
+    const int64_t r0 = tr * kTT, c0 = tc * kTT;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lr0 = warp * 16 + lane / G::kVecPerRow, vec_in_row = lane % G::kVecPerRow;
+    const auto* xv = reinterpret_cast<const typename V::In*>(x + (r0 + lr0) * cols + c0) + vec_in_row;
+    const int64_t vstride = cols / V::kElems * G::kRowsPerLoad;  // lane vectors between this lane's rows
+    typename V::In v[G::kLoads];
+#pragma unroll
+    for (int i = 0; i < G::kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
+
+    if (MODE == 1) {
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) a = fmaxf(a, V::amax(v[i]));
+        a = warp_max<32>(a);
+        if (lane == 0) part[0][warp] = a;
+        __syncthreads();
+        float ta = part[0][0];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) ta = fmaxf(ta, part[0][w]);
+        const float s = scale_from_amax<FMT>(ta);
+        float unused = 0.0f;
+        tile_cast<T, FMT, BYTES, false>(v, f32x2(s, s), q, cols, r0, c0, tile, lr0, vec_in_row, unused);
+        if (threadIdx.x == 0) {
+            scales[tr * tiles_c + tc] = s;
+            scales_t[tc * tiles_r + tr] = s;
+        }
+    } else {
+        // q: one scale per tile row (the row's kVecPerRow lanes reduce together)
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) {
+            const float ra = warp_max<G::kVecPerRow>(V::amax(v[i]));
+            const float s = scale_from_amax<FMT>(ra);
+            const int lr = lr0 + i * G::kRowsPerLoad;
+            st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row,
+                      V::template cast<FMT>(v[i], f32x2(s, s)));
+            if (vec_in_row == 0) scales[(r0 + lr) * tiles_c + tc] = s;
+        }
+        // qt: one scale per tile column
+        ColMax<T, BYTES>::run(v, lane < G::kVecPerRow, &part[warp][vec_in_row * V::kElems]);
+        __syncthreads();
+        if (threadIdx.x < kTT) {
+            const int c = threadIdx.x;
+            float m = part[0][c];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, part[w][c]);
+            const float s = scale_from_amax<FMT>(m);
+            col_scale[c] = s;
+            scales_t[(c0 + c) * tiles_r + tr] = s;
+        }
+        __syncthreads();
+        const float* cs = col_scale + vec_in_row * V::kElems;
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) {
+            const int lr = lr0 + i * G::kRowsPerLoad;
+            *reinterpret_cast<typename V::Out*>(tile + tile_off(lr, vec_in_row * V::kElems)) =
+                PairCast<T, BYTES>::template cast<FMT>(v[i], cs);
+        }
+    }
+    __syncthreads();
+    tile_transpose_out(tile, qt, rows, r0, c0, lane, warp);
+}
+
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+template <typename T, int FMT, int BYTES>
+cudaError_t launch_typed(const void* x, int64_t rows, int64_t cols, int block_rows, uint8_t* q, float* scales,
+                         uint8_t* qt, float* scales_t, cudaStream_t st) {
+    const int64_t tiles = (rows / kTT) * (cols / kTT);
+    if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(tiles));
+    const cudaError_t e =
+        block_rows == 1
+            ? launch_kernel(k_quant_block_transpose<T, FMT, BYTES, 0>, grid, dim3(kThreads), 0, st,
+                            static_cast<const T*>(x), rows, cols, q, scales, qt, scales_t)
+            : launch_kernel(k_quant_block_transpose<T, FMT, BYTES, 1>, grid, dim3(kThreads), 0, st,
+                            static_cast<const T*>(x), rows, cols, q, scales, qt, scales_t);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <typename T, int FMT>
+cudaError_t launch_width(const void* x, int64_t rows, int64_t cols, int block_rows, uint8_t* q, float* scales,
+                         uint8_t* qt, float* scales_t, cudaStream_t st) {
+    // 256-bit lanes when every tile row starts on a 32-byte boundary
+    if (aligned32(x) && (cols * static_cast<int64_t>(sizeof(T))) % 32 == 0)
+        return launch_typed<T, FMT, 32>(x, rows, cols, block_rows, q, scales, qt, scales_t, st);
+    return launch_typed<T, FMT, 16>(x, rows, cols, block_rows, q, scales, qt, scales_t, st);
+}
+
+}  // namespace
+
+cudaError_t launch_quant_block_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int block_rows,
+                                         int fmt, uint8_t* q, float* scales, uint8_t* qt, float* scales_t,
+                                         cudaStream_t st) {
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    if (dtype == 1)
+        return fmt == kE4M3 ? launch_width<uint16_t, kE4M3>(x, rows, cols, block_rows, q, scales, qt, scales_t, st)
+                            : launch_width<uint16_t, kE5M2>(x, rows, cols, block_rows, q, scales, qt, scales_t, st);
+    return fmt == kE4M3 ? launch_width<float, kE4M3>(x, rows, cols, block_rows, q, scales, qt, scales_t, st)
+                        : launch_width<float, kE5M2>(x, rows, cols, block_rows, q, scales, qt, scales_t, st);
+}
+
+}  // namespace fp8q

@@ -288,6 +288,32 @@ int fp8_quantize_per_tensor_transpose(const void *x, int dtype, int64_t rows, in
                                       void *stream);
 
 /*
+ * Blockwise quantization of x together with that of its transpose, from one
+ * read of x.  Follows [MP-handbook] "FP8 training", per_block (1x128
+ * activation blocks, 128x128 weight blocks, s = MAX / max(amax, 1e-12f) per
+ * block): the weight- and data-gradient GEMMs read their operands along the
+ * other dimension, so they need x^T quantized by the same rule.
+ *
+ *   x          [rows, cols] row-major input, FP8_F32 or FP8_BF16; rows and
+ *              cols multiples of 128
+ *   block      (1, 128) or (128, 128)
+ *   q, scales  exactly fp8_quantize_blockwise(x, block): codes [rows, cols],
+ *              scales [rows, cols/128] (1x128) or [rows/128, cols/128]
+ *   qt, scales_t
+ *              exactly fp8_quantize_blockwise(x^T, block): codes [cols, rows]
+ *              and scales [cols, rows/128] (1x128: one scale per 128
+ *              elements of a column of x) or [cols/128, rows/128] (128x128:
+ *              the same blocks as x, so qt = q^T and scales_t = scales^T)
+ * All four outputs are required.  Bit-exact with the two separate calls.
+ * Errors: FP8_ERR_NULL, FP8_ERR_SHAPE (other blocks; rows or cols not a
+ * multiple of 128), FP8_ERR_ALIGN (x, q, qt: 16 bytes; scales: 4),
+ * FP8_ERR_FORMAT, FP8_ERR_DTYPE, FP8_ERR_CUDA.
+ */
+int fp8_quantize_blockwise_transpose(const void *x, int dtype, int64_t rows, int64_t cols,
+                                     int block_rows, int block_cols, int fmt, uint8_t *q,
+                                     float *scales, uint8_t *qt, float *scales_t, void *stream);
+
+/*
  * MX quantization: blocks of 32 consecutive elements of a row share one
  * power-of-two scale.  Follows [MP-handbook] "FP8 training", closing notes
  * (Blackwell's MX formats, MXFP8: every 32 elements share a scale factor in

@@ -179,6 +179,18 @@ def quantize_per_tensor_transpose(x: np.ndarray, fmt: int, scale: float | None =
     return q, qt, s_out[0], a_out[0]
 
 
+def quantize_blockwise_transpose(x: np.ndarray, br: int, bc: int, fmt: int):
+    """The handbook's per_block applied to x and to x^T: (q, scales, qt, scales_t).
+
+    The transposed operand of a weight- or data-gradient GEMM is quantized by the same rule along the
+    other dimension; this is that definition written out, two calls of quantize_blockwise."""
+    if np.asarray(x).ndim != 2:
+        raise ValueError("the transposing blockwise quantize takes a 2-D array")
+    q, s = quantize_blockwise(x, br, bc, fmt)
+    qt, st = quantize_blockwise(np.ascontiguousarray(np.asarray(x).T), br, bc, fmt)
+    return q, s, qt, st
+
+
 def quantize_blockwise(x: np.ndarray, br: int, bc: int, fmt: int):
     """Blockwise quantize of a 2-D array.  Returns (codes, scales [ceil(R/br), ceil(C/bc)])."""
     x, dt = _as_input(x)

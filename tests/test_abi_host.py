@@ -37,7 +37,8 @@ def test_header_declares_the_boundary():
                                            "fp8_selftest_wait_timeout", "fp8_quantize_mx", "fp8_dequantize_mx",
                                            "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise",
                                            "fp8_quantize_delayed_step", "fp8_quantize_blockwise_grouped",
-                                           "fp8_quantize_delayed_step_grouped"])
+                                           "fp8_quantize_delayed_step_grouped",
+                                           "fp8_quantize_blockwise_transpose"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -195,6 +196,30 @@ def test_transpose_validation(L):
     assert f(A16, 1, 4, 64, 0, A16, A16, None, A16, None, None) == ERR_NULL      # qt
     assert f(A16, 1, 4, 64, 0, A16, A16, A1, A16, None, None) == ERR_ALIGN
     assert f(A16, 1, 4, 64, 0, A16, A1, A16, A16, None, None) == ERR_ALIGN
+
+
+def test_blockwise_transpose_validation(L):
+    f = L.fp8_quantize_blockwise_transpose
+    ok = (A16, 1, 256, 384, 1, 128, 0, A16, A16, A16, A16, None)
+    def call(**kw):
+        args = list(ok)
+        names = ["x", "dtype", "rows", "cols", "br", "bc", "fmt", "q", "scales", "qt", "scales_t", "stream"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+    assert call(fmt=9) == ERR_FORMAT
+    assert call(dtype=7) == ERR_DTYPE
+    assert call(br=128, bc=1) == ERR_SHAPE                # only 1x128 and 128x128
+    assert call(br=32) == ERR_SHAPE
+    assert call(rows=200) == ERR_SHAPE                    # rows and cols multiples of 128
+    assert call(cols=100) == ERR_SHAPE
+    assert call(rows=-128) == ERR_SHAPE
+    assert call(rows=0) == OK and call(cols=0, x=None) == OK  # nothing to do
+    for name in ("x", "q", "scales", "qt", "scales_t"):
+        assert call(**{name: None}) == ERR_NULL, name
+    for name in ("x", "q", "qt"):
+        assert call(**{name: A16 + 8}) == ERR_ALIGN, name
+    assert call(scales=A1) == ERR_ALIGN and call(scales_t=A1) == ERR_ALIGN
 
 
 def test_delayed_step_validation(L):

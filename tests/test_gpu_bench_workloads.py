@@ -2,6 +2,7 @@
 
 - MX 1x32 quantize and dequantize of the bf16 16384x7168 activations (outlier channels);
 - the transposing per-tensor cast of the same activations, delayed (given scale) and current;
+- 1x128 quantization of the same activations and of their transpose in one pass;
 - the blockwise GEMM at 16384x4096x7168 on sampled rows of C;
 - 128 weights of 1024x1024 in one grouped 128x128 call;
 - one grouped delayed-scaling step over 128 gradients of 2^20 elements.
@@ -51,6 +52,19 @@ def test_transpose_activations_16384x7168(activations, scale):
     assert_bytes_equal(q, oq, "q")
     # qt is q transposed, by definition of the second output
     assert_bytes_equal(qt, np.ascontiguousarray(oq.T), "qt")
+
+
+def test_blockwise_transpose_activations_16384x7168(activations):
+    a, xh = activations
+    x = to_cuda(a)
+    q, s, qt, st = B.fp8_quantize_blockwise_transpose(x, (1, 128), B.E4M3)
+    oq, os_ = oracle_blockwise(xh, 1, 128, oracle.E4M3)
+    assert_bytes_equal(s, fp32_bits(os_), "scales")
+    assert_bytes_equal(q, oq, "q")
+    del q, s, oq, os_
+    oqt, ost = oracle_blockwise(np.ascontiguousarray(xh.T), 1, 128, oracle.E4M3)
+    assert_bytes_equal(st, fp32_bits(ost), "scales_t")
+    assert_bytes_equal(qt, oqt, "qt")
 
 
 def test_gemm_16384x4096x7168_sampled_rows():

@@ -640,6 +640,49 @@ def test_per_tensor_transpose_16_byte_aligned_input():
     assert_bytes_equal(q, oq, "q")
 
 
+# -- blockwise quantization of x and of x^T in one pass ------------------------------------------
+
+BT_SHAPES = [(128, 128), (256, 384), (384, 128), (128, 1024), (1024, 4096)]
+
+
+def check_blockwise_transpose(x_cpu, block, fmt, what, x=None):
+    R, C = x_cpu.shape
+    br, bc = block
+    x = to_cuda(x_cpu) if x is None else x
+    gq, gt = Guarded((R, C), torch.uint8), Guarded((C, R), torch.uint8)
+    gs, gst = Guarded((R // br, C // bc), torch.float32), Guarded((C // br, R // bc), torch.float32)
+    B.fp8_quantize_blockwise_transpose(x, block, fmt, q=gq.t, scales=gs.t, qt=gt.t, scales_t=gst.t)
+    torch.cuda.synchronize()
+    for g in (gq, gt, gs, gst):
+        g.check()
+    oq, os_, oqt, ost = oracle.quantize_blockwise_transpose(host_input(x_cpu), br, bc, fmt)
+    assert_bytes_equal(gs.t, fp32_bits(os_), f"{what} scales")
+    assert_bytes_equal(gq.t, oq, f"{what} q")
+    assert_bytes_equal(gst.t, fp32_bits(ost), f"{what} scales_t")
+    assert_bytes_equal(gt.t, oqt, f"{what} qt")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("block", [(1, 128), (128, 128)])
+def test_blockwise_transpose(fmt, dtype, block):
+    for i, (R, C) in enumerate(BT_SHAPES):
+        x = inputs.random_matrix(R, C, seed=4300 + i, dtype=dtype, outlier_frac=0.01, factor=1e3)
+        x[:, 3] = 0  # an all-zero column: its 1x128 column blocks get MAX / eps
+        check_blockwise_transpose(x, block, fmt, f"{block} {R}x{C} {dtype}")
+
+
+def test_blockwise_transpose_16_byte_aligned_input():
+    R, C = 256, 512
+    x_cpu = inputs.random_matrix(R, C, seed=4400, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e3)
+    buf = torch.empty(R * C + 8, dtype=torch.bfloat16, device="cuda")
+    x = buf[8:].view(R, C)
+    x.copy_(x_cpu.to("cuda"))
+    assert x.data_ptr() % 32 == 16
+    for block in ((1, 128), (128, 128)):
+        check_blockwise_transpose(x_cpu, block, B.E4M3, f"16-byte aligned {block}", x=x)
+
+
 # -- one delayed-scaling step in one launch ---------------------------------------------------
 
 @pytest.mark.parametrize("fmt", FMTS)

@@ -399,3 +399,37 @@ def test_transposed_output_is_the_per_tensor_codes():
         assert np.array_equal(q, q1) and s == s1 and a == a1
         assert qt.shape == (53, 37)
         assert all(qt[c, r] == q1[r, c] for r in range(37) for c in range(53))
+
+
+# -- blockwise quantization of x and of x^T ---------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+@pytest.mark.parametrize("shape", [(128, 128), (256, 384), (200, 300), (1, 5), (130, 129)])
+def test_square_blocks_commute_with_transposition(fmt, shape):
+    """128x128 blocks of x^T are the blocks of x transposed, so quantizing x^T gives the transposed codes
+    and scales (ragged edges included)."""
+    x = inputs.random_matrix(*shape, seed=7100 + shape[0], dtype=torch.float32, outlier_frac=0.01, factor=1e3)
+    q, s, qt, st = oracle.quantize_blockwise_transpose(x.numpy(), 128, 128, fmt)
+    assert np.array_equal(qt, q.T)
+    assert np.array_equal(st.view(np.uint32), s.T.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_1x128_blocks_of_the_transpose_are_columns(fmt):
+    """For 1x128 blocks, qt's scales are MAX / max(amax, eps) over 128-row runs of x's columns (numpy fp32
+    arithmetic, IEEE division), and every block of qt holds a top code (its amax element maps to MAX)."""
+    R, C = 384, 256
+    x = inputs.random_matrix(R, C, seed=7200, dtype=torch.float32, outlier_frac=0.01, factor=1e3).numpy()
+    x[:128, 5] = 0.0  # an all-zero column block: scale MAX / eps, codes 0
+    q, s, qt, st = oracle.quantize_blockwise_transpose(x, 1, 128, fmt)
+    assert q.shape == (R, C) and s.shape == (R, C // 128) and qt.shape == (C, R) and st.shape == (C, R // 128)
+    amax = np.abs(x).reshape(R // 128, 128, C).max(axis=1).T.astype(np.float32)  # [C, R/128]
+    want = np.float32(oracle.MAX[fmt]) / np.maximum(amax, EPS32)
+    assert np.array_equal(st.view(np.uint32), want.astype(np.float32).view(np.uint32))
+    top = oracle.top_code(fmt)
+    mag = (qt & 0x7F).reshape(C, R // 128, 128).max(axis=2)
+    assert (mag[amax > EPS32] == top).all()
+    assert (qt[5, :128] & 0x7F == 0).all()
+    # q is the plain 1x128 quantization of x
+    q2, s2 = oracle.quantize_blockwise(x, 1, 128, fmt)
+    assert np.array_equal(q, q2) and np.array_equal(s.view(np.uint32), s2.view(np.uint32))
