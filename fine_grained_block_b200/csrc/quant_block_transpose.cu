@@ -120,21 +120,28 @@ struct ColMax<float, BYTES> {
 
 // MODE 0: 1x128 blocks (row scales for q, column scales for qt);
 // MODE 1: 128x128 blocks (one scale per tile for both).
-// Resident CTAs per SM each mode is compiled for (register cap).  Measured on
-// B200 on the bf16 16384x7168 activations: 128x128 runs at 98.7 % of the copy
-// peak with 3 or 4 and 85 % with 2; 1x128, whose column pass holds more
-// registers, spills under the caps of 3 and 4 (68 % and 58 %) and runs
-// best with 2 (73 %).
+// 1x128 reads its tile a second time, from L2, for the column cast instead
+// of holding it in registers across the two barriers of the column pass;
+// with that (and the row scales' divisions shared among a row's lanes) the
+// kernel fits the register cap of 4 CTAs per SM without spilling (bf16; an
+// fp32 tile is twice the registers and keeps the cap of 2).  Measured
+// on B200, bf16 activations 16384x7168, 1x128: 4954 GB/s holding the tile
+// with a cap of 2 CTAs; with the second read 4598 / 5162 / 5213 GB/s for 2 /
+// 3 / 4 CTAs.  128x128: 6462 GB/s (98.7 % of the copy peak) with 3 or 4 CTAs.
+#ifndef FP8Q_BLOCK_TRANSPOSE_RELOAD
+#define FP8Q_BLOCK_TRANSPOSE_RELOAD 1
+#endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
-#define FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS 2
+#define FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS 4
 #endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS
 #define FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS 3
 #endif
 
 template <typename T, int FMT, int BYTES, int MODE>
-__global__ void __launch_bounds__(kThreads, MODE == 0 ? FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
-                                                      : FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS)
+__global__ void __launch_bounds__(kThreads, MODE == 1               ? FP8Q_BLOCK_TRANSPOSE_128X128_MIN_CTAS
+                                           : sizeof(T) == 2         ? FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
+                                                                    : 2)
 k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uint8_t* __restrict__ q,
                         float* __restrict__ scales, uint8_t* __restrict__ qt, float* __restrict__ scales_t) {
     pdl_enter();
@@ -174,11 +181,21 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
             scales_t[tc * tiles_r + tr] = s;
         }
     } else {
-        // q: one scale per tile row (the row's kVecPerRow lanes reduce together)
+        // q: one scale per tile row.  The row's kVecPerRow lanes reduce its
+        // amax together; lane j of the row computes the scale of load j (one
+        // division per lane) and the row's lanes fetch the rest by shuffles.
+        float ra[G::kLoads];
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) ra[i] = warp_max<G::kVecPerRow>(V::amax(v[i]));
+        float mine = 0.0f;
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i)
+            if (i % G::kVecPerRow == vec_in_row) mine = ra[i];
+        const float s_mine = scale_from_amax<FMT>(mine);
+        const int group = lane - vec_in_row;  // first lane of this row
 #pragma unroll
         for (int i = 0; i < G::kLoads; ++i) {
-            const float ra = warp_max<G::kVecPerRow>(V::amax(v[i]));
-            const float s = scale_from_amax<FMT>(ra);
+            const float s = __shfl_sync(0xFFFFFFFFu, s_mine, group + i % G::kVecPerRow);
             const int lr = lr0 + i * G::kRowsPerLoad;
             st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row,
                       V::template cast<FMT>(v[i], f32x2(s, s)));
@@ -198,6 +215,12 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
         }
         __syncthreads();
         const float* cs = col_scale + vec_in_row * V::kElems;
+#if FP8Q_BLOCK_TRANSPOSE_RELOAD
+        // the tile again, from L2 (it was read a moment ago), instead of
+        // holding it in registers across the two barriers above
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
+#endif
 #pragma unroll
         for (int i = 0; i < G::kLoads; ++i) {
             const int lr = lr0 + i * G::kRowsPerLoad;
