@@ -63,7 +63,7 @@ int fp8_quantize_per_tensor(const void* x, int dtype, int64_t n, int fmt, const 
         return FP8_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (amax_out != nullptr) {
-        cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), st);
+        cudaError_t e = fp8q::launch_zero_f32(amax_out, st);
         if (e != cudaSuccess) return FP8_ERR_CUDA;
     }
     if (scale_in == nullptr && n > 0) {
@@ -140,7 +140,7 @@ int fp8_quantize_per_tensor_transpose(const void* x, int dtype, int64_t rows, in
         !aligned(amax_out, 4))
         return FP8_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (amax_out != nullptr && cudaMemsetAsync(amax_out, 0, sizeof(float), st) != cudaSuccess) return FP8_ERR_CUDA;
+    if (amax_out != nullptr && fp8q::launch_zero_f32(amax_out, st) != cudaSuccess) return FP8_ERR_CUDA;
     if (n == 0) {
         // no element: the scale of an empty tensor, as fp8_quantize_per_tensor gives it
         return fp8_quantize_per_tensor(x, dtype, 0, fmt, scale_in, q, scale_out, amax_out, stream);
@@ -159,7 +159,7 @@ int fp8_amax(const void* x, int dtype, int64_t n, float* amax_out, void* stream)
     if (amax_out == nullptr || (n > 0 && x == nullptr)) return FP8_ERR_NULL;
     if (!aligned(x, 16) || !aligned(amax_out, 4)) return FP8_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(amax_out, 0, sizeof(float), st) != cudaSuccess) return FP8_ERR_CUDA;
+    if (fp8q::launch_zero_f32(amax_out, st) != cudaSuccess) return FP8_ERR_CUDA;
     if (n == 0) return FP8_OK;
     return status_of(fp8q::launch_tensor_amax(x, dtype, n, amax_out, st));
 }

@@ -91,6 +91,8 @@ cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_
 
 // *scale_out = MAX / max(*amax_in, eps) (one thread).
 cudaError_t launch_scale_from_amax(const float* amax_in, int fmt, float* scale_out, cudaStream_t stream);
+// *p = 0, in stream order (one thread).
+cudaError_t launch_zero_f32(float* p, cudaStream_t stream);
 
 // Per-tensor cast.  scale_in == nullptr: s from *amax_in (current scaling);
 // else s = *scale_in (delayed), and amax_out (if non-null, zeroed by the

@@ -325,6 +325,14 @@ k_tensor_cast_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, con
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
 }
 
+// Zeroes the amax accumulator before the amax pass.  A kernel rather than a
+// memset, so that the call's launches stay one programmatic-dependent-launch
+// chain (a memset node would make the amax pass wait for a full completion).
+__global__ void k_zero_f32(float* p) {
+    pdl_enter();
+    *p = 0.0f;
+}
+
 template <int FMT>
 __global__ void k_scale_from_amax(const float* amax_in, float* scale_out) {
     pdl_enter();
@@ -547,6 +555,10 @@ cudaError_t launch_tensor_amax(const void* x, int dtype, int64_t n, float* amax_
     if (dtype == 1)
         return aligned32(x) ? amax_typed<uint16_t, 32>(x, n, amax_out, st) : amax_typed<uint16_t, 16>(x, n, amax_out, st);
     return aligned32(x) ? amax_typed<float, 32>(x, n, amax_out, st) : amax_typed<float, 16>(x, n, amax_out, st);
+}
+
+cudaError_t launch_zero_f32(float* p, cudaStream_t st) {
+    return launch_kernel(k_zero_f32, dim3(1), dim3(1), 0, st, p);
 }
 
 cudaError_t launch_scale_from_amax(const float* amax_in, int fmt, float* scale_out, cudaStream_t st) {
