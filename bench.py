@@ -412,7 +412,13 @@ def modes_breakdown(dev, stream, peak):
         "one pass)", 4 * n + 8 * (n // 128), time_in_graph([lambda r, st: raw.check(
             L.fp8_quantize_blockwise_transpose(a.data_ptr(), 1, R_, C_, 1, 128, 0, q.data_ptr(), s.data_ptr(),
                                                qt.data_ptr(), sbt.data_ptr(), st), "block transpose")], 20, dev))
-    del sbt
+    s2_ = torch.empty(R_ // 128, C_ // 128, dtype=torch.float32, device=dev)
+    st2_ = torch.empty(C_ // 128, R_ // 128, dtype=torch.float32, device=dev)
+    put("128x128_e4m3_quant_and_transpose", wl + " (q and qt = q^T with 128x128 tile scales, one pass)",
+        4 * n + 8 * (n // 16384), time_in_graph([lambda r, st: raw.check(
+            L.fp8_quantize_blockwise_transpose(a.data_ptr(), 1, R_, C_, 128, 128, 0, q.data_ptr(), s2_.data_ptr(),
+                                               qt.data_ptr(), st2_.data_ptr(), st), "block transpose")], 20, dev))
+    del sbt, s2_, st2_
     del a, q, s, y, e8, qt
 
     # size sweep point 2^28 (512 MiB bf16): 1x128, 128x128, per-tensor current E5M2, dequant
