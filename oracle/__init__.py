@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.orc_quantize_per_tensor_transpose.restype = c_int
         L.orc_gemm_blockwise.argtypes = [c_void, c_void, c_int, c_void, c_void, c_int, c_i64, c_i64, c_i64, c_void]
         L.orc_gemm_blockwise.restype = c_int
+        L.orc_gemm_blockwise_ex.argtypes = [c_void, c_void, c_int, c_void, c_void, c_int, c_int, c_i64, c_i64, c_i64,
+                                            c_void]
+        L.orc_gemm_blockwise_ex.restype = c_int
         L.orc_mx_exponent.argtypes = [ctypes.c_float, c_int, c_int]
         L.orc_mx_exponent.restype = c_int
         L.orc_quantize_mx.argtypes = [c_void, c_int, c_i64, c_i64, c_int, c_int, c_void, c_void]
@@ -239,8 +242,12 @@ def fake_quantize(x: np.ndarray, fmt: int, br: int = 1, bc: int = 128, scale: fl
     return y.reshape(x.shape), scales
 
 
-def gemm_blockwise(a: np.ndarray, sa: np.ndarray, a_fmt: int, b: np.ndarray, sb: np.ndarray, b_fmt: int):
-    """C [M, N] (float64) = sum over 128-wide K chunks of (dec(a) dec(b)^T) / (sa * sb)."""
+def gemm_blockwise(a: np.ndarray, sa: np.ndarray, a_fmt: int, b: np.ndarray, sb: np.ndarray, b_fmt: int,
+                   b_block: int = 128):
+    """C [M, N] (float64) = sum over 128-wide K chunks of (dec(a) dec(b)^T) / (sa * sb).
+
+    b_block 128: B in 128x128 blocks, sb [ceil(N/128), ceil(K/128)]; b_block 1: B in 1x128 blocks along K
+    (the weight-gradient operand), sb [N, ceil(K/128)]."""
     a = np.ascontiguousarray(a, dtype=np.uint8)
     b = np.ascontiguousarray(b, dtype=np.uint8)
     sa = np.ascontiguousarray(sa, dtype=np.float32)
@@ -248,10 +255,13 @@ def gemm_blockwise(a: np.ndarray, sa: np.ndarray, a_fmt: int, b: np.ndarray, sb:
     M, K = a.shape
     N = b.shape[0]
     nkc = math.ceil(K / 128)
-    if b.shape[1] != K or sa.shape != (M, nkc) or sb.shape != (math.ceil(N / 128), nkc):
+    if b_block not in (1, 128):
+        raise ValueError("gemm_blockwise: b_block is 1 or 128")
+    if b.shape[1] != K or sa.shape != (M, nkc) or sb.shape != (math.ceil(N / b_block), nkc):
         raise ValueError("gemm_blockwise: inconsistent shapes")
     c = np.empty((M, N), dtype=np.float64)
-    _check(lib().orc_gemm_blockwise(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_fmt, M, N, K, _ptr(c)))
+    _check(lib().orc_gemm_blockwise_ex(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_block, b_fmt, M, N, K,
+                                       _ptr(c)))
     return c
 
 

@@ -45,6 +45,9 @@
  *   R18 The transposed per-tensor output holds the same codes as q.
  *   R19 The consumer GEMM divides each 128-chunk partial sum by the two
  *       block scales (the quantizers' multipliers).
+ *   R20 The weight-gradient GEMM takes B with 1x128 blocks along K (the
+ *       transposed quantization of an activation): its scale is per row of
+ *       B and per chunk, sb[n][c]; otherwise the same sum as R19.
  */
 #include <math.h>
 #include <stdint.h>
@@ -544,11 +547,14 @@ int orc_dequantize_mx(const uint8_t *q, int fmt, int64_t rows, int64_t cols, con
  * a [M, K], b [N, K] row-major codes; sa [M, ceil(K/128)],
  * sb [ceil(N/128), ceil(K/128)]; c [M, N] in double.  Each product of two
  * FP8 values is exact in double, the chunk sums and the quotient are rounded
- * in double only: the result is the real value to within a few double ulps. */
-int orc_gemm_blockwise(const uint8_t *a, const float *sa, int a_fmt, const uint8_t *b, const float *sb,
-                       int b_fmt, int64_t M, int64_t N, int64_t K, double *c)
+ * in double only: the result is the real value to within a few double ulps.
+ * b_block_rows 1 (reading R20): B holds 1x128 blocks, sb [N, ceil(K/128)],
+ * and the divisor is sa[m][c] * sb[n][c]. */
+int orc_gemm_blockwise_ex(const uint8_t *a, const float *sa, int a_fmt, const uint8_t *b, const float *sb,
+                          int b_block_rows, int b_fmt, int64_t M, int64_t N, int64_t K, double *c)
 {
     if (!fmt_ok(a_fmt) || !fmt_ok(b_fmt) || M < 0 || N < 0 || K < 0) return ORC_EBADARG;
+    if (b_block_rows != 1 && b_block_rows != 128) return ORC_EBADARG;
     const int64_t nkc = (K + 127) / 128;
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
@@ -558,10 +564,16 @@ int orc_gemm_blockwise(const uint8_t *a, const float *sa, int a_fmt, const uint8
                 double p = 0.0;
                 for (int64_t k = k0; k < k1; ++k)
                     p += orc_fp8_decode(a[m * K + k], a_fmt) * orc_fp8_decode(b[n * K + k], b_fmt);
-                acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / 128) * nkc + kc]);
+                acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / b_block_rows) * nkc + kc]);
             }
             c[m * N + n] = acc;
         }
     }
     return ORC_OK;
+}
+
+int orc_gemm_blockwise(const uint8_t *a, const float *sa, int a_fmt, const uint8_t *b, const float *sb,
+                       int b_fmt, int64_t M, int64_t N, int64_t K, double *c)
+{
+    return orc_gemm_blockwise_ex(a, sa, a_fmt, b, sb, 128, b_fmt, M, N, K, c);
 }

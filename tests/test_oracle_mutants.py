@@ -52,10 +52,11 @@ MUTANTS = [
      [SCALING]),
     ("MX exponent off by one", "int k = emax_elem - (e - 1);", "int k = emax_elem - e;", [MX]),
     ("MX byte stores k, not -k", "(uint8_t)(127 - k)", "(uint8_t)(127 + k)", [MX]),
-    ("GEMM weight scale index transposed", "(double)sb[(n / 128) * nkc + kc]",
-     "(double)sb[kc * ((N + 127) / 128) + (n / 128)]", [GEMM]),
-    ("GEMM drops the activation scale", "acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / 128) * nkc + kc]);",
-     "acc += p / (double)sb[(n / 128) * nkc + kc];", [GEMM]),
+    ("GEMM weight scale index transposed", "(double)sb[(n / b_block_rows) * nkc + kc]",
+     "(double)sb[kc * ((N + b_block_rows - 1) / b_block_rows) + (n / b_block_rows)]", [GEMM]),
+    ("GEMM drops the activation scale",
+     "acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / b_block_rows) * nkc + kc]);",
+     "acc += p / (double)sb[(n / b_block_rows) * nkc + kc];", [GEMM]),
 ]
 
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
