@@ -510,6 +510,33 @@ def modes_breakdown(dev, stream, peak):
             "peak_kind": peak_kind, "us": round(ms * 1e3, 2)}
         del qa, sa, qb, sb, cg
 
+    # the weight-gradient GEMM of the same layer: dW [4096, 7168] = dY^T [4096, 16384] X [16384, 7168], both
+    # operands 1x128 along the 16384 tokens (the transposed outputs of fp8_quantize_blockwise_transpose)
+    Mg, Ng, Kg = 4096, 7168, 16384
+    dyt = inputs.random_matrix(Mg, Kg, seed=8, dtype=torch.bfloat16, scale=1e-3, outlier_frac=1e-3, factor=1e2,
+                               device=dev)
+    xt = inputs.random_matrix(Ng, Kg, seed=9, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e2, device=dev)
+    qa = torch.empty(Mg, Kg, dtype=torch.uint8, device=dev)
+    sa = torch.empty(Mg, Kg // 128, dtype=torch.float32, device=dev)
+    qb = torch.empty(Ng, Kg, dtype=torch.uint8, device=dev)
+    sb = torch.empty(Ng, Kg // 128, dtype=torch.float32, device=dev)
+    raw.check(L.fp8_quantize_blockwise(dyt.data_ptr(), 1, Mg, Kg, 1, 128, 1, qa.data_ptr(), sa.data_ptr(), st0),
+              "1x128")
+    raw.check(L.fp8_quantize_blockwise(xt.data_ptr(), 1, Ng, Kg, 1, 128, 0, qb.data_ptr(), sb.data_ptr(), st0),
+              "1x128")
+    cg = torch.empty(Mg, Ng, dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    del dyt, xt
+    ms = time_in_graph([lambda r, st: raw.check(L.fp8_gemm_blockwise_ex(
+        qa.data_ptr(), sa.data_ptr(), 1, qb.data_ptr(), sb.data_ptr(), 1, 0, Mg, Ng, Kg, cg.data_ptr(), 1, st),
+        "gemm wgrad")], 10, dev)
+    tflops = 2.0 * Mg * Ng * Kg / (ms * 1e-3) / 1e12
+    out[f"gemm_weight_gradient_e5m2xe4m3_{Mg}x{Ng}x{Kg}"] = {
+        "workload": f"dY^T [{Mg}, {Kg}] 1x128-scaled E5M2 x X^T [{Ng}, {Kg}] 1x128-scaled E4M3 -> bf16 dW",
+        "TFLOP_s": round(tflops, 1), "frac_of_peak": round(tflops / fp8_peak, 4), "peak_TFLOP_s": fp8_peak,
+        "peak_kind": peak_kind, "us": round(ms * 1e3, 2)}
+    del qa, sa, qb, sb, cg
+
     # many small tensors: 128 weights of 1024x1024 bf16 (2^20 elements each, 256 MiB in all), 128x128 E4M3,
     # one call per tensor against one grouped call
     from fine_grained_block_b200.binding import FP8BlockTensor

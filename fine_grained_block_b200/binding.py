@@ -56,6 +56,8 @@ SIGNATURES = {
     "fp8_scale_from_amax": (_c_int, [_vp, _c_int, _vp, _vp]),
     "fp8_fake_quantize": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]),
     "fp8_quantize_per_tensor_transpose": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fp8_gemm_blockwise_ex": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _i64, _i64, _i64, _vp, _c_int,
+                                       _vp]),
     "fp8_quantize_blockwise_transpose": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _c_int, _vp, _vp, _vp,
                                                   _vp, _vp]),
     "fp8_quantize_mx": (_c_int, [_vp, _c_int, _i64, _i64, _c_int, _c_int, _vp, _vp, _vp]),
@@ -325,17 +327,25 @@ def fp8_dequantize_mx(q: torch.Tensor, e8m0: torch.Tensor, fmt: int = E4M3, out_
 
 def fp8_gemm_blockwise(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, a_fmt: int = E4M3,
                        b_fmt: int = E4M3, out_dtype=torch.bfloat16, c: torch.Tensor | None = None,
-                       stream=None) -> torch.Tensor:
-    """C [M, N] = A [M, K] (1x128 scales sa) x B [N, K]^T (128x128 scales sb), FP8 tensor cores."""
+                       stream=None, b_block: int = 128) -> torch.Tensor:
+    """C [M, N] = A [M, K] (1x128 scales sa) x B [N, K]^T, FP8 tensor cores.
+
+    b_block 128: B with 128x128 scales sb [N/128, K/128] (fp8_gemm_blockwise); b_block 1: B with 1x128
+    scales sb [N, K/128], the weight-gradient form (fp8_gemm_blockwise_ex)."""
     _need_cuda(a, sa, b, sb, c)
     if a.dim() != 2 or b.dim() != 2 or a.shape[1] != b.shape[1]:
         raise ValueError("fp8_gemm_blockwise takes a [M, K] and b [N, K]")
     M, K = a.shape
     N = b.shape[0]
     c = torch.empty((M, N), dtype=out_dtype, device=a.device) if c is None else c
-    st = load_library().fp8_gemm_blockwise(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_fmt, M, N, K, _ptr(c),
-                                           _DTYPE_CODE[c.dtype], _stream(stream))
-    _check("fp8_gemm_blockwise", st)
+    if b_block == 128:
+        st = load_library().fp8_gemm_blockwise(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_fmt, M, N, K, _ptr(c),
+                                               _DTYPE_CODE[c.dtype], _stream(stream))
+        _check("fp8_gemm_blockwise", st)
+    else:
+        st = load_library().fp8_gemm_blockwise_ex(_ptr(a), _ptr(sa), a_fmt, _ptr(b), _ptr(sb), b_block, b_fmt, M, N,
+                                                  K, _ptr(c), _DTYPE_CODE[c.dtype], _stream(stream))
+        _check("fp8_gemm_blockwise_ex", st)
     return c
 
 

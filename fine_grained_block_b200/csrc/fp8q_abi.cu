@@ -290,10 +290,12 @@ int fp8_dequantize_mx(const uint8_t* q, int fmt, int64_t rows, int64_t cols, con
     return status_of(fp8q::launch_dequant_mx(q, fmt, rows, cols, e8m0, y, out_dtype, static_cast<cudaStream_t>(stream)));
 }
 
-int fp8_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb, int b_fmt,
-                       int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream) {
+int fp8_gemm_blockwise_ex(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb,
+                          int b_block_rows, int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
+                          void* stream) {
     if (!fmt_ok(a_fmt) || !fmt_ok(b_fmt)) return FP8_ERR_FORMAT;
     if (!dtype_ok(c_dtype)) return FP8_ERR_DTYPE;
+    if (b_block_rows != 1 && b_block_rows != 128) return FP8_ERR_SHAPE;
     if (M < 0 || N < 0 || K < 0 || N % 256 != 0 || K % 128 != 0) return FP8_ERR_SHAPE;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || checked_count(M, N) < 0) return FP8_ERR_SHAPE;
     if (M == 0 || N == 0) return FP8_OK;
@@ -307,7 +309,12 @@ int fp8_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8
     if (a == nullptr || sa == nullptr || b == nullptr || sb == nullptr) return FP8_ERR_NULL;
     if (!aligned(a, 16) || !aligned(b, 16) || !aligned(sa, 4) || !aligned(sb, 4)) return FP8_ERR_ALIGN;
     if (!fp8q::gemm_blockwise_supported()) return FP8_ERR_CUDA;
-    return status_of(fp8q::launch_gemm_blockwise(a, sa, a_fmt, b, sb, b_fmt, M, N, K, c, c_dtype, st));
+    return status_of(fp8q::launch_gemm_blockwise(a, sa, a_fmt, b, sb, b_block_rows, b_fmt, M, N, K, c, c_dtype, st));
+}
+
+int fp8_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb, int b_fmt,
+                       int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream) {
+    return fp8_gemm_blockwise_ex(a, sa, a_fmt, b, sb, 128, b_fmt, M, N, K, c, c_dtype, stream);
 }
 
 int fp8_amax_history_update(float* history, int32_t* state, int window, const float* amax, int fmt, float* scale,

@@ -49,11 +49,12 @@ cudaError_t launch_amax_history_update_ex(float* history, int32_t* state, int wi
 // FP8 GEMM with blockwise scales on the tcgen05 tensor cores:
 // C[M, N] = sum over 128-wide K chunks of (A_c B_c^T) / (sa * sb), A [M, K]
 // codes with 1x128 scales sa [M, K/128], B [N, K] codes with 128x128 scales
-// sb [N/128, K/128].  Needs N % 256 == 0, K % 128 == 0, K > 0.
+// sb [N/128, K/128] (b_block_rows 128) or 1x128 scales sb [N, K/128]
+// (b_block_rows 1).  Needs N % 256 == 0, K % 128 == 0, K > 0.
 bool gemm_blockwise_supported();
 cudaError_t launch_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb,
-                                  int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
-                                  cudaStream_t stream);
+                                  int b_block_rows, int b_fmt, int64_t M, int64_t N, int64_t K, void* c,
+                                  int c_dtype, cudaStream_t stream);
 
 // Device address of the status word of the current device (nullptr on failure).
 unsigned int* device_status_word();

@@ -92,10 +92,28 @@ constexpr uint32_t kTmemCols = 2 * kBN;   // two accumulators
 // (and per SM sub-partition: each holds one warp of every warpgroup), or an
 // increase would never be granted.
 constexpr int kLaunchRegs = 168;          // 65536 / 384 rounded down to a multiple of 8
-constexpr int kControlRegs = 40;
-constexpr int kPromoteRegs = 232;
-static_assert(kControlRegs + 2 * kPromoteRegs == 3 * kLaunchRegs, "register split must equal the launch total");
+#ifndef FP8Q_GEMM_B1_CONTROL_REGS
+#define FP8Q_GEMM_B1_CONTROL_REGS 56
+#endif
+// 1x128 B moves registers from the promotion to the control warpgroup, whose
+// warps 2-3 then stage the reciprocal column scales.
+template <int BROW>
+struct Split {
+    static constexpr int kControlRegs = BROW == 1 ? FP8Q_GEMM_B1_CONTROL_REGS : 40;
+    static constexpr int kPromoteRegs = (3 * kLaunchRegs - kControlRegs) / 2;
+    static_assert(kControlRegs + 2 * kPromoteRegs == 3 * kLaunchRegs, "register split must equal the launch total");
+    static_assert(kControlRegs % 8 == 0 && kPromoteRegs % 8 == 0, "setmaxnreg counts are multiples of 8");
+};
 static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the register file");
+
+// B with 1x128 blocks (the weight-gradient operand) has a scale per column
+// and chunk; two otherwise idle warps stage their reciprocals in a ring of
+// kRbSlots chunks ahead of the promotion.
+constexpr int kBarrierBytes = 512;       // shared memory reserved for the mbarriers
+constexpr int kRbSlots = 8;
+constexpr int kRbGroup = 4;               // chunks whose scales one fill round loads together
+constexpr int kRbFillWarps = 2;           // warps 2 and 3
+static_assert(kRbSlots % kRbGroup == 0 && kRbSlots >= 2 * kRbGroup, "the ring holds two fill rounds");
 
 template <bool PAIR>
 struct Cfg {
@@ -106,8 +124,9 @@ struct Cfg {
     static constexpr int kStages = PAIR ? 6 : 4;
     static constexpr int kAccEmptyArrivals = PAIR ? 16 : 8;  // promotion warps releasing an accumulator
     static constexpr uint32_t kFullTx = PAIR ? 2 * kStageBytes : kStageBytes;  // bytes per "full" phase
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* alignment */ + kBarrierBytes;
 };
+constexpr int kRbBytes = kRbSlots * kBN * 4;  // ring of per-column reciprocal B scales (1x128 B only)
 
 template <int STAGES>
 struct Barriers {
@@ -116,10 +135,16 @@ struct Barriers {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
+    uint64_t rb_full[kRbSlots];
+    uint64_t rb_empty[kRbSlots];
     uint32_t tmem_base;
 };
+static_assert(sizeof(Barriers<6>) <= kBarrierBytes, "barriers must fit their reserved bytes");
+static_assert(sizeof(Barriers<4>) <= kBarrierBytes, "barriers must fit their reserved bytes");
 
-template <int OUT, bool PAIR>
+// BROW: rows of a B scale block, 128 (128x128 blocks, sb [N/128, K/128]) or 1
+// (1x128 blocks along K, sb [N, K/128]).
+template <int OUT, bool PAIR, int BROW>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const float* __restrict__ sa, const float* __restrict__ sb, void* __restrict__ c, int64_t M,
@@ -128,6 +153,7 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     auto* bars = reinterpret_cast<Barriers<C::kStages>*>(tiles_smem + C::kStages * C::kStageBytes);
+    float* rb_ring = reinterpret_cast<float*>(tiles_smem + C::kStages * C::kStageBytes + kBarrierBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -151,6 +177,10 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             umma::mbar_init(&bars->acc_empty[b], C::kAccEmptyArrivals);
         }
         umma::mbar_init(&bars->mma_done, 1);
+        for (int r = 0; r < kRbSlots; ++r) {
+            umma::mbar_init(&bars->rb_full[r], kRbFillWarps);
+            umma::mbar_init(&bars->rb_empty[r], 8);  // this CTA's promotion warps
+        }
         umma::fence_mbar_init();
     }
     if (warp == 1) {
@@ -168,7 +198,7 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     // runs on across tiles, so the producer prefetches the next tile and the
     // MMAs start on it while the promotion warps store this one.
     bool timed_out = false;
-    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Split<BROW>::kControlRegs));
     if (warp == 0) {
         // ---- TMA producer ----------------------------------------------------
         if (lane == 0) {
@@ -243,9 +273,44 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             else umma::commit(&bars->mma_done);
             if (!umma::mbar_wait(&bars->mma_done, 0, kWaitLimitNs)) timed_out = true;
         }
+    } else if (BROW == 1 && warp < 4) {
+        // ---- reciprocal column scales of B (1x128 blocks), warps 2-3 ------------
+        // A round loads the scales of up to kRbGroup chunks (16 loads in
+        // flight per thread: the scales of a column are consecutive in K),
+        // then waits for their ring slots and publishes them one by one.
+        const int ft = (warp - 2) * 32 + lane;  // 0..63; columns ft + 64 i of the tile
+        uint32_t g = 0;
+        for (int64_t t = first; t < tiles && !timed_out; t += step) {
+            const float* sb_cols = sb + ((t % tiles_n) * kBN) * kc_stride;
+            for (int kc0 = 0; kc0 < nchunks && !timed_out; kc0 += kRbGroup) {
+                const int cnt = min(kRbGroup, nchunks - kc0);
+                float v[kRbGroup][kBN / 64];
+#pragma unroll
+                for (int u = 0; u < kRbGroup; ++u)
+#pragma unroll
+                    for (int i = 0; i < kBN / 64; ++i)
+                        v[u][i] = (u < cnt) ? __ldg(sb_cols + (ft + 64 * i) * kc_stride + kc0 + u) : 1.0f;
+#pragma unroll
+                for (int u = 0; u < kRbGroup; ++u) {
+                    if (u >= cnt) break;
+                    const uint32_t slot = (g + u) % kRbSlots;
+                    const uint32_t phase = ((g + u) / kRbSlots) & 1u;
+                    if (!umma::mbar_wait(&bars->rb_empty[slot], phase ^ 1u, kWaitLimitNs)) {
+                        timed_out = true;
+                        break;
+                    }
+                    float* rb = rb_ring + slot * kBN;
+#pragma unroll
+                    for (int i = 0; i < kBN / 64; ++i) rb[ft + 64 * i] = __frcp_rn(v[u][i]);
+                    __syncwarp();
+                    if (lane == 0) umma::mbar_arrive(&bars->rb_full[slot]);
+                }
+                g += static_cast<uint32_t>(cnt);
+            }
+        }
     } else if (warp >= 4) {
         // ---- promotion warps -------------------------------------------------
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPromoteRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Split<BROW>::kPromoteRegs));
         const int quarter = warp & 3;            // TMEM lanes this warp may access
         const int half = (warp - 4) >> 2;        // column half of the tile
         const int row = quarter * 32 + lane;     // row within this CTA's 128 = TMEM lane
@@ -257,15 +322,19 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const int64_t m = (t / tiles_n) * C::kTileM + rank * kBM + row;
             const int64_t col0 = (t % tiles_n) * kBN + half * 128;
             const float* sa_row = sa + (m < M ? m : 0) * kc_stride;
-            const float* sb_row = sb + (col0 >> 7) * kc_stride;
+            const float* sb_row = sb + (BROW == 1 ? 0 : (col0 >> 7) * kc_stride);
             float acc[128];
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
             for (int kc = 0; kc < nchunks; ++kc, ++g) {
                 const uint32_t buf = g & 1u;
                 const uint32_t acc_phase = (g >> 1) & 1u;
-                // 1 / (sa * sb): the dequant factor of this chunk for this row and column half
-                const float f = (m < M) ? __frcp_rn(__fmul_rn(__ldg(sa_row + kc), __ldg(sb_row + kc))) : 0.0f;
+                // 128x128 B: 1 / (sa * sb), the dequant factor of this chunk for this row and
+                // column half.  1x128 B: 1 / sa here; 1 / sb per column from the ring.
+                const float f = (m < M) ? (BROW == 1 ? __frcp_rn(__ldg(sa_row + kc))
+                                                     : __frcp_rn(__fmul_rn(__ldg(sa_row + kc), __ldg(sb_row + kc))))
+                                        : 0.0f;
+                const uint32_t slot = g % kRbSlots;
                 if (!umma::mbar_wait(&bars->acc_full[buf], acc_phase, kWaitLimitNs)) {
                     timed_out = true;
                     break;
@@ -286,9 +355,33 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         if (lane == 0)
                             umma::mbar_arrive_cluster(acc_empty0 + buf * static_cast<uint32_t>(sizeof(uint64_t)));
                     }
+                    if (BROW == 1) {
+                        if (h == 0 && !umma::mbar_wait(&bars->rb_full[slot], (g / kRbSlots) & 1u, kWaitLimitNs)) {
+                            timed_out = true;
+                            break;
+                        }
+                        const float4* rb = reinterpret_cast<const float4*>(rb_ring + slot * kBN + half * 128 + h * 64);
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) acc[h * 64 + j] = __fmaf_rn(p[j], f, acc[h * 64 + j]);
+                        for (int j4 = 0; j4 < 16; ++j4) {
+                            const float4 r = rb[j4];
+                            acc[h * 64 + 4 * j4] = __fmaf_rn(__fmul_rn(p[4 * j4], f), r.x, acc[h * 64 + 4 * j4]);
+                            acc[h * 64 + 4 * j4 + 1] =
+                                __fmaf_rn(__fmul_rn(p[4 * j4 + 1], f), r.y, acc[h * 64 + 4 * j4 + 1]);
+                            acc[h * 64 + 4 * j4 + 2] =
+                                __fmaf_rn(__fmul_rn(p[4 * j4 + 2], f), r.z, acc[h * 64 + 4 * j4 + 2]);
+                            acc[h * 64 + 4 * j4 + 3] =
+                                __fmaf_rn(__fmul_rn(p[4 * j4 + 3], f), r.w, acc[h * 64 + 4 * j4 + 3]);
+                        }
+                        if (h == 1) {
+                            __syncwarp();
+                            if (lane == 0) umma::mbar_arrive(&bars->rb_empty[slot]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) acc[h * 64 + j] = __fmaf_rn(p[j], f, acc[h * 64 + j]);
+                    }
                 }
+                if (timed_out) break;
             }
             if (!timed_out && m < M) {
                 if (OUT == 0) {
@@ -357,19 +450,20 @@ bool make_kmajor_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int OUT, bool PAIR>
+template <int OUT, bool PAIR, int BROW>
 cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, const float* sa, const float* sb,
                          void* c, int64_t M, int64_t N, int64_t K, uint32_t idesc, unsigned int* status,
                          cudaStream_t st) {
     using C = Cfg<PAIR>;
-    auto kern = k_gemm_blockwise<OUT, PAIR>;
+    auto kern = k_gemm_blockwise<OUT, PAIR, BROW>;
+    constexpr int kSmem = C::kSmemBytes + (BROW == 1 ? kRbBytes : 0);
     // The shared-memory opt-in, once per device (not inside a stream capture
     // on later calls).
     static std::atomic<bool> opted[128];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
     if (!opted[dev].load(std::memory_order_acquire)) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         opted[dev].store(true, std::memory_order_release);
     }
@@ -377,7 +471,7 @@ cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, con
     if (tiles == 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     int na = 0;
@@ -421,7 +515,7 @@ cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, con
 bool gemm_blockwise_supported() { return tensor_map_encoder() != nullptr; }
 
 cudaError_t launch_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, const uint8_t* b, const float* sb,
-                                  int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
+                                  int b_block_rows, int b_fmt, int64_t M, int64_t N, int64_t K, void* c, int c_dtype,
                                   cudaStream_t st) {
     // A pair pays off once there are two row tiles to share B between.
     const bool pair = M > kBM;
@@ -431,11 +525,15 @@ cudaError_t launch_gemm_blockwise(const uint8_t* a, const float* sa, int a_fmt, 
     unsigned int* status = device_status_word();
     if (status == nullptr) return cudaErrorInvalidValue;
     const uint32_t idesc = umma::instr_desc_f8f6f4(a_fmt, b_fmt, pair ? 2 * kBM : kBM, kBN);
-    if (pair)
-        return c_dtype == 0 ? launch_typed<0, true>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st)
-                            : launch_typed<1, true>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st);
-    return c_dtype == 0 ? launch_typed<0, false>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st)
-                        : launch_typed<1, false>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st);
+#define FP8Q_GEMM_LAUNCH(OUT, PAIR, BROW) \
+    launch_typed<OUT, PAIR, BROW>(map_a, map_b, sa, sb, c, M, N, K, idesc, status, st)
+    if (b_block_rows == 1) {
+        if (pair) return c_dtype == 0 ? FP8Q_GEMM_LAUNCH(0, true, 1) : FP8Q_GEMM_LAUNCH(1, true, 1);
+        return c_dtype == 0 ? FP8Q_GEMM_LAUNCH(0, false, 1) : FP8Q_GEMM_LAUNCH(1, false, 1);
+    }
+    if (pair) return c_dtype == 0 ? FP8Q_GEMM_LAUNCH(0, true, 128) : FP8Q_GEMM_LAUNCH(1, true, 128);
+    return c_dtype == 0 ? FP8Q_GEMM_LAUNCH(0, false, 128) : FP8Q_GEMM_LAUNCH(1, false, 128);
+#undef FP8Q_GEMM_LAUNCH
 }
 
 }  // namespace fp8q

@@ -386,6 +386,24 @@ int fp8_gemm_blockwise(const uint8_t *a, const float *sa, int a_fmt,
                        void *c, int c_dtype, void *stream);
 
 /*
+ * fp8_gemm_blockwise with a choice of B's scale blocks.  b_block_rows 128 is
+ * fp8_gemm_blockwise.  b_block_rows 1 takes B [N, K] quantized with 1x128
+ * blocks along K, sb [N, K/128]: the weight-gradient product dW = dY^T X,
+ * where both operands are activations (or their gradients) quantized along
+ * the token dimension (fp8_quantize_blockwise_transpose gives them):
+ *     C[m][n] = sum over K chunks c of 128:
+ *               (sum_{k in c} decode(a[m][k]) * decode(b[n][k])) / (sa[m][c] * sb[n][c])
+ * With 1x128 B each chunk's partial sum is multiplied by RN(1 / sa) and by
+ * RN(1 / sb[n]) and added in fp32; the bound on the error is that of
+ * fp8_gemm_blockwise.  Other arguments, shapes and errors as there, plus
+ * FP8_ERR_SHAPE for b_block_rows other than 1 or 128.
+ */
+int fp8_gemm_blockwise_ex(const uint8_t *a, const float *sa, int a_fmt,
+                          const uint8_t *b, const float *sb, int b_block_rows, int b_fmt,
+                          int64_t M, int64_t N, int64_t K,
+                          void *c, int c_dtype, void *stream);
+
+/*
  * Delayed scaling: push one amax into the amax history and refresh the scale.
  * Follows [FP8-native] s4.2 DelayedScaler.update: the last `window` amax
  * values are kept; once `window` of them have been seen, the scale becomes

@@ -38,7 +38,7 @@ def test_header_declares_the_boundary():
                                            "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise",
                                            "fp8_quantize_delayed_step", "fp8_quantize_blockwise_grouped",
                                            "fp8_quantize_delayed_step_grouped",
-                                           "fp8_quantize_blockwise_transpose"])
+                                           "fp8_quantize_blockwise_transpose", "fp8_gemm_blockwise_ex"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -196,6 +196,24 @@ def test_transpose_validation(L):
     assert f(A16, 1, 4, 64, 0, A16, A16, None, A16, None, None) == ERR_NULL      # qt
     assert f(A16, 1, 4, 64, 0, A16, A16, A1, A16, None, None) == ERR_ALIGN
     assert f(A16, 1, 4, 64, 0, A16, A1, A16, A16, None, None) == ERR_ALIGN
+
+
+def test_gemm_ex_validation(L):
+    f = L.fp8_gemm_blockwise_ex
+    ok = (A16, A16, 0, A16, A16, 1, 0, 128, 256, 128, A16, 1, None)
+    def call(**kw):
+        args = list(ok)
+        names = ["a", "sa", "a_fmt", "b", "sb", "b_block_rows", "b_fmt", "M", "N", "K", "c", "c_dtype", "stream"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+    assert call(b_block_rows=2) == ERR_SHAPE and call(b_block_rows=0) == ERR_SHAPE
+    assert call(a_fmt=3) == ERR_FORMAT and call(b_fmt=3) == ERR_FORMAT
+    assert call(c_dtype=5) == ERR_DTYPE
+    assert call(N=100) == ERR_SHAPE and call(K=100) == ERR_SHAPE and call(M=-1) == ERR_SHAPE
+    assert call(M=0) == OK
+    assert call(c=None) == ERR_NULL and call(sb=None) == ERR_NULL
+    assert call(a=A16 + 8) == ERR_ALIGN and call(sb=A1) == ERR_ALIGN and call(c=A16 + 4) == ERR_ALIGN
 
 
 def test_blockwise_transpose_validation(L):

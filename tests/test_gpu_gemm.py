@@ -1,7 +1,8 @@
 """GPU parity of the consumer GEMM (fp8_gemm_blockwise) against the oracle.
 
 The tensor cores sum each 128-product chunk in an order of their own, so this
-is not bit-exact.  The bound is derived from the arithmetic: every FP8 product
+is not bit-exact.  With B in 1x128 blocks the factor is RN(1/sa) and RN(1/sb[n])
+applied as two roundings, 3 x 2^-24 instead of 2^-23; the bound below holds.  The bound is derived from the arithmetic: every FP8 product
 is exact in fp32; a chunk sum of 128 products carries at most a relative
 2^-14 of the chunk's absolute sum (allowing an accumulator narrower than fp32,
 the limitation the handbook's promotion works around); the factor
@@ -42,13 +43,13 @@ def oracle_codes(M, N, K, a_fmt, b_fmt, seed):
     return qa, sa, qb, sb
 
 
-def check_gemm(qa, sa, a_fmt, qb, sb, b_fmt, c_gpu, what, rows=None):
+def check_gemm(qa, sa, a_fmt, qb, sb, b_fmt, c_gpu, what, rows=None, b_block=128):
     """Compare c_gpu (torch, [M, N]) with the oracle on the given rows (all by default)."""
     if rows is not None:
         qa, sa = qa[rows], sa[rows]
         c_gpu = c_gpu[torch.as_tensor(rows, device=c_gpu.device)]
-    want = oracle.gemm_blockwise(qa, sa, a_fmt, qb, sb, b_fmt)
-    mag = oracle.gemm_blockwise(qa & 0x7F, sa, a_fmt, qb & 0x7F, sb, b_fmt)
+    want = oracle.gemm_blockwise(qa, sa, a_fmt, qb, sb, b_fmt, b_block=b_block)
+    mag = oracle.gemm_blockwise(qa & 0x7F, sa, a_fmt, qb & 0x7F, sb, b_fmt, b_block=b_block)
     got = c_gpu.float().cpu().numpy().astype(np.float64)
     tol = 2.0 ** -12 * mag
     if c_gpu.dtype == torch.bfloat16:
@@ -121,6 +122,41 @@ def test_gemm_mixed_formats(a_fmt, b_fmt):
                                  b_fmt=b_fmt, out_dtype=torch.float32)
         torch.cuda.synchronize()
         check_gemm(qa, sa, a_fmt, qb, sb, b_fmt, c, f"{M}x{N}x{K} fmts {a_fmt},{b_fmt}")
+
+
+# -- B with 1x128 blocks: the weight-gradient form --------------------------------------------------
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_b_1x128_matches_oracle(out_dtype):
+    """Per-column, per-chunk B scales (sb [N, K/128]): the reciprocal ring and the two-factor promotion."""
+    for i, (M, N, K) in enumerate(SHAPES + [(512, 1024, 1024)]):
+        x = inputs.random_matrix(M, K, seed=5400 + i, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e2)
+        w = inputs.random_matrix(N, K, seed=5500 + i, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e2)
+        qa, sa = oracle.quantize_blockwise(host_input(x), 1, 128, B.E4M3)
+        qb, sb = oracle.quantize_blockwise(host_input(w), 1, 128, B.E4M3)
+        c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
+                                 to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), out_dtype=out_dtype,
+                                 b_block=1)
+        torch.cuda.synchronize()
+        check_gemm(qa, sa, B.E4M3, qb, sb, B.E4M3, c, f"1x128 B {M}x{N}x{K}", b_block=1)
+
+
+def test_weight_gradient_from_the_transposing_quantizer():
+    """dW = dY^T X: dY [T, out] (E5M2) and X [T, in] (E4M3) go through fp8_quantize_blockwise_transpose; its
+    transposed outputs are the GEMM's operands, both 1x128 along the tokens."""
+    T, n_out, n_in = 1024, 256, 512
+    dy = inputs.random_matrix(T, n_out, seed=5600, dtype=torch.bfloat16, scale=1e-3, outlier_frac=1e-3, factor=1e2)
+    x = inputs.random_matrix(T, n_in, seed=5601, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e2)
+    _, _, qdt, sdt = B.fp8_quantize_blockwise_transpose(to_cuda(dy), (1, 128), B.E5M2)
+    _, _, qxt, sxt = B.fp8_quantize_blockwise_transpose(to_cuda(x), (1, 128), B.E4M3)
+    dw = B.fp8_gemm_blockwise(qdt, sdt, qxt, sxt, a_fmt=B.E5M2, b_fmt=B.E4M3, out_dtype=torch.float32, b_block=1)
+    torch.cuda.synchronize()
+    check_gemm(qdt.cpu().numpy(), sdt.cpu().numpy(), B.E5M2, qxt.cpu().numpy(), sxt.cpu().numpy(), B.E4M3, dw,
+               "weight gradient", b_block=1)
+    ref = dy.double().T @ x.double()
+    mag = dy.double().abs().T @ x.double().abs()
+    # E5M2 and E4M3 codes are within 2^-3 and 2^-4 of their inputs: 0.125 + 0.0625 + their product < 0.2
+    assert bool(((dw.double().cpu() - ref).abs() <= 0.2 * mag).all())
 
 
 def test_gemm_reports_no_wait_timeout():
