@@ -39,6 +39,15 @@
 // start on it while the promotion warps store this one.
 // Rows past M arrive as zeros from the copy engine and are not stored.
 //
+// B's scales come in two layouts (template BROW):
+//   128  B in 128x128 blocks (a weight), sb [N/128, K/128]: one factor
+//        1/(sa*sb) per row, chunk and column half;
+//   1    B in 1x128 blocks along K (the weight gradient dW = dY^T X, whose
+//        operands are both quantized along the tokens), sb [N, K/128]: warps
+//        2-3 stage RN(1/sb) for the tile's 256 columns, 4 chunks per round,
+//        in an 8-slot shared-memory ring with its own barriers, and the
+//        promotion multiplies each partial by RN(1/sa) and the column's
+//        reciprocal (56 control / 224 promotion registers).
 // Two variants:
 //   single CTA (M 128 x N 256 per MMA): the CTA loads A (16 KiB) and all of
 //              B (32 KiB) per chunk, 4 stages;
