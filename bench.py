@@ -257,12 +257,12 @@ def run_reference(args):
     from fine_grained_block_b200 import inputs
     w = inputs.weight_4096(seed=1)
     bits = inputs.bf16_bits(w)
-    # size each step's sample so that warm-up + K steps take about a minute
+    # size each step's sample so that warm-up + K steps take about --ref-budget-s seconds (a minute by default)
     probe = bits[:128, :1024].copy()
     oracle_step_seconds(probe, 1)
     t_probe = oracle_step_seconds(probe, 2) / 2
     per_elem = t_probe / probe.size
-    budget = 60.0 / max(1, args.steps + args.warmup)
+    budget = args.ref_budget_s / max(1, args.steps + args.warmup)
     cols = int(max(128, min(COLS, (budget / per_elem / 128) // 128 * 128)))
     sample = bits[:128, :cols].copy()
     for _ in range(args.warmup):
@@ -881,6 +881,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-modes", action="store_true", help="skip the per-mode breakdown")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--ref-budget-s", type=float, default=60.0,
+                    help="reference arm: seconds of oracle work for warm-up + timed steps together")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
