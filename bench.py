@@ -771,6 +771,25 @@ def run_ours(args):
     tq = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
     td = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
     del g_split
+
+    # Single steps, timed one by one: 10 warm-up and 50 timed replays of a one-step graph, each after a
+    # 512 MiB write that flushes L2 (outside the events), median and best.  Each rep also carries the graph
+    # launch and a cold start, so these read lower than the steady-state timed region above.
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    g_one, _ = capture(args.warmup, 1, False)
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rep_ms = []
+    for r in range(10 + 50):
+        flush.zero_()
+        e_a.record(stream)
+        g_one.replay()
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        if r >= 10:
+            rep_ms.append(e_a.elapsed_time(e_b))
+    del g_one, flush
+    rep_med, rep_best = statistics.median(rep_ms), min(rep_ms)
+    rep_med, rep_best = max_over_ranks([rep_med, rep_best], world, device=dev)
     total_ms, tq, td = max_over_ranks([total_ms, tq, td], world, device=dev)
     value = (qb + db) * args.steps * world / (total_ms * 1e-3) / 1e9
 
@@ -854,6 +873,12 @@ def run_ours(args):
                     "d2h_bytes_per_step": hq.numel() + hs.numel() * 4 + hy.numel() * 2, "steps": e2e_steps,
                     "note": "pinned host buffers; uploads, kernels and downloads on three streams, so one "
                             "step's download overlaps the next step's upload"},
+            "per_rep": {"reps": 50, "warmup": 10, "l2": "512 MiB flush before each rep, outside the events",
+                        "median_us": round(rep_med * 1e3, 2), "best_us": round(rep_best * 1e3, 2),
+                        "median_GB_s": round((qb + db) * world / (rep_med * 1e-3) / 1e9, 1),
+                        "best_GB_s": round((qb + db) * world / (rep_best * 1e-3) / 1e9, 1),
+                        "note": "one step per graph replay, events around it: includes the launch and a cold "
+                                "start, which the timed region amortizes"},
             "gpu_launches": 2 * args.steps,
             "timing": f"K steps replayed from CUDA graphs of <= {GRAPH_CHUNK} steps; events around the region only",
             "clocks": clocks.summary(),
