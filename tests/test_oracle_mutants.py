@@ -54,6 +54,9 @@ MUTANTS = [
     ("MX byte stores k, not -k", "(uint8_t)(127 - k)", "(uint8_t)(127 + k)", [MX]),
     ("GEMM weight scale index transposed", "(double)sb[(n / b_block_rows) * nkc + kc]",
      "(double)sb[kc * ((N + b_block_rows - 1) / b_block_rows) + (n / b_block_rows)]", [GEMM]),
+    ("GEMM ignores B's block height (1x128 B read as 128x128)",
+     "acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / b_block_rows) * nkc + kc]);",
+     "acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / 128) * nkc + kc]);", [GEMM]),
     ("GEMM drops the activation scale",
      "acc += p / ((double)sa[m * nkc + kc] * (double)sb[(n / b_block_rows) * nkc + kc]);",
      "acc += p / (double)sb[(n / b_block_rows) * nkc + kc];", [GEMM]),
