@@ -9,8 +9,8 @@ Per-tensor current scaling has one real exchange: the scale of the whole
 tensor needs the amax of all shards (PyTorch-FP8 page s4.1), so each rank
 reduces its shard's amax on its GPU, the ranks all-reduce (MAX) that one
 fp32 value, and each rank then forms the scale and casts its shard.  Delayed
-scaling (s4.2) needs no exchange before the cast; the history update can
-all-reduce the amax the same way off the critical path.
+scaling (s4.2) needs no exchange before the cast; ShardedDelayedScaler
+all-reduces the amax after it, for the history update, off the critical path.
 
 The compute steps are the library's kernels.  ``ShardOps`` bundles them so
 that a test can substitute a CPU implementation and check the collective
@@ -79,3 +79,63 @@ def quantize_blockwise_sharded(x_local: torch.Tensor, block=(1, 128), fmt: int =
     no communication; the result equals the unsharded one restricted to these rows."""
     ops = ops or library_ops()
     return ops.blockwise(x_local, tuple(block), fmt)
+
+
+@dataclass
+class DelayedOps:
+    """The per-shard steps of delayed scaling (default: the CUDA library).
+
+    new_state(window, fmt, algo, alpha, margin, device) -> state with .scale ([1] fp32, the scale the next
+    cast uses); cast_amax(x, state) -> (codes, this shard's amax [1]) with the state's scale;
+    update(state, amax) pushes the (global) amax into the history and refreshes state.scale."""
+    new_state: Callable
+    cast_amax: Callable
+    update: Callable
+
+
+def library_delayed_ops() -> DelayedOps:
+    from . import binding as B
+
+    def new_state(window, fmt, algo, alpha, margin, device):
+        return B.DelayedScaler(window=window, fmt=fmt, device=device, algo=algo, alpha=alpha, margin=margin,
+                               fused=False)
+
+    def cast_amax(x, st):
+        q, _, amax = B.fp8_quantize_per_tensor(x, st.fmt, scale_in=st.scale, scale_out=st.scale_used,
+                                                amax_out=st.amax)
+        return q, amax
+
+    def update(st, amax):
+        if st.algo == B.AMAX_WINDOW_MAX and st.margin == 1.0:
+            B.fp8_amax_history_update(st.history, st.state, amax, st.scale, st.fmt)
+        else:
+            B.fp8_amax_history_update_ex(st.history, st.state, amax, st.scale, st.fmt, st.algo, st.alpha,
+                                         st.margin)
+
+    return DelayedOps(new_state=new_state, cast_amax=cast_amax, update=update)
+
+
+class ShardedDelayedScaler:
+    """Delayed scaling of a row-sharded tensor (PyTorch-FP8 page s4.2, over several GPUs).
+
+    Each step casts this rank's rows with the scale every rank holds, reduces the shard's amax in the same
+    pass, then all-reduces (MAX) that one fp32 and pushes the global amax into the history.  The exchange
+    comes after the cast, so it is off the cast's critical path; every rank's history and next scale stay
+    identical, equal to those of the whole tensor on one GPU."""
+
+    def __init__(self, window: int = 16, fmt: int = 1, group=None, ops: DelayedOps | None = None,
+                 device="cuda", algo: int = 0, alpha: float = 1.0, margin: float = 1.0):
+        self.ops = ops or library_delayed_ops()
+        self.group = group
+        self.state = self.ops.new_state(window, fmt, algo, alpha, margin, device)
+
+    @property
+    def scale(self) -> torch.Tensor:
+        return self.state.scale
+
+    def step(self, x_local: torch.Tensor) -> torch.Tensor:
+        q, amax = self.ops.cast_amax(x_local, self.state)
+        if _world(self.group) > 1:
+            dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=self.group)
+        self.ops.update(self.state, amax)
+        return q

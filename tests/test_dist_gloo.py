@@ -49,6 +49,37 @@ def oracle_ops():
     return sharded.ShardOps(amax=amax, scale_from_amax=scale, cast=cast, blockwise=blockwise)
 
 
+class OracleDelayedState:
+    """A rank's delayed-scaling state kept by the oracle's AmaxHistory."""
+
+    def __init__(self, window, fmt, algo, alpha, margin):
+        self.fmt = fmt
+        self.h = oracle.AmaxHistory(window, fmt, algo=algo, alpha=alpha, margin=margin)
+
+    @property
+    def scale(self):
+        return torch.from_numpy(self.h.scale.copy())
+
+
+def oracle_delayed_ops():
+    def cast_amax(x, st):
+        q, _, a = oracle.quantize_per_tensor(inputs.bf16_bits(x), st.fmt, scale=float(st.h.scale[0]))
+        return torch.from_numpy(q), torch.tensor([float(a)], dtype=torch.float32)
+
+    return sharded.DelayedOps(new_state=lambda w, f, al, a, m, d: OracleDelayedState(w, f, al, a, m),
+                              cast_amax=cast_amax, update=lambda st, amax: st.h.update(float(amax.item())))
+
+
+DELAYED_STEPS, DELAYED_WINDOW = 6, 3
+
+
+def delayed_input(k):
+    """Step k's tensor: the largest element sits in rank (k % 2)'s rows."""
+    x = inputs.random_matrix(300, 256, seed=90 + k, dtype=torch.bfloat16, outlier_frac=0.002, factor=1e2)
+    x[10 if k % 2 == 0 else 250, 3] = torch.tensor(3e3 * (k + 1), dtype=torch.bfloat16)
+    return x
+
+
 def _worker(rank, port, outdir, case):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -68,6 +99,16 @@ def _worker(rank, port, outdir, case):
                 q, s = sharded.quantize_blockwise_sharded(x[r0:r1].contiguous(), block, oracle.E4M3, ops=oracle_ops())
                 np.save(os.path.join(outdir, f"b{block[0]}_q{rank}.npy"), q.numpy())
                 np.save(os.path.join(outdir, f"b{block[0]}_s{rank}.npy"), s.numpy())
+        elif case == "delayed":
+            r0, r1 = sharded.row_shard(300, WORLD, rank, multiple=1)
+            sc = sharded.ShardedDelayedScaler(window=DELAYED_WINDOW, fmt=oracle.E5M2, ops=oracle_delayed_ops(),
+                                              device="cpu")
+            for k in range(DELAYED_STEPS):
+                scale_used = float(sc.scale.item())
+                q = sc.step(delayed_input(k)[r0:r1].contiguous())
+                np.save(os.path.join(outdir, f"d{k}_q{rank}.npy"), q.numpy())
+                np.save(os.path.join(outdir, f"d{k}_s{rank}.npy"),
+                        np.array([scale_used, float(sc.scale.item())], dtype=np.float32))
         elif case == "timing":
             import importlib.util
             root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -141,3 +182,22 @@ def test_bench_timing_is_max_over_ranks():
     out = _run("timing")
     want = [2.0, 5.0, 0.5]
     assert out["t0.npy"].tolist() == want and out["t1.npy"].tolist() == want
+
+
+def test_delayed_scaling_sharded_matches_unsharded():
+    """Each rank casts its rows with the shared scale, then the ranks all-reduce the amax for the history
+    update: codes, scales used and next scales equal the whole tensor's on one device, step after step,
+    although the largest element alternates between the ranks."""
+    out = _run("delayed")
+    ref = oracle.AmaxHistory(DELAYED_WINDOW, oracle.E5M2)
+    for k in range(DELAYED_STEPS):
+        xh = inputs.bf16_bits(delayed_input(k))
+        s_ref = float(ref.scale[0])
+        oq, _, oa = oracle.quantize_per_tensor(xh, oracle.E5M2, scale=s_ref)
+        ref.update(oa)
+        q = np.concatenate([out[f"d{k}_q{r}.npy"].reshape(-1, 256) for r in range(WORLD)])
+        assert np.array_equal(q, oq.reshape(q.shape)), k
+        for r in range(WORLD):
+            used, nxt = out[f"d{k}_s{r}.npy"]
+            assert np.float32(used) == np.float32(s_ref) and np.float32(nxt) == ref.scale[0], (k, r)
+    assert float(ref.scale[0]) != 1.0  # the window filled and the scale moved off its initial value
