@@ -5,9 +5,9 @@
 // (delayed scaling: the scale comes from earlier steps' amax, so the cast
 // needs no global reduction first).
 //
-// Current scaling is two grid-wide passes: k_tensor_amax (at most one
-// atomicMax per CTA into the caller's amax_out), then k_tensor_cast, which
-// turns that amax into s in every CTA.  The cast pass takes its chunks in the
+// Current scaling is two grid-wide passes after k_zero_f32 clears the
+// caller's amax_out: k_tensor_amax (at most one atomicMax per CTA into
+// amax_out), then k_tensor_cast, which turns that amax into s in every CTA.  The cast pass takes its chunks in the
 // reverse order of the amax pass, so its first reads find the most recently
 // read data still in L2.  Delayed scaling is one pass: cast with the given s
 // and reduce this step's amax from the same registers.  Each CTA owns one
