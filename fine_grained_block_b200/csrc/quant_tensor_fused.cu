@@ -8,7 +8,7 @@
 // workspace, and waits at a grid-wide barrier; the last CTA to arrive writes
 // amax_out and scale_out and resets the workspace; then every CTA casts the
 // slice it still holds.  x is read once and the three launches of the
-// two-pass path (memset, amax, cast) become one.
+// two-pass path (zeroing, amax, cast) become one.
 //
 // The launch is cooperative, so all CTAs are co-resident and the barrier
 // cannot deadlock.  The barrier wait is still bounded (about a second); if it
