@@ -22,7 +22,6 @@ import torch
 
 E4M3, E5M2 = 0, 1
 F32, BF16 = 0, 1
-FP8_MAX = {E4M3: 448.0, E5M2: 57344.0}
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp8q.so")

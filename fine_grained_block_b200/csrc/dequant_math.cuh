@@ -1,9 +1,16 @@
 // dequant_math.cuh -- the exact FP8 -> fp32 quotient RN(q / s) used by the
 // dequantize and fake-quantize kernels.
 //
+// The method is Markstein's residual-correction division (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990; also his "IA-64 and Elementary
+// Functions", 2000): a quotient estimate from the rounded reciprocal, its
+// exact residual from one fused multiply-add, and one correction step.
 // Every FP8 value is (1 + j/8) * 2^a.  With r = RN(1/s),
 //     y0 = RN(q * r);  e = RN(q - s * y0) (fma);  y = RN(y0 + e * r) (fma)
-// equals the IEEE quotient for every code as long as no step leaves the
+// The general theorem asks for conditions that are not checked here;
+// instead, for the FP8 dividends this library has, the result is verified
+// to equal the IEEE quotient for every code as long as no step leaves the
 // normal range: tests/c/recip_division_exhaustive.c checks the 8 FP8
 // significands against all 2^23 scale significands.  That holds for |s| in
 // [2^-100, 2^101); other scales use the per-element IEEE division.

@@ -163,6 +163,56 @@ def test_encode_random_fp32_vs_torch(fmt):
     assert np.array_equal(ours, ref)
 
 
+def nearest_code_rule(v: np.ndarray, fmt: int, t: dict) -> np.ndarray:
+    """The encoding's definition, vectorised in float64 and written from the format table alone.
+
+    The finite magnitudes of the table, in code order, are searched for the two neighbours of |v|; the
+    nearer one wins, a tie goes to the even code, and anything beyond the largest value takes the largest
+    code.  The sign bit of v is the code's sign bit (so -0 and negatives that round to zero give 0x80).
+    Every quantity is exact in float64: v is an fp32 value and the table's values have 4 significant bits."""
+    M, bias = t["man_bits"], t["bias"]
+    # magnitudes grow with the code; the finite ones are those up to the table's largest value
+    vals = np.array([v_ for v_ in (_table_value(c, M, bias) for c in range(128)) if v_ <= t["max"]])
+    top = vals.size - 1
+    a = np.abs(v.astype(np.float64))
+    hi = np.minimum(np.searchsorted(vals, a, side="left"), top)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - vals[lo], vals[hi] - a
+    pick = np.where(d_hi < d_lo, hi, lo)
+    tie = (d_hi == d_lo) & (hi != lo)
+    pick = np.where(tie, np.where(hi % 2 == 0, hi, lo), pick)
+    pick = np.where(a >= vals[top], top, pick)
+    pick = np.where(a <= 0.0, 0, pick)
+    sign = (v.view(np.uint32) >> 31).astype(np.int64) << 7
+    return (pick | sign).astype(np.uint8)
+
+
+def _table_value(code: int, M: int, bias: int) -> float:
+    e, m = code >> M, code & ((1 << M) - 1)
+    if e == 0:
+        return m * 2.0 ** (1 - bias - M)
+    return (1 + m / 2 ** M) * 2.0 ** (e - bias)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_encode_ten_million_random_fp32_vs_nearest_code_rule(fmt):
+    """10^7 random fp32 values (log-uniform magnitudes from the fp32 subnormals to 4x the format's
+    largest value, random sign, plus random bit patterns of finite fp32 values) against the encoding's
+    definition: nearest finite code, ties to the even code, saturation beyond the largest value."""
+    t = table()[fmt]
+    rng = np.random.default_rng(7_000_000 + fmt)
+    n = 10_000_000
+    e = rng.uniform(-152, math.log2(t["max"]) + 2, size=n - n // 10)
+    v = (np.exp2(e) * rng.choice([-1.0, 1.0], size=e.size)).astype(np.float32)
+    bits = rng.integers(0, 1 << 32, size=n // 10, dtype=np.uint64).astype(np.uint32)
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]  # finite patterns only
+    v = np.concatenate([v, bits.view(np.float32)])
+    want = nearest_code_rule(v, fmt, t)
+    got = oracle.encode_array(v, fmt)
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, f"{bad.size} mismatches, first {v[bad[0]]!r}: got {got[bad[0]]:#x} want {want[bad[0]]:#x}"
+
+
 @pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
 def test_saturation(fmt):
     top = oracle.top_code(fmt)

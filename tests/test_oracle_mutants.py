@@ -48,6 +48,15 @@ MUTANTS = [
      "const float d = (float)((double)m / (double)margin);", [SCALING]),
     ("EMA weights swapped", "const float beta = (float)(1.0 - (double)alpha);", "const float beta = alpha;",
      [SCALING]),
+    ("EMA as m + alpha * (amax - m), each step rounded",
+     "history[0] = (float)((double)a_part + (double)m_part);",
+     "history[0] = (float)((double)history[0] + (double)(float)((double)alpha * (double)(float)((double)amax - "
+     "(double)history[0]))); (void)a_part; (void)m_part;",
+     [SCALING]),
+    ("EMA sum fused with the amax product (one rounding)",
+     "history[0] = (float)((double)a_part + (double)m_part);",
+     "history[0] = (float)fma((double)alpha, (double)amax, (double)m_part); (void)a_part;",
+     [SCALING]),
     ("transposed copy not transposed", "qt[c * rows + r] = q[r * cols + c];", "qt[r * cols + c] = q[r * cols + c];",
      [SCALING]),
     ("MX exponent off by one", "int k = emax_elem - (e - 1);", "int k = emax_elem - e;", [MX]),

@@ -361,6 +361,31 @@ def test_ema_alpha_one_is_the_latest_amax_and_alpha_zero_the_first(fmt):
             assert s1 == 1.0 and s0 == 1.0  # warm-up: the scale keeps its initial value
 
 
+def test_ema_interior_alpha_hand_example():
+    """One moving-average update at alpha = 5/8, worked by hand from the reading of the PyTorch-FP8
+    page's smoothing (s4.2-4.3): m' = RN(RN(alpha * amax) + RN(RN(1 - alpha) * m)), every step fp32.
+
+    u = 2^-23 (the fp32 spacing in [1, 2)).  m = 1 + 13u, amax = 4 + 8u, 1 - alpha = 3/8 exactly.
+      alpha * amax = 2.5 + 5u.     In [2, 4) the spacing is 2u: 2.5 + 2.5(2u), a tie; the even
+                                   significand is 2.5 + 2(2u) = 2.5 + 4u.
+      (3/8) * m = 0.375 + 4.875u.  In [0.25, 0.5) the spacing is u/4: 0.375 + 19.5(u/4), a tie; the
+                                   even significand is 0.375 + 20(u/4) = 0.375 + 5u.
+      sum = 2.875 + 9u = 2.875 + 4.5(2u), a tie; the even significand is 2.875 + 4(2u) = 2.875 + 8u.
+    So m' = 2.875 + 2^-20 (0x40380004).  Two plausible other orders give other values, so the example
+    tells them apart: the exact value rounded once is 2.875 + 10u (0x40380005), and m + alpha*(amax - m)
+    with each step rounded is 2.875 + 12u (0x40380006)."""
+    h = oracle.AmaxHistory(2, oracle.E4M3, algo=oracle.EMA, alpha=0.625)
+    m0 = np.float32(1 + 13 * 2.0 ** -23)
+    a1 = np.float32(4 + 8 * 2.0 ** -23)
+    assert h.update(m0) == np.float32(1.0)  # warm-up: the first update sets m and keeps the scale
+    assert h.history[0].view(np.uint32) == m0.view(np.uint32)
+    s = h.update(a1)
+    assert int(h.history[0].view(np.uint32)) == 0x40380004
+    assert float(h.history[0]) == 2.875 + 2.0 ** -20
+    # the window (warm-up length 2) is full, so the scale follows from m: RN(448 / m), an IEEE fp32 division
+    assert s.view(np.uint32) == (np.float32(448.0) / np.float32(2.875 + 2.0 ** -20)).view(np.uint32)
+
+
 @pytest.mark.parametrize("alpha", [0.01, 0.1, 0.5, 0.9])
 def test_ema_stays_inside_the_seen_range(alpha):
     seq = _amax_sequence(4, 200)
