@@ -103,7 +103,9 @@ int fp8_quantize_per_tensor_fused_noalloc(const void* x, int dtype, int64_t n, i
     if (n > 0 && (x == nullptr || q == nullptr)) return FP8_ERR_NULL;
     if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale_out, 4) || !aligned(amax_out, 4)) return FP8_ERR_ALIGN;
     if (n == 0) return fp8_quantize_per_tensor(x, dtype, n, fmt, nullptr, q, scale_out, amax_out, stream);
-    if (!fp8q::tensor_fused_fits(x, dtype, n, fmt)) return FP8_ERR_TOO_LARGE;
+    const int fit = fp8q::tensor_fused_fit(x, dtype, n, fmt);
+    if (fit < 0) return FP8_ERR_CUDA;  // the capacity cannot be known on this device
+    if (fit == 0) return FP8_ERR_TOO_LARGE;
     return status_of(fp8q::launch_tensor_fused_noalloc(x, dtype, n, fmt, q, scale_out, amax_out,
                                                        static_cast<cudaStream_t>(stream)));
 }

@@ -65,12 +65,13 @@ unsigned int* device_status_word();
 cudaError_t launch_tensor_fused(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
                                 float* amax_out, void* workspace, cudaStream_t stream, bool* launched);
 
-// Whether x (n elements) is small enough for the one-pass kernel.
-bool tensor_fused_fits(const void* x, int dtype, int64_t n, int fmt);
+// Whether x (n elements) is small enough for the one-pass kernel: 1 yes, 0 no,
+// -1 unknown (a CUDA query failed, or the device has no cooperative launch).
+int tensor_fused_fit(const void* x, int dtype, int64_t n, int fmt);
 
 // The one-pass kernel with its workspace in a fixed array of this module's
 // device memory instead of caller memory (see quant_tensor_fused.cu).  The
-// caller has checked tensor_fused_fits first.
+// caller has checked tensor_fused_fit first.
 cudaError_t launch_tensor_fused_noalloc(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,
                                         float* amax_out, cudaStream_t stream);
 

@@ -137,14 +137,16 @@ k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nve
 
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
-// Largest grid that can be co-resident, or 0 when cooperative launch is unavailable.
+// Largest grid that can be co-resident, or -1 when it cannot be known: a failed
+// CUDA query, or a device without cooperative launch.
 template <typename Kernel>
 int64_t resident_ctas(Kernel k) {
-    int dev = 0, coop = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, 0) != cudaSuccess) return 0;
-    return static_cast<int64_t>(per_sm) * device_sm_count();
+    int dev = 0, coop = 0, per_sm = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return -1;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return -1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, 0) != cudaSuccess) return -1;
+    return static_cast<int64_t>(per_sm) * sms;
 }
 
 template <typename T, int FMT, int BYTES>
@@ -157,7 +159,8 @@ cudaError_t fused_typed(const void* x, int64_t n, uint8_t* q, float* scale_out, 
     const int64_t per_cta = static_cast<int64_t>(kThreads) * kLoads;
     const int64_t grid = std::max<int64_t>(1, (nvec + per_cta - 1) / per_cta);
     *launched = false;
-    if (grid > resident_ctas(kern)) return cudaSuccess;  // too large for one pass: caller falls back
+    const int64_t resident = resident_ctas(kern);
+    if (resident < 0 || grid > resident) return cudaSuccess;  // unknown or too large for one pass: caller falls back
     const typename V::In* xv = static_cast<const typename V::In*>(x);
     const T* tail = static_cast<const T*>(x) + nvec * V::kElems;
     typename V::Out* qv = reinterpret_cast<typename V::Out*>(q);
@@ -181,12 +184,15 @@ cudaError_t fused_width(const void* x, int64_t n, uint8_t* q, float* scale_out, 
     return fused_typed<T, FMT, 16>(x, n, q, scale_out, amax_out, ws, st, launched);
 }
 
+// 1: n elements fit one pass; 0: they do not; -1: the co-resident grid cannot be known.
 template <typename T, int FMT, int BYTES>
-bool fused_fits_typed(int64_t n) {
+int fused_fit_typed(int64_t n) {
     using V = LaneVec<T, BYTES>;
     const int64_t per_cta = static_cast<int64_t>(kThreads) * kLoads;
     const int64_t grid = std::max<int64_t>(1, (n / V::kElems + per_cta - 1) / per_cta);
-    return grid <= resident_ctas(k_tensor_fused<T, FMT, BYTES>);
+    const int64_t resident = resident_ctas(k_tensor_fused<T, FMT, BYTES>);
+    if (resident < 0) return -1;
+    return grid <= resident ? 1 : 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -202,7 +208,9 @@ static_assert(sizeof(Workspace) <= kNoAllocScratchBytes, "the workspace must fit
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch for the current device (looked up on
-// the first call on that device), or nullptr if the lookup failed.
+// the first call on that device and cached for the life of the process), or
+// nullptr if the lookup failed.  The cache does not survive cudaDeviceReset:
+// after a reset the module is loaded again and the array may move.
 void* noalloc_scratch_address() {
     static std::atomic<void*> cache[128];
     int dev = 0;
@@ -217,14 +225,14 @@ void* noalloc_scratch_address() {
 
 }  // namespace
 
-bool tensor_fused_fits(const void* x, int dtype, int64_t n, int fmt) {
+int tensor_fused_fit(const void* x, int dtype, int64_t n, int fmt) {
     const bool w32 = aligned32(x);
     if (dtype == 1) {
-        if (fmt == kE4M3) return w32 ? fused_fits_typed<uint16_t, kE4M3, 32>(n) : fused_fits_typed<uint16_t, kE4M3, 16>(n);
-        return w32 ? fused_fits_typed<uint16_t, kE5M2, 32>(n) : fused_fits_typed<uint16_t, kE5M2, 16>(n);
+        if (fmt == kE4M3) return w32 ? fused_fit_typed<uint16_t, kE4M3, 32>(n) : fused_fit_typed<uint16_t, kE4M3, 16>(n);
+        return w32 ? fused_fit_typed<uint16_t, kE5M2, 32>(n) : fused_fit_typed<uint16_t, kE5M2, 16>(n);
     }
-    if (fmt == kE4M3) return w32 ? fused_fits_typed<float, kE4M3, 32>(n) : fused_fits_typed<float, kE4M3, 16>(n);
-    return w32 ? fused_fits_typed<float, kE5M2, 32>(n) : fused_fits_typed<float, kE5M2, 16>(n);
+    if (fmt == kE4M3) return w32 ? fused_fit_typed<float, kE4M3, 32>(n) : fused_fit_typed<float, kE4M3, 16>(n);
+    return w32 ? fused_fit_typed<float, kE5M2, 32>(n) : fused_fit_typed<float, kE5M2, 16>(n);
 }
 
 cudaError_t launch_tensor_fused_noalloc(const void* x, int dtype, int64_t n, int fmt, uint8_t* q, float* scale_out,

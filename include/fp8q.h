@@ -133,18 +133,33 @@ int fp8_quantize_per_tensor_fused(const void *x, int dtype, int64_t n, int fmt,
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on each device looks up that array's device address
  *     (cudaGetSymbolAddress) with the device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached per device for the
+ *     life of the process, so do not call this entry point after
+ *     cudaDeviceReset (the library's device memory may then have moved).
  *   - Every call clears the workspace (cudaMemsetAsync) before its launch.
  *   - All calls share the one array: calls that can overlap on the GPU
  *     (different streams without ordering between them) race and give wrong
  *     results.  Order such calls, or use fp8_quantize_per_tensor_fused with
  *     one workspace per stream.
- *   - Limit: only tensors that fit the one-pass kernel (fp8_quantize_per_
- *     tensor_fused's on-chip capacity, about 8 MiB of bf16 on a B200) are
- *     accepted; larger ones return FP8_ERR_TOO_LARGE with nothing enqueued.
+ *   - Limit: only tensors that fit the one-pass kernel are accepted; larger
+ *     ones return FP8_ERR_TOO_LARGE with nothing enqueued.  The kernel holds
+ *     x in the registers of the CTAs (256 threads, 4 lane vectors each) that
+ *     can be resident at once, so the largest n is
+ *         C * 1024 * E + (E - 1)
+ *     with E the elements per lane vector and C the co-resident CTAs:
+ *       x 32-byte aligned: 32-byte lanes, E = 16 (bf16) or 8 (fp32);
+ *       x only 16-byte aligned: 16-byte lanes, E = 8 (bf16) or 4 (fp32);
+ *       C = CTAs per SM (from the kernel's registers) x SMs.
+ *     On a B200 (148 SMs) as built here: C = 592 for 32-byte lanes (4 per
+ *     SM) and 740 for 16-byte lanes (5 per SM), so n <= 9,699,343 bf16 or
+ *     4,849,671 fp32 at a 32-byte-aligned x (18.5 MiB), and n <= 6,062,087
+ *     bf16 or 3,031,043 fp32 at an x that is only 16-byte aligned
+ *     (11.6 MiB).  The same tensor can therefore be accepted at one address
+ *     and refused at another.
  *     n == 0 writes amax 0 and its scale, as the other per-tensor calls do.
  * Errors: those of fp8_quantize_per_tensor_fused (without the workspace
- * ones), FP8_ERR_TOO_LARGE.
+ * ones); FP8_ERR_TOO_LARGE; FP8_ERR_CUDA also when the capacity cannot be
+ * known (a failed CUDA query, or a device without cooperative launch).
  */
 int fp8_quantize_per_tensor_fused_noalloc(const void *x, int dtype, int64_t n, int fmt,
                                           uint8_t *q, float *scale_out, float *amax_out,
@@ -516,10 +531,20 @@ int fp8_quantize_delayed_step_grouped(const fp8_delayed_tensor *tensors, int cou
 const char *fp8_status_string(int status);
 
 /* ---- Diagnostics (no counterpart on the pages) ---------------------------
- * Kernels that wait (the grid-wide barrier of the one-pass per-tensor kernel)
- * never wait forever: each wait gives up after about a second, the kernel
- * returns, and it records the event in a device status word.  Results of
- * that launch are then incomplete.
+ * Kernels that wait (the grid-wide barrier of the one-pass per-tensor kernel,
+ * the mbarrier waits of the GEMM) never wait forever: each wait gives up after
+ * about a second, the kernel returns, and it records the event in a device
+ * status word.  Results of that launch are then incomplete.
+ *
+ * The status word is the library's one piece of mutable state besides the
+ * no-allocation entry point's scratch array: one word per device, shared by
+ * every stream, thread and caller on it.  It is written only when a wait
+ * gives up, which does not happen in normal operation.  A set bit says that
+ * some launch on this device timed out since the word was last cleared, not
+ * which one; a caller that needs to know which call it was clears the word,
+ * orders that call alone, and reads the word after it.  The word's address
+ * is cached per device, so the library must not be used after
+ * cudaDeviceReset.
  *
  * Device status bits: */
 #define FP8_DEVICE_STATUS_WAIT_TIMEOUT 0x1u

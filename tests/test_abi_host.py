@@ -147,6 +147,24 @@ def test_fused_per_tensor_validation(L):
     assert f(A16, 1, 16, 0, A4, A16, A16, A16, None) == ERR_ALIGN
 
 
+def test_fused_per_tensor_noalloc_validation(L):
+    """The no-allocation entry point rejects bad arguments before it touches CUDA."""
+    f = L.fp8_quantize_per_tensor_fused_noalloc
+    assert f(A16, 1, 16, 9, A16, A16, A16, None) == ERR_FORMAT
+    assert f(A16, 1, 16, -1, A16, A16, A16, None) == ERR_FORMAT
+    assert f(A16, 5, 16, 0, A16, A16, A16, None) == ERR_DTYPE
+    assert f(A16, 1, -1, 0, A16, A16, A16, None) == ERR_SHAPE
+    assert f(A16, 1, 16, 0, A16, None, A16, None) == ERR_NULL   # scale_out
+    assert f(A16, 1, 16, 0, A16, A16, None, None) == ERR_NULL   # amax_out
+    assert f(A16, 1, 0, 0, A16, None, A16, None) == ERR_NULL    # scale_out is written even for n == 0
+    assert f(None, 1, 16, 0, A16, A16, A16, None) == ERR_NULL   # x
+    assert f(A16, 1, 16, 0, None, A16, A16, None) == ERR_NULL   # q
+    assert f(A16 + 8, 1, 16, 0, A16, A16, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, A16 + 4, A16, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, A16, A16 + 2, A16, None) == ERR_ALIGN
+    assert f(A16, 1, 16, 0, A16, A16, A16 + 1, None) == ERR_ALIGN
+
+
 def test_amax_and_scale_validation(L):
     assert L.fp8_amax(A16, 7, 16, A16, None) == ERR_DTYPE
     assert L.fp8_amax(A16, 1, -1, A16, None) == ERR_SHAPE

@@ -6,16 +6,21 @@ without the workspace argument.  It serves code that may not call cudaMalloc
 or a C caller whose device memory all belongs to another framework's
 allocator): its workspace is a fixed array in the library's own device
 memory.  This test calls it through the C ABI twice in a row on each input
-and requires the same bytes as the existing workspace-taking entry point, the
-same bit-exact bar as every other parity test here.  It depends on no state
-left by other tests, so it passes alone in a fresh process or after them.
+and requires the same bytes as the existing workspace-taking entry point and
+as the oracle, the same bit-exact bar as every other parity test here.  It
+also finds the largest size the entry point accepts, for each element type
+and input alignment, and checks it against the limit the header states.  It
+depends on no state left by other tests, so it passes alone in a fresh
+process or after them.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from fine_grained_block_b200 import binding as B
 from fine_grained_block_b200 import inputs
+from parity_util import host_input
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +44,11 @@ def test_no_alloc_matches_workspace_entry_point_two_calls_in_a_row(fmt, dtype):
         # the existing entry point, with a workspace of its own
         q_ref, s_ref, a_ref = B.fp8_quantize_per_tensor_fused(x, fmt, workspace=B.fused_workspace())
         torch.cuda.synchronize()
+        # and the oracle, directly: current scaling over the whole tensor
+        oq, os_, oa = oracle.quantize_per_tensor(host_input(x.cpu()), fmt)
+        assert np.array_equal(_bits(q_ref), oq), n
+        assert np.array_equal(_bits(s_ref), np.array([os_], np.float32).view(np.int32)), n
+        assert np.array_equal(_bits(a_ref), np.array([oa], np.float32).view(np.int32)), n
         for call in range(2):
             q = torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda")
             s = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda")
@@ -64,3 +74,55 @@ def test_no_alloc_rejects_tensors_beyond_its_limit():
                                                  a.data_ptr(), stream)
     assert rc == FP8_ERR_TOO_LARGE
     assert "too large" in B.fp8_status_string(rc)
+
+
+# The limit the header states: n <= C * 1024 * E + (E - 1), E elements per lane vector (16 or 8 for bf16,
+# 8 or 4 for fp32, at a 32- or only 16-byte-aligned x), C co-resident CTAs; on a 148-SM B200, C = 592 with
+# 32-byte lanes and 740 with 16-byte lanes.
+B200_LIMIT = {(torch.bfloat16, 32): 9_699_343, (torch.bfloat16, 16): 6_062_087,
+              (torch.float32, 32): 4_849_671, (torch.float32, 16): 3_031_043}
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_no_alloc_limit_by_alignment(dtype):
+    """The largest accepted n, found by bisection on the return code (a refused call enqueues nothing), is one
+    full lane vector per thread of every co-resident CTA plus a tail; one more element is refused.  An x that
+    is only 16-byte aligned takes 16-byte lanes, so a size just above that limit is refused there and
+    accepted at a 32-byte-aligned address."""
+    L = B.load_library()
+    stream = torch.cuda.current_stream().cuda_stream
+    cap = 1 << 24
+    esz = torch.empty(0, dtype=dtype).element_size()
+    buf = torch.zeros(cap * esz + 64, dtype=torch.uint8, device="cuda")
+    q = torch.empty(cap + 64, dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    a = torch.empty(1, dtype=torch.float32, device="cuda")
+    base = buf.data_ptr()
+    assert base % 256 == 0
+
+    def call(x_ptr, n):
+        return L.fp8_quantize_per_tensor_fused_noalloc(x_ptr, DT[dtype], n, B.E4M3, q.data_ptr(), s.data_ptr(),
+                                                       a.data_ptr(), stream)
+
+    limits = {}
+    for lane, ptr in ((32, base), (16, base + 16)):
+        lo, hi = 1, cap  # call(lo) accepted, call(hi) refused
+        assert call(ptr, lo) == 0 and call(ptr, hi) == FP8_ERR_TOO_LARGE
+        while hi - lo > 1:
+            mid = (lo + hi) // 2
+            rc = call(ptr, mid)
+            assert rc in (0, FP8_ERR_TOO_LARGE), B.fp8_status_string(rc)
+            lo, hi = (mid, hi) if rc == 0 else (lo, mid)
+        torch.cuda.synchronize()
+        limits[lane] = lo
+        elems = lane // esz
+        assert (lo + 1) % elems == 0  # a whole number of lane vectors plus a tail of elems - 1
+        assert ((lo + 1) // elems) % 1024 == 0  # 1024 lane vectors per CTA
+    assert limits[32] > limits[16]
+    # just above the 16-byte-lane limit: refused at base + 16, accepted at the 32-byte-aligned base
+    n = limits[16] + 1
+    assert call(base + 16, n) == FP8_ERR_TOO_LARGE
+    assert call(base, n) == 0
+    torch.cuda.synchronize()
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert limits[32] == B200_LIMIT[(dtype, 32)] and limits[16] == B200_LIMIT[(dtype, 16)], limits
