@@ -2,26 +2,31 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step is one pass of the hot path over one batch: the bf16 weight
-4096x4096 (N(0, 0.02^2), seed 1 + rank) quantized to E4M3 with one scale per
-128x128 block (amax, scale, saturating cast, code and scale stores) and
-dequantized back to bf16 -- two library launches through the C ABI.  W
-untimed steps, then exactly K steps between barriers and device syncs, timed
+One step is one pass of the hot path over one batch: a bf16 tensor of 2^30
+elements shaped [262144, 4096] (randn with 0.1% of the entries scaled by 1e3,
+seed 4 + rank, drawn on the host so that rank 0's tensor is the one the
+full-size parity tests compare) quantized to E4M3 with one scale per 1x128
+block in a single fused pass (amax, scale, saturating cast, code and scale
+stores) and dequantized back to bf16 -- two library launches through the C ABI.
+W untimed steps, then exactly K steps between barriers and device syncs, timed
 with CUDA events on the launching stream; the max over ranks is reported.
-The K timed steps are captured into CUDA graphs (launch-bound: each kernel
-moves 48 MiB in under 10 us) and timed with events around the whole region;
-a separate instrumented replay gives the split between the two kernels.
-The 32 MiB weight fits in L2, so the steps rotate over enough buffer sets that
-every step reads data last touched more than an L2's worth of traffic ago.
+Each kernel moves about 3.25 GB in roughly half a millisecond, so the steps
+are launched eagerly with an event after every launch: the events give each
+kernel's own duration for the roofline, and their cost (the lost overlap of
+one kernel's tail with the next one's start) is inside the timed region.
+The inputs (2 GiB in, 1 GiB of codes, 2 GiB out) are far larger than the
+126 MB L2, so no flush is needed.
 
 Prints one JSON line (rank 0).  Besides the headline it carries the roofline
-of the dominant kernel, the per-mode breakdown (1x128, 128x128, per-tensor
-current and delayed with the history update, dequant) on the other workload
-shapes, the end-to-end figure with host buffers, the CPU oracle as a baseline,
-SM clocks sampled during the timed region, and the number of library launches.
+of each of the two kernels, the per-mode breakdown (1x128, 128x128, MX,
+per-tensor current and delayed with the history update, the transposing
+casts, dequant, the size sweep, the consumer GEMM) on the other workload
+shapes, the end-to-end figure with host buffers, the CPU oracle as a
+baseline, SM clocks sampled during the timed region, and the number of
+library launches.
 
 --impl reference times the CPU oracle (the plain C reference) on the same
-workload and metric, on a bounded sample per step; rank 0 only.
+workload and metric, on a bounded sample of rows per step; rank 0 only.
 """
 from __future__ import annotations
 
@@ -43,9 +48,11 @@ if ROOT not in sys.path:
 METRIC = "quantize GB/s (in+out bytes) and % of B200 HBM roofline per scaling mode"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
-WORKLOAD = "bf16 weight 4096x4096 N(0,0.02^2); E4M3 128x128 block quantize (1024 fp32 scales) + dequant round trip to bf16"
-ROWS = COLS = 4096
-BLOCK = (128, 128)
+LOG2_N = 30
+ROWS, COLS = (1 << LOG2_N) // 4096, 4096
+BLOCK = (1, 128)
+WORKLOAD = ("bf16 tensor of 2^30 elements as [262144, 4096], randn with 0.1% of entries x1e3 (seed 4 + rank); E4M3 "
+            "1x128 block quantize in one fused pass (262144x32 fp32 scales) + dequant to bf16")
 L2_BYTES = 126 * 1024 * 1024
 GRAPH_CHUNK = 1000
 
@@ -77,7 +84,7 @@ def max_over_ranks(values, world: int, device="cuda"):
     return t.tolist()
 
 
-def step_bytes(rows=ROWS, cols=COLS, br=128, bc=128):
+def step_bytes(rows=ROWS, cols=COLS, br=BLOCK[0], bc=BLOCK[1]):
     """Algorithmic bytes of one step: quantize (read bf16, write codes + scales) + dequant (read codes +
     scales, write bf16)."""
     n = rows * cols
@@ -155,10 +162,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------
 
 KERNEL_SOURCES = {
-    "k_quant_128x128": ["fine_grained_block_b200/csrc/quant_block.cu", "fine_grained_block_b200/csrc/fp8q_device.cuh",
-                        "fine_grained_block_b200/csrc/lane_vec.cuh"],
-    "k_dequant_128x128": ["fine_grained_block_b200/csrc/dequant.cu", "fine_grained_block_b200/csrc/fp8q_device.cuh",
+    "k_quant_rowblocks": ["fine_grained_block_b200/csrc/quant_block.cu", "fine_grained_block_b200/csrc/fp8q_device.cuh",
                           "fine_grained_block_b200/csrc/lane_vec.cuh"],
+    "k_dequant_flat": ["fine_grained_block_b200/csrc/dequant.cu", "fine_grained_block_b200/csrc/dequant_math.cuh",
+                       "fine_grained_block_b200/csrc/fp8q_device.cuh", "fine_grained_block_b200/csrc/lane_vec.cuh"],
 }
 
 
@@ -171,7 +178,8 @@ def source_hash(kernel: str) -> str:
 
 
 def committed_traffic(kernel: str):
-    """dram bytes per launch from profiles/traffic_<kernel>.txt if its source hash still matches."""
+    """DRAM bytes (read + written) per launch from profiles/traffic_<kernel>.txt, or None once the kernel's
+    sources no longer hash to the figure recorded there."""
     path = os.path.join(ROOT, "profiles", f"traffic_{kernel}.txt")
     try:
         kv = {}
@@ -192,24 +200,25 @@ def committed_traffic(kernel: str):
 # ---------------------------------------------------------------------------------
 
 def oracle_step_seconds(x_rows_bits, reps: int):
+    """reps x (1x128 E4M3 quantize + bf16 dequant) of the given rows with the single-threaded C oracle."""
     import oracle
     t0 = time.perf_counter()
     for _ in range(reps):
-        q, s = oracle.quantize_blockwise(x_rows_bits, 128, 128, oracle.E4M3)
-        oracle.dequantize(q, oracle.E4M3, s, 128, 128, out_dtype=oracle.BF16)
+        q, s = oracle.quantize_blockwise(x_rows_bits, *BLOCK, oracle.E4M3)
+        oracle.dequantize(q, oracle.E4M3, s, *BLOCK, out_dtype=oracle.BF16)
     return time.perf_counter() - t0
 
 
 def oracle_step_seconds_threaded(x_rows_bits, reps: int, threads: int):
-    """The same oracle calls, split over 128-row slices (whole 128x128 blocks) on `threads` threads; the
-    oracle is C behind ctypes, which releases the GIL, so the slices run in parallel."""
+    """The same oracle calls, split over 128-row slices (whole blocks) on `threads` threads; the oracle is C
+    behind ctypes, which releases the GIL, so the slices run in parallel."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     slices = [x_rows_bits[r:r + 128] for r in range(0, x_rows_bits.shape[0], 128)]
 
     def one(xs):
-        q, s = oracle.quantize_blockwise(xs, 128, 128, oracle.E4M3)
-        oracle.dequantize(q, oracle.E4M3, s, 128, 128, out_dtype=oracle.BF16)
+        q, s = oracle.quantize_blockwise(xs, *BLOCK, oracle.E4M3)
+        oracle.dequantize(q, oracle.E4M3, s, *BLOCK, out_dtype=oracle.BF16)
 
     with ThreadPoolExecutor(max_workers=threads) as pool:
         t0 = time.perf_counter()
@@ -218,35 +227,32 @@ def oracle_step_seconds_threaded(x_rows_bits, reps: int, threads: int):
         return time.perf_counter() - t0
 
 
-def cpu_baseline_all_cores(budget_s: float = 8.0):
+def cpu_baseline_all_cores(bits, budget_s: float = 8.0):
     """The oracle over all host cores (128-row slices in parallel), next to the single-thread figure."""
-    from fine_grained_block_b200 import inputs
     threads = max(1, len(os.sched_getaffinity(0)))
-    bits = inputs.bf16_bits(inputs.weight_4096(seed=1))
-    t1 = oracle_step_seconds_threaded(bits, 1, threads)
+    rows = 16384
+    xs = bits[:rows]
+    t1 = oracle_step_seconds_threaded(xs, 1, threads)
     reps = max(1, int(budget_s / max(t1, 1e-3)))
-    t = oracle_step_seconds_threaded(bits, reps, threads)
-    qb, db = step_bytes(ROWS, COLS)
+    t = oracle_step_seconds_threaded(xs, reps, threads)
+    qb, db = step_bytes(rows, COLS)
     return {"value": (qb + db) * reps / t / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"the whole seed-1 4096x4096 weight: 128x128 E4M3 quantize + bf16 dequant, the C oracle on "
-                      f"32 slices of 128 rows over {threads} threads, {reps} reps, {t:.1f} s"}
+            "sample": f"rows 0-{rows - 1} of the headline tensor (1/16 of it): 1x128 E4M3 quantize + bf16 dequant, "
+                      f"the C oracle on {rows // 128} slices of 128 rows over {threads} threads, {reps} reps, "
+                      f"{t:.1f} s"}
 
 
-def cpu_baseline(budget_s: float = 12.0):
-    import torch
-    from fine_grained_block_b200 import inputs
-    w = inputs.weight_4096(seed=1)
-    bits = inputs.bf16_bits(w)
-    sample_rows = 1024
+def cpu_baseline(bits, budget_s: float = 12.0):
+    sample_rows = 512
     xs = bits[:sample_rows].copy()
-    oracle_step_seconds(xs[:128], 1)  # build + load outside the timing
+    oracle_step_seconds(xs[:1], 1)  # build + load outside the timing
     t1 = oracle_step_seconds(xs, 1)
     reps = max(1, int(budget_s / max(t1, 1e-3)))
     t = oracle_step_seconds(xs, reps)
     qb, db = step_bytes(sample_rows, COLS)
     return {"value": (qb + db) * reps / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"rows 0-{sample_rows - 1} of the seed-1 4096x4096 weight (1/4 of it): 128x128 E4M3 "
-                      f"quantize + bf16 dequant, single-threaded C oracle, {reps} reps, {t:.1f} s"}
+            "sample": f"rows 0-{sample_rows - 1} of the headline tensor (1/512 of it): 1x128 E4M3 quantize + bf16 "
+                      f"dequant, single-threaded C oracle, {reps} reps, {t:.1f} s"}
 
 
 def run_reference(args):
@@ -255,30 +261,30 @@ def run_reference(args):
         return 0
     import oracle  # noqa: F401  (built on first use)
     from fine_grained_block_b200 import inputs
-    w = inputs.weight_4096(seed=1)
-    bits = inputs.bf16_bits(w)
+    bits = inputs.bf16_bits(inputs.sweep_tensor(LOG2_N, seed=4))
     # size each step's sample so that warm-up + K steps take about --ref-budget-s seconds (a minute by default)
-    probe = bits[:128, :1024].copy()
+    probe = bits[:4].copy()
     oracle_step_seconds(probe, 1)
     t_probe = oracle_step_seconds(probe, 2) / 2
-    per_elem = t_probe / probe.size
+    per_row = t_probe / probe.shape[0]
     budget = args.ref_budget_s / max(1, args.steps + args.warmup)
-    cols = int(max(128, min(COLS, (budget / per_elem / 128) // 128 * 128)))
-    sample = bits[:128, :cols].copy()
+    rows = int(max(1, min(ROWS, budget / per_row)))
+    sample = bits[:rows].copy()
     for _ in range(args.warmup):
         oracle_step_seconds(sample, 1)
     times = [oracle_step_seconds(sample, 1) for _ in range(args.steps)]
     total = sum(times)
-    qb, db = step_bytes(128, cols)
+    qb, db = step_bytes(rows, COLS)
     value = (qb + db) * args.steps / total / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_per_step": f"rows 0-127, cols 0-{cols - 1} (whole 128x128 tiles)",
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "block": list(BLOCK), "fmt": "e4m3",
+                   "sample_per_step": f"rows 0-{rows - 1} of the seed-4 tensor (whole 1x128 blocks)",
                    "parallelism": "rank 0 only (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"128x{cols} slice of the weight per step, single-threaded C oracle"},
+                         "sample": f"{rows}x{COLS} rows of the tensor per step, single-threaded C oracle"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -292,9 +298,9 @@ def run_reference(args):
 class Raw:
     """Direct C-ABI calls with precomputed arguments (the binding's marshalling, done once)."""
 
-    def __init__(self, stream):
+    def __init__(self, stream, lib_path=None):
         from fine_grained_block_b200 import binding
-        self.L = binding.load_library()
+        self.L = binding.load_library(lib_path)
         self.stream = stream.cuda_stream
         self.binding = binding
 
@@ -623,6 +629,21 @@ def modes_breakdown(dev, stream, peak):
             ao_.data_ptr(), st), "per-tensor")], reps, dev)
         row["per_tensor_current_e5m2"] = round(3 * n / (t * 1e-3) / 1e9, 1)
         t = time_in_graph([lambda r, st: raw.check(L.fp8_dequantize(
+            qs_[r % copies].data_ptr(), 1, R, C, 0, 0, so_.data_ptr(), ys_[r % copies].data_ptr(), 1, st),
+            "dequant")], reps, dev)
+        row["per_tensor_dequant_bf16"] = round(3 * n / (t * 1e-3) / 1e9, 1)
+        if R >= 128:
+            for c_ in range(copies):  # every set's 128x128 codes and scales, untimed
+                raw.check(L.fp8_quantize_blockwise(xs_[c_].data_ptr(), 1, R, C, 128, 128, 0, qs_[c_].data_ptr(),
+                                                   st_[c_].data_ptr(), raw.stream), "128x128")
+            t = time_in_graph([lambda r, st: raw.check(L.fp8_dequantize(
+                qs_[r % copies].data_ptr(), 0, R, C, 128, 128, st_[r % copies].data_ptr(),
+                ys_[r % copies].data_ptr(), 1, st), "dequant")], reps, dev)
+            row["128x128_dequant_bf16"] = round((3 * n + 4 * (n // 16384)) / (t * 1e-3) / 1e9, 1)
+        for c_ in range(copies):
+            raw.check(L.fp8_quantize_blockwise(xs_[c_].data_ptr(), 1, R, C, 1, 128, 0, qs_[c_].data_ptr(),
+                                               ss_[c_].data_ptr(), raw.stream), "1x128")
+        t = time_in_graph([lambda r, st: raw.check(L.fp8_dequantize(
             qs_[r % copies].data_ptr(), 0, R, C, 1, 128, ss_[r % copies].data_ptr(), ys_[r % copies].data_ptr(), 1, st),
             "dequant")], reps, dev)
         row["1x128_dequant_bf16"] = round((3 * n + 4 * (n // 128)) / (t * 1e-3) / 1e9, 1)
@@ -655,10 +676,74 @@ def modes_breakdown(dev, stream, peak):
         put(f"per_tensor_current_e4m3_{key}_two_pass", label + " (single call after an L2 flush)", (esz + 1) * nn, t2)
         put(f"per_tensor_current_e4m3_{key}_one_pass", label + " (single call after an L2 flush; cooperative "
             "one-pass kernel)", (esz + 1) * nn, t1)
+        if key == "fp32_1MiB":
+            # the handbook's experiment tensor in 1x128 blocks as well: quantize, then dequant back to fp32
+            R1, C1 = x_small.shape
+            sb_ = torch.empty(R1, C1 // 128, dtype=torch.float32, device=dev)
+            yf_ = torch.empty(R1, C1, dtype=torch.float32, device=dev)
+            bq = lambda r: raw.check(L.fp8_quantize_blockwise(x_small.data_ptr(), 0, R1, C1, 1, 128, 0,
+                                                              qs_.data_ptr(), sb_.data_ptr(), st), "1x128")
+            bd = lambda r: raw.check(L.fp8_dequantize(qs_.data_ptr(), 0, R1, C1, 1, 128, sb_.data_ptr(),
+                                                      yf_.data_ptr(), 0, st), "dequant")
+            tbq, tbd = time_per_launch([bq, bd], 30, 5, stream, lambda: flush_buf.fill_(1))
+            nb1 = (esz + 1) * nn + 4 * (nn // 128)
+            put("1x128_e4m3_fp32_1MiB", label + " (single call after an L2 flush)", nb1, tbq)
+            put("1x128_dequant_fp32_1MiB", label + " (single call after an L2 flush)", nb1, tbd)
+            del sb_, yf_
         del x_small, qs_
     del flush_buf
     out["note"] = ("large modes: back-to-back launches replayed from a CUDA graph, events around the replay; "
                    "frac is of the peak above")
+    return out
+
+
+def weight_roundtrip(dev, raw, peak, steps_list=(20, 2000)):
+    """The bf16 4096x4096 weight (N(0, 0.02^2), seed 1): 128x128 E4M3 quantize + bf16 dequant per step.
+
+    The 32 MiB weight fits in L2, so the steps rotate over enough buffer sets (x, codes, scales, output)
+    that every step reads data last touched more than an L2's worth of traffic ago.  Each kernel moves
+    48 MiB in under 10 us, so K steps are captured into one CUDA graph and timed with events around its
+    replay.  Timed at several K: the replay's fixed cost (the graph launch before the first kernel and the
+    drain after the last) is amortized over K, so K = 20 reads slower per step than K = 2000; the fit
+    t(K) = t0 + K * t_step separates the two."""
+    import torch
+    from fine_grained_block_b200 import inputs
+    L = raw.L
+    R = C = 4096
+    n = R * C
+    qb = 3 * n + 4 * (n // 16384)
+    per_set = n * (2 + 1 + 2) + 4 * 1024
+    nsets = max(2, math.ceil(3 * L2_BYTES / per_set))
+    w0 = inputs.weight_4096(seed=1).to(dev)
+    xs = [w0] + [w0.clone() for _ in range(nsets - 1)]
+    qs = [torch.empty(R, C, dtype=torch.uint8, device=dev) for _ in range(nsets)]
+    ss = [torch.empty(R // 128, C // 128, dtype=torch.float32, device=dev) for _ in range(nsets)]
+    ys = [torch.empty(R, C, dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+
+    def fq(r, st):
+        i = r % nsets
+        raw.check(L.fp8_quantize_blockwise(xs[i].data_ptr(), 1, R, C, 128, 128, 0, qs[i].data_ptr(),
+                                           ss[i].data_ptr(), st), "128x128")
+
+    def fd(r, st):
+        i = r % nsets
+        raw.check(L.fp8_dequantize(qs[i].data_ptr(), 0, R, C, 128, 128, ss[i].data_ptr(), ys[i].data_ptr(), 1, st),
+                  "dequant")
+
+    out = {"workload": "bf16 weight 4096x4096 N(0,0.02^2), seed 1: 128x128 E4M3 quantize + bf16 dequant per step "
+                       f"({nsets} rotating buffer sets, {nsets * per_set >> 20} MiB)", "by_steps": {}}
+    fit = []
+    for K in steps_list:
+        ms = time_in_graph([fq, fd], K, dev) * K
+        fit.append((K, ms))
+        out["by_steps"][str(K)] = {"us_per_step": round(ms / K * 1e3, 3),
+                                   "GB_s": round(2 * qb * K / (ms * 1e-3) / 1e9, 1),
+                                   "frac_of_peak": round(2 * qb * K / (ms * 1e-3) / 1e9 / peak, 4)}
+    (k0, m0), (k1, m1) = fit[0], fit[-1]
+    t_step = (m1 - m0) / (k1 - k0)
+    out["fit"] = {"us_per_step": round(t_step * 1e3, 3), "fixed_us_per_replay": round((m0 - k0 * t_step) * 1e3, 2),
+                  "GB_s_per_step": round(2 * qb / (t_step * 1e-3) / 1e9, 1)}
+    del xs, qs, ss, ys
     return out
 
 
@@ -683,154 +768,97 @@ def run_ours(args):
     L, st = raw.L, raw.stream
     peak, peak_kind = measured_peaks()
 
-    # rotating buffer sets so that no step finds its input in L2
+    # the headline tensor, drawn on the host (rank 0's is the tensor the 2^30 parity test compares)
+    x_cpu = inputs.sweep_tensor(LOG2_N, seed=4 + rank)
+    assert tuple(x_cpu.shape) == (ROWS, COLS)
     qb, db = step_bytes()
-    per_set = ROWS * COLS * (2 + 1 + 2) + 4 * 1024
-    nsets = max(2, math.ceil(3 * L2_BYTES / per_set))
-    w0 = inputs.weight_4096(seed=1 + rank).to(dev)
-    xs = [w0] + [w0.clone() for _ in range(nsets - 1)]
-    qs = [torch.empty(ROWS, COLS, dtype=torch.uint8, device=dev) for _ in range(nsets)]
-    ss = [torch.empty(ROWS // 128, COLS // 128, dtype=torch.float32, device=dev) for _ in range(nsets)]
-    ys = [torch.empty(ROWS, COLS, dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
-    xp = [t.data_ptr() for t in xs]
-    qp = [t.data_ptr() for t in qs]
-    sp = [t.data_ptr() for t in ss]
-    yp = [t.data_ptr() for t in ys]
-    quant = L.fp8_quantize_blockwise
-    deq = L.fp8_dequantize
+    x = x_cpu.to(dev)
+    q = torch.empty(ROWS, COLS, dtype=torch.uint8, device=dev)
+    s = torch.empty(ROWS, COLS // 128, dtype=torch.float32, device=dev)
+    y = torch.empty(ROWS, COLS, dtype=torch.bfloat16, device=dev)
+    quant, deq = L.fp8_quantize_blockwise, L.fp8_dequantize
 
-    def fq(r, stream_handle):
-        i = r % nsets
-        raw.check(quant(xp[i], 1, ROWS, COLS, 128, 128, 0, qp[i], sp[i], stream_handle), "quantize")
+    def fq(bufs, stream_handle):
+        xb, qb_, sb, _ = bufs
+        raw.check(quant(xb.data_ptr(), 1, ROWS, COLS, *BLOCK, 0, qb_.data_ptr(), sb.data_ptr(), stream_handle),
+                  "quantize")
 
-    def fd(r, stream_handle):
-        i = r % nsets
-        raw.check(deq(qp[i], 0, ROWS, COLS, 128, 128, sp[i], yp[i], 1, stream_handle), "dequantize")
+    def fd(bufs, stream_handle):
+        _, qb_, sb, yb = bufs
+        raw.check(deq(qb_.data_ptr(), 0, ROWS, COLS, *BLOCK, sb.data_ptr(), yb.data_ptr(), 1, stream_handle),
+                  "dequantize")
 
-    for r in range(args.warmup):
-        fq(r, st)
-        fd(r, st)
+    main_set = (x, q, s, y)
+    for _ in range(args.warmup):
+        fq(main_set, st)
+        fd(main_set, st)
     torch.cuda.synchronize()
 
-    # The timed steps are captured into CUDA graphs (chunks of <= GRAPH_CHUNK steps) so that host launch
-    # latency does not sit between the kernels.  The timed replay has timing events only around the whole
-    # region: an event node between two kernels serializes them and costs several microseconds per step.
-    def capture(first_step, m, with_events):
-        g = torch.cuda.CUDAGraph()
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(m)] \
-            if with_events else None
-        with torch.cuda.graph(g, stream=cap_stream):
-            cs = torch.cuda.current_stream().cuda_stream
-            for k in range(m):
-                r = first_step + k
-                if with_events:
-                    evs[k][0].record()
-                fq(r, cs)
-                if with_events:
-                    evs[k][1].record()
-                fd(r, cs)
-                if with_events:
-                    evs[k][2].record()
-        return g, evs
-
-    cap_stream = torch.cuda.Stream(dev)
-    chunks = []
-    done = 0
-    while done < args.steps:
-        m = min(GRAPH_CHUNK, args.steps - done)
-        chunks.append(capture(args.warmup + done, m, False)[0])
-        done += m
-    for g in chunks:  # untimed warm replay (graph upload)
-        g.replay()
-    torch.cuda.synchronize()
-    begin, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # The timed region: K steps launched eagerly, an event after every launch.  Each launch runs about
+    # half a millisecond, so the host stays ahead of the device and the queue never drains.
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps + 1)]
     clocks = ClockSampler(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    begin.record(stream)
-    for g in chunks:
-        g.replay()
-    end.record(stream)
+    evs[0].record(stream)
+    for k in range(args.steps):
+        fq(main_set, st)
+        evs[2 * k + 1].record(stream)
+        fd(main_set, st)
+        evs[2 * k + 2].record(stream)
     torch.cuda.synchronize()
     clocks.stop()
     if world > 1:
         dist.barrier()
-    total_ms = begin.elapsed_time(end)
-    del chunks
-
-    # Per-kernel split, from a separate replay with an event before and after every launch (not the
-    # timed region; the events between launches inflate both durations).
-    split_steps = min(args.steps, 200)
-    g_split, evs = capture(args.warmup, split_steps, True)
-    g_split.replay()
-    torch.cuda.synchronize()
-    g_split.replay()
-    torch.cuda.synchronize()
-    tq = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
-    td = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
-    del g_split
-
-    # Single steps, timed one by one: 10 warm-up and 50 timed replays of a one-step graph, each after a
-    # 512 MiB write that flushes L2 (outside the events), median and best.  Each rep also carries the graph
-    # launch and a cold start, so these read lower than the steady-state timed region above.
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    g_one, _ = capture(args.warmup, 1, False)
-    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    rep_ms = []
-    for r in range(10 + 50):
-        flush.zero_()
-        e_a.record(stream)
-        g_one.replay()
-        e_b.record(stream)
-        torch.cuda.synchronize()
-        if r >= 10:
-            rep_ms.append(e_a.elapsed_time(e_b))
-    del g_one, flush
-    rep_med, rep_best = statistics.median(rep_ms), min(rep_ms)
-    rep_med, rep_best = max_over_ranks([rep_med, rep_best], world, device=dev)
-    total_ms, tq, td = max_over_ranks([total_ms, tq, td], world, device=dev)
+    total_ms = evs[0].elapsed_time(evs[-1])
+    tq = [evs[2 * k].elapsed_time(evs[2 * k + 1]) for k in range(args.steps)]
+    td = [evs[2 * k + 1].elapsed_time(evs[2 * k + 2]) for k in range(args.steps)]
+    tq_mean, td_mean = statistics.fmean(tq), statistics.fmean(td)
+    stats = [total_ms, tq_mean, td_mean, statistics.median(tq), min(tq), statistics.median(td), min(td)]
+    total_ms, tq_mean, td_mean, tq_med, tq_best, td_med, td_best = max_over_ranks(stats, world, device=dev)
     value = (qb + db) * args.steps * world / (total_ms * 1e-3) / 1e9
 
-    # end to end through the same C ABI with host buffers: H2D of the input from pinned memory, both
-    # kernels, D2H of codes, scales and the dequantized tensor, every step
-    hx = w0.cpu().pin_memory()
+    # End to end through the same C ABI with host buffers: every step uploads its input from pinned host
+    # memory, runs both kernels and downloads codes, scales and the dequantized tensor.  Upload, compute
+    # and download run on three streams over two device buffer sets, ordered by events per set, so step
+    # r's download (device -> host) overlaps step r+1's upload (host -> device).
+    hx = x_cpu.pin_memory()
     hq = torch.empty(ROWS, COLS, dtype=torch.uint8).pin_memory()
-    hs = torch.empty(ROWS // 128, COLS // 128, dtype=torch.float32).pin_memory()
+    hs = torch.empty(ROWS, COLS // 128, dtype=torch.float32).pin_memory()
     hy = torch.empty(ROWS, COLS, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
-    # Upload, compute and download run on three streams, ordered by events per buffer set: step r's
-    # download (device -> host) overlaps step r+1's upload (host -> device), the two directions of the
-    # link.  Every step still copies its whole input in and its whole result out.
+    sets = [main_set, (torch.empty_like(x), torch.empty_like(q), torch.empty_like(s), torch.empty_like(y))]
+    e2e_steps = max(3, min(args.steps, 10))
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(nsets)]
-    ev_comp = [torch.cuda.Event() for _ in range(nsets)]
-    ev_out = [torch.cuda.Event() for _ in range(nsets)]
-    used = [False] * nsets
+    ev_in = [torch.cuda.Event() for _ in sets]
+    ev_comp = [torch.cuda.Event() for _ in sets]
+    ev_out = [torch.cuda.Event() for _ in sets]
+    used = [False] * len(sets)
 
     def e2e_step(r):
-        i = r % nsets
+        i = r % len(sets)
+        xb, qb_, sb, yb = sets[i]
         with torch.cuda.stream(s_in):
             if used[i]:
-                s_in.wait_event(ev_comp[i])  # the previous use of xs[i] has been read
-            xs[i].copy_(hx, non_blocking=True)
+                s_in.wait_event(ev_comp[i])  # the previous use of this input buffer has been read
+            xb.copy_(hx, non_blocking=True)
             ev_in[i].record(s_in)
         stream.wait_event(ev_in[i])
         if used[i]:
-            stream.wait_event(ev_out[i])  # the previous results in set i have been downloaded
-        fq(r, st)
-        fd(r, st)
+            stream.wait_event(ev_out[i])  # the previous results in this set have been downloaded
+        fq(sets[i], st)
+        fd(sets[i], st)
         ev_comp[i].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp[i])
-            hq.copy_(qs[i], non_blocking=True)
-            hs.copy_(ss[i], non_blocking=True)
-            hy.copy_(ys[i], non_blocking=True)
+            hq.copy_(qb_, non_blocking=True)
+            hs.copy_(sb, non_blocking=True)
+            hy.copy_(yb, non_blocking=True)
             ev_out[i].record(s_out)
         used[i] = True
 
-    for r in range(3):
+    for r in range(2):
         e2e_step(r)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -844,52 +872,47 @@ def run_ours(args):
     torch.cuda.synchronize()
     (te,) = max_over_ranks([e0.elapsed_time(e1)], world, device=dev)
     e2e_value = (qb + db) * e2e_steps * world / (te * 1e-3) / 1e9
+    del sets, main_set, x, q, s, y, hq, hs, hy
+    torch.cuda.empty_cache()
 
     line = None
     if rank == 0:
-        # Both kernels move the same algorithmic bytes per launch (qb == db), so the roofline uses the
-        # average launch duration over the timed region's 2K launches.
-        per_launch_ms = total_ms / (2 * args.steps)
-        achieved = qb / (per_launch_ms * 1e-3) / 1e9
-        traffic = committed_traffic("k_quant_128x128")
+        def roofline(name, nbytes, ms_mean, ms_med, ms_best, share):
+            achieved = nbytes / (ms_mean * 1e-3) / 1e9
+            return {"bound": "hbm", "kernel": name, "achieved": round(achieved, 1), "peak": peak,
+                    "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                    "traffic": committed_traffic(name), "alg_bytes_per_launch": nbytes,
+                    "us_per_launch": round(ms_mean * 1e3, 2), "us_median": round(ms_med * 1e3, 2),
+                    "us_best": round(ms_best * 1e3, 2), "share_of_step": round(share, 4)}
+        share_q = tq_mean / (tq_mean + td_mean)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "block": list(BLOCK), "fmt": "e4m3",
                        "io": "bf16 -> e4m3 codes + fp32 scales -> bf16", "bytes_per_step": qb + db,
-                       "l2": f"{nsets} rotating buffer sets ({nsets * per_set >> 20} MiB) > 126 MB L2; no flush",
-                       "parallelism": f"dp{world}: independent weight per rank (seed 1+rank), no collective"},
-            "roofline": {"bound": "hbm", "kernel": "k_quant_128x128 + k_dequant_128x128",
-                         "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": traffic, "alg_bytes_per_launch": qb,
-                         "us_per_launch": round(per_launch_ms * 1e3, 3),
-                         "note": "the two kernels move equal algorithmic bytes per launch; duration = timed "
-                                 "region / launches; traffic = ncu DRAM bytes of one k_quant_128x128 launch"},
-            "kernels_us": {"k_quant_128x128": round(tq * 1e3, 3), "k_dequant_128x128": round(td * 1e3, 3),
-                           "note": f"separate replay of {split_steps} steps with an event between launches; "
-                                   "those events serialize the kernels and inflate both figures"},
+                       "l2": "inputs larger than L2 (2 GiB in, 1 GiB codes + 32 MiB scales, 2 GiB out per step); "
+                             "no flush",
+                       "parallelism": f"dp{world}: independent tensor per rank (seed 4+rank), no collective"},
+            "roofline": roofline("k_quant_rowblocks", qb, tq_mean, tq_med, tq_best, share_q),
+            "roofline_dequant": roofline("k_dequant_flat", db, td_mean, td_med, td_best, 1 - share_q),
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": hx.numel() * 2,
-                    "d2h_bytes_per_step": hq.numel() + hs.numel() * 4 + hy.numel() * 2, "steps": e2e_steps,
-                    "note": "pinned host buffers; uploads, kernels and downloads on three streams, so one "
-                            "step's download overlaps the next step's upload"},
-            "per_rep": {"reps": 50, "warmup": 10, "l2": "512 MiB flush before each rep, outside the events",
-                        "median_us": round(rep_med * 1e3, 2), "best_us": round(rep_best * 1e3, 2),
-                        "median_GB_s": round((qb + db) * world / (rep_med * 1e-3) / 1e9, 1),
-                        "best_GB_s": round((qb + db) * world / (rep_best * 1e-3) / 1e9, 1),
-                        "note": "one step per graph replay, events around it: includes the launch and a cold "
-                                "start, which the timed region amortizes"},
+                    "d2h_bytes_per_step": ROWS * COLS + ROWS * (COLS // 128) * 4 + ROWS * COLS * 2,
+                    "steps": e2e_steps,
+                    "note": "pinned host buffers; uploads, kernels and downloads on three streams over two device "
+                            "buffer sets, so one step's download overlaps the next step's upload"},
             "gpu_launches": 2 * args.steps,
-            "timing": f"K steps replayed from CUDA graphs of <= {GRAPH_CHUNK} steps; events around the region only",
+            "timing": "K steps launched eagerly, an event after every launch; value = bytes / (last event - first)",
             "clocks": clocks.summary(),
         }
-    del xs, qs, ss, ys
-    torch.cuda.empty_cache()
+    bits = inputs.bf16_bits(x_cpu) if (world == 1 and rank == 0 and not args.no_cpu_baseline) else None
+    del x_cpu, hx
     if world == 1 and not args.no_modes:
         line["modes"] = modes_breakdown(dev, stream, peak)
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
-        line["cpu_baseline_all_cores"] = cpu_baseline_all_cores()
+        line["modes"]["weight_4096_128x128_roundtrip"] = weight_roundtrip(dev, raw, peak)
+    if bits is not None:
+        line["cpu_baseline"] = cpu_baseline(bits)
+        line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(bits)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -898,19 +921,147 @@ def run_ours(args):
     return 0
 
 
+def traffic_probe(args):
+    """One launch of a kernel between L2 cleaners, for an ncu capture of DRAM bytes read and written.
+
+    Sequence: cleaner, kernel, cleaner (and for the headline: quantize, cleaner, dequant, cleaner).  The
+    cleaner is the library's amax kernel over a 512 MiB bf16 buffer: it reads more than the L2 holds and
+    writes 4 bytes, so under `ncu --cache-control none` each probed kernel starts with none of its inputs
+    in L2, and the dirty lines a kernel leaves in L2 are written back during the next cleaner, whose own
+    DRAM writes are those write-backs alone.  A kernel's write traffic is therefore its own
+    dram__bytes_write.sum plus that of the cleaner after it.
+
+    --probe headline   the headline pair (1x128 quantize, dequant) on the 2^n sweep tensor;
+    --probe 128x128    128x128 quantize of the 2^n sweep tensor;
+    --probe bt1x128    1x128 quantize of x and x^T of the bf16 activations 16384x7168;
+    --probe gemm_fwd / gemm_wgrad   the consumer GEMM (timing; its operands are quantized first).
+    --probe-time K     afterwards, also time K back-to-back launches of the probed kernel(s) (not under ncu).
+    --lib PATH         use another build of the library (a variant built with tuning macros)."""
+    import torch
+    from fine_grained_block_b200 import inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    raw = Raw(stream, args.lib)
+    L, st = raw.L, raw.stream
+    if args.probe == "bt1x128":
+        x = inputs.activation_outlier_channels(device=dev)
+    elif args.probe.startswith("gemm"):
+        # the consumer GEMM's operands, quantized by the library: forward (1x128 x 128x128, M N K =
+        # 16384 4096 7168) or weight gradient (1x128 x 1x128, E5M2 x E4M3, 4096 7168 16384)
+        wgrad = args.probe == "gemm_wgrad"
+        Mg, Ng, Kg = (4096, 7168, 16384) if wgrad else (16384, 4096, 7168)
+        xa = inputs.random_matrix(Mg, Kg, seed=8 if wgrad else 6, dtype=torch.bfloat16, scale=1e-3 if wgrad else 1.0,
+                                  outlier_frac=1e-3, factor=1e2, device=dev)
+        xb = inputs.random_matrix(Ng, Kg, seed=9 if wgrad else 7, dtype=torch.bfloat16, scale=1.0 if wgrad else 0.02,
+                                  outlier_frac=1e-3 if wgrad else 0.0, factor=1e2, device=dev)
+        bro = 1 if wgrad else 128
+        qa = torch.empty(Mg, Kg, dtype=torch.uint8, device=dev)
+        sa = torch.empty(Mg, Kg // 128, dtype=torch.float32, device=dev)
+        qbm = torch.empty(Ng, Kg, dtype=torch.uint8, device=dev)
+        sbm = torch.empty(Ng // bro, Kg // 128, dtype=torch.float32, device=dev)
+        raw.check(L.fp8_quantize_blockwise(xa.data_ptr(), 1, Mg, Kg, 1, 128, 1 if wgrad else 0, qa.data_ptr(),
+                                           sa.data_ptr(), st), "1x128")
+        raw.check(L.fp8_quantize_blockwise(xb.data_ptr(), 1, Ng, Kg, bro, 128, 0, qbm.data_ptr(), sbm.data_ptr(), st),
+                  "B")
+        x = torch.empty(Mg, Ng, dtype=torch.bfloat16, device=dev)  # the GEMM's output
+    else:
+        x = inputs.sweep_tensor(args.traffic_log2n, seed=4, device=dev)
+    R, C = x.shape
+    n = x.numel()
+    q = torch.empty(R, C, dtype=torch.uint8, device=dev)
+    cleaner = torch.ones(1 << 28, dtype=torch.bfloat16, device=dev)
+    am = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def clean():
+        raw.check(L.fp8_amax(cleaner.data_ptr(), 1, cleaner.numel(), am.data_ptr(), st), "amax")
+
+    launches = []
+    if args.probe == "headline":
+        s = torch.empty(R, C // 128, dtype=torch.float32, device=dev)
+        y = torch.empty(R, C, dtype=torch.bfloat16, device=dev)
+        qb, db = step_bytes(R, C)
+        launches.append(("k_quant_rowblocks", qb, lambda stream_: raw.check(L.fp8_quantize_blockwise(
+            x.data_ptr(), 1, R, C, *BLOCK, 0, q.data_ptr(), s.data_ptr(), stream_), "quantize")))
+        launches.append(("k_dequant_flat", db, lambda stream_: raw.check(L.fp8_dequantize(
+            q.data_ptr(), 0, R, C, *BLOCK, s.data_ptr(), y.data_ptr(), 1, stream_), "dequantize")))
+    elif args.probe == "128x128":
+        s = torch.empty(R // 128, C // 128, dtype=torch.float32, device=dev)
+        launches.append(("k_quant_128x128", 3 * n + 4 * (n // 16384), lambda stream_: raw.check(
+            L.fp8_quantize_blockwise(x.data_ptr(), 1, R, C, 128, 128, 0, q.data_ptr(), s.data_ptr(), stream_),
+            "128x128")))
+    elif args.probe.startswith("gemm"):
+        s = torch.empty(1, dtype=torch.float32, device=dev)
+        flops = 2.0 * Mg * Ng * Kg
+        launches.append(("k_gemm_blockwise", flops, lambda stream_: raw.check(L.fp8_gemm_blockwise_ex(
+            qa.data_ptr(), sa.data_ptr(), 1 if wgrad else 0, qbm.data_ptr(), sbm.data_ptr(), bro, 0, Mg, Ng, Kg,
+            x.data_ptr(), 1, stream_), "gemm")))
+    else:
+        s = torch.empty(R, C // 128, dtype=torch.float32, device=dev)
+        qt = torch.empty(C, R, dtype=torch.uint8, device=dev)
+        st_ = torch.empty(C, R // 128, dtype=torch.float32, device=dev)
+        launches.append(("k_quant_block_transpose", 4 * n + 8 * (n // 128), lambda stream_: raw.check(
+            L.fp8_quantize_blockwise_transpose(x.data_ptr(), 1, R, C, 1, 128, 0, q.data_ptr(), s.data_ptr(),
+                                               qt.data_ptr(), st_.data_ptr(), stream_), "block transpose")))
+    clean()
+    for _, _, fn in launches:
+        fn(st)
+        clean()
+    torch.cuda.synchronize()
+    same = None
+    if args.lib:
+        # a variant build must give the default build's bytes: rerun the default on copies of the outputs
+        got = [t.clone() for t in (q, s)]
+        if args.probe.startswith("gemm"):  # the GEMM's result is within a bound, not bit-exact: compare loosely
+            got[0] = x.clone()
+        default = Raw(stream)
+        L_var, raw.L = raw.L, default.L
+        L = raw.L
+        for _, _, fn in launches:
+            fn(st)
+        torch.cuda.synchronize()
+        if args.probe.startswith("gemm"):
+            same = bool(torch.allclose(got[0].float(), x.float(), rtol=2e-2, atol=1e-3 * float(x.float().abs().max())))
+        else:
+            same = bool(torch.equal(got[0], q) and torch.equal(got[1].view(torch.int32), s.view(torch.int32)))
+        raw.L = L = L_var
+    out = {"probe": args.probe, "rows": R, "cols": C, "lib": args.lib or "default", "same_as_default": same,
+           "alg_bytes": {name: nb for name, nb, _ in launches},
+           "source_sha256": {k: source_hash(k) for k in KERNEL_SOURCES}}
+    if args.probe_time:
+        del cleaner
+        for name, nb, fn in launches:
+            ms = time_in_graph([lambda r, stream_, fn=fn: fn(stream_)], args.probe_time, dev)
+            rate = nb / (ms * 1e-3) / (1e12 if name == "k_gemm_blockwise" else 1e9)
+            out.setdefault("timing", {})[name] = {"us": round(ms * 1e3, 2),
+                                                  ("TFLOP_s" if name == "k_gemm_blockwise" else "GB_s"): round(rate, 1)}
+    print(json.dumps({"traffic_probe": out}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-modes", action="store_true", help="skip the per-mode breakdown")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--ref-budget-s", type=float, default=60.0,
                     help="reference arm: seconds of oracle work for warm-up + timed steps together")
+    ap.add_argument("--traffic-probe", action="store_true",
+                    help="run one launch of each headline kernel between L2 cleaners (for an ncu DRAM capture)")
+    ap.add_argument("--traffic-log2n", type=int, default=LOG2_N, help="tensor size of --traffic-probe (2^n)")
+    ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad"], default="headline",
+                    help="the kernel(s) of --traffic-probe")
+    ap.add_argument("--probe-time", type=int, default=0, metavar="K",
+                    help="with --traffic-probe: also time K graph-replayed launches of the probed kernel(s)")
+    ap.add_argument("--lib", default=None, help="with --traffic-probe: a variant build of the library")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.traffic_probe:
+        return traffic_probe(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

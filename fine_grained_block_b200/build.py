@@ -80,5 +80,11 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true", help="print nvcc lines and ptxas resource usage")
+    ap.add_argument("--define", action="append", default=[], metavar="NAME=VALUE",
+                    help="a tuning macro for a variant build (with --out)")
+    ap.add_argument("--out", default=None, help="path of a variant library (objects under _build/variants/)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    if a.define and a.out is None:
+        ap.error("--define builds a variant: give its --out path")
+    defines = dict(d.split("=", 1) for d in a.define)
+    print(build(force=a.force, verbose=a.verbose, defines=defines or None, out=a.out))

@@ -82,6 +82,7 @@
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
 #include "launch_util.h"
+#include "tensor_map.h"
 #include "umma.cuh"
 
 namespace fp8q {
@@ -114,6 +115,14 @@ struct Split {
     static_assert(kControlRegs % 8 == 0 && kPromoteRegs % 8 == 0, "setmaxnreg counts are multiples of 8");
 };
 static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the register file");
+
+// 1x128 B: the fill's 16-byte scale loads, and packed f32x2 promotion arithmetic.
+#ifndef FP8Q_GEMM_FILL_VEC4
+#define FP8Q_GEMM_FILL_VEC4 1
+#endif
+#ifndef FP8Q_GEMM_PACKED_B1
+#define FP8Q_GEMM_PACKED_B1 0
+#endif
 
 // B with 1x128 blocks (the weight-gradient operand) has a scale per column
 // and chunk; two otherwise idle warps stage their reciprocals in a ring of
@@ -288,17 +297,33 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // flight per thread: the scales of a column are consecutive in K),
         // then waits for their ring slots and publishes them one by one.
         const int ft = (warp - 2) * 32 + lane;  // 0..63; columns ft + 64 i of the tile
+        // A column's scales are consecutive in K: when every 4-chunk group starts on a 16-byte
+        // boundary, a round takes them with one 16-byte load per column.
+        const bool vec4 = FP8Q_GEMM_FILL_VEC4 && (kc_stride % kRbGroup) == 0 &&
+                          (reinterpret_cast<uintptr_t>(sb) & 15u) == 0;
         uint32_t g = 0;
         for (int64_t t = first; t < tiles && !timed_out; t += step) {
             const float* sb_cols = sb + ((t % tiles_n) * kBN) * kc_stride;
             for (int kc0 = 0; kc0 < nchunks && !timed_out; kc0 += kRbGroup) {
                 const int cnt = min(kRbGroup, nchunks - kc0);
                 float v[kRbGroup][kBN / 64];
+                if (vec4 && cnt == kRbGroup) {
+                    static_assert(kRbGroup == 4, "one float4 per column and round");
 #pragma unroll
-                for (int u = 0; u < kRbGroup; ++u)
+                    for (int i = 0; i < kBN / 64; ++i) {
+                        const float4 w = __ldg(reinterpret_cast<const float4*>(sb_cols + (ft + 64 * i) * kc_stride + kc0));
+                        v[0][i] = w.x;
+                        v[1][i] = w.y;
+                        v[2][i] = w.z;
+                        v[3][i] = w.w;
+                    }
+                } else {
 #pragma unroll
-                    for (int i = 0; i < kBN / 64; ++i)
-                        v[u][i] = (u < cnt) ? __ldg(sb_cols + (ft + 64 * i) * kc_stride + kc0 + u) : 1.0f;
+                    for (int u = 0; u < kRbGroup; ++u)
+#pragma unroll
+                        for (int i = 0; i < kBN / 64; ++i)
+                            v[u][i] = (u < cnt) ? __ldg(sb_cols + (ft + 64 * i) * kc_stride + kc0 + u) : 1.0f;
+                }
 #pragma unroll
                 for (int u = 0; u < kRbGroup; ++u) {
                     if (u >= cnt) break;
@@ -370,6 +395,24 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                             break;
                         }
                         const float4* rb = reinterpret_cast<const float4*>(rb_ring + slot * kBN + half * 128 + h * 64);
+#if FP8Q_GEMM_PACKED_B1
+                        // the same two roundings per element, two elements per instruction:
+                        // RN(p * f) (mul.rn.f32x2), then fma(that, 1/sb, acc) (fma.rn.f32x2)
+                        const uint64_t f2 = f32x2(f, f);
+#pragma unroll
+                        for (int j4 = 0; j4 < 16; ++j4) {
+                            const float4 r = rb[j4];
+                            float* a = acc + h * 64 + 4 * j4;
+                            const float2 lo = f32x2_split(fma_f32x2(mul_f32x2(f32x2(p[4 * j4], p[4 * j4 + 1]), f2),
+                                                                    f32x2(r.x, r.y), f32x2(a[0], a[1])));
+                            const float2 hi = f32x2_split(fma_f32x2(mul_f32x2(f32x2(p[4 * j4 + 2], p[4 * j4 + 3]), f2),
+                                                                    f32x2(r.z, r.w), f32x2(a[2], a[3])));
+                            a[0] = lo.x;
+                            a[1] = lo.y;
+                            a[2] = hi.x;
+                            a[3] = hi.y;
+                        }
+#else
 #pragma unroll
                         for (int j4 = 0; j4 < 16; ++j4) {
                             const float4 r = rb[j4];
@@ -381,6 +424,7 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                             acc[h * 64 + 4 * j4 + 3] =
                                 __fmaf_rn(__fmul_rn(p[4 * j4 + 3], f), r.w, acc[h * 64 + 4 * j4 + 3]);
                         }
+#endif
                         if (h == 1) {
                             __syncwarp();
                             if (lane == 0) umma::mbar_arrive(&bars->rb_empty[slot]);
@@ -430,19 +474,6 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         if (PAIR) umma::tmem_dealloc_pair(tmem, kTmemCols);
         else umma::tmem_dealloc(tmem, kTmemCols);
     }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult res;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &res) == cudaSuccess &&
-            res == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
 }
 
 // [rows, K] bytes, K-major, boxes of box_rows x 128 bytes with the 128-byte

@@ -6,11 +6,21 @@
 // scale, scaled cast, code store, scale store.
 
 #include <algorithm>
+#include <atomic>
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
 #include "launch_util.h"
 #include "lane_vec.cuh"
+
+#ifndef FP8Q_Q128_TMA
+#define FP8Q_Q128_TMA 0
+#endif
+#if FP8Q_Q128_TMA
+#include "fp8q_wait.cuh"
+#include "tensor_map.h"
+#include "umma.cuh"
+#endif
 
 namespace fp8q {
 namespace {
@@ -325,6 +335,135 @@ cudaError_t launch_128x128_typed(const void* x, int64_t rows, int64_t cols, uint
     return cudaGetLastError();
 }
 
+#if FP8Q_Q128_TMA
+// ---------------------------------------------------------------------------
+// A TMA-staged variant of the 128x128 kernel, compiled in only with
+// -DFP8Q_Q128_TMA=1 (bf16, rows and cols multiples of 128).  It exists to
+// measure the alternative the default kernel was chosen over: persistent
+// CTAs keep FP8Q_Q128_TMA_STAGES tiles in flight per CTA, each brought into
+// shared memory by one 2-D TMA load (no multicast) on an mbarrier; the tile is
+// read into registers, its amax reduced (one barrier per tile), the stage
+// reissued for the tile kStages ahead, and the codes cast from registers.
+// ---------------------------------------------------------------------------
+#ifndef FP8Q_Q128_TMA_STAGES
+#define FP8Q_Q128_TMA_STAGES 2
+#endif
+#ifndef FP8Q_Q128_TMA_CTAS
+#define FP8Q_Q128_TMA_CTAS 3
+#endif
+constexpr int kQtStages = FP8Q_Q128_TMA_STAGES;
+constexpr int kQtTileBytes = 128 * 128 * 2;
+constexpr int kQtAlloc = kQtStages * kQtTileBytes + 2 * 8 * 4 + kQtStages * 8 + 128;
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, FP8Q_Q128_TMA_CTAS)
+k_quant_128x128_tma(const __grid_constant__ CUtensorMap map_x, uint4* __restrict__ q, float* __restrict__ scales,
+                    int64_t rows, int64_t cols, unsigned int* status) {
+    using V = LaneVec<uint16_t, 32>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float (*warp_amax)[8] = reinterpret_cast<float (*)[8]>(sm + kQtStages * kQtTileBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kQtStages * kQtTileBytes + 2 * 8 * 4);
+    const int64_t tiles_c = cols / 128, tiles = (rows / 128) * tiles_c;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lr0 = warp * 16 + lane / 8, vec_in_row = lane % 8;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQtStages; ++s) umma::mbar_init(&full[s], 1);
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_enter();
+    auto issue = [&](int64_t t, int s) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        umma::mbar_arrive_expect_tx(&full[s], kQtTileBytes);
+        umma::tma_load_2d(sm + s * kQtTileBytes, &map_x, &full[s], static_cast<int>(tc * 128),
+                          static_cast<int>(tr * 128));
+    };
+    if (threadIdx.x == 0)
+        for (int s = 0; s < kQtStages; ++s) {
+            const int64_t t = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
+            if (t < tiles) issue(t, s);
+        }
+    bool timed_out = false;
+    int i = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int s = i % kQtStages;
+        const bool ok = umma::mbar_wait(&full[s], static_cast<uint32_t>(i / kQtStages) & 1u, kWaitLimitNs);
+        const uint8_t* stage = sm + s * kQtTileBytes;
+        typename V::In v[4];
+        float a = 0.0f;
+        if (ok) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint8_t* p = stage + (lr0 + 4 * k) * 256 + vec_in_row * 32;
+                const uint4 lo = *reinterpret_cast<const uint4*>(p), hi = *reinterpret_cast<const uint4*>(p + 16);
+                v[k] = typename V::In{{lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w}};
+                a = fmaxf(a, V::amax(v[k]));
+            }
+        }
+        a = warp_max<32>(a);
+        if (lane == 0) warp_amax[i & 1][warp] = a;
+        if (__syncthreads_or(!ok)) {
+            timed_out = true;
+            break;
+        }
+        if (threadIdx.x == 0) {  // every thread holds its slice: the stage is free
+            const int64_t tn = t + static_cast<int64_t>(kQtStages) * gridDim.x;
+            if (tn < tiles) issue(tn, s);
+        }
+        float ta = warp_amax[i & 1][0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) ta = fmaxf(ta, warp_amax[i & 1][w]);
+        const float sc = scale_from_amax<FMT>(ta);
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            st_stream(q + ((tr * 128 + lr0 + 4 * k) * cols + tc * 128) / 16 + vec_in_row,
+                      V::template cast<FMT>(v[k], f32x2(sc, sc)));
+        if (threadIdx.x == 0) scales[t] = sc;
+    }
+    if (timed_out) {
+        if (threadIdx.x == 0) {
+            atomicOr(status, kStatusWaitTimeout);
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 1000000ull) {
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int FMT>
+cudaError_t launch_128x128_tma(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales, cudaStream_t st,
+                               bool* launched) {
+    *launched = false;
+    if (rows % 128 != 0 || rows > 0x7FFFFFFF || cols > 0x7FFFFFFF) return cudaSuccess;
+    CUtensorMap map;
+    if (!make_bf16_tile_map(&map, x, rows, cols, 128, 128)) return cudaSuccess;
+    unsigned int* status = device_status_word();
+    if (status == nullptr) return cudaSuccess;
+    auto kern = k_quant_128x128_tma<FMT>;
+    static std::atomic<int> resident[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    int units = resident[dev].load(std::memory_order_acquire);
+    if (units <= 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQtAlloc);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, kQtAlloc);
+        if (e != cudaSuccess) return e;
+        units = std::max(1, per_sm) * device_sm_count();
+        resident[dev].store(units, std::memory_order_release);
+    }
+    const int64_t grid = std::min<int64_t>((rows / 128) * (cols / 128), units);
+    const cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kQtAlloc, st, map,
+                                        reinterpret_cast<uint4*>(q), scales, rows, cols, status);
+    if (e == cudaSuccess) *launched = true;
+    return e;
+}
+#endif  // FP8Q_Q128_TMA
+
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 template <typename T, int FMT>
@@ -360,6 +499,14 @@ cudaError_t launch_quant_1x128(const void* x, int dtype, int64_t nblocks, int fm
 
 cudaError_t launch_quant_128x128(const void* x, int dtype, int64_t rows, int64_t cols, int fmt, uint8_t* q,
                                  float* scales, cudaStream_t st) {
+#if FP8Q_Q128_TMA
+    if (dtype == 1) {
+        bool launched = false;
+        const cudaError_t e = fmt == kE4M3 ? launch_128x128_tma<kE4M3>(x, rows, cols, q, scales, st, &launched)
+                                           : launch_128x128_tma<kE5M2>(x, rows, cols, q, scales, st, &launched);
+        if (e != cudaSuccess || launched) return e;
+    }
+#endif
     const bool w32 = aligned32(x);
     if (dtype == 1) {
         if (w32)

@@ -24,12 +24,15 @@
 // Both casts are RN_fp32(x * s) then the saturating RNE cast, as everywhere.
 
 #include <algorithm>
+#include <atomic>
 
 #include "fp8q_device.cuh"
 #include "fp8q_launch.h"
 #include "launch_util.h"
 #include "lane_vec.cuh"
+#include "tensor_map.h"
 #include "tile_transpose.cuh"
+#include "umma.cuh"
 
 namespace fp8q {
 namespace {
@@ -128,6 +131,9 @@ struct ColMax<float, BYTES> {
 // on B200, bf16 activations 16384x7168, 1x128: 4954 GB/s holding the tile
 // with a cap of 2 CTAs; with the second read 4598 / 5162 / 5213 GB/s for 2 /
 // 3 / 4 CTAs.  128x128: 6462 GB/s (98.7 % of the copy peak) with 3 or 4 CTAs.
+#ifndef FP8Q_BT_TMA
+#define FP8Q_BT_TMA 1
+#endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_RELOAD
 #define FP8Q_BLOCK_TRANSPOSE_RELOAD 1
 #endif
@@ -232,6 +238,195 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
     tile_transpose_out(tile, qt, rows, r0, c0, lane, warp);
 }
 
+// ---------------------------------------------------------------------------
+// 1x128 blocks of bf16 x and x^T, TMA-staged and persistent.
+//
+// The register-tile kernel above spends most of a tile's time computing
+// (two casts, the row and column reductions, three barriers) with nothing in
+// flight to HBM, and its column pass reads the tile a second time from L2.
+// Here each CTA walks tiles first, first + step, ... and keeps the next
+// kStages tiles in flight: a 2-D TMA load (no multicast) brings each 128x128
+// bf16 tile (32 KiB) into a shared-memory stage, completing on the stage's
+// mbarrier, and is issued for tile i + kStages as soon as tile i's last read
+// of the stage is behind a barrier.  Both passes read the tile from shared
+// memory, with the lane geometry of the register kernel (16 tile rows per
+// warp, one 32-byte slice per lane and load), so the arithmetic is the same:
+// row amax -> row scale -> q; column amax (lane, warp row groups, warps) ->
+// column scale -> codes into the swizzled code tile -> qt.
+// Waits are bounded; a wait that runs out sets the device status bit, the
+// CTA stops, and it waits (bounded) for its loads in flight before it exits.
+// ---------------------------------------------------------------------------
+#ifndef FP8Q_BT_TMA_STAGES
+#define FP8Q_BT_TMA_STAGES 2
+#endif
+#ifndef FP8Q_BT_TMA_CTAS
+#define FP8Q_BT_TMA_CTAS 2
+#endif
+constexpr int kBtStages = FP8Q_BT_TMA_STAGES;
+constexpr int kBtTileBytes = kTT * kTT * 2;  // one bf16 tile
+struct BtSmem {
+    static constexpr int kStage = 0;
+    static constexpr int kCode = kBtStages * kBtTileBytes;
+    static constexpr int kPart = kCode + kTT * kTT;
+    static constexpr int kColScale = kPart + kWarps * kTT * 4;
+    static constexpr int kBars = kColScale + kTT * 4;
+    static constexpr int kBytes = kBars + kBtStages * 8;
+    static constexpr int kAlloc = kBytes + 128;  // alignment slack
+};
+
+__device__ __forceinline__ Words<8> lds32(const uint8_t* p) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint4 b = *reinterpret_cast<const uint4*>(p + 16);
+    return Words<8>{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, FP8Q_BT_TMA_CTAS)
+k_quant_block_transpose_tma(const __grid_constant__ CUtensorMap map_x, int64_t rows, int64_t cols,
+                            uint8_t* __restrict__ q, float* __restrict__ scales, uint8_t* __restrict__ qt,
+                            float* __restrict__ scales_t, unsigned int* status) {
+    using V = LaneVec<uint16_t, 32>;
+    using G = TileGeom<uint16_t, 32>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t* tile = sm + BtSmem::kCode;
+    float (*part)[kTT] = reinterpret_cast<float (*)[kTT]>(sm + BtSmem::kPart);
+    float* col_scale = reinterpret_cast<float*>(sm + BtSmem::kColScale);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + BtSmem::kBars);
+
+    const int64_t tiles_c = cols / kTT, tiles_r = rows / kTT;
+    const int64_t tiles = tiles_r * tiles_c;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lr0 = warp * 16 + lane / G::kVecPerRow, vec_in_row = lane % G::kVecPerRow;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBtStages; ++s) umma::mbar_init(&full[s], 1);
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_enter();  // x may come from the previous kernel
+
+    auto issue = [&](int64_t t, int s) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        umma::mbar_arrive_expect_tx(&full[s], kBtTileBytes);
+        umma::tma_load_2d(sm + BtSmem::kStage + s * kBtTileBytes, &map_x, &full[s], static_cast<int>(tc * kTT),
+                          static_cast<int>(tr * kTT));
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBtStages; ++s) {
+            const int64_t t = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
+            if (t < tiles) issue(t, s);
+        }
+    }
+
+    bool timed_out = false;
+    int i = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int s = i % kBtStages;
+        const uint32_t parity = static_cast<uint32_t>(i / kBtStages) & 1u;
+        const bool ok = umma::mbar_wait(&full[s], parity, kWaitLimitNs);
+        const uint8_t* stage = sm + BtSmem::kStage + s * kBtTileBytes;
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t r0 = tr * kTT, c0 = tc * kTT;
+
+        typename V::In v[G::kLoads];
+        if (ok) {
+#pragma unroll
+            for (int k = 0; k < G::kLoads; ++k)
+                v[k] = lds32(stage + (lr0 + k * G::kRowsPerLoad) * (kTT * 2) + vec_in_row * 32);
+            // q: one scale per tile row, as in the register kernel
+            float ra[G::kLoads];
+#pragma unroll
+            for (int k = 0; k < G::kLoads; ++k) ra[k] = warp_max<G::kVecPerRow>(V::amax(v[k]));
+            float mine = 0.0f;
+#pragma unroll
+            for (int k = 0; k < G::kLoads; ++k)
+                if (k % G::kVecPerRow == vec_in_row) mine = ra[k];
+            const float s_mine = scale_from_amax<FMT>(mine);
+            const int group = lane - vec_in_row;
+#pragma unroll
+            for (int k = 0; k < G::kLoads; ++k) {
+                const float sc = __shfl_sync(0xFFFFFFFFu, s_mine, group + k % G::kVecPerRow);
+                const int lr = lr0 + k * G::kRowsPerLoad;
+                st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row,
+                          V::template cast<FMT>(v[k], f32x2(sc, sc)));
+                if (vec_in_row == 0) scales[(r0 + lr) * tiles_c + tc] = sc;
+            }
+            ColMax<uint16_t, 32>::run(v, lane < G::kVecPerRow, &part[warp][vec_in_row * V::kElems]);
+        }
+        if (__syncthreads_or(!ok)) {
+            timed_out = true;
+            break;
+        }
+        if (threadIdx.x < kTT) {
+            const int c = threadIdx.x;
+            float m = part[0][c];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, part[w][c]);
+            const float sc = scale_from_amax<FMT>(m);
+            col_scale[c] = sc;
+            scales_t[(c0 + c) * tiles_r + tr] = sc;
+        }
+        __syncthreads();
+        const float* cs = col_scale + vec_in_row * V::kElems;
+#pragma unroll
+        for (int k = 0; k < G::kLoads; ++k) {
+            const int lr = lr0 + k * G::kRowsPerLoad;
+            const typename V::In w = lds32(stage + lr * (kTT * 2) + vec_in_row * 32);
+            *reinterpret_cast<typename V::Out*>(tile + tile_off(lr, vec_in_row * V::kElems)) =
+                PairCast<uint16_t, 32>::template cast<FMT>(w, cs);
+        }
+        __syncthreads();  // the stage is read and the code tile complete
+        if (threadIdx.x == 0) {
+            const int64_t tn = t + static_cast<int64_t>(kBtStages) * gridDim.x;
+            if (tn < tiles) issue(tn, s);
+        }
+        tile_transpose_out(tile, qt, rows, r0, c0, lane, warp);
+    }
+    if (timed_out) {
+        if (threadIdx.x == 0) {
+            atomicOr(status, kStatusWaitTimeout);
+            // loads may still be landing in this CTA's shared memory: let them finish (bounded)
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 1000000ull) {
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int FMT>
+cudaError_t launch_bt_tma(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales, uint8_t* qt,
+                          float* scales_t, cudaStream_t st, bool* launched) {
+    *launched = false;
+    const int64_t tiles = (rows / kTT) * (cols / kTT);
+    if (rows > 0x7FFFFFFF || cols > 0x7FFFFFFF) return cudaSuccess;  // TMA coordinates are 32-bit
+    CUtensorMap map;
+    if (!make_bf16_tile_map(&map, x, rows, cols, kTT, kTT)) return cudaSuccess;
+    unsigned int* status = device_status_word();
+    if (status == nullptr) return cudaSuccess;
+    auto kern = k_quant_block_transpose_tma<FMT>;
+    // The shared-memory opt-in and the co-resident grid, once per device.
+    static std::atomic<int> resident[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    int units = resident[dev].load(std::memory_order_acquire);
+    if (units <= 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BtSmem::kAlloc);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, BtSmem::kAlloc);
+        if (e != cudaSuccess) return e;
+        units = std::max(1, per_sm) * device_sm_count();
+        resident[dev].store(units, std::memory_order_release);
+    }
+    const int64_t grid = std::min<int64_t>(tiles, units);
+    const cudaError_t e = launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), BtSmem::kAlloc, st,
+                                        map, rows, cols, q, scales, qt, scales_t, status);
+    if (e == cudaSuccess) *launched = true;
+    return e;
+}
+
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 template <typename T, int FMT, int BYTES>
@@ -264,6 +459,15 @@ cudaError_t launch_quant_block_transpose(const void* x, int dtype, int64_t rows,
                                          int fmt, uint8_t* q, float* scales, uint8_t* qt, float* scales_t,
                                          cudaStream_t st) {
     if (rows == 0 || cols == 0) return cudaSuccess;
+#if FP8Q_BT_TMA
+    if (dtype == 1 && block_rows == 1) {
+        // bf16 in 1x128 blocks: the TMA-staged persistent kernel, where the driver offers tensor maps
+        bool launched = false;
+        const cudaError_t e = fmt == kE4M3 ? launch_bt_tma<kE4M3>(x, rows, cols, q, scales, qt, scales_t, st, &launched)
+                                           : launch_bt_tma<kE5M2>(x, rows, cols, q, scales, qt, scales_t, st, &launched);
+        if (e != cudaSuccess || launched) return e;
+    }
+#endif
     if (dtype == 1)
         return fmt == kE4M3 ? launch_width<uint16_t, kE4M3>(x, rows, cols, block_rows, q, scales, qt, scales_t, st)
                             : launch_width<uint16_t, kE5M2>(x, rows, cols, block_rows, q, scales, qt, scales_t, st);

@@ -84,6 +84,15 @@ def oracle_per_tensor(x: np.ndarray, fmt: int, scale=None):
     return q, s, a
 
 
+def oracle_cast(x: np.ndarray, fmt: int, scale) -> np.ndarray:
+    """oracle.quantize_per_tensor's codes for a given scale, in chunks (no amax pass)."""
+    flat = x.reshape(-1)
+    step = max(1, math.ceil(flat.size / (NTHREADS * 4)))
+    parts = list(_pool.map(lambda i: oracle.quantize_per_tensor(flat[i:i + step], fmt, scale=float(scale))[0],
+                           range(0, flat.size, step)))
+    return np.concatenate(parts).reshape(x.shape) if parts else np.zeros(x.shape, np.uint8)
+
+
 def oracle_dequant(q: np.ndarray, fmt: int, scales: np.ndarray, br: int, bc: int, out_dtype: int):
     if q.ndim == 1:
         q = q.reshape(1, -1)

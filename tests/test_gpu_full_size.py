@@ -1,9 +1,8 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the benchmark uses.
 
-Full element-by-element comparison with the (threaded) oracle up to 2^26
-elements; the 2^30 sweep point is compared on sampled rows / tile rows (each
-block's result depends only on its block, and the per-tensor scale comes from
-the oracle's amax over the whole tensor), plus invariants over every block.
+Every element is compared with the (threaded) oracle: the 16384x7168
+activations, 32 delayed steps of the 8192x8192 gradients, and the size sweep
+from 2^20 to 2^30 elements in all three of its modes with their dequant.
 """
 import math
 
@@ -14,8 +13,8 @@ import torch
 import oracle
 from fine_grained_block_b200 import binding as B
 from fine_grained_block_b200 import inputs
-from parity_util import (assert_bytes_equal, fp32_bits, host_input, oracle_amax, oracle_blockwise, oracle_dequant,
-                         oracle_per_tensor, to_cuda)
+from parity_util import (assert_bytes_equal, fp32_bits, host_input, oracle_amax, oracle_blockwise, oracle_cast,
+                         oracle_dequant, oracle_per_tensor, to_cuda)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -59,69 +58,43 @@ def test_gradients_8192_delayed_e5m2_32_steps():
     assert min(zero_frac[:W]) > 0.1 and max(zero_frac[W:]) < 1e-3
 
 
-@pytest.mark.parametrize("log2_n", [20, 24, 26])
+def _row_chunks(R, rows_per_chunk):
+    return [(r0, min(R, r0 + rows_per_chunk)) for r0 in range(0, R, rows_per_chunk)]
+
+
+@pytest.mark.parametrize("log2_n", [20, 22, 24, 26, 28, 30])
 def test_sweep_full(log2_n):
+    """The size sweep, every element: 1x128 E4M3, 128x128 E4M3 and per-tensor current E5M2, each with its
+    bf16 dequant, compared with the oracle in chunks of 2^24 elements (whole block rows), so the host holds
+    one chunk of expected values at a time."""
     t = inputs.sweep_tensor(log2_n)
     xh = host_input(t)
     x = to_cuda(t)
-    for block in ((1, 128), (128, 128)):
-        q, s = B.fp8_quantize_blockwise(x, block, B.E4M3)
-        oq, os_ = oracle_blockwise(xh, *block, oracle.E4M3)
-        assert_bytes_equal(s, fp32_bits(os_), f"{block} scales")
-        assert_bytes_equal(q, oq, f"{block} codes")
-        y = B.fp8_dequantize(q, s, block, B.E4M3, torch.bfloat16)
-        assert_bytes_equal(y, oracle_dequant(oq, oracle.E4M3, os_, *block, oracle.BF16), f"{block} dequant")
-    q, s, a = B.fp8_quantize_per_tensor(x, B.E5M2)
-    oq, os_, oa = oracle_per_tensor(xh, oracle.E5M2)
-    assert_bytes_equal(a, fp32_bits([oa]), "amax")
-    assert_bytes_equal(s, fp32_bits([os_]), "scale")
-    assert_bytes_equal(q, oq, "per-tensor codes")
-    y = B.fp8_dequantize(q, s, (0, 0), B.E5M2, torch.bfloat16)
-    assert_bytes_equal(y, oracle_dequant(oq, oracle.E5M2, np.array([os_], np.float32), 0, 0, oracle.BF16),
-                       "per-tensor dequant")
-
-
-def test_sweep_2pow30_sampled():
-    t = inputs.sweep_tensor(30)
-    xh = host_input(t)
-    R, C = xh.shape
-    x = to_cuda(t)
     del t
-    rng = np.random.default_rng(30)
-    top_e4 = oracle.top_code(oracle.E4M3)
-    # 1x128: sampled rows, plus the first and last
-    q, s = B.fp8_quantize_blockwise(x, (1, 128), B.E4M3)
-    rows = np.unique(np.concatenate([[0, R - 1], rng.integers(0, R, 254)]))
-    for r in rows:
-        oq, os_ = oracle.quantize_blockwise(xh[r:r + 1], 1, 128, oracle.E4M3)
-        assert_bytes_equal(q[r:r + 1], oq, f"1x128 row {r}")
-        assert_bytes_equal(s[r:r + 1], fp32_bits(os_), f"1x128 scales row {r}")
-    assert bool(((q & 0x7F).view(R, C // 128, 128).amax(dim=2) == top_e4).all())
-    y = B.fp8_dequantize(q, s, (1, 128), B.E4M3, torch.bfloat16)
-    for r in rows[:32]:
-        oq = q[r:r + 1].cpu().numpy()
-        assert_bytes_equal(y[r:r + 1], oracle.dequantize(oq, oracle.E4M3, s[r:r + 1].cpu().numpy(), 1, 128,
-                                                         oracle.BF16), f"1x128 dequant row {r}")
-    del q, s, y
-    # 128x128: sampled tile rows, plus the first and last
-    q, s = B.fp8_quantize_blockwise(x, (128, 128), B.E4M3)
-    for tr in np.unique(np.concatenate([[0, R // 128 - 1], rng.integers(0, R // 128, 6)])):
-        sl = slice(tr * 128, tr * 128 + 128)
-        oq, os_ = oracle_blockwise(xh[sl], 128, 128, oracle.E4M3)
-        assert_bytes_equal(q[sl], oq, f"128x128 tile row {tr}")
-        assert_bytes_equal(s[tr:tr + 1], fp32_bits(os_), f"128x128 scales tile row {tr}")
-    mag = (q & 0x7F).view(R // 128, 128, C // 128, 128)
-    assert bool((mag.amax(dim=(1, 3)) == top_e4).all())
-    del q, s, mag
-    # per-tensor E5M2: amax over the whole tensor from the oracle; codes on sampled rows
+    R, C = xh.shape
+    chunks = _row_chunks(R, max(128, (1 << 24) // C))
+    for block in ((1, 128), (128, 128)):
+        br = block[0]
+        q, s = B.fp8_quantize_blockwise(x, block, B.E4M3)
+        y = B.fp8_dequantize(q, s, block, B.E4M3, torch.bfloat16)
+        for r0, r1 in chunks:
+            oq, os_ = oracle_blockwise(xh[r0:r1], *block, oracle.E4M3)
+            assert_bytes_equal(s[r0 // br:math.ceil(r1 / br)], fp32_bits(os_), f"{block} scales rows {r0}..")
+            assert_bytes_equal(q[r0:r1], oq, f"{block} codes rows {r0}..")
+            assert_bytes_equal(y[r0:r1], oracle_dequant(oq, oracle.E4M3, os_, *block, oracle.BF16),
+                               f"{block} dequant rows {r0}..")
+        del q, s, y
     q, s, a = B.fp8_quantize_per_tensor(x, B.E5M2)
+    y = B.fp8_dequantize(q, s, (0, 0), B.E5M2, torch.bfloat16)
     oa = oracle_amax(xh)
     os_ = oracle.scale_from_amax(oa, oracle.E5M2)
-    assert_bytes_equal(a, fp32_bits([oa]), "amax 2^30")
-    assert_bytes_equal(s, fp32_bits([os_]), "scale 2^30")
-    for r in rows[:64]:
-        oq, _, _ = oracle.quantize_per_tensor(xh[r], oracle.E5M2, scale=float(os_))
-        assert_bytes_equal(q[r], oq, f"per-tensor row {r}")
+    assert_bytes_equal(a, fp32_bits([oa]), "amax")
+    assert_bytes_equal(s, fp32_bits([os_]), "scale")
+    for r0, r1 in chunks:
+        oq = oracle_cast(xh[r0:r1], oracle.E5M2, os_)
+        assert_bytes_equal(q[r0:r1], oq, f"per-tensor codes rows {r0}..")
+        assert_bytes_equal(y[r0:r1], oracle_dequant(oq, oracle.E5M2, np.array([os_], np.float32), 0, 0,
+                                                    oracle.BF16), f"per-tensor dequant rows {r0}..")
 
 
 def test_fake_quant_activations_16384x7168():

@@ -1,9 +1,10 @@
 """GPU parity past the 32-bit index range: a bf16 tensor of [2^19 + 256, 4096] = 2^31 + 2^20 elements.
 
-Element indices pass 2^31 and the input's byte offsets pass 2^32, so every kernel's index arithmetic
-must be 64-bit.  Expected values come from the oracle on sampled rows: the first row, the rows on
-both sides of element 2^31, random rows, and the last rows (block results depend only on their
-block).  The per-tensor amax is the oracle's over the whole tensor.
+Element indices pass 2^31 and the input's byte offsets pass 2^31 (at element 2^30) and 2^32 (at element
+2^31), so every kernel's index arithmetic must be 64-bit.  Expected values come from the oracle on whole
+bands of rows: 256 rows around each of those crossings, the first and last 256 rows, and random rows
+(block results depend only on their block).  The transposed copy is compared on the whole qt rows whose
+flat index passes 2^31.  The per-tensor amax is the oracle's over the whole tensor.
 """
 import numpy as np
 import pytest
@@ -20,12 +21,17 @@ R, C = (1 << 19) + 256, 4096
 EDGE = (1 << 31) // C  # the first row past element 2^31
 
 
+HALF = (1 << 30) // C  # the first row whose bf16 byte offset passes 2^31
+BANDS = [(0, 256), (HALF - 128, HALF + 128), (EDGE - 128, EDGE + 128), (R - 256, R)]
+
+
 @pytest.fixture(scope="module")
 def big():
     x = inputs.random_matrix(R, C, seed=31, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e3, device="cuda")
     rng = np.random.default_rng(31)
-    rows = np.unique(np.concatenate([[0, EDGE - 1, EDGE, EDGE + 1, R - 129, R - 1], rng.integers(0, R, 24)]))
-    tile_rows = np.unique(np.concatenate([[0, EDGE // 128 - 1, EDGE // 128, R // 128 - 1],
+    band_rows = np.concatenate([np.arange(a, b) for a, b in BANDS])
+    rows = np.unique(np.concatenate([band_rows, rng.integers(0, R, 24)]))
+    tile_rows = np.unique(np.concatenate([[a // 128 + i for a, b in BANDS for i in range((b - a) // 128)],
                                           rng.integers(0, R // 128, 3)]))
     yield x, rows, tile_rows
     del x
@@ -118,3 +124,9 @@ def test_max_size_transpose(big):
     assert_bytes_equal(q[idx], oq, "transpose q rows")
     # qt column r is q row r
     assert_bytes_equal(qt[:, idx].t().contiguous(), oq, "transpose qt columns")
+    # the whole qt rows whose flat index c * R + r passes 2^31 (and the last one): x's columns c
+    c0 = (1 << 31) // R
+    assert c0 * R < (1 << 31) < (c0 + 1) * R
+    for c in sorted({c0, C - 1}):
+        oqc, _, _ = oracle.quantize_per_tensor(host_input(x[:, c].contiguous().cpu()), oracle.E4M3, scale=0.25)
+        assert_bytes_equal(qt[c], oqc, f"transpose qt row {c}")

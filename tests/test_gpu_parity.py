@@ -672,6 +672,15 @@ def test_blockwise_transpose(fmt, dtype, block):
         check_blockwise_transpose(x, block, fmt, f"{block} {R}x{C} {dtype}")
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_blockwise_transpose_many_tiles_per_cta(fmt):
+    """bf16 1x128 with several times more tiles than resident CTAs, so each CTA of the persistent kernel
+    reuses its shared-memory stages (both mbarrier parities) many times."""
+    x = inputs.random_matrix(4096, 8192, seed=4350 + fmt, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e3)
+    x[:, 130] = 0
+    check_blockwise_transpose(x, (1, 128), fmt, "1x128 4096x8192 bf16")
+
+
 def test_blockwise_transpose_16_byte_aligned_input():
     R, C = 256, 512
     x_cpu = inputs.random_matrix(R, C, seed=4400, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e3)
