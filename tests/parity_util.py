@@ -108,6 +108,16 @@ def oracle_dequant(q: np.ndarray, fmt: int, scales: np.ndarray, br: int, bc: int
     return np.concatenate(parts)
 
 
+def oracle_gemm(qa, sa, a_fmt, qb, sb, b_fmt, b_block=128):
+    """oracle.gemm_blockwise over row chunks of A in parallel (each chunk's rows are the oracle's own
+    computation)."""
+    M = qa.shape[0]
+    per = max(1, math.ceil(M / (NTHREADS * 2)))
+    parts = list(_pool.map(lambda r: oracle.gemm_blockwise(qa[r:r + per], sa[r:r + per], a_fmt, qb, sb, b_fmt,
+                                                           b_block=b_block), range(0, M, per)))
+    return np.concatenate(parts)
+
+
 def oracle_mx(x: np.ndarray, fmt: int, rule: int):
     """oracle.quantize_mx in row chunks: (codes, e8m0)."""
     R, C = x.shape

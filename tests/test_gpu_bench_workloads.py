@@ -3,7 +3,7 @@
 - MX 1x32 quantize and dequantize of the bf16 16384x7168 activations (outlier channels);
 - the transposing per-tensor cast of the same activations, delayed (given scale) and current;
 - 1x128 quantization of the same activations and of their transpose in one pass;
-- the blockwise GEMM at 16384x4096x7168 on sampled rows of C;
+- the blockwise GEMM at 16384x4096x7168: the whole last 256-row tile row of C and sampled rows;
 - 128 weights of 1024x1024 in one grouped 128x128 call;
 - one grouped delayed-scaling step over 128 gradients of 2^20 elements.
 
@@ -16,8 +16,8 @@ import torch
 import oracle
 from fine_grained_block_b200 import binding as B
 from fine_grained_block_b200 import inputs
-from parity_util import (assert_bytes_equal, fp32_bits, host_input, oracle_blockwise, oracle_dequant_mx, oracle_mx,
-                         oracle_per_tensor, to_cuda)
+from parity_util import (assert_bytes_equal, fp32_bits, host_input, oracle_blockwise, oracle_dequant_mx, oracle_gemm,
+                         oracle_mx, oracle_per_tensor, to_cuda)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -67,7 +67,9 @@ def test_blockwise_transpose_activations_16384x7168(activations):
     assert_bytes_equal(qt, oqt, "qt")
 
 
-def test_gemm_16384x4096x7168_sampled_rows():
+def test_gemm_16384x4096x7168_full_last_tile_row_and_sampled_rows():
+    """The benchmark's GEMM shape: every output of the last 256-row tile row (one CTA pair's tiles, the
+    last round of the persistent schedule, all 16 column tiles) and 12 sampled rows elsewhere."""
     M, N, K = 16384, 4096, 7168
     x = inputs.random_matrix(M, K, seed=6, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e2)
     w = inputs.random_matrix(N, K, seed=7, dtype=torch.bfloat16, scale=0.02)
@@ -76,9 +78,9 @@ def test_gemm_16384x4096x7168_sampled_rows():
     c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
                              to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
-    rows = [0, 1, 127, 128, 255, 256, 4095, 8191, 8192, 12000, 16256, 16383]
-    want = oracle.gemm_blockwise(qa[rows], sa[rows], oracle.E4M3, qb, sb, oracle.E4M3)
-    mag = oracle.gemm_blockwise(qa[rows] & 0x7F, sa[rows], oracle.E4M3, qb & 0x7F, sb, oracle.E4M3)
+    rows = [0, 1, 127, 128, 255, 256, 4095, 8191, 8192, 12000, 15000, 16000] + list(range(M - 256, M))
+    want = oracle_gemm(qa[rows], sa[rows], oracle.E4M3, qb, sb, oracle.E4M3)
+    mag = oracle_gemm(qa[rows] & 0x7F, sa[rows], oracle.E4M3, qb & 0x7F, sb, oracle.E4M3)
     got = c[torch.as_tensor(rows, device="cuda")].float().cpu().numpy().astype(np.float64)
     # fp32 sums of 56 promoted chunks (2^-12 of the absolute sum), then one bf16 rounding of the result
     tol = 2.0 ** -12 * mag + 2.0 ** -8 * np.abs(want)

@@ -116,8 +116,8 @@ def test_no_alloc_limit_by_alignment(dtype):
         torch.cuda.synchronize()
         limits[lane] = lo
         elems = lane // esz
-        assert (lo + 1) % elems == 0  # a whole number of lane vectors plus a tail of elems - 1
-        assert ((lo + 1) // elems) % 1024 == 0  # 1024 lane vectors per CTA
+        # a whole number of CTAs of 1024 lane vectors, plus a tail of elems - 1
+        assert (lo - (elems - 1)) % (1024 * elems) == 0, lo
     assert limits[32] > limits[16]
     # just above the 16-byte-lane limit: refused at base + 16, accepted at the 32-byte-aligned base
     n = limits[16] + 1
