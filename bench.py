@@ -255,6 +255,97 @@ def cpu_baseline(bits, budget_s: float = 12.0):
                       f"dequant, single-threaded C oracle, {reps} reps, {t:.1f} s"}
 
 
+def oracle_by_config(args):
+    """The CPU oracle's throughput on a sample of each workload in BASELINE's list, single-threaded and over
+    every host core (independent row slices in parallel), in GB/s of the same algorithmic bytes.  Host only;
+    prints one JSON line."""
+    import oracle
+    import torch
+    from concurrent.futures import ThreadPoolExecutor
+    from fine_grained_block_b200 import inputs
+    threads = max(1, len(os.sched_getaffinity(0)))
+    pool = ThreadPoolExecutor(max_workers=threads)
+
+    def rate(fn, xs, nbytes, budget=args.oracle_budget_s):
+        """GB/s of fn over the row slices xs, single-threaded and on all cores."""
+        t0 = time.perf_counter()
+        fn(xs[0])
+        one = time.perf_counter() - t0
+        reps = max(1, int(budget / max(one * len(xs), 1e-4)))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            for x in xs:
+                fn(x)
+        t1 = time.perf_counter() - t0
+        preps = max(1, int(budget / max(t1 / reps / threads, 1e-4)))
+        t0 = time.perf_counter()
+        for _ in range(preps):
+            list(pool.map(fn, xs))
+        tn = time.perf_counter() - t0
+        return {"one_core": round(nbytes * reps / t1 / 1e9, 4), "all_cores": round(nbytes * preps / tn / 1e9, 3),
+                "cores": threads}
+
+    def q_deq(br, bc, fmt, out=oracle.BF16):
+        def f(x):
+            q, sc = oracle.quantize_blockwise(x, br, bc, fmt)
+            oracle.dequantize(q, fmt, sc, br, bc, out_dtype=out)
+        return f
+
+    out = {}
+    # 1: the handbook's fp32 256x1024 tensor (outliers x1e4), E4M3 per tensor and 1x128, each + dequant
+    x1 = inputs.relerr_outlier_tensors()[1][1].numpy()
+    n1 = x1.size
+
+    def pt_deq(x):
+        q, sc, _ = oracle.quantize_per_tensor(x, oracle.E4M3)
+        oracle.dequantize(q, oracle.E4M3, np.array([sc], np.float32), 0, 0, out_dtype=oracle.F32)
+    import numpy as np
+    out["1_fp32_256x1024_per_tensor_e4m3_and_dequant"] = rate(pt_deq, [x1], 2 * 5 * n1)
+    out["1_fp32_256x1024_1x128_e4m3_and_dequant"] = rate(q_deq(1, 128, oracle.E4M3, oracle.F32),
+                                                           [x1[r:r + 16] for r in range(0, x1.shape[0], 16)],
+                                                           2 * (5 * n1 + 4 * (n1 // 128)))
+    # 2: the bf16 4096^2 weight, 128x128 + dequant, on its 32 slices of 128 rows
+    w = inputs.bf16_bits(inputs.weight_4096(seed=1))[:4096]
+    sl = [w[r:r + 128] for r in range(0, w.shape[0], 128)]
+    out["2_bf16_weight_4096_128x128_e4m3_and_dequant"] = rate(q_deq(128, 128, oracle.E4M3), sl,
+                                                              2 * (3 * w.size + 4 * (w.size // 16384)))
+    # 3: the bf16 activations 16384x7168, 1x128 quantize, on 128-row slices of the first 4096 rows
+    a = inputs.bf16_bits(inputs.activation_outlier_channels())[:4096]
+    sl = [a[r:r + 128] for r in range(0, a.shape[0], 128)]
+    out["3_bf16_activations_16384x7168_1x128_e4m3"] = rate(
+        lambda x: oracle.quantize_blockwise(x, 1, 128, oracle.E4M3), sl, 3 * a.size + 4 * (a.size // 128))
+    # 4: a delayed E5M2 step of the 8192^2 gradients (cast with the given scale + amax, history update)
+    g = inputs.bf16_bits(inputs.gradient_step(inputs.gradient_base(), 20))[:4096]
+    sl = [g[r:r + 128] for r in range(0, g.shape[0], 128)]
+    h = oracle.AmaxHistory(16, oracle.E5M2)
+
+    def delayed(x):
+        _, _, am = oracle.quantize_per_tensor(x, oracle.E5M2, scale=0.5)
+        return am
+    r4 = rate(delayed, sl, 3 * g.size)
+    t0 = time.perf_counter()
+    for _ in range(1000):
+        h.update(1.0)
+    r4["history_update_us"] = round((time.perf_counter() - t0) * 1e3, 3)
+    out["4_bf16_gradients_8192x8192_delayed_e5m2"] = r4
+    # 5: the headline tensor's first rows: 1x128, 128x128 and per-tensor E5M2, each + dequant
+    x5 = inputs.bf16_bits(inputs.sweep_tensor(LOG2_N, seed=4))[:4096]
+    sl = [x5[r:r + 128] for r in range(0, x5.shape[0], 128)]
+    n5 = x5.size
+    out["5_bf16_2^30_1x128_e4m3_and_dequant"] = rate(q_deq(1, 128, oracle.E4M3), sl, 2 * (3 * n5 + 4 * (n5 // 128)))
+    out["5_bf16_2^30_128x128_e4m3_and_dequant"] = rate(q_deq(128, 128, oracle.E4M3), sl,
+                                                       2 * (3 * n5 + 4 * (n5 // 16384)))
+
+    def pt5(x):
+        q, sc, _ = oracle.quantize_per_tensor(x, oracle.E5M2)
+        oracle.dequantize(q, oracle.E5M2, np.array([sc], np.float32), 0, 0, out_dtype=oracle.BF16)
+    out["5_bf16_2^30_per_tensor_e5m2_and_dequant"] = rate(pt5, sl, 6 * n5)
+    print(json.dumps({"oracle_by_config": out, "note": "samples: config 1 whole (per tensor) or in 16-row slices "
+                      "(1x128); configs 2-5 the first 4096 rows in 128-row slices; per-tensor slices each take their own amax (the oracle's work per "
+                      "element is the same)"}))
+    return 0
+
+
 def run_reference(args):
     rank = env_int("RANK", 0)
     if rank != 0:
@@ -1061,9 +1152,14 @@ def main():
     ap.add_argument("--probe-time", type=int, default=0, metavar="K",
                     help="with --traffic-probe: also time K graph-replayed launches of the probed kernel(s)")
     ap.add_argument("--lib", default=None, help="with --traffic-probe: a variant build of the library")
+    ap.add_argument("--oracle-by-config", action="store_true",
+                    help="time the CPU oracle on a sample of each configuration (host only)")
+    ap.add_argument("--oracle-budget-s", type=float, default=1.5, help="seconds per leg of --oracle-by-config")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.oracle_by_config:
+        return oracle_by_config(args)
     if args.traffic_probe:
         return traffic_probe(args)
     if args.impl == "reference":

@@ -43,7 +43,7 @@ constexpr int kWarps = kThreads / 32;
 // Cast of one lane vector with a scale per element (column scales): cs[e] is
 // the scale of element e, read from shared memory pair by pair.
 // {cs[2p], cs[2p+1]} as packed fp32 operands (one 8-byte shared load).
-__device__ __forceinline__ uint64_t pair(const float* cs, int p) {
+[[maybe_unused]] __device__ __forceinline__ uint64_t pair(const float* cs, int p) {
     const float2 s = reinterpret_cast<const float2*>(cs)[p];
     return f32x2(s.x, s.y);
 }
@@ -62,6 +62,17 @@ struct PairCast<uint16_t, BYTES> {
                    (scale_cast_bf16x2<FMT>(v.w[2 * k + 1], pair(cs, 2 * k + 1)) << 16);
         return CodeWords<V::kWords / 2>::make(c);
     }
+    // the same with the pairs already in registers: s2[p] = {cs[2p], cs[2p+1]}
+    template <int FMT>
+    static __device__ __forceinline__ typename V::Out cast_regs(const typename V::In& v,
+                                                                const uint64_t (&s2)[V::kElems / 2]) {
+        uint32_t c[V::kWords / 2];
+#pragma unroll
+        for (int k = 0; k < V::kWords / 2; ++k)
+            c[k] = scale_cast_bf16x2<FMT>(v.w[2 * k], s2[2 * k]) |
+                   (scale_cast_bf16x2<FMT>(v.w[2 * k + 1], s2[2 * k + 1]) << 16);
+        return CodeWords<V::kWords / 2>::make(c);
+    }
 };
 template <int BYTES>
 struct PairCast<float, BYTES> {
@@ -73,6 +84,16 @@ struct PairCast<float, BYTES> {
         for (int k = 0; k < V::kWords / 4; ++k)
             c[k] = scale_cast_f32x2<FMT>(v.w[4 * k], v.w[4 * k + 1], pair(cs, 2 * k)) |
                    (scale_cast_f32x2<FMT>(v.w[4 * k + 2], v.w[4 * k + 3], pair(cs, 2 * k + 1)) << 16);
+        return CodeWords<V::kWords / 4>::make(c);
+    }
+    template <int FMT>
+    static __device__ __forceinline__ typename V::Out cast_regs(const typename V::In& v,
+                                                                const uint64_t (&s2)[V::kElems / 2]) {
+        uint32_t c[V::kWords / 4];
+#pragma unroll
+        for (int k = 0; k < V::kWords / 4; ++k)
+            c[k] = scale_cast_f32x2<FMT>(v.w[4 * k], v.w[4 * k + 1], s2[2 * k]) |
+                   (scale_cast_f32x2<FMT>(v.w[4 * k + 2], v.w[4 * k + 3], s2[2 * k + 1]) << 16);
         return CodeWords<V::kWords / 4>::make(c);
     }
 };
@@ -124,18 +145,25 @@ struct ColMax<float, BYTES> {
 // MODE 0: 1x128 blocks (row scales for q, column scales for qt);
 // MODE 1: 128x128 blocks (one scale per tile for both).
 // 1x128 reads its tile a second time, from L2, for the column cast instead
-// of holding it in registers across the two barriers of the column pass;
-// with that (and the row scales' divisions shared among a row's lanes) the
-// kernel fits the register cap of 4 CTAs per SM without spilling (bf16; an
-// fp32 tile is twice the registers and keeps the cap of 2).  Measured
-// on B200, bf16 activations 16384x7168, 1x128: 4954 GB/s holding the tile
-// with a cap of 2 CTAs; with the second read 4598 / 5162 / 5213 GB/s for 2 /
-// 3 / 4 CTAs.  128x128: 6462 GB/s (98.7 % of the copy peak) with 3 or 4 CTAs.
+// of holding it in registers through the row pass and the column pass; with
+// that (and the row scales' divisions shared among a row's lanes) the kernel
+// fits the register cap of 4 CTAs per SM without spilling (bf16; an fp32
+// tile is twice the registers and keeps the cap of 2).  Measured on B200,
+// bf16 activations 16384x7168, 1x128: 4954 GB/s holding the tile with a cap
+// of 2 CTAs (4544 with a cap of 3); with the second read issued after the
+// column pass's barriers 4598 / 5162 / 5210 GB/s for caps of 2 / 3 / 4 CTAs,
+// and 5437 GB/s with it issued before them (RELOAD 2), so that the loads are
+// in flight across the barriers.  The column cast takes this lane's 16
+// column scales into registers once (SCALE_REGS).  128x128: 6462 GB/s
+// (98.7 % of the copy peak) with 3 or 4 CTAs.
 #ifndef FP8Q_BT_TMA
 #define FP8Q_BT_TMA 0
 #endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_RELOAD
-#define FP8Q_BLOCK_TRANSPOSE_RELOAD 1
+#define FP8Q_BLOCK_TRANSPOSE_RELOAD 2
+#endif
+#ifndef FP8Q_BLOCK_TRANSPOSE_SCALE_REGS
+#define FP8Q_BLOCK_TRANSPOSE_SCALE_REGS 1
 #endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
 #define FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS 4
@@ -199,6 +227,11 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
             if (i % G::kVecPerRow == vec_in_row) mine = ra[i];
         const float s_mine = scale_from_amax<FMT>(mine);
         const int group = lane - vec_in_row;  // first lane of this row
+#if FP8Q_BLOCK_TRANSPOSE_RELOAD == 3
+        // qt's column maxima first; then each row is cast to q and its registers
+        // reloaded from L2 at once, so the reloads start as early as they can
+        ColMax<T, BYTES>::run(v, lane < G::kVecPerRow, &part[warp][vec_in_row * V::kElems]);
+#endif
 #pragma unroll
         for (int i = 0; i < G::kLoads; ++i) {
             const float s = __shfl_sync(0xFFFFFFFFu, s_mine, group + i % G::kVecPerRow);
@@ -206,9 +239,20 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
             st_stream(reinterpret_cast<typename V::Out*>(q + (r0 + lr) * cols + c0) + vec_in_row,
                       V::template cast<FMT>(v[i], f32x2(s, s)));
             if (vec_in_row == 0) scales[(r0 + lr) * tiles_c + tc] = s;
+#if FP8Q_BLOCK_TRANSPOSE_RELOAD == 3
+            v[i] = ld_words_stream(xv + i * vstride);
+#endif
         }
+#if FP8Q_BLOCK_TRANSPOSE_RELOAD != 3
         // qt: one scale per tile column
         ColMax<T, BYTES>::run(v, lane < G::kVecPerRow, &part[warp][vec_in_row * V::kElems]);
+#endif
+#if FP8Q_BLOCK_TRANSPOSE_RELOAD == 2
+        // the tile again, from L2, issued now so that the loads are in flight
+        // across the two barriers of the column pass
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
+#endif
         __syncthreads();
         if (threadIdx.x < kTT) {
             const int c = threadIdx.x;
@@ -221,23 +265,41 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
         }
         __syncthreads();
         const float* cs = col_scale + vec_in_row * V::kElems;
-#if FP8Q_BLOCK_TRANSPOSE_RELOAD
+#if FP8Q_BLOCK_TRANSPOSE_RELOAD == 1
         // the tile again, from L2 (it was read a moment ago), instead of
         // holding it in registers across the two barriers above
 #pragma unroll
         for (int i = 0; i < G::kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
 #endif
+#if FP8Q_BLOCK_TRANSPOSE_SCALE_REGS
+        // this lane's column scales are the same for all its rows: into registers once, as packed pairs
+        uint64_t cs2[V::kElems / 2];
+#pragma unroll
+        for (int p4 = 0; p4 < V::kElems / 4; ++p4) {
+            const float4 c4 = reinterpret_cast<const float4*>(cs)[p4];
+            cs2[2 * p4] = f32x2(c4.x, c4.y);
+            cs2[2 * p4 + 1] = f32x2(c4.z, c4.w);
+        }
+#pragma unroll
+        for (int i = 0; i < G::kLoads; ++i) {
+            const int lr = lr0 + i * G::kRowsPerLoad;
+            *reinterpret_cast<typename V::Out*>(tile + tile_off(lr, vec_in_row * V::kElems)) =
+                PairCast<T, BYTES>::template cast_regs<FMT>(v[i], cs2);
+        }
+#else
 #pragma unroll
         for (int i = 0; i < G::kLoads; ++i) {
             const int lr = lr0 + i * G::kRowsPerLoad;
             *reinterpret_cast<typename V::Out*>(tile + tile_off(lr, vec_in_row * V::kElems)) =
                 PairCast<T, BYTES>::template cast<FMT>(v[i], cs);
         }
+#endif
     }
     __syncthreads();
     tile_transpose_out(tile, qt, rows, r0, c0, lane, warp);
 }
 
+#if FP8Q_BT_TMA
 // ---------------------------------------------------------------------------
 // 1x128 blocks of bf16 x and x^T, TMA-staged and persistent: the measured
 // alternative to the register-tile kernel above, compiled in only with
@@ -434,6 +496,7 @@ cudaError_t launch_bt_tma(const void* x, int64_t rows, int64_t cols, uint8_t* q,
     if (e == cudaSuccess) *launched = true;
     return e;
 }
+#endif  // FP8Q_BT_TMA
 
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
