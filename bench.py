@@ -684,6 +684,32 @@ def modes_breakdown(dev, stream, peak):
             "grouped step")], 16, dev))
     del gx_, gq_, gst_, gws_, garr
 
+    # many small per-tensor current-scaling casts: 128 bf16 tensors of 2^20 elements, E4M3, each with its own
+    # amax and scale; one fp8_quantize_per_tensor call per tensor against one grouped call (3 launches)
+    from fine_grained_block_b200.binding import FP8CurrentTensor
+    cx_ = [inputs.random_matrix(1, 1 << 20, seed=500 + i, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e3,
+                                device=dev).reshape(-1) for i in range(128)]
+    cq_ = [torch.empty(1 << 20, dtype=torch.uint8, device=dev) for _ in cx_]
+    cs_ = torch.empty(len(cx_), dtype=torch.float32, device=dev)
+    ca_ = torch.empty(len(cx_), dtype=torch.float32, device=dev)
+    carr = (FP8CurrentTensor * len(cx_))(*[FP8CurrentTensor(x_.data_ptr(), q_.data_ptr(), x_.numel(),
+                                                            cs_[i:i + 1].data_ptr(), ca_[i:i + 1].data_ptr())
+                                           for i, (x_, q_) in enumerate(zip(cx_, cq_))])
+    cnb = 3 * sum(x_.numel() for x_ in cx_)
+
+    def current_one_by_one(r, st):
+        for i, (x_, q_) in enumerate(zip(cx_, cq_)):
+            raw.check(L.fp8_quantize_per_tensor(x_.data_ptr(), 1, x_.numel(), 0, None, q_.data_ptr(),
+                                                cs_[i:i + 1].data_ptr(), ca_[i:i + 1].data_ptr(), st), "per-tensor")
+    put("128_tensors_2^20_per_tensor_current_e4m3_one_call_each", "128 bf16 tensors of 2^20 elements, N(0,1) with "
+        "0.1% x1e3, seeds 500..627 (128 x 3 launches; alg bytes 3/elem)", cnb, time_in_graph([current_one_by_one], 4,
+                                                                                           dev))
+    put("128_tensors_2^20_per_tensor_current_e4m3_grouped", "the same 128 tensors in one "
+        "fp8_quantize_per_tensor_grouped call (3 launches; alg bytes 3/elem)", cnb, time_in_graph([
+            lambda r, st: raw.check(L.fp8_quantize_per_tensor_grouped(carr, len(cx_), 1, 0, st), "grouped current")],
+            16, dev))
+    del cx_, cq_, cs_, ca_, carr
+
     # size sweep 2^20 .. 2^30 elements (bf16, 0.1% x1e3 outliers, seed 4): GB/s per mode and size.  Sizes
     # whose buffers fit in L2 rotate over enough copies that every launch reads from HBM.
     sweep = {}

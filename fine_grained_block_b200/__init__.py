@@ -13,6 +13,7 @@ _BINDING_NAMES = (
     "fp8_quantize_mx", "fp8_dequantize_mx", "MX_FIT", "MX_OCP", "fp8_quantize_per_tensor_transpose", "fp8_quantize_blockwise_transpose",
     "fp8_gemm_blockwise", "fp8_quantize_delayed_step", "DelayedScaler",
     "fp8_quantize_blockwise_grouped", "FP8BlockTensor", "fp8_quantize_delayed_step_grouped", "FP8DelayedTensor",
+    "fp8_quantize_per_tensor_grouped", "FP8CurrentTensor",
     "E4M3", "E5M2", "F32", "BF16",
 )
 

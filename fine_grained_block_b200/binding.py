@@ -33,6 +33,12 @@ class FP8BlockTensor(ctypes.Structure):
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
+class FP8CurrentTensor(ctypes.Structure):
+    """struct fp8_current_tensor of include/fp8q.h."""
+    _fields_ = [("x", ctypes.c_void_p), ("q", ctypes.c_void_p), ("n", ctypes.c_int64),
+                ("scale_out", ctypes.c_void_p), ("amax_out", ctypes.c_void_p)]
+
+
 class FP8DelayedTensor(ctypes.Structure):
     """struct fp8_delayed_tensor of include/fp8q.h."""
     _fields_ = [("x", ctypes.c_void_p), ("q", ctypes.c_void_p), ("n", ctypes.c_int64), ("scale", ctypes.c_void_p),
@@ -68,6 +74,7 @@ SIGNATURES = {
                                                 _c_int, _vp]),
     "fp8_quantize_delayed_step_grouped": (_c_int, [ctypes.POINTER(FP8DelayedTensor), _c_int, _c_int, _c_int, _c_int,
                                                    _c_int, ctypes.c_float, ctypes.c_float, _vp, _vp]),
+    "fp8_quantize_per_tensor_grouped": (_c_int, [ctypes.POINTER(FP8CurrentTensor), _c_int, _c_int, _c_int, _vp]),
     "fp8_status_string": (ctypes.c_char_p, [_c_int]),
     "fp8_device_status": (_c_int, [_vp, _c_int, _vp]),
     "fp8_selftest_wait_timeout": (_c_int, [ctypes.c_uint32, _vp]),
@@ -465,6 +472,29 @@ def fp8_quantize_delayed_step_grouped(xs, scalers, qs=None, workspace: torch.Ten
                                                           _stream(stream))
     _check("fp8_quantize_delayed_step_grouped", st)
     return qs
+
+
+def fp8_quantize_per_tensor_grouped(xs, fmt: int = E4M3, qs=None, scales=None, amaxes=None, stream=None):
+    """Per-tensor current scaling of several tensors in three launches per 128 tensors: each tensor gets
+    its own amax and scale, exactly as from fp8_quantize_per_tensor(x, fmt).  Returns (codes, scales, amaxes),
+    lists of CUDA tensors (codes in each x's shape, scales and amaxes of one element)."""
+    xs = list(xs)
+    if not xs:
+        return [], [], []
+    dt = xs[0].dtype
+    dev = xs[0].device
+    qs = [torch.empty(x.shape, dtype=torch.uint8, device=x.device) for x in xs] if qs is None else list(qs)
+    scales = [torch.empty(1, dtype=torch.float32, device=dev) for _ in xs] if scales is None else list(scales)
+    amaxes = [torch.empty(1, dtype=torch.float32, device=dev) for _ in xs] if amaxes is None else list(amaxes)
+    arr = (FP8CurrentTensor * len(xs))()
+    for i, (x, q, s_, a_) in enumerate(zip(xs, qs, scales, amaxes)):
+        _need_cuda(x, q, s_, a_)
+        if x.dtype != dt:
+            raise ValueError("grouped tensors must share one dtype")
+        arr[i] = FP8CurrentTensor(_ptr(x), _ptr(q), x.numel(), _ptr(s_), _ptr(a_))
+    st = load_library().fp8_quantize_per_tensor_grouped(arr, len(xs), _DTYPE_CODE[dt], fmt, _stream(stream))
+    _check("fp8_quantize_per_tensor_grouped", st)
+    return qs, scales, amaxes
 
 
 class DelayedScaler:

@@ -402,6 +402,25 @@ int fp8_quantize_delayed_step_grouped(const fp8_delayed_tensor* tensors, int cou
                                                               workspace, static_cast<cudaStream_t>(stream)));
 }
 
+int fp8_quantize_per_tensor_grouped(const fp8_current_tensor* tensors, int count, int dtype, int fmt, void* stream) {
+    if (!fmt_ok(fmt)) return FP8_ERR_FORMAT;
+    if (!dtype_ok(dtype)) return FP8_ERR_DTYPE;
+    if (count < 0) return FP8_ERR_ARG;
+    if (count == 0) return FP8_OK;
+    if (tensors == nullptr) return FP8_ERR_NULL;
+    for (int i = 0; i < count; ++i) {
+        const fp8_current_tensor& t = tensors[i];
+        if (t.n < 0 || t.n > (INT64_MAX >> 4)) return FP8_ERR_SHAPE;
+        if (t.scale_out == nullptr || t.amax_out == nullptr) return FP8_ERR_NULL;
+        if (t.n > 0 && (t.x == nullptr || t.q == nullptr)) return FP8_ERR_NULL;
+        if (!aligned(t.x, 16) || !aligned(t.q, 16) || !aligned(t.scale_out, 4) || !aligned(t.amax_out, 4))
+            return FP8_ERR_ALIGN;
+    }
+    static_assert(sizeof(fp8_current_tensor) == sizeof(fp8q::CurrentTensor), "descriptor layouts must agree");
+    return status_of(fp8q::launch_tensor_current_grouped(reinterpret_cast<const fp8q::CurrentTensor*>(tensors), count,
+                                                         dtype, fmt, static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_device_status(uint32_t* status, int clear, void* stream) {
     if (status == nullptr) return FP8_ERR_NULL;
     if (!aligned(status, 4)) return FP8_ERR_ALIGN;

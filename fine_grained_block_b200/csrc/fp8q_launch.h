@@ -139,6 +139,18 @@ cudaError_t launch_tensor_delayed_step_grouped(const DelayedTensor* tensors, int
                                                int algo, float alpha, float margin, void* workspace,
                                                cudaStream_t stream);
 
+// Per-tensor current scaling of many tensors: zero every amax_out, one amax
+// pass and one cast pass over all of them (up to 128 tensors per launch).
+struct CurrentTensor {
+    const void* x;
+    uint8_t* q;
+    int64_t n;
+    float* scale_out;
+    float* amax_out;
+};
+cudaError_t launch_tensor_current_grouped(const CurrentTensor* tensors, int count, int dtype, int fmt,
+                                          cudaStream_t stream);
+
 // Fused quantize -> dequantize round trip in x's dtype.  block_rows 0: per
 // tensor with *scale_in; 1 or 128: block scales (written to `scales` if it is
 // non-null).

@@ -252,6 +252,95 @@ k_tensor_cast_delayed_step_grouped(const __grid_constant__ StepTable tab) {
                                     tab.ws + lo, b - tab.start[lo], tab.start[lo + 1] - tab.start[lo]);
 }
 
+// Per-tensor current scaling of many tensors in three launches: every
+// tensor's amax_out is cleared, then one amax pass and one cast pass run over
+// all tensors' chunks, numbered consecutively across the group (a CTA finds
+// its tensor by binary search over the start indices, which travel in the
+// kernel parameters with the descriptors).  Each tensor keeps its own amax and
+// scale; the per-CTA work is that of k_tensor_amax and k_tensor_cast, and the
+// cast pass again takes the chunks last-to-first.
+constexpr int kCurGroupMax = 128;  // tensors per launch (a 6.2 KiB parameter block)
+
+struct CurTable {
+    int count;
+    int64_t start[kCurGroupMax + 1];
+    CurrentTensor e[kCurGroupMax];
+};
+static_assert(sizeof(CurTable) <= 16384, "the grouped parameter block must stay well inside 32 KiB");
+
+__device__ __forceinline__ int find_tensor(const CurTable& tab, int64_t b) {
+    int lo = 0, hi = tab.count;  // start[lo] <= b < start[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tab.start[mid] <= b) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+__global__ void k_zero_group_amax(const __grid_constant__ CurTable tab) {
+    pdl_enter();
+    for (int i = threadIdx.x; i < tab.count; i += blockDim.x) *tab.e[i].amax_out = 0.0f;
+}
+
+template <typename T, int BYTES>
+__global__ void __launch_bounds__(kThreads) k_tensor_amax_grouped(const __grid_constant__ CurTable tab) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    const int t = find_tensor(tab, blockIdx.x);
+    const CurrentTensor& e = tab.e[t];
+    const int64_t nvec = e.n / V::kElems;
+    const int tail_n = static_cast<int>(e.n - nvec * V::kElems);
+    const int64_t chunk = static_cast<int64_t>(blockIdx.x) - tab.start[t];
+    const auto* x = static_cast<const typename V::In*>(e.x);
+    const int64_t base = chunk * kThreads * kUnroll + threadIdx.x;
+    typename V::In v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * kThreads;
+        v[u] = (i < nvec) ? ld_words_stream(x + i) : V::zero();
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) a = fmaxf(a, V::amax(v[u]));
+    if (chunk == 0 && threadIdx.x < tail_n)
+        a = fmaxf(a, fabsf(load_scalar(static_cast<const T*>(e.x) + nvec * V::kElems, threadIdx.x)));
+    cta_amax_to_global(a, e.amax_out);
+}
+
+template <typename T, int FMT, int BYTES>
+__global__ void __launch_bounds__(kThreads) k_tensor_cast_grouped(const __grid_constant__ CurTable tab) {
+    pdl_enter();
+    using V = LaneVec<T, BYTES>;
+    const int64_t b = tab.start[tab.count] - 1 - blockIdx.x;  // last-to-first
+    const int t = find_tensor(tab, b);
+    const CurrentTensor& e = tab.e[t];
+    const int64_t nvec = e.n / V::kElems;
+    const int tail_n = static_cast<int>(e.n - nvec * V::kElems);
+    const int64_t chunk = b - tab.start[t];
+    const auto* x = static_cast<const typename V::In*>(e.x);
+    auto* q = reinterpret_cast<typename V::Out*>(e.q);
+    const int64_t base = chunk * kThreads * kUnroll + threadIdx.x;
+    typename V::In v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * kThreads;
+        v[u] = (i < nvec) ? ld_words_stream(x + i) : V::zero();
+    }
+    const float s = scale_from_amax<FMT>(*e.amax_out);
+    const uint64_t s2 = f32x2(s, s);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * kThreads;
+        if (i < nvec) st_stream(q + i, V::template cast<FMT>(v[u], s2));
+    }
+    if (chunk == 0 && threadIdx.x < tail_n) {
+        const float xv = load_scalar(static_cast<const T*>(e.x) + nvec * V::kElems, threadIdx.x);
+        e.q[nvec * V::kElems + threadIdx.x] = static_cast<uint8_t>(cvt_fp8x2<FMT>(__fmul_rn(xv, s), 0.0f) & 0xFFu);
+    }
+    if (chunk == 0 && threadIdx.x == 0) *e.scale_out = s;
+}
+
 // ---------------------------------------------------------------------------
 // Per-tensor cast with a second, transposed output: q [R, C] (optional) and
 // qt [C, R] with qt[c][r] = q[r][c] -- the copy a weight-gradient GEMM reads
@@ -536,6 +625,52 @@ cudaError_t launch_tensor_delayed_step_grouped(const DelayedTensor* t, int count
                    : delayed_grouped_width<uint16_t, kE5M2>(t, count, window, algo, alpha, margin, workspace, st);
     return fmt == kE4M3 ? delayed_grouped_width<float, kE4M3>(t, count, window, algo, alpha, margin, workspace, st)
                         : delayed_grouped_width<float, kE5M2>(t, count, window, algo, alpha, margin, workspace, st);
+}
+
+namespace {
+
+template <typename T, int FMT, int BYTES>
+cudaError_t current_grouped_typed(const CurrentTensor* t, int count, cudaStream_t st) {
+    using V = LaneVec<T, BYTES>;
+    CurTable tab;
+    for (int first = 0; first < count; first += kCurGroupMax) {
+        tab.count = std::min(kCurGroupMax, count - first);
+        int64_t units = 0;
+        for (int i = 0; i < tab.count; ++i) {
+            tab.e[i] = t[first + i];
+            tab.start[i] = units;
+            units += chunk_grid(t[first + i].n / V::kElems);  // at least 1: every tensor's scale is written
+        }
+        tab.start[tab.count] = units;
+        if (units > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        cudaError_t e = launch_kernel(k_zero_group_amax, dim3(1), dim3(kCurGroupMax), 0, st, tab);
+        if (e != cudaSuccess) return e;
+        e = launch_kernel(k_tensor_amax_grouped<T, BYTES>, dim3(static_cast<unsigned>(units)), dim3(kThreads), 0, st,
+                          tab);
+        if (e != cudaSuccess) return e;
+        e = launch_kernel(k_tensor_cast_grouped<T, FMT, BYTES>, dim3(static_cast<unsigned>(units)), dim3(kThreads),
+                          0, st, tab);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T, int FMT>
+cudaError_t current_grouped_width(const CurrentTensor* t, int count, cudaStream_t st) {
+    bool w32 = true;  // 256-bit lanes only when every tensor allows them
+    for (int i = 0; i < count; ++i) w32 = w32 && aligned32(t[i].x);
+    return w32 ? current_grouped_typed<T, FMT, 32>(t, count, st) : current_grouped_typed<T, FMT, 16>(t, count, st);
+}
+
+}  // namespace
+
+cudaError_t launch_tensor_current_grouped(const CurrentTensor* t, int count, int dtype, int fmt, cudaStream_t st) {
+    if (count <= 0) return cudaSuccess;
+    if (dtype == 1)
+        return fmt == kE4M3 ? current_grouped_width<uint16_t, kE4M3>(t, count, st)
+                            : current_grouped_width<uint16_t, kE5M2>(t, count, st);
+    return fmt == kE4M3 ? current_grouped_width<float, kE4M3>(t, count, st)
+                        : current_grouped_width<float, kE5M2>(t, count, st);
 }
 
 cudaError_t launch_tensor_cast_transpose(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,

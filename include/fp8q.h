@@ -527,6 +527,34 @@ int fp8_quantize_delayed_step_grouped(const fp8_delayed_tensor *tensors, int cou
                                       int fmt, int window, int algo, float alpha, float margin,
                                       void *workspace, void *stream);
 
+/*
+ * Per-tensor current scaling (fp8_quantize_per_tensor with scale_in NULL) of
+ * `count` tensors in three launches per 128 tensors, whatever their sizes:
+ * every amax_out is cleared, then one amax pass and one cast pass run over the
+ * chunks of all the tensors.  Each tensor gets its own amax and scale: its
+ * codes, scale_out and amax_out come out exactly as from its own call.  All
+ * tensors share dtype and fmt.  [MP-handbook] "FP8 training" per_tensor;
+ * [FP8-native] s4.1.  For the many small tensors of a training step, whose
+ * single calls are dominated by their fixed cost.
+ *
+ *   tensors    host array of `count` descriptors (read during the call);
+ *              each holds the device pointers of one current-scaling
+ *              fp8_quantize_per_tensor call and its element count n.  The
+ *              scale_out and amax_out words of different tensors must be
+ *              distinct (each amax is cleared, then reduced into atomically).
+ * Errors: those of fp8_quantize_per_tensor with current scaling, for any
+ * tensor; FP8_ERR_ARG for count < 0.
+ */
+typedef struct fp8_current_tensor {
+    const void *x;      /* [n] input */
+    uint8_t *q;         /* [n] codes */
+    int64_t n;
+    float *scale_out;   /* [1] the scale used */
+    float *amax_out;    /* [1] amax(x) */
+} fp8_current_tensor;
+int fp8_quantize_per_tensor_grouped(const fp8_current_tensor *tensors, int count, int dtype, int fmt,
+                                    void *stream);
+
 /* Static, human-readable text for a status code (never NULL). */
 const char *fp8_status_string(int status);
 

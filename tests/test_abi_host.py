@@ -37,7 +37,7 @@ def test_header_declares_the_boundary():
                                            "fp8_selftest_wait_timeout", "fp8_quantize_mx", "fp8_dequantize_mx",
                                            "fp8_quantize_per_tensor_transpose", "fp8_gemm_blockwise",
                                            "fp8_quantize_delayed_step", "fp8_quantize_blockwise_grouped",
-                                           "fp8_quantize_delayed_step_grouped",
+                                           "fp8_quantize_delayed_step_grouped", "fp8_quantize_per_tensor_grouped",
                                            "fp8_quantize_blockwise_transpose", "fp8_gemm_blockwise_ex"])
 
 
@@ -163,6 +163,27 @@ def test_fused_per_tensor_noalloc_validation(L):
     assert f(A16, 1, 16, 0, A16 + 4, A16, A16, None) == ERR_ALIGN
     assert f(A16, 1, 16, 0, A16, A16 + 2, A16, None) == ERR_ALIGN
     assert f(A16, 1, 16, 0, A16, A16, A16 + 1, None) == ERR_ALIGN
+
+
+def test_per_tensor_grouped_validation(L):
+    from fine_grained_block_b200.binding import FP8CurrentTensor
+    f = L.fp8_quantize_per_tensor_grouped
+
+    def arr(*ts):
+        return (FP8CurrentTensor * len(ts))(*ts)
+    good = FP8CurrentTensor(A16, A16, 16, A16, A16)
+    assert f(arr(good), 1, 1, 9, None) == ERR_FORMAT
+    assert f(arr(good), 1, 7, 0, None) == ERR_DTYPE
+    assert f(arr(good), -1, 1, 0, None) == ERR_ARG
+    assert f(None, 0, 1, 0, None) == OK          # nothing to do
+    assert f(None, 2, 1, 0, None) == ERR_NULL
+    assert f(arr(good, FP8CurrentTensor(A16, A16, -1, A16, A16)), 2, 1, 0, None) == ERR_SHAPE
+    assert f(arr(good, FP8CurrentTensor(A16, A16, 16, None, A16)), 2, 1, 0, None) == ERR_NULL
+    assert f(arr(good, FP8CurrentTensor(A16, A16, 16, A16, None)), 2, 1, 0, None) == ERR_NULL
+    assert f(arr(good, FP8CurrentTensor(None, A16, 16, A16, A16)), 2, 1, 0, None) == ERR_NULL
+    assert f(arr(good, FP8CurrentTensor(A16 + 8, A16, 16, A16, A16)), 2, 1, 0, None) == ERR_ALIGN
+    assert f(arr(good, FP8CurrentTensor(A16, A16 + 4, 16, A16, A16)), 2, 1, 0, None) == ERR_ALIGN
+    assert f(arr(good, FP8CurrentTensor(A16, A16, 16, A16 + 2, A16)), 2, 1, 0, None) == ERR_ALIGN
 
 
 def test_amax_and_scale_validation(L):

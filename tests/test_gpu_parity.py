@@ -756,6 +756,35 @@ def test_grouped_matches_oracle(fmt, dtype, block):
 
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_grouped_current_scaling_matches_oracle(fmt, dtype):
+    """fp8_quantize_per_tensor_grouped over 140 tensors (more than one launch of 128; empty, one-element,
+    ragged and multi-chunk ones; outlier magnitudes that differ per tensor) == the oracle's current scaling
+    of each tensor on its own, codes, scale and amax bit for bit, twice in a row (the amax outputs are
+    cleared by the call, whatever they held), with 16- and 32-byte lanes."""
+    sizes = [0, 1, 7, 4097, 1 << 16, (1 << 20) + 3] + [1000 * (i + 1) + (i % 9) for i in range(134)]
+    xs_cpu = [inputs.random_matrix(1, max(n, 1), seed=9500 + i, dtype=dtype, outlier_frac=1e-3,
+                                   factor=10.0 ** (i % 5)).reshape(-1)[:n] for i, n in enumerate(sizes)]
+    refs = [oracle.quantize_per_tensor(host_input(x), fmt) for x in xs_cpu]
+    xs = [to_cuda(x) for x in xs_cpu]
+    # one tensor 16- but not 32-byte aligned: the whole group takes 16-byte lanes
+    esz = xs_cpu[4].element_size()
+    buf = torch.empty(xs_cpu[4].numel() + 16 // esz, dtype=dtype, device="cuda")
+    x16 = buf[16 // esz:]
+    x16.copy_(xs_cpu[4].to("cuda"))
+    for lanes, group in (("32-byte", xs), ("16-byte", xs[:4] + [x16] + xs[5:])):
+        amaxes = [torch.full((1,), 1e30, dtype=torch.float32, device="cuda") for _ in xs]  # stale values
+        for call in range(2):
+            qs, ss, aa = B.fp8_quantize_per_tensor_grouped(group, fmt, amaxes=amaxes)
+            torch.cuda.synchronize()
+            for i, (oq, os_, oa) in enumerate(refs):
+                what = f"{lanes} call {call} tensor {i}"
+                assert_bytes_equal(aa[i], fp32_bits([oa]), what + " amax")
+                assert_bytes_equal(ss[i], fp32_bits([os_]), what + " scale")
+                assert_bytes_equal(qs[i], oq, what + " codes")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("algo,alpha,margin,window", [(0, 1.0, 1.0, 3), (1, 0.5, 1.1, 2)])
 def test_grouped_delayed_steps_match_single_calls_and_oracle(fmt, dtype, algo, alpha, margin, window):
     """fp8_quantize_delayed_step_grouped over 140 tensors (more than one launch of 128, with empty and ragged
