@@ -120,6 +120,11 @@ struct Split {
 };
 static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the register file");
 
+// Tile order: -1 picks per call (row tile fastest when M < N), 0 column tile
+// fastest, 1 row tile fastest.
+#ifndef FP8Q_GEMM_RASTER
+#define FP8Q_GEMM_RASTER -1
+#endif
 // 1x128 B: the fill's 16-byte scale loads, and packed f32x2 promotion arithmetic.
 #ifndef FP8Q_GEMM_FILL_VEC4
 #define FP8Q_GEMM_FILL_VEC4 1
@@ -170,7 +175,7 @@ template <int OUT, bool PAIR, int BROW>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const float* __restrict__ sa, const float* __restrict__ sb, void* __restrict__ c, int64_t M,
-                 int64_t N, int64_t K, uint32_t idesc, unsigned int* status) {
+                 int64_t N, int64_t K, uint32_t idesc, unsigned int* status, int row_fastest) {
     using C = Cfg<PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,9 +186,15 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const int lane = threadIdx.x & 31;
     const uint32_t rank = PAIR ? umma::cluster_ctarank() : 0u;  // 0: this CTA issues the MMAs
     // Persistent: this CTA (pair) takes tiles first, first + step, ...; a tile is
-    // C::kTileM rows x kBN columns, numbered with the column tile fastest.
+    // C::kTileM rows x kBN columns, numbered with the column tile fastest, or
+    // with the row tile fastest when row_fastest is set (the host picks the
+    // order in which the operand that every wave of tiles reads whole is the
+    // smaller one, so that it stays in L2 from one wave to the next).
     const int64_t tiles_n = N / kBN;
-    const int64_t tiles = ((M + C::kTileM - 1) / C::kTileM) * tiles_n;
+    const int64_t tiles_m = (M + C::kTileM - 1) / C::kTileM;
+    const int64_t tiles = tiles_m * tiles_n;
+    auto tile_row = [&](int64_t t) { return row_fastest ? t % tiles_m : t / tiles_n; };
+    auto tile_col = [&](int64_t t) { return row_fastest ? t / tiles_m : t % tiles_n; };
     const int64_t first = PAIR ? blockIdx.x / 2 : blockIdx.x;
     const int64_t step = PAIR ? gridDim.x / 2 : gridDim.x;
     const int nchunks = static_cast<int>(K / kBK);
@@ -226,8 +237,8 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         if (lane == 0) {
             uint32_t g = 0;
             for (int64_t t = first; t < tiles && !timed_out; t += step) {
-                const int m0 = static_cast<int>((t / tiles_n) * C::kTileM + rank * kBM);
-                const int n0 = static_cast<int>((t % tiles_n) * kBN);
+                const int m0 = static_cast<int>(tile_row(t) * C::kTileM + rank * kBM);
+                const int n0 = static_cast<int>(tile_col(t) * kBN);
                 for (int kc = 0; kc < nchunks; ++kc, ++g) {
                     const uint32_t s = g % C::kStages;
                     const uint32_t phase = (g / C::kStages) & 1u;
@@ -307,7 +318,7 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                           (reinterpret_cast<uintptr_t>(sb) & 15u) == 0;
         uint32_t g = 0;
         for (int64_t t = first; t < tiles && !timed_out; t += step) {
-            const float* sb_cols = sb + ((t % tiles_n) * kBN) * kc_stride;
+            const float* sb_cols = sb + (tile_col(t) * kBN) * kc_stride;
             for (int kc0 = 0; kc0 < nchunks && !timed_out; kc0 += kRbGroup) {
                 const int cnt = min(kRbGroup, nchunks - kc0);
                 float v[kRbGroup][kBN / 64];
@@ -357,8 +368,8 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
         uint32_t g = 0;
         for (int64_t t = first; t < tiles && !timed_out; t += step) {
-            const int64_t m = (t / tiles_n) * C::kTileM + rank * kBM + row;
-            const int64_t col0 = (t % tiles_n) * kBN + half * 128;
+            const int64_t m = tile_row(t) * C::kTileM + rank * kBM + row;
+            const int64_t col0 = tile_col(t) * kBN + half * 128;
             const float* sa_row = sa + (m < M ? m : 0) * kc_stride;
             const float* sb_row = sb + (BROW == 1 ? 0 : (col0 >> 7) * kc_stride);
             float acc[128];
@@ -550,7 +561,13 @@ cudaError_t launch_typed(const CUtensorMap& map_a, const CUtensorMap& map_b, con
     }
     const int64_t ctas = std::min<int64_t>(tiles, units) * (PAIR ? 2 : 1);
     cfg.gridDim = dim3(static_cast<unsigned>(ctas));
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, sa, sb, c, M, N, K, idesc, status);
+#if FP8Q_GEMM_RASTER < 0
+    const int row_fastest = M < N ? 1 : 0;  // each wave reads all of A (row fastest) or all of B
+#else
+    const int row_fastest = FP8Q_GEMM_RASTER;
+#endif
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, kern, map_a, map_b, sa, sb, c, M, N, K, idesc, status, row_fastest);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

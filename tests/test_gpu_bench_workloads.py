@@ -4,6 +4,7 @@
 - the transposing per-tensor cast of the same activations, delayed (given scale) and current;
 - 1x128 quantization of the same activations and of their transpose in one pass;
 - the blockwise GEMM at 16384x4096x7168: the whole last 256-row tile row of C and sampled rows;
+- the weight-gradient GEMM at 4096x7168x16384 (B in 1x128 blocks): whole sampled rows of dW;
 - 128 weights of 1024x1024 in one grouped 128x128 call;
 - one grouped delayed-scaling step over 128 gradients of 2^20 elements.
 
@@ -83,6 +84,27 @@ def test_gemm_16384x4096x7168_full_last_tile_row_and_sampled_rows():
     mag = oracle_gemm(qa[rows] & 0x7F, sa[rows], oracle.E4M3, qb & 0x7F, sb, oracle.E4M3)
     got = c[torch.as_tensor(rows, device="cuda")].float().cpu().numpy().astype(np.float64)
     # fp32 sums of 56 promoted chunks (2^-12 of the absolute sum), then one bf16 rounding of the result
+    tol = 2.0 ** -12 * mag + 2.0 ** -8 * np.abs(want)
+    bad = np.abs(got - want) > tol
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} sampled outputs outside the bound"
+
+
+def test_weight_gradient_gemm_4096x7168x16384_sampled_rows():
+    """The benchmark's weight-gradient GEMM shape (B in 1x128 blocks, E5M2 x E4M3; M < N, so the row tile
+    is fastest): whole rows of dW from every row tile, against the oracle."""
+    M, N, K = 4096, 7168, 16384
+    dyt = inputs.random_matrix(M, K, seed=8, dtype=torch.bfloat16, scale=1e-3, outlier_frac=1e-3, factor=1e2)
+    xt = inputs.random_matrix(N, K, seed=9, dtype=torch.bfloat16, outlier_frac=1e-3, factor=1e2)
+    qa, sa = oracle_blockwise(host_input(dyt), 1, 128, oracle.E5M2)
+    qb, sb = oracle_blockwise(host_input(xt), 1, 128, oracle.E4M3)
+    c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
+                             to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), a_fmt=B.E5M2,
+                             b_fmt=B.E4M3, out_dtype=torch.bfloat16, b_block=1)
+    torch.cuda.synchronize()
+    rows = [0, 255, 256, 1000, 2047, 2048, 3333, 4095]
+    want = oracle_gemm(qa[rows], sa[rows], oracle.E5M2, qb, sb, oracle.E4M3, b_block=1)
+    mag = oracle_gemm(qa[rows] & 0x7F, sa[rows], oracle.E5M2, qb & 0x7F, sb, oracle.E4M3, b_block=1)
+    got = c[torch.as_tensor(rows, device="cuda")].float().cpu().numpy().astype(np.float64)
     tol = 2.0 ** -12 * mag + 2.0 ** -8 * np.abs(want)
     bad = np.abs(got - want) > tol
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} sampled outputs outside the bound"

@@ -102,6 +102,25 @@ def test_gemm_large_sampled_rows():
     check_gemm(qa, sa, B.E4M3, qb, sb, B.E4M3, c, "4096^3 sampled rows", rows=rows)
 
 
+@pytest.mark.parametrize("b_block", [128, 1])
+def test_gemm_more_tiles_than_pairs_row_tile_order(b_block):
+    """M < N: the persistent CTA pairs take the tiles with the row tile fastest.  1024 x 8192 is 4 x 32 =
+    128 pair tiles, more than the 74 pairs, so pairs take several tiles; sampled rows cover every row tile
+    and every column tile."""
+    M, N, K = 1024, 8192, 256
+    x = inputs.random_matrix(M, K, seed=5150 + b_block, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e2)
+    w = inputs.random_matrix(N, K, seed=5160 + b_block, dtype=torch.bfloat16, scale=0.02, outlier_frac=0.01,
+                             factor=1e2)
+    qa, sa = oracle.quantize_blockwise(host_input(x), 1, 128, B.E4M3)
+    qb, sb = oracle.quantize_blockwise(host_input(w), b_block, 128, B.E4M3)
+    c = B.fp8_gemm_blockwise(to_cuda(torch.from_numpy(qa)), to_cuda(torch.from_numpy(sa)),
+                             to_cuda(torch.from_numpy(qb)), to_cuda(torch.from_numpy(sb)), out_dtype=torch.float32,
+                             b_block=b_block)
+    torch.cuda.synchronize()
+    rows = [0, 127, 128, 255, 256, 511, 512, 700, 767, 768, 1023]
+    check_gemm(qa, sa, B.E4M3, qb, sb, B.E4M3, c, f"{M}x{N}x{K} B block {b_block}", rows=rows, b_block=b_block)
+
+
 def test_gemm_k_zero_and_empty():
     a = torch.zeros(64, 0, dtype=torch.uint8, device="cuda")
     b = torch.zeros(256, 0, dtype=torch.uint8, device="cuda")
