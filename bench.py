@@ -256,9 +256,10 @@ def cpu_baseline(bits, budget_s: float = 12.0):
 
 
 def oracle_by_config(args):
-    """The CPU oracle's throughput on a sample of each workload in BASELINE's list, single-threaded and over
-    every host core (independent row slices in parallel), in GB/s of the same algorithmic bytes.  Host only;
-    prints one JSON line."""
+    """The CPU oracle's throughput on a sample of each benchmark workload (the handbook's fp32 tensor, the
+    4096^2 weight, the 16384x7168 activations, the 8192^2 gradients, the size sweep's 2^30 tensor),
+    single-threaded and over every host core (independent row slices in parallel), in GB/s of the same
+    algorithmic bytes.  Host only; prints one JSON line."""
     import oracle
     import torch
     from concurrent.futures import ThreadPoolExecutor

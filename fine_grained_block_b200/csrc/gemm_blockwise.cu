@@ -120,6 +120,10 @@ struct Split {
 };
 static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the register file");
 
+// The promotion loads its row's scales one chunk ahead.
+#ifndef FP8Q_GEMM_PREFETCH_SCALES
+#define FP8Q_GEMM_PREFETCH_SCALES 1
+#endif
 // Tile order: -1 picks per call (row tile fastest when M < N), 0 column tile
 // fastest, 1 row tile fastest.
 #ifndef FP8Q_GEMM_RASTER
@@ -375,14 +379,29 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             float acc[128];
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+#if FP8Q_GEMM_PREFETCH_SCALES
+            // this row's scales one chunk ahead, so their load latency is not on the hand-back path
+            float sa_next = (m < M && nchunks > 0) ? __ldg(sa_row) : 1.0f;
+            float sb_next = (BROW != 1 && m < M && nchunks > 0) ? __ldg(sb_row) : 1.0f;
+#endif
             for (int kc = 0; kc < nchunks; ++kc, ++g) {
                 const uint32_t buf = g & 1u;
                 const uint32_t acc_phase = (g >> 1) & 1u;
                 // 128x128 B: 1 / (sa * sb), the dequant factor of this chunk for this row and
                 // column half.  1x128 B: 1 / sa here; 1 / sb per column from the ring.
+#if FP8Q_GEMM_PREFETCH_SCALES
+                const float sa_cur = sa_next, sb_cur = sb_next;
+                if (m < M && kc + 1 < nchunks) {
+                    sa_next = __ldg(sa_row + kc + 1);
+                    if (BROW != 1) sb_next = __ldg(sb_row + kc + 1);
+                }
+                const float f = (m < M) ? (BROW == 1 ? __frcp_rn(sa_cur) : __frcp_rn(__fmul_rn(sa_cur, sb_cur)))
+                                        : 0.0f;
+#else
                 const float f = (m < M) ? (BROW == 1 ? __frcp_rn(__ldg(sa_row + kc))
                                                      : __frcp_rn(__fmul_rn(__ldg(sa_row + kc), __ldg(sb_row + kc))))
                                         : 0.0f;
+#endif
                 const uint32_t slot = g % kRbSlots;
                 if (!umma::mbar_wait(&bars->acc_full[buf], acc_phase, kWaitLimitNs)) {
                     timed_out = true;
