@@ -1056,7 +1056,9 @@ def traffic_probe(args):
     --probe headline   the headline pair (1x128 quantize, dequant) on the 2^n sweep tensor;
     --probe 128x128    128x128 quantize of the 2^n sweep tensor;
     --probe bt1x128    1x128 quantize of x and x^T of the bf16 activations 16384x7168;
-    --probe gemm_fwd / gemm_wgrad   the consumer GEMM (timing; its operands are quantized first).
+    --probe gemm_fwd / gemm_wgrad   the consumer GEMM (timing; its operands are quantized first);
+    --probe gemm_wgrad_e4m3         the weight-gradient shape with both operands E4M3;
+    --probe gemm_wgrad_b128         the weight-gradient shape with B in 128x128 blocks (the forward form).
     --probe-time K     afterwards, also time K back-to-back launches of the probed kernel(s) (not under ncu).
     --lib PATH         use another build of the library (a variant built with tuning macros)."""
     import torch
@@ -1071,19 +1073,20 @@ def traffic_probe(args):
     elif args.probe.startswith("gemm"):
         # the consumer GEMM's operands, quantized by the library: forward (1x128 x 128x128, M N K =
         # 16384 4096 7168) or weight gradient (1x128 x 1x128, E5M2 x E4M3, 4096 7168 16384)
-        wgrad = args.probe == "gemm_wgrad"
+        wgrad = args.probe.startswith("gemm_wgrad")
         Mg, Ng, Kg = (4096, 7168, 16384) if wgrad else (16384, 4096, 7168)
+        a_fmt = 1 if args.probe == "gemm_wgrad" else 0  # gemm_wgrad_e4m3: both operands E4M3
         xa = inputs.random_matrix(Mg, Kg, seed=8 if wgrad else 6, dtype=torch.bfloat16, scale=1e-3 if wgrad else 1.0,
                                   outlier_frac=1e-3, factor=1e2, device=dev)
         xb = inputs.random_matrix(Ng, Kg, seed=9 if wgrad else 7, dtype=torch.bfloat16, scale=1.0 if wgrad else 0.02,
                                   outlier_frac=1e-3 if wgrad else 0.0, factor=1e2, device=dev)
-        bro = 1 if wgrad else 128
+        bro = 1 if wgrad and args.probe != "gemm_wgrad_b128" else 128  # gemm_wgrad_b128: B in 128x128 blocks
         qa = torch.empty(Mg, Kg, dtype=torch.uint8, device=dev)
         sa = torch.empty(Mg, Kg // 128, dtype=torch.float32, device=dev)
         qbm = torch.empty(Ng, Kg, dtype=torch.uint8, device=dev)
         sbm = torch.empty(Ng // bro, Kg // 128, dtype=torch.float32, device=dev)
-        raw.check(L.fp8_quantize_blockwise(xa.data_ptr(), 1, Mg, Kg, 1, 128, 1 if wgrad else 0, qa.data_ptr(),
-                                           sa.data_ptr(), st), "1x128")
+        raw.check(L.fp8_quantize_blockwise(xa.data_ptr(), 1, Mg, Kg, 1, 128, a_fmt, qa.data_ptr(), sa.data_ptr(),
+                                           st), "1x128")
         raw.check(L.fp8_quantize_blockwise(xb.data_ptr(), 1, Ng, Kg, bro, 128, 0, qbm.data_ptr(), sbm.data_ptr(), st),
                   "B")
         x = torch.empty(Mg, Ng, dtype=torch.bfloat16, device=dev)  # the GEMM's output
@@ -1116,7 +1119,7 @@ def traffic_probe(args):
         s = torch.empty(1, dtype=torch.float32, device=dev)
         flops = 2.0 * Mg * Ng * Kg
         launches.append(("k_gemm_blockwise", flops, lambda stream_: raw.check(L.fp8_gemm_blockwise_ex(
-            qa.data_ptr(), sa.data_ptr(), 1 if wgrad else 0, qbm.data_ptr(), sbm.data_ptr(), bro, 0, Mg, Ng, Kg,
+            qa.data_ptr(), sa.data_ptr(), a_fmt, qbm.data_ptr(), sbm.data_ptr(), bro, 0, Mg, Ng, Kg,
             x.data_ptr(), 1, stream_), "gemm")))
     else:
         s = torch.empty(R, C // 128, dtype=torch.float32, device=dev)
@@ -1174,7 +1177,9 @@ def main():
     ap.add_argument("--traffic-probe", action="store_true",
                     help="run one launch of each headline kernel between L2 cleaners (for an ncu DRAM capture)")
     ap.add_argument("--traffic-log2n", type=int, default=LOG2_N, help="tensor size of --traffic-probe (2^n)")
-    ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad"], default="headline",
+    ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad", "gemm_wgrad_e4m3",
+                                        "gemm_wgrad_b128"],
+                    default="headline",
                     help="the kernel(s) of --traffic-probe")
     ap.add_argument("--probe-time", type=int, default=0, metavar="K",
                     help="with --traffic-probe: also time K graph-replayed launches of the probed kernel(s)")

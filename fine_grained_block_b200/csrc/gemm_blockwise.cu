@@ -51,7 +51,8 @@
 //        reciprocal, two elements per f32x2 instruction (56 control / 224
 //        promotion registers).  Measured at 4096 x 7168 x 16384: 816 TF/s
 //        with a scalar load per column and chunk, 874 with the 16-byte
-//        loads, 901 with the packed arithmetic as well.
+//        loads, 901 with the packed arithmetic as well, 1056-1060 with the
+//        row scales loaded ahead (FP8Q_GEMM_PREFETCH_SCALES).
 // Two variants:
 //   single CTA (M 128 x N 256 per MMA): the CTA loads A (16 KiB) and all of
 //              B (32 KiB) per chunk, 4 stages;
@@ -120,9 +121,9 @@ struct Split {
 };
 static_assert(kLaunchRegs * kThreads <= 65536, "launch registers exceed the register file");
 
-// The promotion loads its row's scales one chunk ahead.
+// The promotion loads its row's scales this many chunks ahead (0: in the chunk that uses them).
 #ifndef FP8Q_GEMM_PREFETCH_SCALES
-#define FP8Q_GEMM_PREFETCH_SCALES 1
+#define FP8Q_GEMM_PREFETCH_SCALES 2
 #endif
 // Tile order: -1 picks per call (row tile fastest when M < N), 0 column tile
 // fastest, 1 row tile fastest.
@@ -380,9 +381,15 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 #if FP8Q_GEMM_PREFETCH_SCALES
-            // this row's scales one chunk ahead, so their load latency is not on the hand-back path
-            float sa_next = (m < M && nchunks > 0) ? __ldg(sa_row) : 1.0f;
-            float sb_next = (BROW != 1 && m < M && nchunks > 0) ? __ldg(sb_row) : 1.0f;
+            // this row's scales FP8Q_GEMM_PREFETCH_SCALES chunks ahead, so that their load latency is
+            // not on the accumulator hand-back path
+            constexpr int kAhead = FP8Q_GEMM_PREFETCH_SCALES;
+            float sa_q[kAhead], sb_q[kAhead];
+#pragma unroll
+            for (int d = 0; d < kAhead; ++d) {
+                sa_q[d] = (m < M && d < nchunks) ? __ldg(sa_row + d) : 1.0f;
+                sb_q[d] = (BROW != 1 && m < M && d < nchunks) ? __ldg(sb_row + d) : 1.0f;
+            }
 #endif
             for (int kc = 0; kc < nchunks; ++kc, ++g) {
                 const uint32_t buf = g & 1u;
@@ -390,10 +397,15 @@ k_gemm_blockwise(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 // 128x128 B: 1 / (sa * sb), the dequant factor of this chunk for this row and
                 // column half.  1x128 B: 1 / sa here; 1 / sb per column from the ring.
 #if FP8Q_GEMM_PREFETCH_SCALES
-                const float sa_cur = sa_next, sb_cur = sb_next;
-                if (m < M && kc + 1 < nchunks) {
-                    sa_next = __ldg(sa_row + kc + 1);
-                    if (BROW != 1) sb_next = __ldg(sb_row + kc + 1);
+                const float sa_cur = sa_q[0], sb_cur = sb_q[0];
+#pragma unroll
+                for (int d = 0; d + 1 < kAhead; ++d) {
+                    sa_q[d] = sa_q[d + 1];
+                    sb_q[d] = sb_q[d + 1];
+                }
+                if (m < M && kc + kAhead < nchunks) {
+                    sa_q[kAhead - 1] = __ldg(sa_row + kc + kAhead);
+                    if (BROW != 1) sb_q[kAhead - 1] = __ldg(sb_row + kc + kAhead);
                 }
                 const float f = (m < M) ? (BROW == 1 ? __frcp_rn(sa_cur) : __frcp_rn(__fmul_rn(sa_cur, sb_cur)))
                                         : 0.0f;
