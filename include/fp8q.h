@@ -94,10 +94,12 @@ int fp8_quantize_per_tensor(const void *x, int dtype, int64_t n, int fmt,
 
 /*
  * Per-tensor CURRENT scaling in one pass over x, for tensors small enough to
- * be held on chip by the CTAs that fit on the GPU at once (about 8-9 MiB of
- * input on a B200; larger tensors transparently take the two-pass path of
- * fp8_quantize_per_tensor and do not touch the workspace).  Same results as
- * fp8_quantize_per_tensor with scale_in == NULL.
+ * be held on chip by the CTAs that fit on the GPU at once (on a B200 up to
+ * 18.5 MiB of input when x is 32-byte aligned, 11.6 MiB when it is only
+ * 16-byte aligned: the exact element counts are stated with
+ * fp8_quantize_per_tensor_fused_noalloc).  Larger tensors transparently take
+ * the two-pass path of fp8_quantize_per_tensor and do not touch the
+ * workspace.  Same results as fp8_quantize_per_tensor with scale_in == NULL.
  *
  *   x, dtype, n, fmt, q, scale_out, amax_out   as fp8_quantize_per_tensor
  *              (scale_out and amax_out both required)
