@@ -1058,7 +1058,8 @@ def traffic_probe(args):
     --probe bt1x128    1x128 quantize of x and x^T of the bf16 activations 16384x7168;
     --probe gemm_fwd / gemm_wgrad   the consumer GEMM (timing; its operands are quantized first);
     --probe gemm_wgrad_e4m3         the weight-gradient shape with both operands E4M3;
-    --probe gemm_wgrad_b128         the weight-gradient shape with B in 128x128 blocks (the forward form).
+    --probe gemm_wgrad_b128         the weight-gradient shape with B in 128x128 blocks (the forward form);
+    --probe gemm_wgrad_f32out       the weight-gradient GEMM writing fp32 instead of bf16.
     --probe-time K     afterwards, also time K back-to-back launches of the probed kernel(s) (not under ncu).
     --lib PATH         use another build of the library (a variant built with tuning macros)."""
     import torch
@@ -1075,7 +1076,7 @@ def traffic_probe(args):
         # 16384 4096 7168) or weight gradient (1x128 x 1x128, E5M2 x E4M3, 4096 7168 16384)
         wgrad = args.probe.startswith("gemm_wgrad")
         Mg, Ng, Kg = (4096, 7168, 16384) if wgrad else (16384, 4096, 7168)
-        a_fmt = 1 if args.probe == "gemm_wgrad" else 0  # gemm_wgrad_e4m3: both operands E4M3
+        a_fmt = 1 if args.probe in ("gemm_wgrad", "gemm_wgrad_f32out") else 0  # gemm_wgrad_e4m3: both E4M3
         xa = inputs.random_matrix(Mg, Kg, seed=8 if wgrad else 6, dtype=torch.bfloat16, scale=1e-3 if wgrad else 1.0,
                                   outlier_frac=1e-3, factor=1e2, device=dev)
         xb = inputs.random_matrix(Ng, Kg, seed=9 if wgrad else 7, dtype=torch.bfloat16, scale=1.0 if wgrad else 0.02,
@@ -1089,7 +1090,8 @@ def traffic_probe(args):
                                            st), "1x128")
         raw.check(L.fp8_quantize_blockwise(xb.data_ptr(), 1, Ng, Kg, bro, 128, 0, qbm.data_ptr(), sbm.data_ptr(), st),
                   "B")
-        x = torch.empty(Mg, Ng, dtype=torch.bfloat16, device=dev)  # the GEMM's output
+        out_f32 = args.probe == "gemm_wgrad_f32out"  # the weight-gradient GEMM writing fp32
+        x = torch.empty(Mg, Ng, dtype=torch.float32 if out_f32 else torch.bfloat16, device=dev)  # the GEMM's output
     else:
         x = inputs.sweep_tensor(args.traffic_log2n, seed=4, device=dev)
     R, C = x.shape
@@ -1120,7 +1122,7 @@ def traffic_probe(args):
         flops = 2.0 * Mg * Ng * Kg
         launches.append(("k_gemm_blockwise", flops, lambda stream_: raw.check(L.fp8_gemm_blockwise_ex(
             qa.data_ptr(), sa.data_ptr(), a_fmt, qbm.data_ptr(), sbm.data_ptr(), bro, 0, Mg, Ng, Kg,
-            x.data_ptr(), 1, stream_), "gemm")))
+            x.data_ptr(), 0 if out_f32 else 1, stream_), "gemm")))
     else:
         s = torch.empty(R, C // 128, dtype=torch.float32, device=dev)
         qt = torch.empty(C, R, dtype=torch.uint8, device=dev)
@@ -1178,7 +1180,7 @@ def main():
                     help="run one launch of each headline kernel between L2 cleaners (for an ncu DRAM capture)")
     ap.add_argument("--traffic-log2n", type=int, default=LOG2_N, help="tensor size of --traffic-probe (2^n)")
     ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad", "gemm_wgrad_e4m3",
-                                        "gemm_wgrad_b128"],
+                                        "gemm_wgrad_b128", "gemm_wgrad_f32out"],
                     default="headline",
                     help="the kernel(s) of --traffic-probe")
     ap.add_argument("--probe-time", type=int, default=0, metavar="K",
