@@ -124,6 +124,28 @@ struct ColMax<uint16_t, BYTES> {
             }
         }
     }
+    // The same maxima left packed, one word per column pair: colmax_w[k] holds columns 2k and 2k + 1 of
+    // this lane's slice as two |bf16| halves, stored with 16-byte shared stores.
+    static __device__ __forceinline__ void run_packed(const typename V::In (&v)[G::kLoads], bool write,
+                                                      uint32_t* colmax_w) {
+        uint32_t mw[V::kWords];
+#pragma unroll
+        for (int k = 0; k < V::kWords; ++k) {
+            uint32_t m = v[0].w[k];
+#pragma unroll
+            for (int i = 1; i < G::kLoads; ++i) m = xabsmax_bf16x2(m, v[i].w[k]);
+#pragma unroll
+            for (int off = G::kVecPerRow; off < 32; off <<= 1)
+                m = xabsmax_bf16x2(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+            mw[k] = m & 0x7FFF7FFFu;
+        }
+        if (write) {
+#pragma unroll
+            for (int k4 = 0; k4 < V::kWords / 4; ++k4)
+                reinterpret_cast<uint4*>(colmax_w)[k4] = make_uint4(mw[4 * k4], mw[4 * k4 + 1], mw[4 * k4 + 2],
+                                                                    mw[4 * k4 + 3]);
+        }
+    }
 };
 template <int BYTES>
 struct ColMax<float, BYTES> {
@@ -154,8 +176,11 @@ struct ColMax<float, BYTES> {
 // column pass's barriers 4598 / 5162 / 5210 GB/s for caps of 2 / 3 / 4 CTAs,
 // and 5437 GB/s with it issued before them (RELOAD 2), so that the loads are
 // in flight across the barriers.  The column cast takes this lane's 16
-// column scales into registers once (SCALE_REGS).  128x128: 6462 GB/s
-// (98.7 % of the copy peak) with 3 or 4 CTAs.
+// column scales into registers once (SCALE_REGS).  Keeping bf16 column
+// maxima as packed |bf16| pairs through shared memory (PACKED_PART: two
+// 16-byte stores per writing lane instead of 16 scalar ones, no unpacking)
+// gives 5567-5573 GB/s against 5429-5431.  128x128: 6462 GB/s (98.7 % of the
+// copy peak) with 3 or 4 CTAs.
 #ifndef FP8Q_BT_TMA
 #define FP8Q_BT_TMA 0
 #endif
@@ -164,6 +189,10 @@ struct ColMax<float, BYTES> {
 #endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_SCALE_REGS
 #define FP8Q_BLOCK_TRANSPOSE_SCALE_REGS 1
+#endif
+// bf16 column maxima kept as packed |bf16| pairs through shared memory
+#ifndef FP8Q_BLOCK_TRANSPOSE_PACKED_PART
+#define FP8Q_BLOCK_TRANSPOSE_PACKED_PART 1
 #endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
 #define FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS 4
@@ -182,7 +211,10 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
     using V = LaneVec<T, BYTES>;
     using G = TileGeom<T, BYTES>;
     __shared__ __align__(16) uint8_t tile[kTT * kTT];
-    __shared__ float part[kWarps][kTT];  // per-warp column maxima (MODE 0); warp maxima (MODE 1)
+    __shared__ __align__(16) float part[kWarps][kTT];  // per-warp column maxima (MODE 0); warp maxima (MODE 1)
+    // bf16, MODE 0 with packed partials: the same storage as [kWarps][kTT / 2] words of |bf16| pairs
+    uint32_t (*part_w)[kTT] = reinterpret_cast<uint32_t (*)[kTT]>(part);
+    constexpr bool kPackedPart = FP8Q_BLOCK_TRANSPOSE_PACKED_PART && sizeof(T) == 2;
     __shared__ __align__(16) float col_scale[kTT];
 
     const int64_t tiles_c = cols / kTT, tiles_r = rows / kTT;
@@ -245,7 +277,10 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
         }
 #if FP8Q_BLOCK_TRANSPOSE_RELOAD != 3
         // qt: one scale per tile column
-        ColMax<T, BYTES>::run(v, lane < G::kVecPerRow, &part[warp][vec_in_row * V::kElems]);
+        if constexpr (kPackedPart)
+            ColMax<T, BYTES>::run_packed(v, lane < G::kVecPerRow, &part_w[warp][vec_in_row * V::kElems / 2]);
+        else
+            ColMax<T, BYTES>::run(v, lane < G::kVecPerRow, &part[warp][vec_in_row * V::kElems]);
 #endif
 #if FP8Q_BLOCK_TRANSPOSE_RELOAD == 2
         // the tile again, from L2, issued now so that the loads are in flight
@@ -256,9 +291,17 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
         __syncthreads();
         if (threadIdx.x < kTT) {
             const int c = threadIdx.x;
-            float m = part[0][c];
+            float m;
+            if constexpr (kPackedPart) {
+                uint32_t mw = part_w[0][c >> 1];
 #pragma unroll
-            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, part[w][c]);
+                for (int w = 1; w < kWarps; ++w) mw = xabsmax_bf16x2(mw, part_w[w][c >> 1]);
+                m = __uint_as_float((c & 1) ? (mw & 0xFFFF0000u) : (mw << 16));
+            } else {
+                m = part[0][c];
+#pragma unroll
+                for (int w = 1; w < kWarps; ++w) m = fmaxf(m, part[w][c]);
+            }
             const float s = scale_from_amax<FMT>(m);
             col_scale[c] = s;
             scales_t[(c0 + c) * tiles_r + tr] = s;
