@@ -1138,7 +1138,8 @@ def traffic_probe(args):
     same = None
     if args.lib:
         # a variant build must give the default build's bytes: rerun the default on copies of the outputs
-        got = [t.clone() for t in (q, s)]
+        outs = (q, s, qt, st_) if args.probe == "bt1x128" else (q, s)
+        got = [t.clone() for t in outs]
         if args.probe.startswith("gemm"):  # the GEMM's result is within a bound, not bit-exact: compare loosely
             got[0] = x.clone()
         default = Raw(stream)
@@ -1150,7 +1151,9 @@ def traffic_probe(args):
         if args.probe.startswith("gemm"):
             same = bool(torch.allclose(got[0].float(), x.float(), rtol=2e-2, atol=1e-3 * float(x.float().abs().max())))
         else:
-            same = bool(torch.equal(got[0], q) and torch.equal(got[1].view(torch.int32), s.view(torch.int32)))
+            same = all(torch.equal(g.view(torch.int32) if g.dtype == torch.float32 else g,
+                                   o.view(torch.int32) if o.dtype == torch.float32 else o)
+                       for g, o in zip(got, outs))
         raw.L = L = L_var
     out = {"probe": args.probe, "rows": R, "cols": C, "lib": args.lib or "default", "same_as_default": same,
            "alg_bytes": {name: nb for name, nb, _ in launches},
