@@ -15,11 +15,23 @@
 // runs out the CTA records the wait-timeout bit in the device status word and
 // returns without writing its codes.
 //
-// Workspace (16 bytes of device memory, zero before the first use, left zero
-// after every call): {arrivals, generation, amax bits, unused}.  Calls that
-// share a workspace must not overlap on the device.
+// Workspace (16 bytes of device memory, zero before the first use; every call
+// leaves it ready for the next): {arrivals, amax bits, result}, where result
+// packs the amax bits of the last completed call (low half) with the count of
+// completed calls (high half).  Calls that share a workspace must not overlap
+// on the device.
+//
+// The barrier keeps the chain of dependent global-memory trips short.  Each
+// CTA reads the call count when it starts, while its loads of x are in
+// flight.  At the barrier it folds its amax in (an atomic max, fenced) and
+// arrives (an atomic add).  The last to arrive reads the final amax, writes
+// amax_out and scale_out, clears the arrival count and the running amax, and
+// publishes {amax, count + 1} in the result word with one 64-bit store.  The
+// others spin on that word until its count moves on and take the amax from
+// it, so they need no further read.
 
 #include <algorithm>
+#include <cstddef>
 #include <atomic>
 
 #include "fp8q_device.cuh"
@@ -35,22 +47,40 @@ constexpr int kThreads = 256;
 constexpr int kLoads = 4;  // lane vectors per thread held in registers
 
 struct Workspace {
-    unsigned int arrivals;
-    unsigned int generation;
-    unsigned int amax_bits;
-    unsigned int unused;
+    unsigned int arrivals;        // CTAs of the current call that have arrived
+    unsigned int amax_bits;       // running max of the current call's CTA maxima
+    unsigned long long result;    // {amax bits of the last completed call, completed calls}
 };
 static_assert(sizeof(Workspace) == 16, "workspace layout");
+static_assert(offsetof(Workspace, result) == 8, "the result word is 8-byte aligned in a 16-byte-aligned workspace");
 
-__device__ __forceinline__ unsigned int ld_volatile(const unsigned int* p) {
-    unsigned int v;
-    asm volatile("ld.volatile.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ float ld_volatile(const float* p) {
-    float v;
-    asm volatile("ld.volatile.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
-    return v;
+__device__ __forceinline__ void st_volatile_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Spin until the call count in the result word differs from `count`; the word
+// then holds the amax of this call.  False if limit_ns passes first.
+__device__ __forceinline__ bool wait_for_result(const unsigned long long* word, unsigned int count,
+                                                unsigned long long* out, uint64_t limit_ns) {
+    unsigned long long r = ld_volatile_u64(word);
+    if (static_cast<unsigned int>(r >> 32) != count) {
+        *out = r;
+        return true;
+    }
+    const uint64_t start = global_timer_ns();
+    for (;;) {
+        r = ld_volatile_u64(word);
+        if (static_cast<unsigned int>(r >> 32) != count) {
+            *out = r;
+            return true;
+        }
+        if (global_timer_ns() - start > limit_ns) return false;
+    }
 }
 
 template <typename T>
@@ -72,6 +102,9 @@ k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nve
     __shared__ float cta_result;
     __shared__ int cta_ok;
 
+    // the call count, read while the loads below are in flight: it cannot move before this CTA arrives
+    unsigned int count = 0;
+    if (threadIdx.x == 0) count = static_cast<unsigned int>(ld_volatile_u64(&ws->result) >> 32);
     const int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads * kLoads + threadIdx.x;
     typename V::In v[kLoads];
 #pragma unroll
@@ -95,27 +128,27 @@ k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nve
         float m = warp_amax[0];
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_amax[w]);
-        // contribute this CTA's amax (skipped when the running maximum is already as large)
-        if (__float_as_uint(m) > ld_volatile(&ws->amax_bits)) atomicMax(&ws->amax_bits, __float_as_uint(m));
-        const unsigned int gen = ld_volatile(&ws->generation);  // read before arriving
+        // contribute this CTA's amax; the fence orders it before the arrival
+        atomicMax(&ws->amax_bits, __float_as_uint(m));
         __threadfence();
         const unsigned int arrived = atomicAdd(&ws->arrivals, 1u);
         bool ok = true;
         float amax;
         if (arrived == gridDim.x - 1) {
-            // last to arrive: every other CTA's atomicMax is ordered before its arrival
+            // last to arrive: every other CTA's atomicMax was performed before its arrival
             __threadfence();
-            amax = __uint_as_float(atomicOr(&ws->amax_bits, 0u));
+            const unsigned int bits = atomicOr(&ws->amax_bits, 0u);
+            amax = __uint_as_float(bits);
             *amax_out = amax;
             *scale_out = scale_from_amax<FMT>(amax);
             ws->amax_bits = 0u;
             ws->arrivals = 0u;
-            __threadfence();
-            atomicAdd(&ws->generation, 1u);  // releases the waiting CTAs
+            // the waiting CTAs read nothing but this word, so no fence is needed before it
+            st_volatile_u64(&ws->result, (static_cast<unsigned long long>(count + 1u) << 32) | bits);
         } else {
-            ok = wait_for_change(&ws->generation, gen, kWaitLimitNs);
-            __threadfence();
-            amax = ld_volatile(amax_out);
+            unsigned long long r = 0;
+            ok = wait_for_result(&ws->result, count, &r, kWaitLimitNs);
+            amax = __uint_as_float(static_cast<unsigned int>(r));
         }
         if (!ok) atomicOr(status, kStatusWaitTimeout);
         cta_result = amax;

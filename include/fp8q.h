@@ -105,8 +105,11 @@ int fp8_quantize_per_tensor(const void *x, int dtype, int64_t n, int fmt,
  *              (scale_out and amax_out both required)
  *   workspace  FP8_FUSED_WORKSPACE_BYTES of caller-owned device memory,
  *              16-byte aligned, zeroed once before its first use; every call
- *              leaves it zeroed again.  Calls that share a workspace must not
- *              overlap on the device (use one workspace per stream).
+ *              leaves it ready for the next one (it keeps a count of
+ *              completed calls and the last amax), and zeroing it again
+ *              between calls is also allowed.  Calls that share a workspace
+ *              must not overlap on the device (use one workspace per stream).
+ *              After FP8_DEVICE_STATUS_WAIT_TIMEOUT, zero it before reuse.
  * The one-pass kernel holds its slice of x in registers, meets the other CTAs
  * at a grid-wide barrier (a cooperative launch, so every CTA is resident),
  * and then casts.  The barrier wait gives up after about a second, sets
