@@ -128,15 +128,15 @@ k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nve
         float m = warp_amax[0];
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_amax[w]);
-        // contribute this CTA's amax; the fence orders it before the arrival
+        // contribute this CTA's amax, then arrive: the arrival's release half orders the max before it,
+        // and its acquire half makes every earlier arrival's max visible to the last CTA
         atomicMax(&ws->amax_bits, __float_as_uint(m));
-        __threadfence();
-        const unsigned int arrived = atomicAdd(&ws->arrivals, 1u);
+        unsigned int arrived;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(&ws->arrivals) : "memory");
         bool ok = true;
         float amax;
         if (arrived == gridDim.x - 1) {
             // last to arrive: every other CTA's atomicMax was performed before its arrival
-            __threadfence();
             const unsigned int bits = atomicOr(&ws->amax_bits, 0u);
             amax = __uint_as_float(bits);
             *amax_out = amax;
