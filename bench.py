@@ -1059,7 +1059,10 @@ def traffic_probe(args):
     --probe gemm_fwd / gemm_wgrad   the consumer GEMM (timing; its operands are quantized first);
     --probe gemm_wgrad_e4m3         the weight-gradient shape with both operands E4M3;
     --probe gemm_wgrad_b128         the weight-gradient shape with B in 128x128 blocks (the forward form);
-    --probe gemm_wgrad_f32out       the weight-gradient GEMM writing fp32 instead of bf16.
+    --probe gemm_wgrad_f32out       the weight-gradient GEMM writing fp32 instead of bf16;
+    --probe per_tensor_1mib         per-tensor current scaling of the fp32 256x1024 experiment tensor in one
+                                    pass (k_tensor_fused; --probe-time: each call timed alone after an L2
+                                    flush, beside the two-pass path).
     --probe-time K     afterwards, also time K back-to-back launches of the probed kernel(s) (not under ncu).
     --lib PATH         use another build of the library (a variant built with tuning macros)."""
     import torch
@@ -1071,6 +1074,8 @@ def traffic_probe(args):
     L, st = raw.L, raw.stream
     if args.probe == "bt1x128":
         x = inputs.activation_outlier_channels(device=dev)
+    elif args.probe == "per_tensor_1mib":
+        x = inputs.relerr_outlier_tensors()[1][1].to(dev)
     elif args.probe.startswith("gemm"):
         # the consumer GEMM's operands, quantized by the library: forward (1x128 x 128x128, M N K =
         # 16384 4096 7168) or weight gradient (1x128 x 1x128, E5M2 x E4M3, 4096 7168 16384)
@@ -1117,6 +1122,13 @@ def traffic_probe(args):
         launches.append(("k_quant_128x128", 3 * n + 4 * (n // 16384), lambda stream_: raw.check(
             L.fp8_quantize_blockwise(x.data_ptr(), 1, R, C, 128, 128, 0, q.data_ptr(), s.data_ptr(), stream_),
             "128x128")))
+    elif args.probe == "per_tensor_1mib":
+        s = torch.empty(1, dtype=torch.float32, device=dev)
+        am1 = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.zeros(4, dtype=torch.int32, device=dev)
+        launches.append(("k_tensor_fused", 5 * n, lambda stream_: raw.check(L.fp8_quantize_per_tensor_fused(
+            x.data_ptr(), 0, n, 0, q.data_ptr(), s.data_ptr(), am1.data_ptr(), ws.data_ptr(), stream_),
+            "fused per-tensor")))
     elif args.probe.startswith("gemm"):
         s = torch.empty(1, dtype=torch.float32, device=dev)
         flops = 2.0 * Mg * Ng * Kg
@@ -1158,7 +1170,16 @@ def traffic_probe(args):
     out = {"probe": args.probe, "rows": R, "cols": C, "lib": args.lib or "default", "same_as_default": same,
            "alg_bytes": {name: nb for name, nb, _ in launches},
            "source_sha256": {k: source_hash(k) for k in KERNEL_SOURCES}}
-    if args.probe_time:
+    if args.probe_time and args.probe == "per_tensor_1mib":
+        # a 1 MiB call is latency-bound: time each call alone after an L2 flush, beside the two-pass path
+        two = lambda r: raw.check(L.fp8_quantize_per_tensor(x.data_ptr(), 0, n, 0, None, q.data_ptr(),
+                                                            s.data_ptr(), am1.data_ptr(), st), "per-tensor")
+        t_one, t_two = time_per_launch([lambda r: launches[0][2](st), two], args.probe_time, 5, stream,
+                                       lambda: cleaner.fill_(1))
+        out["timing"] = {"k_tensor_fused": {"us": round(t_one * 1e3, 2), "GB_s": round(5 * n / (t_one * 1e-3) / 1e9, 1)},
+                         "two_pass": {"us": round(t_two * 1e3, 2), "GB_s": round(5 * n / (t_two * 1e-3) / 1e9, 1)},
+                         "note": "each call timed alone after an L2 flush"}
+    elif args.probe_time:
         del cleaner
         for name, nb, fn in launches:
             ms = time_in_graph([lambda r, stream_, fn=fn: fn(stream_)], args.probe_time, dev)
@@ -1183,7 +1204,7 @@ def main():
                     help="run one launch of each headline kernel between L2 cleaners (for an ncu DRAM capture)")
     ap.add_argument("--traffic-log2n", type=int, default=LOG2_N, help="tensor size of --traffic-probe (2^n)")
     ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad", "gemm_wgrad_e4m3",
-                                        "gemm_wgrad_b128", "gemm_wgrad_f32out"],
+                                        "gemm_wgrad_b128", "gemm_wgrad_f32out", "per_tensor_1mib"],
                     default="headline",
                     help="the kernel(s) of --traffic-probe")
     ap.add_argument("--probe-time", type=int, default=0, metavar="K",
