@@ -990,6 +990,31 @@ def run_ours(args):
     torch.cuda.synchronize()
     (te,) = max_over_ranks([e0.elapsed_time(e1)], world, device=dev)
     e2e_value = (qb + db) * e2e_steps * world / (te * 1e-3) / 1e9
+
+    # The link alone: the same uploads and downloads with no kernels, the two directions at once, as the
+    # bound the e2e figure is read against.
+    torch.cuda.synchronize()
+    l0, l1, l_in = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                    torch.cuda.Event())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    l0.record(s_in)
+    s_out.wait_event(l0)
+    for r in range(e2e_steps):
+        xb, qb_, sb, yb = sets[r % len(sets)]
+        with torch.cuda.stream(s_in):
+            xb.copy_(hx, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            hq.copy_(qb_, non_blocking=True)
+            hs.copy_(sb, non_blocking=True)
+            hy.copy_(yb, non_blocking=True)
+    l_in.record(s_in)
+    s_out.wait_event(l_in)
+    l1.record(s_out)
+    torch.cuda.synchronize()
+    (tl,) = max_over_ranks([l0.elapsed_time(l1)], world, device=dev)
+    link_value = (qb + db) * e2e_steps * world / (tl * 1e-3) / 1e9
     del sets, main_set, x, q, s, y, hq, hs, hy
     torch.cuda.empty_cache()
 
@@ -1022,7 +1047,10 @@ def run_ours(args):
                     "d2h_bytes_per_step": ROWS * COLS + ROWS * (COLS // 128) * 4 + ROWS * COLS * 2,
                     "steps": e2e_steps,
                     "note": "pinned host buffers; uploads, kernels and downloads on three streams over two device "
-                            "buffer sets, so one step's download overlaps the next step's upload"},
+                            "buffer sets, so one step's download overlaps the next step's upload",
+                    "link_bound": {"value": round(link_value, 2), "unit": UNIT,
+                                   "note": "the same uploads and downloads with no kernels, both directions at once"},
+                    "frac_of_link_bound": round(e2e_value / link_value, 4)},
             "gpu_launches": 2 * args.steps,
             "timing": "K steps launched eagerly, an event after every launch; value = bytes / (last event - first)",
             "clocks": clocks.summary(),
