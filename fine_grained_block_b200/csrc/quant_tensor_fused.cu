@@ -171,15 +171,24 @@ k_tensor_fused(const typename LaneVec<T, BYTES>::In* __restrict__ x, int64_t nve
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // Largest grid that can be co-resident, or -1 when it cannot be known: a failed
-// CUDA query, or a device without cooperative launch.
+// CUDA query, or a device without cooperative launch.  A known answer is kept
+// per device (one cache per kernel), so calls after the first make one CUDA
+// call here (cudaGetDevice) instead of four.
 template <typename Kernel>
 int64_t resident_ctas(Kernel k) {
+    static std::atomic<int64_t> cache[128];
     int dev = 0, coop = 0, per_sm = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 128) {
+        const int64_t known = cache[dev].load(std::memory_order_acquire);
+        if (known > 0) return known;
+    }
     if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return -1;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return -1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, 0) != cudaSuccess) return -1;
-    return static_cast<int64_t>(per_sm) * sms;
+    const int64_t units = static_cast<int64_t>(per_sm) * sms;
+    if (units > 0 && dev >= 0 && dev < 128) cache[dev].store(units, std::memory_order_release);
+    return units;
 }
 
 template <typename T, int FMT, int BYTES>
