@@ -1085,6 +1085,7 @@ def traffic_probe(args):
     --probe 128x128    128x128 quantize of the 2^n sweep tensor;
     --probe bt1x128    1x128 quantize of x and x^T of the bf16 activations 16384x7168;
     --probe gemm_fwd / gemm_wgrad   the consumer GEMM (timing; its operands are quantized first);
+    --probe gemm_4096               the forward GEMM at 4096 x 4096 x 4096;
     --probe gemm_wgrad_e4m3         the weight-gradient shape with both operands E4M3;
     --probe gemm_wgrad_b128         the weight-gradient shape with B in 128x128 blocks (the forward form);
     --probe gemm_wgrad_f32out       the weight-gradient GEMM writing fp32 instead of bf16;
@@ -1108,7 +1109,8 @@ def traffic_probe(args):
         # the consumer GEMM's operands, quantized by the library: forward (1x128 x 128x128, M N K =
         # 16384 4096 7168) or weight gradient (1x128 x 1x128, E5M2 x E4M3, 4096 7168 16384)
         wgrad = args.probe.startswith("gemm_wgrad")
-        Mg, Ng, Kg = (4096, 7168, 16384) if wgrad else (16384, 4096, 7168)
+        Mg, Ng, Kg = (4096, 7168, 16384) if wgrad else (4096, 4096, 4096) if args.probe == "gemm_4096" else \
+            (16384, 4096, 7168)
         a_fmt = 1 if args.probe in ("gemm_wgrad", "gemm_wgrad_f32out") else 0  # gemm_wgrad_e4m3: both E4M3
         xa = inputs.random_matrix(Mg, Kg, seed=8 if wgrad else 6, dtype=torch.bfloat16, scale=1e-3 if wgrad else 1.0,
                                   outlier_frac=1e-3, factor=1e2, device=dev)
@@ -1232,7 +1234,7 @@ def main():
                     help="run one launch of each headline kernel between L2 cleaners (for an ncu DRAM capture)")
     ap.add_argument("--traffic-log2n", type=int, default=LOG2_N, help="tensor size of --traffic-probe (2^n)")
     ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad", "gemm_wgrad_e4m3",
-                                        "gemm_wgrad_b128", "gemm_wgrad_f32out", "per_tensor_1mib"],
+                                        "gemm_wgrad_b128", "gemm_wgrad_f32out", "gemm_4096", "per_tensor_1mib"],
                     default="headline",
                     help="the kernel(s) of --traffic-probe")
     ap.add_argument("--probe-time", type=int, default=0, metavar="K",
