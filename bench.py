@@ -1071,6 +1071,174 @@ def run_ours(args):
     return 0
 
 
+KERNEL_PROBES = {
+    "q128_weight4096": "k_quant_128x128: 128x128 E4M3 quantize of the bf16 weight 4096x4096",
+    "dq128_weight4096": "k_dequant_128x128: its codes back to bf16",
+    "fake_1x128_act": "k_fake_quant_1x128: 1x128 E4M3 round trip of the bf16 activations 16384x7168",
+    "mx_act": "k_quant_rowblocks (Pow2Scale): MX 1x32 E4M3 quantize of the activations",
+    "dqmx_act": "k_dequant_mx: those MX codes back to bf16",
+    "cast_transpose_act": "k_tensor_cast_transpose: per-tensor E4M3 q and qt of the activations, delayed scale",
+    "delayed_step_grads": "k_tensor_cast_delayed_step: one delayed E5M2 step (W 16) on the gradients 8192x8192",
+    "delayed_step_grouped": "k_tensor_cast_delayed_step_grouped: 128 bf16 tensors of 2^20 in one call",
+    "grouped_weights": "k_quant_grouped: 128 bf16 weights 1024x1024, 128x128 E4M3, in one call",
+    "per_tensor_sweep28": "k_tensor_amax then k_tensor_cast: per-tensor current E5M2 of the sweep tensor 2^28",
+}
+
+
+def kernel_probe(args):
+    """One launch of a named kernel on the workload its profile covers, between L2 cleaners (as in
+    --traffic-probe), for an ncu capture; --probe-time K then times K single launches, each after an L2
+    flush.  The workloads are those of `bench.py` modes, and small enough for a full ncu capture."""
+    import torch
+    from fine_grained_block_b200 import inputs
+    from fine_grained_block_b200.binding import FP8BlockTensor, FP8DelayedTensor
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    raw = Raw(stream, args.lib)
+    L, st = raw.L, raw.stream
+    f32, u8, bf16 = torch.float32, torch.uint8, torch.bfloat16
+    name = args.probe
+    pre = []       # launches run once before the captured ones (the codes a dequant reads)
+    launches = []  # (kernel, algorithmic bytes, fn(stream))
+    keep = []      # tensors the launches use
+    if name in ("q128_weight4096", "dq128_weight4096"):
+        w = inputs.weight_4096(device=dev)
+        R, C = w.shape
+        n = w.numel()
+        q = torch.empty(R, C, dtype=u8, device=dev)
+        s = torch.empty(R // 128, C // 128, dtype=f32, device=dev)
+        y = torch.empty(R, C, dtype=bf16, device=dev)
+        quant = lambda s_: raw.check(L.fp8_quantize_blockwise(w.data_ptr(), 1, R, C, 128, 128, 0, q.data_ptr(),
+                                                              s.data_ptr(), s_), "128x128")
+        if name == "q128_weight4096":
+            launches.append(("k_quant_128x128", 3 * n + 4 * (n // 16384), quant))
+            outs = (q, s)
+        else:
+            pre.append(quant)
+            launches.append(("k_dequant_128x128", 3 * n + 4 * (n // 16384), lambda s_: raw.check(L.fp8_dequantize(
+                q.data_ptr(), 0, R, C, 128, 128, s.data_ptr(), y.data_ptr(), 1, s_), "dequant")))
+            outs = (y,)
+        keep += [w, q, s, y]
+    elif name in ("fake_1x128_act", "mx_act", "dqmx_act", "cast_transpose_act"):
+        a = inputs.activation_outlier_channels(device=dev)
+        R, C = a.shape
+        n = a.numel()
+        q = torch.empty(R, C, dtype=u8, device=dev)
+        y = torch.empty(R, C, dtype=bf16, device=dev)
+        e8 = torch.empty(R, C // 32, dtype=u8, device=dev)
+        qt = torch.empty(C, R, dtype=u8, device=dev)
+        sc = torch.full((1,), 0.25, dtype=f32, device=dev)
+        so = torch.empty(1, dtype=f32, device=dev)
+        ao = torch.empty(1, dtype=f32, device=dev)
+        mx = lambda s_: raw.check(L.fp8_quantize_mx(a.data_ptr(), 1, R, C, 0, 0, q.data_ptr(), e8.data_ptr(), s_), "mx")
+        if name == "fake_1x128_act":
+            launches.append(("k_fake_quant_1x128", 4 * n, lambda s_: raw.check(L.fp8_fake_quantize(
+                a.data_ptr(), 1, R, C, 1, 128, 0, None, y.data_ptr(), None, s_), "fake quant")))
+            outs = (y,)
+        elif name == "mx_act":
+            launches.append(("k_quant_rowblocks", 3 * n + n // 32, mx))
+            outs = (q, e8)
+        elif name == "dqmx_act":
+            pre.append(mx)
+            launches.append(("k_dequant_mx", 3 * n + n // 32, lambda s_: raw.check(L.fp8_dequantize_mx(
+                q.data_ptr(), 0, R, C, e8.data_ptr(), y.data_ptr(), 1, s_), "mx dequant")))
+            outs = (y,)
+        else:
+            launches.append(("k_tensor_cast_transpose", 4 * n, lambda s_: raw.check(
+                L.fp8_quantize_per_tensor_transpose(a.data_ptr(), 1, R, C, 0, sc.data_ptr(), q.data_ptr(),
+                                                    qt.data_ptr(), so.data_ptr(), ao.data_ptr(), s_), "transpose")))
+            outs = (q, qt, ao)
+        keep += [a, q, y, e8, qt, sc, so, ao]
+    elif name == "delayed_step_grads":
+        g = inputs.gradient_step(inputs.gradient_base(device=dev), 0)
+        n = g.numel()
+        q = torch.empty(g.shape, dtype=u8, device=dev)
+        scale = torch.ones(1, dtype=f32, device=dev)
+        hist = torch.zeros(16, dtype=f32, device=dev)
+        state = torch.zeros(2, dtype=torch.int32, device=dev)
+        used = torch.empty(1, dtype=f32, device=dev)
+        amax = torch.empty(1, dtype=f32, device=dev)
+        ws = torch.zeros(4, dtype=torch.int32, device=dev)
+        launches.append(("k_tensor_cast_delayed_step", 3 * n, lambda s_: raw.check(L.fp8_quantize_delayed_step(
+            g.data_ptr(), 1, n, 1, scale.data_ptr(), hist.data_ptr(), state.data_ptr(), 16, 0, 1.0, 1.0,
+            q.data_ptr(), used.data_ptr(), amax.data_ptr(), ws.data_ptr(), s_), "delayed step")))
+        outs = (q, amax)
+        keep += [g, q, scale, hist, state, used, amax, ws]
+    elif name == "delayed_step_grouped":
+        gx = [inputs.random_matrix(1, 1 << 20, seed=300 + i, dtype=bf16, scale=1e-3, device=dev).reshape(-1)
+              for i in range(128)]
+        gq = [torch.empty(1 << 20, dtype=u8, device=dev) for _ in gx]
+        gst = [(torch.ones(1, device=dev), torch.zeros(16, device=dev), torch.zeros(2, dtype=torch.int32, device=dev),
+                torch.empty(1, device=dev), torch.empty(1, device=dev)) for _ in gx]
+        gws = torch.zeros(len(gx) * 4, dtype=torch.int32, device=dev)
+        garr = (FP8DelayedTensor * len(gx))(*[FP8DelayedTensor(x_.data_ptr(), q_.data_ptr(), x_.numel(), sc_.data_ptr(),
+                                                                h_.data_ptr(), stt_.data_ptr(), su_.data_ptr(),
+                                                                am_.data_ptr())
+                                               for x_, q_, (sc_, h_, stt_, su_, am_) in zip(gx, gq, gst)])
+        launches.append(("k_tensor_cast_delayed_step_grouped", 3 * sum(x_.numel() for x_ in gx), lambda s_: raw.check(
+            L.fp8_quantize_delayed_step_grouped(garr, len(gx), 1, 1, 16, 0, 1.0, 1.0, gws.data_ptr(), s_),
+            "grouped step")))
+        outs = tuple(gq[:4])
+        keep += [gx, gq, gst, gws, garr]
+    elif name == "grouped_weights":
+        ws_ = [inputs.random_matrix(1024, 1024, seed=100 + i, dtype=bf16, scale=0.02, device=dev) for i in range(128)]
+        wq = [torch.empty(1024, 1024, dtype=u8, device=dev) for _ in ws_]
+        wsc = [torch.empty(8, 8, dtype=f32, device=dev) for _ in ws_]
+        arr = (FP8BlockTensor * len(ws_))(*[FP8BlockTensor(w.data_ptr(), q_.data_ptr(), s_.data_ptr(), 1024, 1024)
+                                            for w, q_, s_ in zip(ws_, wq, wsc)])
+        launches.append(("k_quant_grouped", sum(3 * w.numel() + 4 * 64 for w in ws_), lambda s_: raw.check(
+            L.fp8_quantize_blockwise_grouped(arr, len(ws_), 1, 128, 128, 0, s_), "grouped")))
+        outs = tuple(wq[:4]) + tuple(wsc[:4])
+        keep += [ws_, wq, wsc, arr]
+    else:  # per_tensor_sweep28
+        x = inputs.sweep_tensor(28, device=dev)
+        n = x.numel()
+        q = torch.empty(x.shape, dtype=u8, device=dev)
+        so = torch.empty(1, dtype=f32, device=dev)
+        ao = torch.empty(1, dtype=f32, device=dev)
+        launches.append(("k_tensor_amax + k_tensor_cast", 3 * n, lambda s_: raw.check(L.fp8_quantize_per_tensor(
+            x.data_ptr(), 1, n, 1, None, q.data_ptr(), so.data_ptr(), ao.data_ptr(), s_), "per-tensor")))
+        outs = (q, so, ao)
+        keep += [x, q, so, ao]
+    cleaner = torch.ones(1 << 28, dtype=bf16, device=dev)
+    am = torch.empty(1, dtype=f32, device=dev)
+
+    def clean():
+        raw.check(L.fp8_amax(cleaner.data_ptr(), 1, cleaner.numel(), am.data_ptr(), st), "amax")
+
+    for fn in pre:
+        fn(st)
+    clean()
+    for _, _, fn in launches:
+        fn(st)
+        clean()
+    torch.cuda.synchronize()
+    same = None
+    if args.lib:
+        # a variant build must give the default build's bytes: rerun the default on copies of the outputs
+        got = [t.clone() for t in outs]
+        L_var, raw.L = raw.L, Raw(stream).L
+        L = raw.L
+        for fn in pre:
+            fn(st)
+        for _, _, fn in launches:
+            fn(st)
+        torch.cuda.synchronize()
+        bits = lambda t: t.view(torch.int32) if t.dtype == f32 else t.view(torch.int16) if t.dtype == bf16 else t
+        same = all(torch.equal(bits(g_), bits(o_)) for g_, o_ in zip(got, outs))
+        raw.L = L = L_var
+    out = {"probe": name, "what": KERNEL_PROBES[name], "lib": args.lib or "default", "same_as_default": same,
+           "alg_bytes": {k: nb for k, nb, _ in launches}}
+    if args.probe_time:
+        for k, nb, fn in launches:
+            (ms,) = time_per_launch([lambda r, fn=fn: fn(st)], args.probe_time, 3, stream, lambda: cleaner.fill_(1))
+            out.setdefault("timing", {})[k] = {"us": round(ms * 1e3, 2), "GB_s": round(nb / (ms * 1e-3) / 1e9, 1),
+                                               "note": "each launch alone after an L2 flush"}
+    print(json.dumps({"kernel_probe": out}))
+    return 0
+
+
 def traffic_probe(args):
     """One launch of a kernel between L2 cleaners, for an ncu capture of DRAM bytes read and written.
 
@@ -1093,7 +1261,8 @@ def traffic_probe(args):
                                     pass (k_tensor_fused; --probe-time: each call timed alone after an L2
                                     flush, beside the two-pass path).
     --probe-time K     afterwards, also time K back-to-back launches of the probed kernel(s) (not under ncu).
-    --lib PATH         use another build of the library (a variant built with tuning macros)."""
+    --lib PATH         use another build of the library (a variant built with tuning macros).
+    The kernels of the other modes have probes of their own (KERNEL_PROBES, run by kernel_probe)."""
     import torch
     from fine_grained_block_b200 import inputs
     dev = torch.device("cuda", 0)
@@ -1234,7 +1403,8 @@ def main():
                     help="run one launch of each headline kernel between L2 cleaners (for an ncu DRAM capture)")
     ap.add_argument("--traffic-log2n", type=int, default=LOG2_N, help="tensor size of --traffic-probe (2^n)")
     ap.add_argument("--probe", choices=["headline", "128x128", "bt1x128", "gemm_fwd", "gemm_wgrad", "gemm_wgrad_e4m3",
-                                        "gemm_wgrad_b128", "gemm_wgrad_f32out", "gemm_4096", "per_tensor_1mib"],
+                                        "gemm_wgrad_b128", "gemm_wgrad_f32out", "gemm_4096", "per_tensor_1mib",
+                                        *KERNEL_PROBES],
                     default="headline",
                     help="the kernel(s) of --traffic-probe")
     ap.add_argument("--probe-time", type=int, default=0, metavar="K",
@@ -1248,6 +1418,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.oracle_by_config:
         return oracle_by_config(args)
+    if args.traffic_probe and args.probe in KERNEL_PROBES:
+        return kernel_probe(args)
     if args.traffic_probe:
         return traffic_probe(args)
     if args.impl == "reference":
