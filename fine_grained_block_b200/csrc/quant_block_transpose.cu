@@ -179,8 +179,11 @@ struct ColMax<float, BYTES> {
 // column scales into registers once (SCALE_REGS).  Keeping bf16 column
 // maxima as packed |bf16| pairs through shared memory (PACKED_PART: two
 // 16-byte stores per writing lane instead of 16 scalar ones, no unpacking)
-// gives 5567-5573 GB/s against 5429-5431.  128x128: 6462 GB/s (98.7 % of the
-// copy peak) with 3 or 4 CTAs.
+// gives 5567-5573 GB/s against 5429-5431.  Every warp forming the column
+// scales its lanes need (SCALES_IN_WARP: 4 per lane, shared by shuffles)
+// instead of 128 threads forming them behind a second barrier: 5658-5663
+// against 5590-5594 GB/s.  128x128: 6462 GB/s (98.7 % of the copy peak)
+// with 3 or 4 CTAs.
 #ifndef FP8Q_BT_TMA
 #define FP8Q_BT_TMA 0
 #endif
@@ -193,6 +196,10 @@ struct ColMax<float, BYTES> {
 // bf16 column maxima kept as packed |bf16| pairs through shared memory
 #ifndef FP8Q_BLOCK_TRANSPOSE_PACKED_PART
 #define FP8Q_BLOCK_TRANSPOSE_PACKED_PART 1
+#endif
+// 1x128, bf16 with 32-byte lanes: each warp forms the column scales it needs (no second barrier).
+#ifndef FP8Q_BT_SCALES_IN_WARP
+#define FP8Q_BT_SCALES_IN_WARP 1
 #endif
 #ifndef FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS
 #define FP8Q_BLOCK_TRANSPOSE_1X128_MIN_CTAS 4
@@ -288,6 +295,47 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
 #pragma unroll
         for (int i = 0; i < G::kLoads; ++i) v[i] = ld_words_stream(xv + i * vstride);
 #endif
+#if FP8Q_BT_SCALES_IN_WARP
+        if constexpr (kPackedPart && BYTES == 32 && FP8Q_BLOCK_TRANSPOSE_SCALE_REGS) {
+            __syncthreads();
+            // Every warp forms the column scales its lanes need, with no second barrier: the 4 lanes
+            // that hold the same 16 columns (one per row group) each reduce 4 of them over the 8 warps'
+            // packed maxima and share them by shuffles.  Warp 0 stores scales_t.
+            const int rowgrp = lane / G::kVecPerRow;
+            const int w0 = vec_in_row * (V::kElems / 2) + rowgrp * 2;
+            uint32_t ma = part_w[0][w0], mb = part_w[0][w0 + 1];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) {
+                ma = xabsmax_bf16x2(ma, part_w[w][w0]);
+                mb = xabsmax_bf16x2(mb, part_w[w][w0 + 1]);
+            }
+            float s4[4] = {scale_from_amax<FMT>(__uint_as_float(ma << 16)),
+                           scale_from_amax<FMT>(__uint_as_float(ma & 0xFFFF0000u)),
+                           scale_from_amax<FMT>(__uint_as_float(mb << 16)),
+                           scale_from_amax<FMT>(__uint_as_float(mb & 0xFFFF0000u))};
+            if (warp == 0) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    scales_t[(c0 + vec_in_row * V::kElems + rowgrp * 4 + k) * tiles_r + tr] = s4[k];
+            }
+            uint64_t cs2[V::kElems / 2];
+#pragma unroll
+            for (int g = 0; g < V::kElems / 4; ++g) {
+                const int src = g * G::kVecPerRow + vec_in_row;
+                const float a = __shfl_sync(0xFFFFFFFFu, s4[0], src), b = __shfl_sync(0xFFFFFFFFu, s4[1], src);
+                const float c_ = __shfl_sync(0xFFFFFFFFu, s4[2], src), d = __shfl_sync(0xFFFFFFFFu, s4[3], src);
+                cs2[2 * g] = f32x2(a, b);
+                cs2[2 * g + 1] = f32x2(c_, d);
+            }
+#pragma unroll
+            for (int i = 0; i < G::kLoads; ++i) {
+                const int lr = lr0 + i * G::kRowsPerLoad;
+                *reinterpret_cast<typename V::Out*>(tile + tile_off(lr, vec_in_row * V::kElems)) =
+                    PairCast<T, BYTES>::template cast_regs<FMT>(v[i], cs2);
+            }
+        } else
+#endif
+        {
         __syncthreads();
         if (threadIdx.x < kTT) {
             const int c = threadIdx.x;
@@ -337,6 +385,7 @@ k_quant_block_transpose(const T* __restrict__ x, int64_t rows, int64_t cols, uin
                 PairCast<T, BYTES>::template cast<FMT>(v[i], cs);
         }
 #endif
+        }
     }
     __syncthreads();
     tile_transpose_out(tile, qt, rows, r0, c0, lane, warp);
