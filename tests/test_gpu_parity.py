@@ -692,6 +692,31 @@ def test_blockwise_transpose_many_tiles_per_cta(fmt):
     check_blockwise_transpose(x, (1, 128), fmt, "1x128 4096x8192 bf16")
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_blockwise_transpose_edge_values(fmt):
+    """Special rows and columns through x and x^T at once: zero and negative-zero runs, fp32 subnormals,
+    values near the type's maximum, a binade ladder, constant runs, an all-zero 128x128 tile, and columns
+    of each kind, so that row blocks and column blocks both meet them (finite inputs, the contract)."""
+    R, C = 256, 512
+    x = inputs.random_matrix(R, C, seed=78, dtype=torch.float32)
+    x[0, :128] = 0.0
+    x[1, :128] = -0.0
+    x[2, :128] = 1e-42
+    x[3, :128] = torch.linspace(-1e-30, 1e-30, 128)
+    x[4, 128:256] = 3.0e38
+    x[5, 256:384] = torch.tensor([2.0 ** k for k in range(-64, 64)])
+    x[6, :] = 1.0
+    x[128:256, 384:512] = 0.0
+    x[:128, 7] = -0.0                       # a column block of negative zeros
+    x[:128, 8] = 1e-42                      # a column block of subnormals
+    x[:, 9] = torch.tensor([2.0 ** (k % 128 - 64) for k in range(R)])  # binade ladders down a column
+    x[128:, 10] = 2.5e38
+    for dtype in (torch.float32, torch.bfloat16):
+        xd = x.to(dtype)
+        for block in ((1, 128), (128, 128)):
+            check_blockwise_transpose(xd, block, fmt, f"edge {block} {dtype}")
+
+
 def test_blockwise_transpose_16_byte_aligned_input():
     R, C = 256, 512
     x_cpu = inputs.random_matrix(R, C, seed=4400, dtype=torch.bfloat16, outlier_frac=0.01, factor=1e3)
