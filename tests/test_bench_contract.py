@@ -59,3 +59,21 @@ def test_reference_arm_under_two_ranks_prints_once():
     lines = json_lines(r.stdout)
     assert len(lines) == 1
     check_line(lines[0], 2, 1, 3)
+
+
+def test_profile_commands_name_existing_probes():
+    """Every ncu summary under profiles/ names the command that made it; each `--probe` it uses must be one
+    that bench.py offers, so the command still runs as written."""
+    import glob
+    import re
+    help_text = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True,
+                               text=True, check=True, timeout=120).stdout
+    m = re.search(r"--probe \{([^}]*)\}", help_text)
+    assert m, "bench.py --help lists no probe choices"
+    offered = set(m.group(1).replace("\n", "").replace(" ", "").split(","))
+    used = set()
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*")):
+        with open(path, encoding="utf-8") as f:
+            used |= set(re.findall(r"--probe ([a-z0-9_]+)", f.read()))
+    assert used, "no profile names a probe"
+    assert used <= offered, sorted(used - offered)
